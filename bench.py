@@ -1,0 +1,350 @@
+"""Benchmark: RNS-CKKS hybrid key switching at N=2^16 (config 3) on B200.
+
+One step = one pass of the whole key-switching path over one batch of synthetic input:
+  d   = tensor(x, y)            (ct x ct product, 36 limbs)
+  r   = relin(d)                (key switch #1: ModUp, ChaCha12 inner product, ModDown)
+  out = rotate(r, g = 5)        (automorphism + key switch #2)
+at N=2^16, 36 ciphertext + 12 special primes (< 2^30), dnum 3, full level.  The metric is
+key-switches/s (2 per step) over all ranks; rotations/s is reported beside it.
+
+Inputs are synthetic: uniform residues for the ciphertexts and for the keys' stored b halves
+(the cost of every kernel is data independent), seeded per rank.  Three independent buffer
+and key sets (> 126 MB L2 in total) are cycled so that consecutive steps never find their
+inputs in L2.
+
+--impl reference times the CPU oracle (the plain C restatement of the same path) on the host
+cores instead, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+CONFIG_KEY = "3"
+METRIC = "key-switches/s (rotations/s) at N=2^16, 32-bit RNS; % of HBM roofline"
+KS_PER_STEP = 2          # relin + rotation
+ROT_PER_STEP = 1
+N_SETS = 3
+
+
+def _env_int(name, default):
+    try:
+        return int(os.environ.get(name, default))
+    except ValueError:
+        return default
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import fhe_key_switching_b200 as ks
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    cfg = W.CONFIGS[CONFIG_KEY]
+    n, lvl = cfg.n, cfg.level
+    na = lvl + 1
+    q, p = ks.ckks_gen_primes(cfg.log_n, cfg.n_q, cfg.n_p)
+    ctx = ks.Context(cfg.log_n, q, p, cfg.dnum)
+    g = ks.galois_element(cfg.log_n, cfg.rot_steps[0])
+    nd = -(-cfg.n_q // cfg.alpha)
+    mods = q + p
+
+    def residues(moduli, seed_tag):
+        a = W.uniform_residues(moduli, n, W.rng(cfg.seed, W.TAG_SYNTH, rank, seed_tag))
+        return torch.from_numpy(a).to(dev)
+
+    sets = []
+    for s in range(N_SETS):
+        x = residues(q[:na] * 2, 10 * s + 1).view(2, na, n)
+        y = residues(q[:na] * 2, 10 * s + 2).view(2, na, n)
+        b_rel = residues(mods * nd, 10 * s + 3).view(nd, len(mods), n)
+        b_rot = residues(mods * nd, 10 * s + 4).view(nd, len(mods), n)
+        sets.append(dict(x=x, y=y, b_rel=b_rel, b_rot=b_rot,
+                         k_rel=ks.make_evk(b_rel, cfg.chacha_seed, 0),
+                         k_rot=ks.make_evk(b_rot, cfg.chacha_seed, g)))
+    d = torch.empty((3, na, n), dtype=torch.uint32, device=dev)
+    r = torch.empty((2, na, n), dtype=torch.uint32, device=dev)
+    out = torch.empty((2, na, n), dtype=torch.uint32, device=dev)
+    ws = ctx.workspace(lvl, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        st = sets[i % N_SETS]
+        ks.ckks_tensor(ctx, st["x"], st["y"], lvl, d, stream)
+        ks.ckks_relin(ctx, d, lvl, st["k_rel"], r, ws, stream)
+        ks.ckks_rotate(ctx, r, lvl, g, st["k_rot"], out, ws, stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    value = KS_PER_STEP * args.steps * world / (ms / 1e3)
+
+    # end to end: pinned host inputs copied in, result copied out, every step
+    h_x = [s["x"].cpu().pin_memory() for s in sets]
+    h_y = [s["y"].cpu().pin_memory() for s in sets]
+    h_out = torch.empty((2, na, n), dtype=torch.uint32).pin_memory()
+    dx, dy = torch.empty_like(sets[0]["x"]), torch.empty_like(sets[0]["y"])
+
+    def step_e2e(i):
+        st = sets[i % N_SETS]
+        dx.copy_(h_x[i % N_SETS], non_blocking=True)
+        dy.copy_(h_y[i % N_SETS], non_blocking=True)
+        ks.ckks_tensor(ctx, dx, dy, lvl, d, stream)
+        ks.ckks_relin(ctx, d, lvl, st["k_rel"], r, ws, stream)
+        ks.ckks_rotate(ctx, r, lvl, g, st["k_rot"], out, ws, stream)
+        h_out.copy_(out, non_blocking=True)
+
+    for i in range(args.warmup):
+        step_e2e(i)
+    torch.cuda.synchronize()
+    barrier()
+    e0.record(stream)
+    for i in range(args.steps):
+        step_e2e(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms_e2e = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+    e2e_value = KS_PER_STEP * args.steps * world / (ms_e2e / 1e3)
+    h2d = (sets[0]["x"].numel() + sets[0]["y"].numel()) * 4
+    d2h = out.numel() * 4
+
+    cpu = cpu_baseline() if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
+
+    if rank == 0:
+        line = {
+            "metric": METRIC,
+            "value": value,
+            "unit": "key-switches/s",
+            "rotations_per_s": ROT_PER_STEP * args.steps * world / (ms / 1e3),
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms_per_step,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "u32",
+            "data": "synthetic",
+            "config": {"workload": "config 3: N=2^16, 36+12 primes < 2^30, dnum 3, level 35; "
+                                   "step = tensor + relin + rotate(1)",
+                       "log_n": cfg.log_n, "n_q": cfg.n_q, "n_p": cfg.n_p, "dnum": cfg.dnum,
+                       "level": lvl, "key_switches_per_step": KS_PER_STEP,
+                       "l2": f"{N_SETS} rotating input/key sets (~{N_SETS * 150} MiB > 126 MB L2)",
+                       "parallelism": f"replicas x{world}"},
+            "e2e": {"value": e2e_value, "unit": "key-switches/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": args.steps * LAUNCHES_PER_STEP,
+            "clocks": clk,
+            "roofline": None,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+# kernels launched by one step: tensor (1) + 2 key switches x 13 (+0 automorphism kernels:
+# the rotation gathers inside the inverse-NTT load, the inner product and the combine)
+LAUNCHES_PER_STEP = 1 + 2 * 13
+
+
+def _oracle_sample():
+    """Bounded CPU sample of the same step: one relinearisation and one rotation at config 3,
+    timed on the oracle with synthetic residues (cost is data independent)."""
+    import numpy as np
+    import oracle
+
+    cfg = W.CONFIGS[CONFIG_KEY]
+    ctx = oracle.Ctx(cfg.log_n, cfg.n_q, cfg.n_p)
+    n, lvl = cfg.n, cfg.level
+    na = lvl + 1
+    nd = -(-cfg.n_q // cfg.alpha)
+    gen = W.rng(cfg.seed, W.TAG_SYNTH, 99)
+    x = W.uniform_residues(ctx.q[:na] * 2, n, gen).reshape(2, na, n)
+    y = W.uniform_residues(ctx.q[:na] * 2, n, gen).reshape(2, na, n)
+    b = W.uniform_residues(ctx.mod * nd, n, gen).reshape(nd, len(ctx.mod), n)
+    g = ctx.galois(1)
+
+    def one_step():
+        dd = ctx.tensor(x, y, lvl)
+        rr = ctx.relin(dd, lvl, cfg.alpha, b, cfg.chacha_seed, 0)
+        ctx.rotate(rr, lvl, cfg.alpha, g, b, cfg.chacha_seed, g)
+
+    return one_step
+
+
+def _omp_threads():
+    v = os.environ.get("OMP_NUM_THREADS")
+    return int(v) if v and v.isdigit() else (os.cpu_count() or 1)
+
+
+def cpu_baseline(max_seconds: float = 20.0):
+    one_step = _oracle_sample()
+    one_step()                              # warm (tables, page faults)
+    t0 = time.perf_counter()
+    k = 0
+    while True:
+        one_step()
+        k += 1
+        if time.perf_counter() - t0 > max_seconds / 2 or k >= 8:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": KS_PER_STEP * k / dt, "unit": "key-switches/s", "cores": _omp_threads(),
+            "kind": "oracle",
+            "sample": f"{k} steps of config 3 (tensor + relin + rotate, 2 key switches each) "
+                      "on synthetic residues, plain C oracle with OpenMP over limbs"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    one_step = _oracle_sample()
+    for _ in range(args.warmup):
+        one_step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        one_step()
+    dt = time.perf_counter() - t0
+    value = KS_PER_STEP * args.steps / dt
+    cfg = W.CONFIGS[CONFIG_KEY]
+    line = {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": value,
+        "unit": "key-switches/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": 1e3 * dt / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "u32",
+        "data": "synthetic",
+        "config": {"workload": "config 3: N=2^16, 36+12 primes < 2^30, dnum 3, level 35; "
+                               "step = tensor + relin + rotate(1)",
+                   "log_n": cfg.log_n, "n_q": cfg.n_q, "n_p": cfg.n_p, "dnum": cfg.dnum,
+                   "level": cfg.level, "key_switches_per_step": KS_PER_STEP},
+        "cpu_baseline": {"kind": "oracle", "cores": _omp_threads(), "value": value,
+                         "unit": "key-switches/s",
+                         "sample": f"{args.steps} timed steps of config 3 on the host cores"},
+        "e2e": {"value": value, "unit": "key-switches/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    rank = _env_int("RANK", 0)
+    world = _env_int("WORLD_SIZE", 1)
+    local_rank = _env_int("LOCAL_RANK", 0)
+    if args.impl == "reference":
+        if args.steps > 3:
+            args.steps = 3          # each oracle step is seconds of CPU work
+        args.warmup = min(args.warmup, 1)
+        run_reference(args, rank, world)
+        return
+    run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,237 @@
+"""B200 (sm_100a) RNS-CKKS hybrid key switching with in-kernel ChaCha12 key regeneration.
+
+Thin Python binding of the C ABI in ``include/ckks_ks.h`` (argument marshalling only: every
+step of the key-switching path runs in the library's CUDA kernels).  PyTorch supplies device
+memory and streams.  The functions keep the C names; buffers are CUDA tensors of dtype
+uint32 or int32 (reinterpreted), contiguous, laid out as the header states.
+
+There is no CPU fallback: if the compiled library is missing, importing this package raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "_build", "libckks_ks.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"CUDA library {LIB_PATH} is not built; run `python -m fhe_key_switching_b200.build` "
+        "(nvcc, sm_100a) first")
+
+_L = ctypes.CDLL(LIB_PATH)
+
+CKKS_OK, CKKS_ERR_ARG, CKKS_ERR_UNSUPPORTED, CKKS_ERR_ALIGN = 0, -1, -2, -3
+CKKS_ERR_WORKSPACE, CKKS_ERR_CUDA, CKKS_ERR_TIMEOUT = -4, -5, -6
+
+_u32p = ctypes.POINTER(ctypes.c_uint32)
+_vp = ctypes.c_void_p
+_ci, _cu, _sz = ctypes.c_int, ctypes.c_uint32, ctypes.c_size_t
+
+
+class ckks_params(ctypes.Structure):
+    _fields_ = [("log_n", _cu), ("n_q", _cu), ("n_p", _cu), ("dnum", _cu),
+                ("q", _u32p), ("p", _u32p)]
+
+
+class ckks_evk(ctypes.Structure):
+    _fields_ = [("b", _vp), ("a", _vp), ("seed", ctypes.c_uint8 * 32), ("key_id", _cu)]
+
+
+_SIGS = {
+    "ckks_gen_primes": (_ci, [_cu, _cu, _cu, _u32p, _u32p]),
+    "ckks_ctx_create": (_ci, [ctypes.POINTER(ckks_params), ctypes.POINTER(_vp)]),
+    "ckks_ctx_destroy": (None, [_vp]),
+    "ckks_ntt_fwd": (_ci, [_vp, _vp, _ci, _ci, _vp]),
+    "ckks_ntt_inv": (_ci, [_vp, _vp, _ci, _ci, _vp]),
+    "ckks_automorph": (_ci, [_vp, _vp, _vp, _ci, _cu, _vp]),
+    "ckks_modup": (_ci, [_vp, _vp, _ci, _vp, _vp, _sz, _vp]),
+    "ckks_inner_product": (_ci, [_vp, _vp, _ci, ctypes.POINTER(ckks_evk), _vp, _vp]),
+    "ckks_moddown": (_ci, [_vp, _vp, _ci, _vp, _vp, _sz, _vp]),
+    "ckks_keyswitch": (_ci, [_vp, _vp, _ci, ctypes.POINTER(ckks_evk), _vp, _vp, _sz, _vp]),
+    "ckks_rotate": (_ci, [_vp, _vp, _ci, _cu, ctypes.POINTER(ckks_evk), _vp, _vp, _sz, _vp]),
+    "ckks_rotate_hoisted": (_ci, [_vp, _vp, _ci, _ci, _u32p, ctypes.POINTER(ckks_evk), _vp, _vp,
+                                  _sz, _vp]),
+    "ckks_relin": (_ci, [_vp, _vp, _ci, ctypes.POINTER(ckks_evk), _vp, _vp, _sz, _vp]),
+    "ckks_tensor": (_ci, [_vp, _vp, _vp, _ci, _vp, _vp]),
+    "ckks_chacha_expand": (_ci, [_vp, ctypes.POINTER(ctypes.c_uint8), _cu, _ci, _ci, _vp, _vp]),
+    "ckks_workspace_bytes": (_sz, [_vp, _ci, _ci]),
+    "ckks_sync_status": (_ci, [_vp, _vp, _ci]),
+    "ckks_last_error": (ctypes.c_char_p, []),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _f = getattr(_L, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+EXPORTED = tuple(_SIGS)
+
+
+class CkksError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        msg = _L.ckks_last_error().decode(errors="replace")
+        super().__init__(f"{where} failed ({code}): {msg}")
+        self.code = code
+
+
+def _check(code: int, where: str) -> int:
+    if code != CKKS_OK:
+        raise CkksError(code, where)
+    return code
+
+
+def _ptr(t) -> int:
+    """Device pointer of a CUDA tensor (no copy, no dtype conversion)."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+# ----------------------------------------------------------------------------- parameters
+
+def ckks_gen_primes(log_n: int, n_q: int, n_p: int):
+    """The library's prime chain rule; returns (q list, p list)."""
+    q = (ctypes.c_uint32 * max(n_q, 1))()
+    p = (ctypes.c_uint32 * max(n_p, 1))()
+    _check(_L.ckks_gen_primes(log_n, n_q, n_p, q, p), "ckks_gen_primes")
+    return list(q)[:n_q], list(p)[:n_p]
+
+
+class Context:
+    """Owns a ckks_ctx (device tables for one parameter set)."""
+
+    def __init__(self, log_n: int, q, p, dnum: int):
+        qa = (ctypes.c_uint32 * len(q))(*q)
+        pa = (ctypes.c_uint32 * len(p))(*p)
+        prm = ckks_params(log_n, len(q), len(p), dnum, qa, pa)
+        h = _vp()
+        _check(_L.ckks_ctx_create(ctypes.byref(prm), ctypes.byref(h)), "ckks_ctx_create")
+        self.handle = h
+        self.log_n, self.n, self.q, self.p, self.dnum = log_n, 1 << log_n, list(q), list(p), dnum
+        self.n_q, self.n_p = len(q), len(p)
+        self.alpha = -(-self.n_q // dnum)
+
+    def close(self):
+        if getattr(self, "handle", None):
+            _L.ckks_ctx_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    @property
+    def _as_parameter_(self):
+        return self.handle
+
+    def workspace_bytes(self, level: int, n_rot: int = 1) -> int:
+        return int(_L.ckks_workspace_bytes(self.handle, level, n_rot))
+
+    def workspace(self, level: int, n_rot: int = 1, device=None):
+        import torch
+        return torch.empty(self.workspace_bytes(level, n_rot), dtype=torch.uint8,
+                           device=device or torch.device("cuda", torch.cuda.current_device()))
+
+
+def ckks_ctx_create(log_n: int, q, p, dnum: int) -> Context:
+    return Context(log_n, q, p, dnum)
+
+
+def make_evk(b, seed: bytes, key_id: int, a=None) -> ckks_evk:
+    """Key-switching key record: b (and optionally a stored a) are CUDA tensors
+    [D][n_q+n_p][N]; the caller keeps them alive while the record is used."""
+    k = ckks_evk()
+    k.b = _ptr(b)
+    k.a = _ptr(a) if a is not None else None
+    if len(seed) != 32:
+        raise ValueError("seed must be 32 bytes")
+    ctypes.memmove(k.seed, seed, 32)
+    k.key_id = key_id
+    return k
+
+
+# ----------------------------------------------------------------------------- operations
+
+def ckks_ntt_fwd(ctx, poly, first_limb: int, n_limbs: int, stream=None):
+    _check(_L.ckks_ntt_fwd(ctx.handle, _ptr(poly), first_limb, n_limbs, _stream(stream)), "ckks_ntt_fwd")
+
+
+def ckks_ntt_inv(ctx, poly, first_limb: int, n_limbs: int, stream=None):
+    _check(_L.ckks_ntt_inv(ctx.handle, _ptr(poly), first_limb, n_limbs, _stream(stream)), "ckks_ntt_inv")
+
+
+def ckks_automorph(ctx, inp, out, n_limbs: int, galois: int, stream=None):
+    _check(_L.ckks_automorph(ctx.handle, _ptr(inp), _ptr(out), n_limbs, galois, _stream(stream)),
+           "ckks_automorph")
+
+
+def ckks_modup(ctx, c, level: int, dtilde, ws, stream=None):
+    _check(_L.ckks_modup(ctx.handle, _ptr(c), level, _ptr(dtilde), _ptr(ws), ws.numel() * ws.element_size(),
+                         _stream(stream)), "ckks_modup")
+
+
+def ckks_inner_product(ctx, dtilde, level: int, evk: ckks_evk, acc, stream=None):
+    _check(_L.ckks_inner_product(ctx.handle, _ptr(dtilde), level, ctypes.byref(evk), _ptr(acc),
+                                 _stream(stream)), "ckks_inner_product")
+
+
+def ckks_moddown(ctx, acc, level: int, out, ws, stream=None):
+    _check(_L.ckks_moddown(ctx.handle, _ptr(acc), level, _ptr(out), _ptr(ws), ws.numel() * ws.element_size(),
+                           _stream(stream)), "ckks_moddown")
+
+
+def ckks_keyswitch(ctx, c, level: int, evk: ckks_evk, out, ws, stream=None):
+    _check(_L.ckks_keyswitch(ctx.handle, _ptr(c), level, ctypes.byref(evk), _ptr(out), _ptr(ws),
+                             ws.numel() * ws.element_size(), _stream(stream)), "ckks_keyswitch")
+
+
+def ckks_rotate(ctx, ct, level: int, galois: int, evk: ckks_evk, out, ws, stream=None):
+    _check(_L.ckks_rotate(ctx.handle, _ptr(ct), level, galois, ctypes.byref(evk), _ptr(out), _ptr(ws),
+                          ws.numel() * ws.element_size(), _stream(stream)), "ckks_rotate")
+
+
+def ckks_rotate_hoisted(ctx, ct, level: int, galois, evks, out, ws, stream=None):
+    n = len(galois)
+    ga = (ctypes.c_uint32 * max(n, 1))(*galois)
+    ka = (ckks_evk * max(n, 1))(*evks)
+    _check(_L.ckks_rotate_hoisted(ctx.handle, _ptr(ct), level, n, ga, ka, _ptr(out), _ptr(ws),
+                                  ws.numel() * ws.element_size(), _stream(stream)), "ckks_rotate_hoisted")
+
+
+def ckks_relin(ctx, d, level: int, evk: ckks_evk, out, ws, stream=None):
+    _check(_L.ckks_relin(ctx.handle, _ptr(d), level, ctypes.byref(evk), _ptr(out), _ptr(ws),
+                         ws.numel() * ws.element_size(), _stream(stream)), "ckks_relin")
+
+
+def ckks_tensor(ctx, x, y, level: int, d, stream=None):
+    _check(_L.ckks_tensor(ctx.handle, _ptr(x), _ptr(y), level, _ptr(d), _stream(stream)), "ckks_tensor")
+
+
+def ckks_chacha_expand(ctx, seed: bytes, key_id: int, digit: int, limb: int, out, stream=None):
+    sb = (ctypes.c_uint8 * 32).from_buffer_copy(seed)
+    _check(_L.ckks_chacha_expand(ctx.handle, sb, key_id, digit, limb, _ptr(out), _stream(stream)),
+           "ckks_chacha_expand")
+
+
+def ckks_sync_status(ctx, stream=None, timeout_ms: int = 10000) -> int:
+    return int(_L.ckks_sync_status(ctx.handle if ctx is not None else None, _stream(stream), timeout_ms))
+
+
+def galois_element(log_n: int, r: int) -> int:
+    """Galois element of a rotation by r slots: 5^r mod 2N (r < 0: 5^(N/2+r))."""
+    n = 1 << log_n
+    return pow(5, r % (n // 2), 2 * n)

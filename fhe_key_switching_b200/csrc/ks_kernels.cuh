@@ -1,0 +1,316 @@
+// ks_kernels.cuh -- base conversion, ChaCha12-fused key inner product, ModDown combine,
+// tensor product and automorphism kernels.
+#pragma once
+#include "ntt.cuh"
+
+// ---------------------------------------------------------------- ChaCha12
+// Block function (Bernstein 2008) with the RFC 8439 sec. 2.3 state: "expand 32-byte k",
+// the key as 8 little-endian words, a 32-bit block counter, three nonce words; 12 rounds
+// (6 column/diagonal double rounds) then the feed-forward addition.
+struct ChachaKey {
+    u32 k[8];
+};
+
+__device__ __forceinline__ u32 rotl(u32 v, int c) { return __funnelshift_l(v, v, c); }
+
+#define CKKS_QR(a, b, c, d)                 \
+    a += b; d ^= a; d = rotl(d, 16);        \
+    c += d; b ^= c; b = rotl(b, 12);        \
+    a += b; d ^= a; d = rotl(d, 8);         \
+    c += d; b ^= c; b = rotl(b, 7);
+
+__device__ __forceinline__ void chacha12_block(const ChachaKey &key, u32 counter, u32 n0, u32 n1,
+                                               u32 n2, u32 (&o)[16]) {
+    const u32 c0 = 0x61707865u, c1 = 0x3320646eu, c2 = 0x79622d32u, c3 = 0x6b206574u;
+    u32 x0 = c0, x1 = c1, x2 = c2, x3 = c3;
+    u32 x4 = key.k[0], x5 = key.k[1], x6 = key.k[2], x7 = key.k[3];
+    u32 x8 = key.k[4], x9 = key.k[5], x10 = key.k[6], x11 = key.k[7];
+    u32 x12 = counter, x13 = n0, x14 = n1, x15 = n2;
+#pragma unroll
+    for (int r = 0; r < 6; r++) {
+        CKKS_QR(x0, x4, x8, x12) CKKS_QR(x1, x5, x9, x13)
+        CKKS_QR(x2, x6, x10, x14) CKKS_QR(x3, x7, x11, x15)
+        CKKS_QR(x0, x5, x10, x15) CKKS_QR(x1, x6, x11, x12)
+        CKKS_QR(x2, x7, x8, x13) CKKS_QR(x3, x4, x9, x14)
+    }
+    o[0] = x0 + c0; o[1] = x1 + c1; o[2] = x2 + c2; o[3] = x3 + c3;
+    o[4] = x4 + key.k[0]; o[5] = x5 + key.k[1]; o[6] = x6 + key.k[2]; o[7] = x7 + key.k[3];
+    o[8] = x8 + key.k[4]; o[9] = x9 + key.k[5]; o[10] = x10 + key.k[6]; o[11] = x11 + key.k[7];
+    o[12] = x12 + counter; o[13] = x13 + n0; o[14] = x14 + n1; o[15] = x15 + n2;
+}
+
+// a[n] for the 8 coefficients of block b: 64-bit LE word m = (o[2m] | o[2m+1] << 32) mod q,
+// lazily in [0, 4q) (canonical when CANON).
+template <bool CANON>
+__device__ __forceinline__ void chacha_coeffs(const ChachaKey &key, u32 key_id, u32 digit, u32 limb,
+                                              u32 block, const PrimeInfo &pi, u32 (&a)[8]) {
+    u32 o[16];
+    chacha12_block(key, block, key_id, digit, limb, o);
+#pragma unroll
+    for (int m = 0; m < 8; m++) {
+        u32 v = shoup_mul(o[2 * m + 1], pi.r64, pi.r64p, pi.q) + shoup_mul(o[2 * m], 1u, pi.onep, pi.q);
+        if (CANON) v = csub(csub(v, 2 * pi.q), pi.q);
+        a[m] = v;
+    }
+}
+
+__global__ void k_chacha_expand(ChachaKey key, u32 key_id, u32 digit, u32 limb,
+                                const PrimeInfo *pinfo, u32 *out, int n) {
+    const int b = blockIdx.x * blockDim.x + threadIdx.x;
+    if (b >= n / 8) return;
+    const PrimeInfo pi = pinfo[limb];
+    u32 a[8];
+    chacha_coeffs<true>(key, key_id, digit, limb, (u32)b, pi, a);
+    uint4 *o = reinterpret_cast<uint4 *>(out + 8 * b);
+    o[0] = make_uint4(a[0], a[1], a[2], a[3]);
+    o[1] = make_uint4(a[4], a[5], a[6], a[7]);
+}
+
+// ---------------------------------------------------------------- fast base conversion
+// For group g (a ModUp digit or a ModDown operand) with inputs y_i (coefficient domain,
+// canonical, already multiplied by (D/r_i)^-1) and every target k of the group:
+//   out_k = sum_i y_i [D/r_i]_t - v [D]_t  (mod t),  v = #{i : y_i > (r_i - 1)/2},
+// i.e. the sum over the centred representatives y_i - r_i [y_i > (r_i-1)/2].
+struct BconvArgs {
+    const u32 *y;            // input rows
+    u32 *out;                // output rows
+    const PrimeInfo *pinfo;
+    const u32 *bmat;         // per group config: [n_in][n_primes] = [D/r_i]_t
+    const u32 *negd;         // per group config: [n_primes] = [-D]_t
+    JobMap map;              // targets: per_group, split, bases, out rows, skip_alpha
+    int n_primes;            // row length of bmat/negd tables (global limbs)
+    int log_n;
+    // inputs of group g: rows in_row0 + g * in_group_rows + i, primes in_prime0 + g*in_prime_step + i
+    int in_row0, in_group_rows, in_prime0, in_prime_step;
+    int n_in_full;           // inputs per group (the last group may have fewer: n_in_last)
+    int n_in_last;
+    int n_groups;
+    int cfg_per_group;       // table config index = g * cfg_per_group + (n_in(g) - 1) (ModUp), or 0
+    int cfg_stride;          // words per config in bmat = max_in * n_primes
+};
+
+constexpr int BCONV_THREADS = 256;
+constexpr int BCONV_MAX_IN = 64;
+
+__global__ void __launch_bounds__(BCONV_THREADS)
+k_bconv(BconvArgs a) {
+    extern __shared__ u32 smb[];          // [n_in][per_group] constants, then [per_group] negd
+    const int g = blockIdx.y;
+    const int n = 1 << a.log_n;
+    const int n_in = (g == a.n_groups - 1) ? a.n_in_last : a.n_in_full;
+    const int cfg = a.cfg_per_group ? g * a.cfg_per_group + (n_in - 1) : 0;
+    const u32 *bm = a.bmat + (size_t)cfg * a.cfg_stride;
+    const u32 *nd = a.negd + (size_t)cfg * a.n_primes;
+    const int T = a.map.per_group;
+    // stage the conversion constants of this group's targets in shared memory
+    for (int idx = threadIdx.x; idx < (n_in + 1) * T; idx += blockDim.x) {
+        const int i = idx / T, kk = idx - i * T;
+        const int t = kk < a.map.split ? a.map.lo_base + kk : a.map.hi_base + (kk - a.map.split);
+        smb[idx] = (i < n_in) ? bm[(size_t)i * a.n_primes + t] : nd[t];
+    }
+    __syncthreads();
+    const int c = blockIdx.x * blockDim.x + threadIdx.x;   // coefficient
+    if (c >= n) return;
+    u32 y[BCONV_MAX_IN];
+    u32 v = 0;
+    const int row0 = a.in_row0 + g * a.in_group_rows;
+    const int p0 = a.in_prime0 + g * a.in_prime_step;
+    for (int i = 0; i < n_in; i++) {
+        y[i] = a.y[(size_t)(row0 + i) * n + c];
+        v += (y[i] > a.pinfo[p0 + i].half) ? 1u : 0u;
+    }
+    const int lo = a.map.skip_alpha > 0 ? g * a.map.skip_alpha : 0;
+    const int hi = a.map.skip_alpha > 0 ? min(lo + a.map.skip_alpha, a.map.split) : 0;
+    for (int kk = 0; kk < T; kk++) {
+        if (kk >= lo && kk < hi) continue;
+        const int t = kk < a.map.split ? a.map.lo_base + kk : a.map.hi_base + (kk - a.map.split);
+        const PrimeInfo pi = a.pinfo[t];
+        u64 acc = (u64)v * smb[n_in * T + kk];
+        for (int i = 0; i < n_in; i++) {
+            acc += (u64)y[i] * smb[i * T + kk];
+            if ((i % 14) == 13) acc = reduce64_lazy(acc, pi.q, pi.r64, pi.r64p, pi.onep);
+        }
+        const u32 r = reduce64(acc, pi.q, pi.r64, pi.r64p, pi.onep);
+        a.out[((size_t)g * a.map.out_group_rows + a.map.out_k_base + kk) * n + c] = r;
+    }
+}
+
+// ---------------------------------------------------------------- key inner product
+// acc0[u] = sum_j dt_j[u] b_j[t], acc1[u] = sum_j dt_j[u] a_j[t] over the active digits, with
+// a_j[t] regenerated by ChaCha12 (or read from a stored a half).  For u inside digit j the
+// extended digit equals the input polynomial itself (cdig).  hoist_g != 0: every dt row is
+// read through kappa_{hoist_g} (hoisted rotation); cdig_g != 0: cdig is read through
+// kappa_{cdig_g} (single rotation, whose ModUp input was kappa_g(c1)).
+struct IpArgs {
+    const u32 *dt;           // [beta][ext][N]
+    const u32 *cdig;         // [l+1][N]: digit limbs (nullptr: read them from dt)
+    const u32 *b;            // [D][n_primes][N]
+    const u32 *a_stored;     // nullptr: regenerate
+    u32 *acc;                // [2][ext][N]
+    const PrimeInfo *pinfo;
+    ChachaKey key;
+    u32 key_id;
+    int log_n, level, n_q, n_primes, alpha, beta, ext;
+    u32 hoist_g, cdig_g;
+};
+
+constexpr int IP_THREADS = 128;
+
+__global__ void __launch_bounds__(IP_THREADS)
+k_inner_product(IpArgs a) {
+    const int n = 1 << a.log_n;
+    const int blk = blockIdx.x * blockDim.x + threadIdx.x;   // 8 coefficients each
+    if (blk >= n / 8) return;
+    const int u = blockIdx.y;
+    const int na = a.level + 1;
+    const int t = u < na ? u : a.n_q + (u - na);
+    const PrimeInfo pi = a.pinfo[t];
+    u64 s0[8], s1[8];
+#pragma unroll
+    for (int m = 0; m < 8; m++) s0[m] = s1[m] = 0;
+    for (int j = 0; j < a.beta; j++) {
+        const bool in_digit = a.cdig && u < na && u >= j * a.alpha && u < min(j * a.alpha + a.alpha, na);
+        const u32 *src = in_digit ? a.cdig + (size_t)u * n : a.dt + ((size_t)j * a.ext + u) * n;
+        const u32 g = in_digit ? (a.hoist_g ? a.hoist_g : a.cdig_g) : a.hoist_g;
+        u32 d[8];
+        if (g) {
+#pragma unroll
+            for (int m = 0; m < 8; m++) d[m] = src[automorph_src((u32)(8 * blk + m), g, a.log_n)];
+        } else {
+            const uint4 *s4 = reinterpret_cast<const uint4 *>(src + 8 * blk);
+            const uint4 p = s4[0], q4 = s4[1];
+            d[0] = p.x; d[1] = p.y; d[2] = p.z; d[3] = p.w;
+            d[4] = q4.x; d[5] = q4.y; d[6] = q4.z; d[7] = q4.w;
+        }
+        const uint4 *b4 = reinterpret_cast<const uint4 *>(a.b + ((size_t)j * a.n_primes + t) * n + 8 * blk);
+        const uint4 bp = b4[0], bq = b4[1];
+        const u32 bb[8] = {bp.x, bp.y, bp.z, bp.w, bq.x, bq.y, bq.z, bq.w};
+        u32 av[8];
+        if (a.a_stored) {
+            const uint4 *a4 = reinterpret_cast<const uint4 *>(a.a_stored + ((size_t)j * a.n_primes + t) * n + 8 * blk);
+            const uint4 ap = a4[0], aq = a4[1];
+            av[0] = ap.x; av[1] = ap.y; av[2] = ap.z; av[3] = ap.w;
+            av[4] = aq.x; av[5] = aq.y; av[6] = aq.z; av[7] = aq.w;
+        } else {
+            chacha_coeffs<false>(a.key, a.key_id, (u32)j, (u32)t, (u32)blk, pi, av);
+        }
+#pragma unroll
+        for (int m = 0; m < 8; m++) {
+            s0[m] += (u64)d[m] * bb[m];          // < 2^60 per term
+            s1[m] += (u64)d[m] * av[m];          // a lazy < 4q: < 2^62 per term
+        }
+        if ((j & 1) == 1) {
+#pragma unroll
+            for (int m = 0; m < 8; m++) {
+                s0[m] = reduce64_lazy(s0[m], pi.q, pi.r64, pi.r64p, pi.onep);
+                s1[m] = reduce64_lazy(s1[m], pi.q, pi.r64, pi.r64p, pi.onep);
+            }
+        }
+    }
+    u32 r0[8], r1[8];
+#pragma unroll
+    for (int m = 0; m < 8; m++) {
+        r0[m] = reduce64(s0[m], pi.q, pi.r64, pi.r64p, pi.onep);
+        r1[m] = reduce64(s1[m], pi.q, pi.r64, pi.r64p, pi.onep);
+    }
+    uint4 *o0 = reinterpret_cast<uint4 *>(a.acc + (size_t)u * n + 8 * blk);
+    uint4 *o1 = reinterpret_cast<uint4 *>(a.acc + ((size_t)a.ext + u) * n + 8 * blk);
+    o0[0] = make_uint4(r0[0], r0[1], r0[2], r0[3]);
+    o0[1] = make_uint4(r0[4], r0[5], r0[6], r0[7]);
+    o1[0] = make_uint4(r1[0], r1[1], r1[2], r1[3]);
+    o1[1] = make_uint4(r1[4], r1[5], r1[6], r1[7]);
+}
+
+// ---------------------------------------------------------------- ModDown combine
+// out_c[i] = (acc_c[i] - conv_c[i]) [P^-1]_{q_i} + add_c[i]   (mod q_i), c = 0, 1.
+// add: nullptr, or [2][l+1][N] rows (relinearisation), or component 0 only gathered through
+// kappa_{add_g} (rotation, add0_only).
+struct CombineArgs {
+    const u32 *acc;          // [2][ext][N]  (Q rows 0..l of each component used)
+    const u32 *conv;         // [2][l+1][N]
+    const u32 *add;          // see above
+    u32 *out;                // [2][l+1][N]
+    const PrimeInfo *pinfo;
+    const tw_t *pinv;        // [n_q] (P^-1 mod q_i, Shoup)
+    int log_n, level, ext;
+    int add_comps;           // 0, 1 (component 0 only) or 2
+    u32 add_g;               // gather add through kappa_g
+};
+
+__global__ void k_moddown_combine(CombineArgs a) {
+    const int n = 1 << a.log_n;
+    const int c4 = blockIdx.x * blockDim.x + threadIdx.x;    // 4 coefficients each
+    if (c4 >= n / 4) return;
+    const int i = blockIdx.y, comp = blockIdx.z;
+    const int na = a.level + 1;
+    const PrimeInfo pi = a.pinfo[i];
+    const u32 q = pi.q;
+    const tw_t w = a.pinv[i];
+    const uint4 av = reinterpret_cast<const uint4 *>(a.acc + ((size_t)comp * a.ext + i) * n)[c4];
+    const uint4 cv = reinterpret_cast<const uint4 *>(a.conv + ((size_t)comp * na + i) * n)[c4];
+    u32 r[4] = {av.x + q - cv.x, av.y + q - cv.y, av.z + q - cv.z, av.w + q - cv.w};
+#pragma unroll
+    for (int m = 0; m < 4; m++) r[m] = csub(shoup_mul(r[m], w.x, w.y, q), q);
+    if (comp < a.add_comps) {
+        const u32 *src = a.add + ((size_t)comp * na + i) * n;
+        u32 ad[4];
+        if (a.add_g) {
+#pragma unroll
+            for (int m = 0; m < 4; m++) ad[m] = src[automorph_src((u32)(4 * c4 + m), a.add_g, a.log_n)];
+        } else {
+            const uint4 t = reinterpret_cast<const uint4 *>(src)[c4];
+            ad[0] = t.x; ad[1] = t.y; ad[2] = t.z; ad[3] = t.w;
+        }
+#pragma unroll
+        for (int m = 0; m < 4; m++) r[m] = csub(r[m] + ad[m], q);
+    }
+    reinterpret_cast<uint4 *>(a.out + ((size_t)comp * na + i) * n)[c4] = make_uint4(r[0], r[1], r[2], r[3]);
+}
+
+// ---------------------------------------------------------------- tensor product
+__global__ void k_tensor(const u32 *x, const u32 *y, u32 *d, const PrimeInfo *pinfo, int log_n,
+                         int level) {
+    const int n = 1 << log_n;
+    const int c4 = blockIdx.x * blockDim.x + threadIdx.x;
+    if (c4 >= n / 4) return;
+    const int i = blockIdx.y;
+    const size_t pl = (size_t)(level + 1) * n;
+    const PrimeInfo pi = pinfo[i];
+    const size_t off = (size_t)i * n;
+    const uint4 x0 = reinterpret_cast<const uint4 *>(x + off)[c4];
+    const uint4 x1 = reinterpret_cast<const uint4 *>(x + pl + off)[c4];
+    const uint4 y0 = reinterpret_cast<const uint4 *>(y + off)[c4];
+    const uint4 y1 = reinterpret_cast<const uint4 *>(y + pl + off)[c4];
+    const u32 a0[4] = {x0.x, x0.y, x0.z, x0.w}, a1[4] = {x1.x, x1.y, x1.z, x1.w};
+    const u32 b0[4] = {y0.x, y0.y, y0.z, y0.w}, b1[4] = {y1.x, y1.y, y1.z, y1.w};
+    u32 r0[4], r1[4], r2[4];
+#pragma unroll
+    for (int m = 0; m < 4; m++) {
+        r0[m] = reduce64((u64)a0[m] * b0[m], pi.q, pi.r64, pi.r64p, pi.onep);
+        r1[m] = reduce64((u64)a0[m] * b1[m] + (u64)a1[m] * b0[m], pi.q, pi.r64, pi.r64p, pi.onep);
+        r2[m] = reduce64((u64)a1[m] * b1[m], pi.q, pi.r64, pi.r64p, pi.onep);
+    }
+    reinterpret_cast<uint4 *>(d + off)[c4] = make_uint4(r0[0], r0[1], r0[2], r0[3]);
+    reinterpret_cast<uint4 *>(d + pl + off)[c4] = make_uint4(r1[0], r1[1], r1[2], r1[3]);
+    reinterpret_cast<uint4 *>(d + 2 * pl + off)[c4] = make_uint4(r2[0], r2[1], r2[2], r2[3]);
+}
+
+// ---------------------------------------------------------------- automorphism
+__global__ void k_automorph(const u32 *in, u32 *out, int log_n, u32 g) {
+    const int n = 1 << log_n;
+    const int k = blockIdx.x * blockDim.x + threadIdx.x;
+    if (k >= n) return;
+    const size_t off = (size_t)blockIdx.y * n;
+    out[off + k] = in[off + automorph_src((u32)k, g, log_n)];
+}
+
+// digit limbs of the extended output: dtilde[j][u] = c[u] for u inside digit j
+__global__ void k_copy_digit_limbs(const u32 *c, u32 *dt, int log_n, int level, int alpha, int ext) {
+    const int n = 1 << log_n;
+    const int c4 = blockIdx.x * blockDim.x + threadIdx.x;
+    if (c4 >= n / 4) return;
+    const int u = blockIdx.y;            // 0..level
+    const int j = u / alpha;
+    reinterpret_cast<uint4 *>(dt + ((size_t)j * ext + u) * n)[c4] =
+        reinterpret_cast<const uint4 *>(c + (size_t)u * n)[c4];
+}

@@ -1,0 +1,270 @@
+// ntt.cuh -- two-pass negacyclic NTT for N = R1 * 256 (R1 = 2^r1, 4 <= r1 <= 8).
+//
+// Definition (the library's evaluation domain): A[k] = sum_n a[n] psi^((2 brv(k)+1) n) mod q.
+// Schedule: the iterative Cooley-Tukey transform with the psi powers merged into the
+// twiddles; global stage s pairs j and j + N/2^(s+1) with twiddle psi^brv(idx),
+// idx = 2^s + (j >> (log_n - s)).  Its output is the definition above in bit-reversed order.
+//
+// The N coefficients are viewed as a R1 x 256 row-major matrix (j = 256*m + col for the
+// column pass, j = 256*row + m for the row pass):
+//   column pass = global stages 0 .. r1-1: independent length-R1 transforms down each
+//                 column, twiddle idx = 2^s + (m >> (r1 - s));
+//   row pass    = global stages r1 .. log_n-1: independent length-256 transforms along each
+//                 row, twiddle idx = ((R1 + row) << s) + (m >> (8 - s)), s = 0..7 local.
+// Each pass runs 16 elements per thread in two register rounds with one shared-memory
+// exchange between them:
+//   round 0: the top 4 bits of m vary in registers (m = lo + (R/16) u, u = 0..15),
+//   round 1: the remaining low bits (m = 16 lo + u).
+// The inverse passes undo the forward stages in reverse order with Gentleman-Sande
+// butterflies and the psi^-brv(idx) table.
+#pragma once
+#include "modarith.cuh"
+
+// Twiddle record: (w, Shoup companion of w).
+typedef uint2 tw_t;
+
+// ---------------------------------------------------------------- register blocks
+
+// Forward round over the top 4 bits: stage s (0..3) pairs (u, u + (8 >> s)); group g = u /
+// (16 >> s) uses idx = (base << s) + g.
+__device__ __forceinline__ void fwd_top4(u32 (&x)[16], const tw_t *__restrict__ tw, u32 base,
+                                         u32 q, u32 two_q) {
+#pragma unroll
+    for (int s = 0; s < 4; s++) {
+        const int d = 8 >> s;
+#pragma unroll
+        for (int g = 0; g < (1 << s); g++) {
+            const tw_t w = __ldg(tw + (base << s) + g);
+#pragma unroll
+            for (int i = 0; i < d; i++) ct_bfly(x[2 * d * g + i], x[2 * d * g + i + d], w.x, w.y, q, two_q);
+        }
+    }
+}
+
+// Forward round over the low RLOG-4 bits of m = 16 lo + u: global-in-pass stage s = 4 ..
+// RLOG-1 pairs (u, u + d), d = 2^(RLOG-1-s); group g = u / 2d uses
+// idx = (base << s) + (lo << (s - RLOG + 4)) + g.
+template <int RLOG>
+__device__ __forceinline__ void fwd_low(u32 (&x)[16], const tw_t *__restrict__ tw, u32 base, u32 lo,
+                                        u32 q, u32 two_q) {
+#pragma unroll
+    for (int s = 4; s < RLOG; s++) {
+        const int d = 1 << (RLOG - 1 - s);
+        const u32 gbase = (base << s) + (lo << (s - RLOG + 4));
+#pragma unroll
+        for (int g = 0; g < 16 / (2 * d); g++) {
+            const tw_t w = __ldg(tw + gbase + g);
+#pragma unroll
+            for (int i = 0; i < d; i++) ct_bfly(x[2 * d * g + i], x[2 * d * g + i + d], w.x, w.y, q, two_q);
+        }
+    }
+}
+
+template <int RLOG>
+__device__ __forceinline__ void inv_low(u32 (&x)[16], const tw_t *__restrict__ tw, u32 base, u32 lo,
+                                        u32 q, u32 two_q) {
+#pragma unroll
+    for (int s = RLOG - 1; s >= 4; s--) {
+        const int d = 1 << (RLOG - 1 - s);
+        const u32 gbase = (base << s) + (lo << (s - RLOG + 4));
+#pragma unroll
+        for (int g = 0; g < 16 / (2 * d); g++) {
+            const tw_t w = __ldg(tw + gbase + g);
+#pragma unroll
+            for (int i = 0; i < d; i++) gs_bfly(x[2 * d * g + i], x[2 * d * g + i + d], w.x, w.y, q, two_q);
+        }
+    }
+}
+
+__device__ __forceinline__ void inv_top4(u32 (&x)[16], const tw_t *__restrict__ tw, u32 base,
+                                         u32 q, u32 two_q) {
+#pragma unroll
+    for (int s = 3; s >= 0; s--) {
+        const int d = 8 >> s;
+#pragma unroll
+        for (int g = 0; g < (1 << s); g++) {
+            const tw_t w = __ldg(tw + (base << s) + g);
+#pragma unroll
+            for (int i = 0; i < d; i++) gs_bfly(x[2 * d * g + i], x[2 * d * g + i + d], w.x, w.y, q, two_q);
+        }
+    }
+}
+
+// ---------------------------------------------------------------- job mapping
+// A launch processes a batch of limbs ("jobs", blockIdx.y).  Job y belongs to group
+// g = y / per_group at position k = y % per_group; its prime is global limb lo_base + k for
+// k < split, hi_base + (k - split) otherwise (the extended basis q_0..q_l, p_0..).  With
+// skip_alpha > 0, positions inside digit g ([g*alpha, min(g*alpha+alpha, split))) are skipped
+// (ModUp leaves digit limbs untouched).
+struct JobMap {
+    int per_group, split, lo_base, hi_base;
+    int in_group_rows, out_group_rows, in_k_base, out_k_base;
+    int skip_alpha;
+};
+
+__device__ __forceinline__ bool map_job(const JobMap &m, int y, int &prime, size_t &in_row,
+                                        size_t &out_row, int &k) {
+    const int g = y / m.per_group;
+    k = y - g * m.per_group;
+    if (m.skip_alpha > 0) {
+        const int lo = g * m.skip_alpha;
+        const int hi = min(lo + m.skip_alpha, m.split);
+        if (k >= lo && k < hi) return false;
+    }
+    prime = k < m.split ? m.lo_base + k : m.hi_base + (k - m.split);
+    in_row = (size_t)g * m.in_group_rows + m.in_k_base + k;
+    out_row = (size_t)g * m.out_group_rows + m.out_k_base + k;
+    return true;
+}
+
+// Evaluation-domain automorphism source index: out[k] = in[src(k)] with
+// 2 brv(src)+1 = (2 brv(k)+1) g mod 2N.
+__device__ __forceinline__ u32 automorph_src(u32 k, u32 g, int log_n) {
+    const u32 kb = __brev(k) >> (32 - log_n);
+    const u32 e = ((2u * kb + 1u) * g) & ((2u << log_n) - 1u);
+    return __brev((e - 1u) >> 1) >> (32 - log_n);
+}
+
+struct NttArgs {
+    const u32 *in;
+    u32 *out;
+    const tw_t *tw;         // [n_primes][N] forward or inverse table
+    const PrimeInfo *pinfo; // [n_primes]
+    const tw_t *scale;      // per-k output scale (inverse column pass), or nullptr
+    JobMap map;
+    int log_n;
+    u32 galois;             // inverse row pass: gather input through kappa_g (0 = none)
+};
+
+// ---------------------------------------------------------------- column pass (stages 0..r1-1)
+// Block: (R1/16) "lo" values x CPB columns; warp = 32 consecutive columns at one lo.
+template <int R1LOG>
+struct ColCfg {
+    static constexpr int R1 = 1 << R1LOG;
+    static constexpr int LOS = R1 / 16;                       // threads per column
+    static constexpr int CPB = (8192 / R1) < 256 ? (8192 / R1) : 256;  // columns per block
+    static constexpr int THREADS = LOS * CPB;
+};
+
+// FWD: forward stages, output lazy in [0, 4q).  !FWD: inverse stages, output multiplied by
+// scale[k] (or N^-1 when scale is null) and canonical.
+template <int R1LOG, bool FWD>
+__global__ void __launch_bounds__(ColCfg<R1LOG>::THREADS)
+k_ntt_col(NttArgs a) {
+    using C = ColCfg<R1LOG>;
+    __shared__ u32 sm[C::R1 * C::CPB];
+    int prime, k;
+    size_t in_row, out_row;
+    if (!map_job(a.map, blockIdx.y, prime, in_row, out_row, k)) return;
+    const int n = 1 << a.log_n;
+    const PrimeInfo pi = a.pinfo[prime];
+    const u32 q = pi.q, two_q = 2 * q;
+    const tw_t *tw = a.tw + (size_t)prime * n;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int cgroups = C::CPB / 32;
+    const int lo = warp / cgroups;
+    const int ccol = (warp % cgroups) * 32 + lane;          // column within block
+    const int col = blockIdx.x * C::CPB + ccol;
+    const u32 *src = a.in + in_row * n;
+    u32 *dst = a.out + out_row * n;
+    u32 x[16];
+    if (FWD) {
+#pragma unroll
+        for (int u = 0; u < 16; u++) x[u] = src[(size_t)(lo + C::LOS * u) * 256 + col];
+        fwd_top4(x, tw, 1u, q, two_q);
+#pragma unroll
+        for (int u = 0; u < 16; u++) sm[(lo + C::LOS * u) * C::CPB + ccol] = x[u];
+        __syncthreads();
+#pragma unroll
+        for (int u = 0; u < 16; u++) x[u] = sm[(16 * lo + u) * C::CPB + ccol];
+        fwd_low<R1LOG>(x, tw, 1u, (u32)lo, q, two_q);
+#pragma unroll
+        for (int u = 0; u < 16; u++) dst[(size_t)(16 * lo + u) * 256 + col] = x[u];
+    } else {
+#pragma unroll
+        for (int u = 0; u < 16; u++) x[u] = src[(size_t)(16 * lo + u) * 256 + col];
+        inv_low<R1LOG>(x, tw, 1u, (u32)lo, q, two_q);
+#pragma unroll
+        for (int u = 0; u < 16; u++) sm[(16 * lo + u) * C::CPB + ccol] = x[u];
+        __syncthreads();
+#pragma unroll
+        for (int u = 0; u < 16; u++) x[u] = sm[(lo + C::LOS * u) * C::CPB + ccol];
+        inv_top4(x, tw, 1u, q, two_q);
+        u32 w = pi.n_inv, wp = pi.n_invp;
+        if (a.scale) { const tw_t s = a.scale[k]; w = s.x; wp = s.y; }
+#pragma unroll
+        for (int u = 0; u < 16; u++)
+            dst[(size_t)(lo + C::LOS * u) * 256 + col] = csub(shoup_mul(x[u], w, wp, q), q);
+    }
+}
+
+// ---------------------------------------------------------------- row pass (stages r1..log_n-1)
+// Block: 16 rows x 16 threads.  The register exchange stays inside a warp (2 rows per warp).
+// Shared layout per row: element m at m + (m >> 4) (row stride 272), conflict-free for both
+// the lo + 16u and the 16 lo + u patterns.
+constexpr int ROW_THREADS = 256;
+
+// FWD: forward stages, canonical output.  !FWD: inverse stages (input gathered through
+// kappa_g when galois != 0), output lazy in [0, 2q).
+template <bool FWD>
+__global__ void __launch_bounds__(ROW_THREADS)
+k_ntt_row(NttArgs a) {
+    __shared__ u32 sm[16 * 272];
+    int prime, k;
+    size_t in_row, out_row;
+    if (!map_job(a.map, blockIdx.y, prime, in_row, out_row, k)) return;
+    const int n = 1 << a.log_n;
+    const PrimeInfo pi = a.pinfo[prime];
+    const u32 q = pi.q, two_q = 2 * q;
+    const tw_t *tw = a.tw + (size_t)prime * n;
+    const int r = threadIdx.x >> 4, lo = threadIdx.x & 15;
+    const int row = blockIdx.x * 16 + r;
+    const u32 base = (u32)(n >> 8) + (u32)row;
+    const u32 *src = a.in + in_row * n;
+    u32 *dst = a.out + out_row * n + (size_t)row * 256;
+    u32 *srow = sm + r * 272;
+    u32 x[16];
+    if (FWD) {
+        const u32 *s = src + (size_t)row * 256;
+#pragma unroll
+        for (int u = 0; u < 16; u++) x[u] = s[lo + 16 * u];
+        fwd_top4(x, tw, base, q, two_q);
+#pragma unroll
+        for (int u = 0; u < 16; u++) srow[lo + 17 * u] = x[u];
+        __syncwarp();
+#pragma unroll
+        for (int u = 0; u < 16; u++) x[u] = srow[17 * lo + u];
+        fwd_low<8>(x, tw, base, (u32)lo, q, two_q);
+#pragma unroll
+        for (int v = 0; v < 4; v++) {
+            uint4 o;
+            o.x = csub(csub(x[4 * v + 0], two_q), q);
+            o.y = csub(csub(x[4 * v + 1], two_q), q);
+            o.z = csub(csub(x[4 * v + 2], two_q), q);
+            o.w = csub(csub(x[4 * v + 3], two_q), q);
+            reinterpret_cast<uint4 *>(dst + 16 * lo)[v] = o;
+        }
+    } else {
+        if (a.galois) {
+#pragma unroll
+            for (int u = 0; u < 16; u++)
+                x[u] = src[automorph_src((u32)(row * 256 + 16 * lo + u), a.galois, a.log_n)];
+        } else {
+            const uint4 *s4 = reinterpret_cast<const uint4 *>(src + (size_t)row * 256 + 16 * lo);
+#pragma unroll
+            for (int v = 0; v < 4; v++) {
+                const uint4 t = s4[v];
+                x[4 * v] = t.x; x[4 * v + 1] = t.y; x[4 * v + 2] = t.z; x[4 * v + 3] = t.w;
+            }
+        }
+        inv_low<8>(x, tw, base, (u32)lo, q, two_q);
+#pragma unroll
+        for (int u = 0; u < 16; u++) srow[17 * lo + u] = x[u];
+        __syncwarp();
+#pragma unroll
+        for (int u = 0; u < 16; u++) x[u] = srow[lo + 17 * u];
+        inv_top4(x, tw, base, q, two_q);
+#pragma unroll
+        for (int u = 0; u < 16; u++) dst[lo + 16 * u] = x[u];
+    }
+}

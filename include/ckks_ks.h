@@ -1,0 +1,170 @@
+/*
+ * ckks_ks.h -- C ABI of the B200 (sm_100a) RNS-CKKS hybrid key-switching library.
+ *
+ * What the library computes.  The Perseus write-up ("Perseus: A Full-Stack System for
+ * Homomorphic Model Inference", ai4snews, Interpretation, 2nd paragraph) describes a 32-bit
+ * RNS CKKS runtime whose key-switching keys store only their b half: the uniformly random
+ * a half is regenerated inside the two kernels that use the key by a counter-mode ChaCha12
+ * expander, halving key storage.  Key switching is the core of every rotation and
+ * relinearisation.  The pages give no formulas; the operations below follow full-RNS CKKS
+ * and fast base conversion (Cheon, Han, Kim, Kim, Song, SAC 2018) and hybrid key switching
+ * with dnum gadget digits (Han, Ki, CT-RSA 2020), with the conventions listed here.
+ *
+ * Conventions (every entry point):
+ *  - N = 2^log_n, 12 <= log_n <= 16.  Primes are NTT friendly (q = 1 mod 2N) and below 2^30.
+ *  - Chain: ciphertext primes q_0..q_{n_q-1}, special primes p_0..p_{n_p-1}; "global limb
+ *    index" t = 0..n_q-1 for q_t and n_q + i for p_i.  `level` l means l+1 active ciphertext
+ *    limbs q_0..q_l.  The extended basis at level l is q_0..q_l, p_0..p_{n_p-1}
+ *    (ext = l + 1 + n_p limbs, in that order).
+ *  - Gadget digits: alpha = ceil(n_q / dnum) primes per digit; digit j holds q_{j*alpha} ..
+ *    q_{min((j+1)*alpha, l+1)-1}; beta = ceil((l+1)/alpha) digits are active at level l.
+ *  - Polynomials are uint32 [limb][N] row-major, residues canonical in [0, q) on input and
+ *    output.  Evaluation ("NTT") domain: storage index k holds a(psi^(2*brv(k)+1)) with
+ *    psi the primitive 2N-th root chosen as h^((q-1)/2N) for the smallest h >= 2 with
+ *    psi^N = -1, brv the log_n-bit reversal.  Ciphertexts are [2][l+1][N], the tensor
+ *    product is [3][l+1][N]; all in the evaluation domain.
+ *  - Device pointers must be 16-byte aligned.  Outputs must not alias inputs unless the
+ *    entry point says so.  The caller owns every buffer and the stream.
+ *  - Every call is asynchronous on `stream`; nothing synchronises the device, nothing
+ *    allocates device memory except ckks_ctx_create.  The workspace `ws` is caller-owned
+ *    device memory of at least ckks_workspace_bytes(...) bytes; calls on different streams
+ *    need different workspaces.
+ *  - Return codes: CKKS_OK (0) or a negative CKKS_ERR_*; ckks_last_error() gives a message
+ *    (thread-local).  No C++ exception crosses this boundary.
+ */
+#ifndef CKKS_KS_H
+#define CKKS_KS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same underlying type as cudaStream_t; NULL means the legacy default stream. */
+typedef struct CUstream_st *ckks_stream_t;
+
+enum {
+    CKKS_OK = 0,
+    CKKS_ERR_ARG = -1,          /* null pointer or bad argument */
+    CKKS_ERR_UNSUPPORTED = -2,  /* log_n outside 12..16, prime >= 2^30 or not 1 mod 2N, level > L ... */
+    CKKS_ERR_ALIGN = -3,        /* a device pointer is not 16-byte aligned */
+    CKKS_ERR_WORKSPACE = -4,    /* workspace smaller than ckks_workspace_bytes() */
+    CKKS_ERR_CUDA = -5,         /* a CUDA call or kernel launch failed */
+    CKKS_ERR_TIMEOUT = -6       /* ckks_sync_status: stream still busy at the deadline */
+};
+
+typedef struct ckks_ctx ckks_ctx; /* opaque; owns read-only device tables only */
+
+/* Parameter set.  q: n_q ciphertext primes, p: n_p special primes (host arrays, copied).
+ * dnum: number of gadget digits the keys of this context are generated with. */
+typedef struct {
+    uint32_t log_n, n_q, n_p, dnum;
+    const uint32_t *q, *p;
+} ckks_params;
+
+/* Key-switching key (from a secret s' to s), evaluation domain, full chain.
+ *  b:  device, [D][n_q+n_p][N], D = ceil(n_q/alpha) digits:
+ *      b_j[t] = -a_j[t]*s[t] + e_j[t] + [t in digit j]*[P]_{q_t}*s'[t]   (mod t).
+ *  a:  NULL (default): the a half is regenerated in-kernel (see ckks_chacha_expand);
+ *      non-NULL: device [D][n_q+n_p][N] stored a half (ablation that reads it from HBM).
+ *  seed, key_id: the ChaCha12 key and the first nonce word; key_id is 0 for the
+ *      relinearisation key and the Galois element g for the rotation key of kappa_g. */
+typedef struct {
+    const uint32_t *b;
+    const uint32_t *a;
+    uint8_t seed[32];
+    uint32_t key_id;
+} ckks_evk;
+
+/* Prime chain rule: scan x = 1 (mod 2N) downward from the largest such x below 2^30, keep
+ * primes in order; the first n_p found are the special primes p_0 > p_1 > ..., the next n_q
+ * the ciphertext primes q_0 > q_1 > ...  Host only; q_out/p_out are host arrays. */
+int ckks_gen_primes(uint32_t log_n, uint32_t n_q, uint32_t n_p, uint32_t *q_out, uint32_t *p_out);
+
+/* Builds the device tables (twiddles, base-conversion constants) for a parameter set on the
+ * current CUDA device.  Synchronous.  The context may then be used from any stream. */
+int ckks_ctx_create(const ckks_params *params, ckks_ctx **ctx_out);
+void ckks_ctx_destroy(ckks_ctx *ctx);
+
+/* Forward / inverse negacyclic NTT, in place, on n_limbs consecutive rows of `poly`; row r
+ * uses the prime of global limb first_limb + r.  Forward: coefficients -> evaluation domain
+ * as defined above (A[k] = sum_n a[n] psi^((2 brv(k)+1) n)); inverse: its exact inverse
+ * (including the N^-1 scale). */
+int ckks_ntt_fwd(ckks_ctx *ctx, uint32_t *poly, int first_limb, int n_limbs, ckks_stream_t stream);
+int ckks_ntt_inv(ckks_ctx *ctx, uint32_t *poly, int first_limb, int n_limbs, ckks_stream_t stream);
+
+/* Automorphism kappa_g (g odd, 0 < g < 2N) in the evaluation domain on n_limbs rows:
+ * out[k] = in[k'] with 2 brv(k')+1 = (2 brv(k)+1) g mod 2N.  out must not alias in. */
+int ckks_automorph(ckks_ctx *ctx, const uint32_t *in, uint32_t *out, int n_limbs, uint32_t galois,
+                   ckks_stream_t stream);
+
+/* ModUp (hybrid key switching): c [l+1][N] -> dtilde [beta][ext][N].  For each active digit
+ * j, digit limbs keep their evaluation values; every other extended limb t receives
+ * NTT_t(FastBConv(iNTT(digit j's limbs))) with the centred lift
+ * y_i = [x_i (D_j/q_i)^-1]_{q_i} in (-q_i/2, q_i/2], out_t = sum_i y_i [D_j/q_i]_t mod t. */
+int ckks_modup(ckks_ctx *ctx, const uint32_t *c, int level, uint32_t *dtilde, void *ws,
+               size_t ws_bytes, ckks_stream_t stream);
+
+/* Key inner product (the kernel that uses the key): acc [2][ext][N],
+ * acc0[u] = sum_j dtilde_j[u] * b_j[t], acc1[u] = sum_j dtilde_j[u] * a_j[t] (mod t), t the
+ * global limb of extended position u; a_j[t] regenerated by ChaCha12 unless evk->a is set. */
+int ckks_inner_product(ckks_ctx *ctx, const uint32_t *dtilde, int level, const ckks_evk *evk,
+                       uint32_t *acc, ckks_stream_t stream);
+
+/* ModDown: acc [ext][N] -> out [l+1][N]; iNTT of the special limbs, centred FastBConv
+ * P -> q_i, NTT, out_i = (acc_i - conv_i) [P^-1]_{q_i}. */
+int ckks_moddown(ckks_ctx *ctx, const uint32_t *acc, int level, uint32_t *out, void *ws,
+                 size_t ws_bytes, ckks_stream_t stream);
+
+/* Key switching of one polynomial c [l+1][N]: out [2][l+1][N] = (ModDown(acc0), ModDown(acc1)). */
+int ckks_keyswitch(ckks_ctx *ctx, const uint32_t *c, int level, const ckks_evk *evk, uint32_t *out,
+                   void *ws, size_t ws_bytes, ckks_stream_t stream);
+
+/* Rotation by the Galois element g: kappa_g on both components, key switching of
+ * kappa_g(c1) with the key for kappa_g(s), kappa_g(c0) added to the first output component.
+ * ct, out: [2][l+1][N]. */
+int ckks_rotate(ckks_ctx *ctx, const uint32_t *ct, int level, uint32_t galois, const ckks_evk *evk,
+                uint32_t *out, void *ws, size_t ws_bytes, ckks_stream_t stream);
+
+/* Hoisted rotations: one ModUp of c1, then for each r the extended digits permuted by
+ * kappa_{g_r}, the inner product with keys[r], ModDown and kappa_{g_r}(c0) added.
+ * galois, keys: host arrays of n_rot entries; out: [n_rot][2][l+1][N].  (With the centred
+ * lift, ModUp commutes with kappa_g, so each output equals ckks_rotate bit for bit.) */
+int ckks_rotate_hoisted(ckks_ctx *ctx, const uint32_t *ct, int level, int n_rot,
+                        const uint32_t *galois, const ckks_evk *keys, uint32_t *out, void *ws,
+                        size_t ws_bytes, ckks_stream_t stream);
+
+/* Relinearisation: d [3][l+1][N] (decrypting under 1, s, s^2) -> out [2][l+1][N] =
+ * (d0, d1) + keyswitch(d2) with the key for s^2. */
+int ckks_relin(ckks_ctx *ctx, const uint32_t *d, int level, const ckks_evk *evk, uint32_t *out,
+               void *ws, size_t ws_bytes, ckks_stream_t stream);
+
+/* Tensor product of x = (x0, x1), y = (y0, y1) [2][l+1][N]: d [3][l+1][N] =
+ * (x0 y0, x0 y1 + x1 y0, x1 y1) pointwise mod q_i. */
+int ckks_tensor(ckks_ctx *ctx, const uint32_t *x, const uint32_t *y, int level, uint32_t *d,
+                ckks_stream_t stream);
+
+/* The key's regenerated uniform half for one (digit, global limb): out [N] (device),
+ * out[n] = w mod q_t with w = (x[2m] | x[2m+1] << 32), m = n mod 8, x = ChaCha12 block
+ * (RFC 8439 state: key = seed as 8 LE words, counter = n/8, nonce = (key_id, digit, limb)). */
+int ckks_chacha_expand(ckks_ctx *ctx, const uint8_t seed[32], uint32_t key_id, int digit, int limb,
+                       uint32_t *out, ckks_stream_t stream);
+
+/* Workspace bytes for keyswitch/rotate/relin/modup/moddown at `level`
+ * (n_rot > 1: rotate_hoisted with n_rot rotations). */
+size_t ckks_workspace_bytes(const ckks_ctx *ctx, int level, int n_rot);
+
+/* Waits for `stream` with a deadline (polling, no device-side wait): CKKS_OK when the
+ * stream is idle and no CUDA error is pending, CKKS_ERR_TIMEOUT at the deadline,
+ * CKKS_ERR_CUDA on an asynchronous error. */
+int ckks_sync_status(ckks_ctx *ctx, ckks_stream_t stream, int timeout_ms);
+
+/* Message of the last error on this thread ("" if none). */
+const char *ckks_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CKKS_KS_H */

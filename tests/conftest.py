@@ -14,6 +14,15 @@ def pytest_configure(config):
 
 
 @pytest.fixture(scope="session")
+def ks_lib():
+    """The CUDA library, built in-tree (nvcc cross-compiles for sm_100a without a GPU)."""
+    from fhe_key_switching_b200 import build as _build
+    _build.build()
+    import fhe_key_switching_b200 as ks
+    return ks
+
+
+@pytest.fixture(scope="session")
 def oracle_mod():
     import oracle
     oracle.lib()
