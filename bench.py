@@ -235,9 +235,9 @@ def run_ours(args, rank, world, local_rank):
         dist.destroy_process_group()
 
 
-# kernels launched by one step: tensor (1) + 2 key switches x 13 (+0 automorphism kernels:
-# the rotation gathers inside the inverse-NTT load, the inner product and the combine)
-LAUNCHES_PER_STEP = 1 + 2 * 13
+# kernels launched by one step: tensor (1) + 2 key switches x 10 (ModUp 4, inner product with
+# the last ModUp and first ModDown NTT passes 2, ModDown 4 including the fused combine)
+LAUNCHES_PER_STEP = 1 + 2 * 10
 
 
 def _oracle_sample():

@@ -87,51 +87,145 @@ struct BconvArgs {
     int n_groups;
     int cfg_per_group;       // table config index = g * cfg_per_group + (n_in(g) - 1) (ModUp), or 0
     int cfg_stride;          // words per config in bmat = max_in * n_primes
+    int g_base;              // logical group of blockIdx.y = 0 (a launch may cover a subset)
 };
 
 constexpr int BCONV_THREADS = 256;
 constexpr int BCONV_MAX_IN = 64;
+constexpr int BCONV_TCHUNK = 12;      // targets per block (blockIdx.z splits the target list)
 
+// MAXIN: compile-time bound on the group's input count (inputs live in registers).
+// Each thread converts 2 consecutive coefficients.
+template <int MAXIN>
 __global__ void __launch_bounds__(BCONV_THREADS)
 k_bconv(BconvArgs a) {
-    extern __shared__ u32 smb[];          // [n_in][per_group] constants, then [per_group] negd
-    const int g = blockIdx.y;
+    extern __shared__ u32 smb[];          // [n_in + 1][T] constants (row n_in: [-D]_t), then half[n_in]
+    const int g = a.g_base + blockIdx.y;
     const int n = 1 << a.log_n;
     const int n_in = (g == a.n_groups - 1) ? a.n_in_last : a.n_in_full;
     const int cfg = a.cfg_per_group ? g * a.cfg_per_group + (n_in - 1) : 0;
     const u32 *bm = a.bmat + (size_t)cfg * a.cfg_stride;
     const u32 *nd = a.negd + (size_t)cfg * a.n_primes;
     const int T = a.map.per_group;
-    // stage the conversion constants of this group's targets in shared memory
+    const int row0 = a.in_row0 + g * a.in_group_rows;
+    const int p0 = a.in_prime0 + g * a.in_prime_step;
+    u32 *half = smb + (n_in + 1) * T;
     for (int idx = threadIdx.x; idx < (n_in + 1) * T; idx += blockDim.x) {
         const int i = idx / T, kk = idx - i * T;
         const int t = kk < a.map.split ? a.map.lo_base + kk : a.map.hi_base + (kk - a.map.split);
         smb[idx] = (i < n_in) ? bm[(size_t)i * a.n_primes + t] : nd[t];
     }
+    for (int i = threadIdx.x; i < n_in; i += blockDim.x) half[i] = a.pinfo[p0 + i].half;
     __syncthreads();
-    const int c = blockIdx.x * blockDim.x + threadIdx.x;   // coefficient
-    if (c >= n) return;
-    u32 y[BCONV_MAX_IN];
-    u32 v = 0;
-    const int row0 = a.in_row0 + g * a.in_group_rows;
-    const int p0 = a.in_prime0 + g * a.in_prime_step;
-    for (int i = 0; i < n_in; i++) {
-        y[i] = a.y[(size_t)(row0 + i) * n + c];
-        v += (y[i] > a.pinfo[p0 + i].half) ? 1u : 0u;
+    const int c2 = blockIdx.x * blockDim.x + threadIdx.x;   // coefficient pair
+    if (2 * c2 >= n) return;
+    u32 y0[MAXIN], y1[MAXIN];
+    u32 v0 = 0, v1 = 0;
+#pragma unroll
+    for (int i = 0; i < MAXIN; i++) {
+        if (i < n_in) {
+            const uint2 t = reinterpret_cast<const uint2 *>(a.y + (size_t)(row0 + i) * n)[c2];
+            const u32 h = half[i];
+            y0[i] = t.x; y1[i] = t.y;
+            v0 += t.x > h ? 1u : 0u;
+            v1 += t.y > h ? 1u : 0u;
+        }
     }
     const int lo = a.map.skip_alpha > 0 ? g * a.map.skip_alpha : 0;
     const int hi = a.map.skip_alpha > 0 ? min(lo + a.map.skip_alpha, a.map.split) : 0;
-    for (int kk = 0; kk < T; kk++) {
+    const int k_end = min(T, (int)(blockIdx.z + 1) * BCONV_TCHUNK);
+    for (int kk = blockIdx.z * BCONV_TCHUNK; kk < k_end; kk++) {
         if (kk >= lo && kk < hi) continue;
         const int t = kk < a.map.split ? a.map.lo_base + kk : a.map.hi_base + (kk - a.map.split);
         const PrimeInfo pi = a.pinfo[t];
-        u64 acc = (u64)v * smb[n_in * T + kk];
-        for (int i = 0; i < n_in; i++) {
-            acc += (u64)y[i] * smb[i * T + kk];
-            if ((i % 14) == 13) acc = reduce64_lazy(acc, pi.q, pi.r64, pi.r64p, pi.onep);
+        const u32 nd_t = smb[n_in * T + kk];
+        u64 s0 = (u64)v0 * nd_t, s1 = (u64)v1 * nd_t;
+#pragma unroll
+        for (int i = 0; i < MAXIN; i++) {
+            if (i < n_in) {
+                const u32 bc = smb[i * T + kk];
+                s0 += (u64)y0[i] * bc;
+                s1 += (u64)y1[i] * bc;
+                if ((i % 14) == 13) {          // keep the 64-bit sums below 2^64
+                    s0 = reduce64_lazy(s0, pi.q, pi.r64, pi.r64p, pi.onep);
+                    s1 = reduce64_lazy(s1, pi.q, pi.r64, pi.r64p, pi.onep);
+                }
+            }
         }
-        const u32 r = reduce64(acc, pi.q, pi.r64, pi.r64p, pi.onep);
-        a.out[((size_t)g * a.map.out_group_rows + a.map.out_k_base + kk) * n + c] = r;
+        const uint2 r = make_uint2(reduce64(s0, pi.q, pi.r64, pi.r64p, pi.onep),
+                                   reduce64(s1, pi.q, pi.r64, pi.r64p, pi.onep));
+        reinterpret_cast<uint2 *>(a.out + ((size_t)g * a.map.out_group_rows + a.map.out_k_base + kk) * n)[c2] = r;
+    }
+}
+
+// Exact-count variant: NIN inputs known at compile time; each thread converts 2 consecutive
+// coefficients for 4 targets at a time (8 independent 64-bit sums).  Constants are staged as
+// [NIN + 1][T4] with T4 = T rounded up to 4 (row NIN holds [-D]_t, multiplied by the count v
+// of negative representatives), so one 128-bit shared load gives 4 targets' constants.
+template <int NIN>
+__global__ void __launch_bounds__(BCONV_THREADS)
+k_bconv_n(BconvArgs a) {
+    extern __shared__ __align__(16) u32 smc[];
+    const int g = a.g_base + blockIdx.y;
+    const int n = 1 << a.log_n;
+    const int cfg = a.cfg_per_group ? g * a.cfg_per_group + (NIN - 1) : 0;
+    const u32 *bm = a.bmat + (size_t)cfg * a.cfg_stride;
+    const u32 *nd = a.negd + (size_t)cfg * a.n_primes;
+    const int T = a.map.per_group;
+    const int T4 = (T + 3) & ~3;
+    const int row0 = a.in_row0 + g * a.in_group_rows;
+    const int p0 = a.in_prime0 + g * a.in_prime_step;
+    for (int idx = threadIdx.x; idx < (NIN + 1) * T4; idx += blockDim.x) {
+        const int i = idx / T4, kk = idx - i * T4;
+        u32 val = 0;
+        if (kk < T) {
+            const int t = kk < a.map.split ? a.map.lo_base + kk : a.map.hi_base + (kk - a.map.split);
+            val = (i < NIN) ? bm[(size_t)i * a.n_primes + t] : nd[t];
+        }
+        smc[idx] = val;
+    }
+    __syncthreads();
+    const int c2 = blockIdx.x * blockDim.x + threadIdx.x;   // coefficient pair
+    if (2 * c2 >= n) return;
+    u32 y0[NIN + 1], y1[NIN + 1];
+    u32 v0 = 0, v1 = 0;
+#pragma unroll
+    for (int i = 0; i < NIN; i++) {
+        const uint2 t = reinterpret_cast<const uint2 *>(a.y + (size_t)(row0 + i) * n)[c2];
+        const u32 h = a.pinfo[p0 + i].half;
+        y0[i] = t.x; y1[i] = t.y;
+        v0 += t.x > h ? 1u : 0u;
+        v1 += t.y > h ? 1u : 0u;
+    }
+    y0[NIN] = v0; y1[NIN] = v1;
+    const int lo = a.map.skip_alpha > 0 ? g * a.map.skip_alpha : 0;
+    const int hi = a.map.skip_alpha > 0 ? min(lo + a.map.skip_alpha, a.map.split) : 0;
+    const int k_beg = blockIdx.z * BCONV_TCHUNK;
+    const int k_end = min(T, k_beg + BCONV_TCHUNK);
+    for (int k4 = k_beg; k4 < k_end; k4 += 4) {
+        u64 s0[4], s1[4];
+#pragma unroll
+        for (int m = 0; m < 4; m++) s0[m] = s1[m] = 0;
+#pragma unroll
+        for (int i = 0; i <= NIN; i++) {
+            const uint4 b4 = *reinterpret_cast<const uint4 *>(smc + i * T4 + k4);
+            const u32 bb[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+            for (int m = 0; m < 4; m++) {
+                s0[m] += (u64)y0[i] * bb[m];
+                s1[m] += (u64)y1[i] * bb[m];
+            }
+        }
+#pragma unroll
+        for (int m = 0; m < 4; m++) {
+            const int kk = k4 + m;
+            if (kk >= k_end || (kk >= lo && kk < hi)) continue;
+            const int t = kk < a.map.split ? a.map.lo_base + kk : a.map.hi_base + (kk - a.map.split);
+            const PrimeInfo pi = a.pinfo[t];
+            const uint2 r = make_uint2(reduce64(s0[m], pi.q, pi.r64, pi.r64p, pi.onep),
+                                       reduce64(s1[m], pi.q, pi.r64, pi.r64p, pi.onep));
+            reinterpret_cast<uint2 *>(a.out + ((size_t)g * a.map.out_group_rows + a.map.out_k_base + kk) * n)[c2] = r;
+        }
     }
 }
 
@@ -313,4 +407,215 @@ __global__ void k_copy_digit_limbs(const u32 *c, u32 *dt, int log_n, int level, 
     const int j = u / alpha;
     reinterpret_cast<uint4 *>(dt + ((size_t)j * ext + u) * n)[c4] =
         reinterpret_cast<const uint4 *>(c + (size_t)u * n)[c4];
+}
+
+// ---------------------------------------------------------------- fused row kernels
+// Both kernels use the row-pass geometry of k_ntt_row (16 rows x 16 threads per block); at
+// the end of a forward row pass thread (r, lo) holds the 16 consecutive evaluation slots
+// k = 256*row + 16*lo + v, v = 0..15.
+
+__device__ __forceinline__ void load16_vec(const u32 *p, u32 (&x)[16]) {
+    const uint4 *p4 = reinterpret_cast<const uint4 *>(p);
+#pragma unroll
+    for (int v = 0; v < 4; v++) {
+        const uint4 t = p4[v];
+        x[4 * v] = t.x; x[4 * v + 1] = t.y; x[4 * v + 2] = t.z; x[4 * v + 3] = t.w;
+    }
+}
+
+__device__ __forceinline__ void store16_vec(u32 *p, const u32 (&x)[16]) {
+    uint4 *p4 = reinterpret_cast<uint4 *>(p);
+#pragma unroll
+    for (int v = 0; v < 4; v++) p4[v] = make_uint4(x[4 * v], x[4 * v + 1], x[4 * v + 2], x[4 * v + 3]);
+}
+
+// Forward row pass of one row held as round-0 input x[v] = row element lo + 16 v; returns the
+// canonical evaluation values of elements 16 lo + v.  srow: this row's 272-word exchange area.
+__device__ __forceinline__ void row_fwd_regs(u32 (&x)[16], const tw_t *tw, u32 base, int lo, u32 *srow,
+                                             u32 q) {
+    const u32 two_q = 2 * q;
+    fwd_top4(x, tw, base, q, two_q);
+#pragma unroll
+    for (int u = 0; u < 16; u++) srow[lo + 17 * u] = x[u];
+    __syncwarp();
+#pragma unroll
+    for (int u = 0; u < 16; u++) x[u] = srow[17 * lo + u];
+    __syncwarp();
+    fwd_low<8>(x, tw, base, (u32)lo, q, two_q);
+#pragma unroll
+    for (int u = 0; u < 16; u++) x[u] = csub(csub(x[u], two_q), q);
+}
+
+// Inverse row pass of one row held as x[v] = element 16 lo + v (values in [0, 2q)); returns
+// elements lo + 16 v, lazily in [0, 2q).
+__device__ __forceinline__ void row_inv_regs(u32 (&x)[16], const tw_t *tw, u32 base, int lo, u32 *srow,
+                                             u32 q) {
+    const u32 two_q = 2 * q;
+    inv_low<8>(x, tw, base, (u32)lo, q, two_q);
+#pragma unroll
+    for (int u = 0; u < 16; u++) srow[17 * lo + u] = x[u];
+    __syncwarp();
+#pragma unroll
+    for (int u = 0; u < 16; u++) x[u] = srow[lo + 17 * u];
+    __syncwarp();
+    inv_top4(x, tw, base, q, two_q);
+}
+
+// Key inner product fused with the last forward NTT pass of ModUp.  Block (row block, u): for every active digit
+// j, the extended digit dt_j[u] is completed in registers (forward row pass of the column-pass
+// output x[j][u], or the input polynomial itself for u inside digit j), the key's a half for
+// (digit j, limb t) is regenerated by ChaCha12 for the same 16 slots, and
+//   acc0 += dt_j[u] * b_j[t],  acc1 += dt_j[u] * a_j[t]   (Montgomery products, mod t).
+// Rotations: hoist_g != 0 reads every dt_j[u] through kappa_{hoist_g} (hoisted rotation:
+// the source row is transformed, then permuted inside the row); cdig_g != 0 reads only the
+// input polynomial's digit limbs through kappa_{cdig_g} (single rotation).
+// Output: acc rows, canonical evaluation values.
+struct IpRowArgs {
+    const u32 *x;            // [beta][ext][N] ModUp column-pass output (non-digit limbs)
+    const u32 *cdig;         // [l+1][N] input polynomial, evaluation domain
+    const u32 *b;            // [D][n_primes][N]
+    const u32 *a_stored;     // nullptr: regenerate
+    u32 *acc;                // [2][ext][N]
+    const tw_t *twf, *twi;
+    const PrimeInfo *pinfo;
+    ChachaKey key;
+    u32 key_id;
+    int log_n, level, n_q, n_primes, alpha, beta, ext;
+    u32 hoist_g, cdig_g;
+};
+
+__global__ void __launch_bounds__(ROW_THREADS)
+k_ip_row(IpRowArgs a) {
+    __shared__ u32 sm[16 * 272];
+    const int n = 1 << a.log_n;
+    const int na = a.level + 1;
+    const int u = blockIdx.y;
+    const int t = u < na ? u : a.n_q + (u - na);
+    const PrimeInfo pi = a.pinfo[t];
+    const u32 q = pi.q, two_q = 2 * q;
+    const int r = threadIdx.x >> 4, lo = threadIdx.x & 15;
+    const int row = blockIdx.x * 16 + r;
+    const u32 R1 = (u32)(n >> 8);
+    u32 *srow = sm + r * 272;
+    const int k0 = row * 256 + 16 * lo;              // first evaluation slot of this thread
+    const tw_t *twf = a.twf + (size_t)t * n;
+    // hoisted rotation: source row of this row under kappa_g
+    const int src_row = a.hoist_g ? (int)(automorph_src((u32)(row * 256), a.hoist_g, a.log_n) >> 8) : row;
+    u32 acc0[16], acc1[16];
+#pragma unroll
+    for (int v = 0; v < 16; v++) acc0[v] = acc1[v] = 0;
+    for (int j = 0; j < a.beta; j++) {
+        const bool in_digit = u < na && u >= j * a.alpha && u < min(j * a.alpha + a.alpha, na);
+        u32 x[16];
+        if (in_digit) {
+            const u32 *src = a.cdig + (size_t)u * n;
+            const u32 g = a.hoist_g ? a.hoist_g : a.cdig_g;
+            if (g) {
+#pragma unroll
+                for (int v = 0; v < 16; v++) x[v] = src[automorph_src((u32)(k0 + v), g, a.log_n)];
+            } else {
+                load16_vec(src + k0, x);
+            }
+        } else {
+            const u32 *src = a.x + ((size_t)j * a.ext + u) * n + (size_t)src_row * 256;
+#pragma unroll
+            for (int v = 0; v < 16; v++) x[v] = src[lo + 16 * v];
+            row_fwd_regs(x, twf, R1 + (u32)src_row, lo, srow, q);
+            if (a.hoist_g) {            // permute inside the row: slot k takes source slot src(k)
+#pragma unroll
+                for (int v = 0; v < 16; v++) srow[17 * lo + v] = x[v];
+                __syncwarp();
+#pragma unroll
+                for (int v = 0; v < 16; v++) {
+                    const u32 m = automorph_src((u32)(k0 + v), a.hoist_g, a.log_n) & 255u;
+                    x[v] = srow[m + (m >> 4)];
+                }
+                __syncwarp();
+            }
+        }
+        u32 bv[16], av[16];
+        load16_vec(a.b + ((size_t)j * a.n_primes + t) * n + k0, bv);
+        if (a.a_stored) {
+            load16_vec(a.a_stored + ((size_t)j * a.n_primes + t) * n + k0, av);
+        } else {
+            u32 h[8];
+            chacha_coeffs<false>(a.key, a.key_id, (u32)j, (u32)t, (u32)(k0 >> 3), pi, h);
+#pragma unroll
+            for (int v = 0; v < 8; v++) av[v] = h[v];
+            chacha_coeffs<false>(a.key, a.key_id, (u32)j, (u32)t, (u32)(k0 >> 3) + 1u, pi, h);
+#pragma unroll
+            for (int v = 0; v < 8; v++) av[8 + v] = h[v];
+        }
+#pragma unroll
+        for (int v = 0; v < 16; v++) {
+            acc0[v] = csub(acc0[v] + mont_mul(x[v], bv[v], q, pi.qinv), two_q);
+            acc1[v] = csub(acc1[v] + mont_mul(x[v], av[v], q, pi.qinv), two_q);
+        }
+    }
+    // undo the Montgomery factor 2^-32
+#pragma unroll
+    for (int v = 0; v < 16; v++) {
+        acc0[v] = shoup_mul(acc0[v], pi.r64, pi.r64p, q);
+        acc1[v] = shoup_mul(acc1[v], pi.r64, pi.r64p, q);
+    }
+    u32 *o0 = a.acc + (size_t)u * n + (size_t)row * 256;
+    u32 *o1 = a.acc + ((size_t)a.ext + u) * n + (size_t)row * 256;
+#pragma unroll
+    for (int v = 0; v < 16; v++) { acc0[v] = csub(acc0[v], q); acc1[v] = csub(acc1[v], q); }
+    store16_vec(o0 + 16 * lo, acc0);
+    store16_vec(o1 + 16 * lo, acc1);
+}
+
+// Last forward NTT pass of ModDown's converted limbs fused with the combine:
+//   out_c[i] = (acc_c[i] - conv_c[i]) [P^-1]_{q_i} + add_c[i]   (mod q_i).
+// conv: column-pass output [n_comp][l+1][N]; acc: [2][ext][N] (rows 0..l of each component).
+// add: nullptr, [2][l+1][N] (both components), or component 0 only, gathered through
+// kappa_{add_g} when add_g != 0.
+struct RowCombineArgs {
+    const u32 *conv;
+    const u32 *acc;
+    const u32 *add;
+    u32 *out;                // [n_comp][l+1][N]
+    const tw_t *twf;
+    const PrimeInfo *pinfo;
+    const tw_t *pinv;
+    int log_n, level, ext, acc_comp_rows, add_comps;
+    u32 add_g;
+};
+
+__global__ void __launch_bounds__(ROW_THREADS)
+k_row_combine(RowCombineArgs a) {
+    __shared__ u32 sm[16 * 272];
+    const int n = 1 << a.log_n;
+    const int i = blockIdx.y, comp = blockIdx.z;
+    const int na = a.level + 1;
+    const PrimeInfo pi = a.pinfo[i];
+    const u32 q = pi.q;
+    const int r = threadIdx.x >> 4, lo = threadIdx.x & 15;
+    const int row = blockIdx.x * 16 + r;
+    const int k0 = row * 256 + 16 * lo;
+    u32 *srow = sm + r * 272;
+    u32 x[16];
+    const u32 *src = a.conv + ((size_t)comp * na + i) * n + (size_t)row * 256;
+#pragma unroll
+    for (int v = 0; v < 16; v++) x[v] = src[lo + 16 * v];
+    row_fwd_regs(x, a.twf + (size_t)i * n, (u32)(n >> 8) + (u32)row, lo, srow, q);
+    u32 ac[16];
+    load16_vec(a.acc + ((size_t)comp * a.acc_comp_rows + i) * n + k0, ac);
+    const tw_t w = a.pinv[i];
+#pragma unroll
+    for (int v = 0; v < 16; v++) x[v] = csub(shoup_mul(ac[v] + q - x[v], w.x, w.y, q), q);
+    if (comp < a.add_comps) {
+        const u32 *ad = a.add + ((size_t)comp * na + i) * n;
+        u32 y[16];
+        if (a.add_g) {
+#pragma unroll
+            for (int v = 0; v < 16; v++) y[v] = ad[automorph_src((u32)(k0 + v), a.add_g, a.log_n)];
+        } else {
+            load16_vec(ad + k0, y);
+        }
+#pragma unroll
+        for (int v = 0; v < 16; v++) x[v] = csub(x[v] + y[v], q);
+    }
+    store16_vec(a.out + ((size_t)comp * na + i) * n + k0, x);
 }

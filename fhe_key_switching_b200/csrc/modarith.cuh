@@ -57,5 +57,14 @@ struct PrimeInfo {
     u32 n_inv;    // N^-1 mod q
     u32 n_invp;   // Shoup companion
     u32 half;     // (q - 1) / 2, the centred-lift threshold
-    u32 pad;
+    u32 qinv;     // -q^-1 mod 2^32 (Montgomery)
 };
+
+// Montgomery product a*b*2^-32 mod q, in [0, 2q) whenever a*b < 4q^2 (e.g. a < q, b < 4q).
+__device__ __forceinline__ u32 mont_mul(u32 a, u32 b, u32 q, u32 qinv) {
+    const u32 lo = a * b;
+    const u32 hi = __umulhi(a, b);
+    const u32 m = lo * qinv;
+    // (a*b + m*q) / 2^32: the low words cancel, with a carry exactly when lo != 0
+    return hi + __umulhi(m, q) + (lo != 0u ? 1u : 0u);
+}
