@@ -151,6 +151,8 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # the dominant kernel's launches are bracketed by events on the launching stream
+    ks.ckks_prof_begin(ctx, DOMINANT, KS_PER_STEP * args.steps)
     e0.record(stream)
     for i in range(args.steps):
         step(i)
@@ -158,6 +160,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
+    dom_launches, dom_ms = ks.ckks_prof_end(ctx)
     ms = e0.elapsed_time(e1)
     if world > 1:
         t = torch.tensor([ms], device=dev, dtype=torch.float64)
@@ -227,12 +230,83 @@ def run_ours(args, rank, world, local_rank):
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": args.steps * LAUNCHES_PER_STEP,
             "clocks": clk,
-            "roofline": None,
+            "roofline": roofline(cfg, dom_launches, dom_ms, clk),
+            "hbm_fraction_step": {"b_min_bytes_per_step": step_bytes_min(cfg),
+                                  "frac": step_bytes_min(cfg) / (ms_per_step / 1e3) / (HBM_PEAK_GBS * 1e9),
+                                  "peak_gbs": HBM_PEAK_GBS, "peak_source": PEAK_SOURCE},
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+DOMINANT = "ip_row"      # the fused NTT-row-pass + ChaCha12 + key inner-product kernel
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d.get("sm_max_mhz", 1965.0)), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, 1965.0, "fallback"
+
+
+HBM_PEAK_GBS, SM_MAX_MHZ, PEAK_SOURCE = _peaks()
+N_SM = 148
+
+
+def alu_peak_tops(mhz: float) -> float:
+    """int32 issue peak: 148 SMs x 4 sub-partitions x 32 lanes x 1 instruction/clock."""
+    return N_SM * 4 * 32 * mhz * 1e6 / 1e12
+
+
+def ip_row_ops(cfg) -> float:
+    """Algorithmic int32 operations of one k_ip_row launch (one key switch), with the unit costs
+    of the op model: ChaCha12 block 608 (8 coefficients), 64-bit word reduction 8, NTT butterfly
+    8, variable modular product 6, modular addition 2.  Units: beta*ext (digit, limb) pairs of N
+    coefficients; the row pass (8 of log N stages) runs on the pairs outside their digit."""
+    na = cfg.level + 1
+    ext = na + cfg.n_p
+    beta = -(-na // cfg.alpha)
+    pairs = beta * ext
+    n = cfg.n
+    chacha = pairs * n / 8 * 608
+    a_red = pairs * n * 8
+    ntt = (pairs - na) * 8 * (n / 2) * 8
+    macs = 2 * pairs * n * 6 + 2 * pairs * n * 2
+    return chacha + a_red + ntt + macs
+
+
+def roofline(cfg, launches, total_ms, clk):
+    if not launches:
+        return None
+    avg_s = total_ms / launches / 1e3
+    achieved = ip_row_ops(cfg) / avg_s / 1e12
+    peak = alu_peak_tops(SM_MAX_MHZ)
+    return {"kernel": "k_ip_row (ModUp last NTT pass + ChaCha12 + key inner product)",
+            "bound": "alu", "achieved": achieved, "peak": peak, "unit": "Tops (int32)",
+            "frac": achieved / peak, "traffic": IP_ROW_TRAFFIC, "launches": launches,
+            "avg_launch_us": avg_s * 1e6,
+            "peak_source": f"derived: {N_SM} SMs x 128 int32 lanes x {SM_MAX_MHZ:.0f} MHz"}
+
+
+# DRAM bytes (read + write) of one k_ip_row launch from an ncu capture of the current kernel;
+# None when the kernel changed after the capture.
+IP_ROW_TRAFFIC = None
+
+
+def step_bytes_min(cfg) -> int:
+    """Compulsory HBM bytes of one step: inputs, the keys' stored b halves and outputs of the
+    tensor product (4 -> 3 polys), the relinearisation (3 polys + key -> 2) and the rotation
+    (2 polys + key -> 2); the a halves are regenerated, intermediates are not counted."""
+    na = cfg.level + 1
+    nd = -(-cfg.n_q // cfg.alpha)
+    key = nd * (cfg.n_q + cfg.n_p)
+    limbs = (4 + 3) * na + (3 * na + key + 2 * na) + (2 * na + key + 2 * na)
+    return limbs * cfg.n * 4
 
 
 # kernels launched by one step: tensor (1) + 2 key switches x 10 (ModUp 4, inner product with

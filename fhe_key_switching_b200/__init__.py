@@ -58,6 +58,8 @@ _SIGS = {
     "ckks_chacha_expand": (_ci, [_vp, ctypes.POINTER(ctypes.c_uint8), _cu, _ci, _ci, _vp, _vp]),
     "ckks_workspace_bytes": (_sz, [_vp, _ci, _ci]),
     "ckks_sync_status": (_ci, [_vp, _vp, _ci]),
+    "ckks_prof_begin": (_ci, [_vp, ctypes.c_char_p, _ci]),
+    "ckks_prof_end": (_ci, [_vp, ctypes.POINTER(_ci), ctypes.POINTER(ctypes.c_double)]),
     "ckks_last_error": (ctypes.c_char_p, []),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -229,6 +231,18 @@ def ckks_chacha_expand(ctx, seed: bytes, key_id: int, digit: int, limb: int, out
 
 def ckks_sync_status(ctx, stream=None, timeout_ms: int = 10000) -> int:
     return int(_L.ckks_sync_status(ctx.handle if ctx is not None else None, _stream(stream), timeout_ms))
+
+
+def ckks_prof_begin(ctx, kernel: str, max_launches: int):
+    _check(_L.ckks_prof_begin(ctx.handle, kernel.encode(), max_launches), "ckks_prof_begin")
+
+
+def ckks_prof_end(ctx):
+    """(launches, total_ms) recorded since ckks_prof_begin."""
+    n = _ci()
+    ms = ctypes.c_double()
+    _check(_L.ckks_prof_end(ctx.handle, ctypes.byref(n), ctypes.byref(ms)), "ckks_prof_end")
+    return n.value, ms.value
 
 
 def galois_element(log_n: int, r: int) -> int:

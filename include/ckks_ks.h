@@ -161,6 +161,16 @@ size_t ckks_workspace_bytes(const ckks_ctx *ctx, int level, int n_rot);
  * CKKS_ERR_CUDA on an asynchronous error. */
 int ckks_sync_status(ckks_ctx *ctx, ckks_stream_t stream, int timeout_ms);
 
+/* Kernel timing.  Between ckks_prof_begin and ckks_prof_end, every launch of the kernel named
+ * `kernel` ("ip_row", "bconv", "ntt_col_fwd", "ntt_col_inv", "ntt_row_fwd", "ntt_row_inv",
+ * "row_combine", "tensor") made through `ctx` is bracketed by CUDA events recorded on its
+ * launching stream; up to max_launches launches are recorded (the events are created by
+ * ckks_prof_begin, outside any timed region).  ckks_prof_end synchronises on the last event and
+ * returns the number of recorded launches and their summed device time in milliseconds.
+ * Not thread-safe: one profiling session per context at a time. */
+int ckks_prof_begin(ckks_ctx *ctx, const char *kernel, int max_launches);
+int ckks_prof_end(ckks_ctx *ctx, int *launches, double *total_ms);
+
 /* Message of the last error on this thread ("" if none). */
 const char *ckks_last_error(void);
 
