@@ -58,6 +58,7 @@ _SIGS = {
     "ckks_chacha_expand": (_ci, [_vp, ctypes.POINTER(ctypes.c_uint8), _cu, _ci, _ci, _vp, _vp]),
     "ckks_workspace_bytes": (_sz, [_vp, _ci, _ci]),
     "ckks_sync_status": (_ci, [_vp, _vp, _ci]),
+    "ckks_keyswitch_noalloc": (_ci, [_vp, _vp, _ci, ctypes.POINTER(ckks_evk), _vp, _vp]),
     "ckks_prof_begin": (_ci, [_vp, ctypes.c_char_p, _ci]),
     "ckks_prof_end": (_ci, [_vp, ctypes.POINTER(_ci), ctypes.POINTER(ctypes.c_double)]),
     "ckks_last_error": (ctypes.c_char_p, []),
@@ -199,6 +200,16 @@ def ckks_moddown(ctx, acc, level: int, out, ws, stream=None):
 def ckks_keyswitch(ctx, c, level: int, evk: ckks_evk, out, ws, stream=None):
     _check(_L.ckks_keyswitch(ctx.handle, _ptr(c), level, ctypes.byref(evk), _ptr(out), _ptr(ws),
                              ws.numel() * ws.element_size(), _stream(stream)), "ckks_keyswitch")
+
+
+def ckks_keyswitch_noalloc(ctx, c, level: int, evk: ckks_evk, out, stream=None):
+    """ckks_keyswitch with the library's fixed device workspace: allocates nothing (for callers
+    whose host framework owns all device memory); calls must not overlap on the GPU."""
+    _check(_L.ckks_keyswitch_noalloc(ctx.handle, _ptr(c), level, ctypes.byref(evk), _ptr(out),
+                                     _stream(stream)), "ckks_keyswitch_noalloc")
+
+
+NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
 def ckks_rotate(ctx, ct, level: int, galois: int, evk: ckks_evk, out, ws, stream=None):

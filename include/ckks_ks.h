@@ -152,6 +152,26 @@ int ckks_tensor(ckks_ctx *ctx, const uint32_t *x, const uint32_t *y, int level, 
 int ckks_chacha_expand(ckks_ctx *ctx, const uint8_t seed[32], uint32_t key_id, int digit, int limb,
                        uint32_t *out, ckks_stream_t stream);
 
+/* Key switching without any device allocation, for callers that must not allocate device
+ * memory themselves: code that runs inside a host framework which owns every device
+ * allocation (a serving runtime with its own memory pool that forbids third-party cudaMalloc),
+ * or a latency-critical loop where a cudaMalloc, which may synchronise the device, is not
+ * acceptable.  Same operation and output as ckks_keyswitch; the workspace is a fixed array in
+ * the library's device memory (CKKS_NOALLOC_SCRATCH_BYTES, present on every GPU that loads the
+ * library until the process exits) instead of a caller buffer.
+ *  - Returns CKKS_ERR_WORKSPACE when ckks_workspace_bytes(ctx, level, 1) exceeds that size
+ *    (N=2^12 and N=2^14 parameter sets fit; N=2^16 with 36+12 primes does not).
+ *  - The first call on a device looks up the array's device address (once per device, with
+ *    that device current) and should come before any stream capture on that device.
+ *  - Every call on a device shares the one array: calls that may overlap on the GPU (different
+ *    streams, or different host threads) race on it; serialise them.  Nothing in the array
+ *    needs to start at zero, so the previous call's contents are harmless.
+ *  - Allocates nothing: no cudaMalloc, no cudaFree.
+ * (This entry point is an engineering addition; the pages describe nothing like it.) */
+#define CKKS_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+int ckks_keyswitch_noalloc(ckks_ctx *ctx, const uint32_t *c, int level, const ckks_evk *evk,
+                           uint32_t *out, ckks_stream_t stream);
+
 /* Workspace bytes for keyswitch/rotate/relin/modup/moddown at `level`
  * (n_rot > 1: rotate_hoisted with n_rot rotations). */
 size_t ckks_workspace_bytes(const ckks_ctx *ctx, int level, int n_rot);
