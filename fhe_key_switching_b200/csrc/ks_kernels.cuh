@@ -461,62 +461,12 @@ __device__ __forceinline__ void row_inv_regs(u32 (&x)[16], const tw_t *tw, u32 b
     inv_top4(x, tw, base, q, two_q);
 }
 
-// ---------------------------------------------------------------- bulk copies (TMA)
-// 1-D bulk global->shared copies completing on an mbarrier (no multicast).  Every wait is
-// bounded: after WAIT_LIMIT polls the kernel records KS_ERR_WAIT in the device error word.
-constexpr u32 KS_ERR_WAIT = 1u;
-constexpr int WAIT_LIMIT = 1 << 24;
-
-__device__ __forceinline__ u32 smem_u32(const void *p) { return (u32)__cvta_generic_to_shared(p); }
-
-__device__ __forceinline__ void mbar_init(uint64_t *bar, u32 count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_fence_init() {
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, u32 bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, u32 parity) {
-    u32 ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-// bounded wait; false (and the error word set) if the phase did not complete
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, u32 parity, u32 *err) {
-    for (int it = 0; it < WAIT_LIMIT; it++)
-        if (mbar_try_wait(bar, parity)) return true;
-    if (err) atomicOr(err, KS_ERR_WAIT);
-    return false;
-}
-__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, u32 bytes, uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_u32(dst)),
-        "l"(src), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
-__device__ __forceinline__ void fence_proxy_async() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 // Key inner product fused with the last forward NTT pass of ModUp.  Block (16 rows, u): for
 // every active digit j, the extended digit dt_j[u] is completed in registers (forward row
 // pass of the column-pass output x[j][u], or the input polynomial itself for u inside digit
 // j), the key's a half for (digit j, limb t) is regenerated by ChaCha12 for the same 16
 // slots, and
 //   acc0 += dt_j[u] * b_j[t],  acc1 += dt_j[u] * a_j[t]   (Montgomery products, mod t).
-// The 16-row source tile and the b (and stored a) tile of digit j+1 are brought into shared
-// memory by bulk copies while digit j is computed (three stages, one mbarrier each; a block
-// barrier is needed only when a stage is refilled, i.e. beyond three digits).
 // Rotations: hoist_g != 0 reads every dt_j[u] through kappa_{hoist_g} (hoisted rotation:
 // the source row is transformed, then permuted inside the row); cdig_g != 0 reads only the
 // input polynomial's digit limbs through kappa_{cdig_g} (single rotation).
@@ -529,117 +479,48 @@ struct IpRowArgs {
     u32 *acc;                // [2][ext][N]
     const tw_t *twf, *twi;
     const PrimeInfo *pinfo;
-    u32 *err;                // device error word
     ChachaKey key;
     u32 key_id;
     int log_n, level, n_q, n_primes, alpha, beta, ext;
     u32 hoist_g, cdig_g;
 };
 
-constexpr int IPR_ROWS = 8;                              // rows per block (16 threads each)
-constexpr int IPR_THREADS = IPR_ROWS * 16;
-constexpr int IPR_TILE = IPR_ROWS * 256;                 // words per tile
-constexpr int IPR_XCH = IPR_ROWS * 272;                  // row-exchange words
-constexpr int IPR_STAGES = 3;                            // digits in flight (no reuse when beta <= 3)
-
-__host__ __device__ constexpr size_t ip_row_smem(bool stored_a) {
-    return (size_t)(IPR_STAGES * (stored_a ? 3 : 2) * IPR_TILE + IPR_XCH) * sizeof(u32) +
-           IPR_STAGES * sizeof(uint64_t);
-}
-
-// Producer side of k_ip_row: one thread issues the bulk copies of digit j's tiles into the
-// stage at dst (completing on *bar): the 16 source rows (permuted rows for rotations), the b
-// rows and, for the stored-a ablation, the a rows.
-__device__ __forceinline__ void ip_issue(const IpRowArgs &a, int j, u32 *dst, int stage_words, uint64_t *bar,
-                                      int u, int t, int row0, int na, u32 gdig) {
-    const int n = 1 << a.log_n;
-    const bool dig = u < na && u >= j * a.alpha && u < min(j * a.alpha + a.alpha, na);
-    const u32 g = dig ? gdig : a.hoist_g;
-    const u32 *src = dig ? a.cdig + (size_t)u * n : a.x + ((size_t)j * a.ext + u) * n;
-    mbar_expect_tx(bar, (u32)(stage_words * sizeof(u32)));
-    if (g) {
-        for (int rr = 0; rr < IPR_ROWS; rr++) {
-            const int sr = (int)(automorph_src((u32)((row0 + rr) * 256), g, a.log_n) >> 8);
-            bulk_g2s(dst + rr * 256, src + (size_t)sr * 256, 1024u, bar);
-        }
-    } else {
-        bulk_g2s(dst, src + (size_t)row0 * 256, (u32)(IPR_TILE * sizeof(u32)), bar);
-    }
-    bulk_g2s(dst + IPR_TILE, a.b + ((size_t)j * a.n_primes + t) * n + (size_t)row0 * 256,
-             (u32)(IPR_TILE * sizeof(u32)), bar);
-    if (a.a_stored)
-        bulk_g2s(dst + 2 * IPR_TILE, a.a_stored + ((size_t)j * a.n_primes + t) * n + (size_t)row0 * 256,
-                 (u32)(IPR_TILE * sizeof(u32)), bar);
-}
-
-__global__ void __launch_bounds__(IPR_THREADS, 4)
+__global__ void __launch_bounds__(ROW_THREADS)
 k_ip_row(IpRowArgs a) {
-    extern __shared__ __align__(128) u32 smi[];
+    __shared__ u32 sm[16 * 272];
     const int n = 1 << a.log_n;
     const int na = a.level + 1;
     const int u = blockIdx.y;
     const int t = u < na ? u : a.n_q + (u - na);
-    const int ntile = a.a_stored ? 3 : 2;
-    const int stage_words = ntile * IPR_TILE;       // stage s starts at smi + s * stage_words
-    u32 *xch = smi + IPR_STAGES * ntile * IPR_TILE;
-    uint64_t *bar = reinterpret_cast<uint64_t *>(xch + IPR_XCH);
     const PrimeInfo pi = a.pinfo[t];
     const u32 q = pi.q, two_q = 2 * q;
     const int r = threadIdx.x >> 4, lo = threadIdx.x & 15;
-    const int row0 = blockIdx.x * IPR_ROWS;
-    const int row = row0 + r;
+    const int row = blockIdx.x * 16 + r;
     const u32 R1 = (u32)(n >> 8);
-    u32 *srow = xch + r * 272;
-    const int k0 = row * 256 + 16 * lo;
+    u32 *srow = sm + r * 272;
+    const int k0 = row * 256 + 16 * lo;              // first evaluation slot of this thread
     const tw_t *twf = a.twf + (size_t)t * n;
-    const u32 gdig = a.hoist_g ? a.hoist_g : a.cdig_g;   // gather for digit limbs
-    if (threadIdx.x == 0) {
-        for (int st = 0; st < IPR_STAGES; st++) mbar_init(&bar[st], 1);
-        mbar_fence_init();
-    }
-    __syncthreads();
-    if (threadIdx.x == 0)
-        for (int j = 0; j < min(a.beta, IPR_STAGES - 1); j++)
-            ip_issue(a, j, smi + j * stage_words, stage_words, bar + j, u, t, row0, na, gdig);
     // hoisted rotation: source row of this row under kappa_g
     const int src_row = a.hoist_g ? (int)(automorph_src((u32)(row * 256), a.hoist_g, a.log_n) >> 8) : row;
     u32 acc0[16], acc1[16];
 #pragma unroll
     for (int v = 0; v < 16; v++) acc0[v] = acc1[v] = 0;
-    bool ok = true;
     for (int j = 0; j < a.beta; j++) {
-        const int s = j % IPR_STAGES;
-        // digit j+2 goes to the stage of digit j-1 (released by the barrier ending digit j-1)
-        const int jn = j + IPR_STAGES - 1;
-        if (threadIdx.x == 0 && jn < a.beta) {
-            const int sn = jn % IPR_STAGES;
-            fence_proxy_async();
-            ip_issue(a, jn, smi + sn * stage_words, stage_words, bar + sn, u, t, row0, na, gdig);
-        }
-        // the key's a half for these 16 slots: ChaCha12 (independent of the copies in flight)
-        u32 av[16];
-        if (!a.a_stored) {
-            u32 h[8];
-            chacha_coeffs<false>(a.key, a.key_id, (u32)j, (u32)t, (u32)(k0 >> 3), pi, h);
-#pragma unroll
-            for (int v = 0; v < 8; v++) av[v] = h[v];
-            chacha_coeffs<false>(a.key, a.key_id, (u32)j, (u32)t, (u32)(k0 >> 3) + 1u, pi, h);
-#pragma unroll
-            for (int v = 0; v < 8; v++) av[8 + v] = h[v];
-        }
-        if (!mbar_wait(&bar[s], (u32)((j / IPR_STAGES) & 1), a.err)) { ok = false; break; }
-        const u32 *tile = smi + s * stage_words + r * 256;
+        const bool in_digit = u < na && u >= j * a.alpha && u < min(j * a.alpha + a.alpha, na);
         u32 x[16];
-        if (u < na && u >= j * a.alpha && u < min(j * a.alpha + a.alpha, na)) {
-            if (gdig) {
+        if (in_digit) {
+            const u32 *src = a.cdig + (size_t)u * n;
+            const u32 g = a.hoist_g ? a.hoist_g : a.cdig_g;
+            if (g) {
 #pragma unroll
-                for (int v = 0; v < 16; v++) x[v] = tile[automorph_src((u32)(k0 + v), gdig, a.log_n) & 255u];
+                for (int v = 0; v < 16; v++) x[v] = src[automorph_src((u32)(k0 + v), g, a.log_n)];
             } else {
-                load16_vec(tile + 16 * lo, x);
+                load16_vec(src + k0, x);
             }
         } else {
+            const u32 *src = a.x + ((size_t)j * a.ext + u) * n + (size_t)src_row * 256;
 #pragma unroll
-            for (int v = 0; v < 16; v++) x[v] = tile[lo + 16 * v];
+            for (int v = 0; v < 16; v++) x[v] = src[lo + 16 * v];
             row_fwd_regs(x, twf, R1 + (u32)src_row, lo, srow, q);
             if (a.hoist_g) {            // permute inside the row: slot k takes source slot src(k)
 #pragma unroll
@@ -653,25 +534,37 @@ k_ip_row(IpRowArgs a) {
                 __syncwarp();
             }
         }
-        u32 bv[16];
-        load16_vec(tile + IPR_TILE + 16 * lo, bv);
-        if (a.a_stored) load16_vec(tile + 2 * IPR_TILE + 16 * lo, av);
+        u32 bv[16], av[16];
+        load16_vec(a.b + ((size_t)j * a.n_primes + t) * n + k0, bv);
+        if (a.a_stored) {
+            load16_vec(a.a_stored + ((size_t)j * a.n_primes + t) * n + k0, av);
+        } else {
+            u32 h[8];
+            chacha_coeffs<false>(a.key, a.key_id, (u32)j, (u32)t, (u32)(k0 >> 3), pi, h);
+#pragma unroll
+            for (int v = 0; v < 8; v++) av[v] = h[v];
+            chacha_coeffs<false>(a.key, a.key_id, (u32)j, (u32)t, (u32)(k0 >> 3) + 1u, pi, h);
+#pragma unroll
+            for (int v = 0; v < 8; v++) av[8 + v] = h[v];
+        }
 #pragma unroll
         for (int v = 0; v < 16; v++) {
             acc0[v] = csub(acc0[v] + mont_mul(x[v], bv[v], q, pi.qinv), two_q);
             acc1[v] = csub(acc1[v] + mont_mul(x[v], av[v], q, pi.qinv), two_q);
         }
-        if (j + IPR_STAGES < a.beta) __syncthreads();   // stage s will be refilled
     }
-    if (!ok) return;    // (a failed wait means the copies never completed; nothing to drain)
-    // undo the Montgomery factor 2^-32, canonical output
+    // undo the Montgomery factor 2^-32
 #pragma unroll
     for (int v = 0; v < 16; v++) {
-        acc0[v] = csub(shoup_mul(acc0[v], pi.r64, pi.r64p, q), q);
-        acc1[v] = csub(shoup_mul(acc1[v], pi.r64, pi.r64p, q), q);
+        acc0[v] = shoup_mul(acc0[v], pi.r64, pi.r64p, q);
+        acc1[v] = shoup_mul(acc1[v], pi.r64, pi.r64p, q);
     }
-    store16_vec(a.acc + (size_t)u * n + k0, acc0);
-    store16_vec(a.acc + ((size_t)a.ext + u) * n + k0, acc1);
+    u32 *o0 = a.acc + (size_t)u * n + (size_t)row * 256;
+    u32 *o1 = a.acc + ((size_t)a.ext + u) * n + (size_t)row * 256;
+#pragma unroll
+    for (int v = 0; v < 16; v++) { acc0[v] = csub(acc0[v], q); acc1[v] = csub(acc1[v], q); }
+    store16_vec(o0 + 16 * lo, acc0);
+    store16_vec(o1 + 16 * lo, acc1);
 }
 
 // Last forward NTT pass of ModDown's converted limbs fused with the combine:
