@@ -1,16 +1,19 @@
 """Benchmark: RNS-CKKS hybrid key switching at N=2^16 (config 3) on B200.
 
-One step = one pass of the whole key-switching path over one batch of synthetic input:
+One step = one pass of the whole key-switching path over one batch of B independent units
+of config 3 (default B = 8), each unit
   d   = tensor(x, y)            (ct x ct product, 36 limbs)
   r   = relin(d)                (key switch #1: ModUp, ChaCha12 inner product, ModDown)
   out = rotate(r, g = 5)        (automorphism + key switch #2)
-at N=2^16, 36 ciphertext + 12 special primes (< 2^30), dnum 3, full level.  The metric is
-key-switches/s (2 per step) over all ranks; rotations/s is reported beside it.
+at N=2^16, 36 ciphertext + 12 special primes (< 2^30), dnum 3, full level.  The batch runs
+through the batched entry points (one launch per kernel covers all B units).  Every unit has
+its own relinearisation and rotation keys.  The metric is key-switches/s (2 per unit) over all
+ranks; rotations/s is reported beside it.
 
 Inputs are synthetic: uniform residues for the ciphertexts and for the keys' stored b halves
 (the cost of every kernel is data independent), seeded per rank.  Three independent buffer
-and key sets (> 126 MB L2 in total) are cycled so that consecutive steps never find their
-inputs in L2.
+and key sets (each larger than the 126 MB L2) are cycled so that consecutive steps never find
+their inputs in L2.
 
 --impl reference times the CPU oracle (the plain C restatement of the same path) on the host
 cores instead, on a bounded sample of the same workload.
@@ -33,8 +36,8 @@ import workloads as W  # noqa: E402
 
 CONFIG_KEY = "3"
 METRIC = "key-switches/s (rotations/s) at N=2^16, 32-bit RNS; % of HBM roofline"
-KS_PER_STEP = 2          # relin + rotation
-ROT_PER_STEP = 1
+KS_PER_UNIT = 2          # relin + rotation
+ROT_PER_UNIT = 1
 N_SETS = 3
 
 
@@ -116,26 +119,28 @@ def run_ours(args, rank, world, local_rank):
         a = W.uniform_residues(moduli, n, W.rng(cfg.seed, W.TAG_SYNTH, rank, seed_tag))
         return torch.from_numpy(a).to(dev)
 
+    B = args.batch
     sets = []
     for s in range(N_SETS):
-        x = residues(q[:na] * 2, 10 * s + 1).view(2, na, n)
-        y = residues(q[:na] * 2, 10 * s + 2).view(2, na, n)
-        b_rel = residues(mods * nd, 10 * s + 3).view(nd, len(mods), n)
-        b_rot = residues(mods * nd, 10 * s + 4).view(nd, len(mods), n)
+        x = residues(q[:na] * 2 * B, 10 * s + 1).view(B, 2, na, n)
+        y = residues(q[:na] * 2 * B, 10 * s + 2).view(B, 2, na, n)
+        b_rel = residues(mods * nd * B, 10 * s + 3).view(B, nd, len(mods), n)
+        b_rot = residues(mods * nd * B, 10 * s + 4).view(B, nd, len(mods), n)
         sets.append(dict(x=x, y=y, b_rel=b_rel, b_rot=b_rot,
-                         k_rel=ks.make_evk(b_rel, cfg.chacha_seed, 0),
-                         k_rot=ks.make_evk(b_rot, cfg.chacha_seed, g)))
-    d = torch.empty((3, na, n), dtype=torch.uint32, device=dev)
-    r = torch.empty((2, na, n), dtype=torch.uint32, device=dev)
-    out = torch.empty((2, na, n), dtype=torch.uint32, device=dev)
-    ws = ctx.workspace(lvl, device=dev)
+                         k_rel=[ks.make_evk(b_rel[i], cfg.chacha_seed, 0) for i in range(B)],
+                         k_rot=[ks.make_evk(b_rot[i], cfg.chacha_seed, g) for i in range(B)]))
+    d = torch.empty((B, 3, na, n), dtype=torch.uint32, device=dev)
+    r = torch.empty((B, 2, na, n), dtype=torch.uint32, device=dev)
+    out = torch.empty((B, 2, na, n), dtype=torch.uint32, device=dev)
+    ws = ctx.workspace(lvl, B, device=dev)
     stream = torch.cuda.current_stream(dev)
+    gal = [g] * B
 
     def step(i):
         st = sets[i % N_SETS]
-        ks.ckks_tensor(ctx, st["x"], st["y"], lvl, d, stream)
-        ks.ckks_relin(ctx, d, lvl, st["k_rel"], r, ws, stream)
-        ks.ckks_rotate(ctx, r, lvl, g, st["k_rot"], out, ws, stream)
+        ks.ckks_tensor_batch(ctx, B, st["x"], st["y"], lvl, d, stream)
+        ks.ckks_relin_batch(ctx, d, lvl, st["k_rel"], r, ws, stream)
+        ks.ckks_rotate_batch(ctx, r, lvl, gal, st["k_rot"], out, ws, stream)
 
     def barrier():
         if world > 1:
@@ -152,7 +157,7 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     # the dominant kernel's launches are bracketed by events on the launching stream
-    ks.ckks_prof_begin(ctx, DOMINANT, KS_PER_STEP * args.steps)
+    ks.ckks_prof_begin(ctx, DOMINANT, KS_PER_UNIT * args.steps)
     e0.record(stream)
     for i in range(args.steps):
         step(i)
@@ -167,21 +172,21 @@ def run_ours(args, rank, world, local_rank):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
     ms_per_step = ms / args.steps
-    value = KS_PER_STEP * args.steps * world / (ms / 1e3)
+    value = KS_PER_UNIT * B * args.steps * world / (ms / 1e3)
 
     # end to end: pinned host inputs copied in, result copied out, every step
     h_x = [s["x"].cpu().pin_memory() for s in sets]
     h_y = [s["y"].cpu().pin_memory() for s in sets]
-    h_out = torch.empty((2, na, n), dtype=torch.uint32).pin_memory()
+    h_out = torch.empty((B, 2, na, n), dtype=torch.uint32).pin_memory()
     dx, dy = torch.empty_like(sets[0]["x"]), torch.empty_like(sets[0]["y"])
 
     def step_e2e(i):
         st = sets[i % N_SETS]
         dx.copy_(h_x[i % N_SETS], non_blocking=True)
         dy.copy_(h_y[i % N_SETS], non_blocking=True)
-        ks.ckks_tensor(ctx, dx, dy, lvl, d, stream)
-        ks.ckks_relin(ctx, d, lvl, st["k_rel"], r, ws, stream)
-        ks.ckks_rotate(ctx, r, lvl, g, st["k_rot"], out, ws, stream)
+        ks.ckks_tensor_batch(ctx, B, dx, dy, lvl, d, stream)
+        ks.ckks_relin_batch(ctx, d, lvl, st["k_rel"], r, ws, stream)
+        ks.ckks_rotate_batch(ctx, r, lvl, gal, st["k_rot"], out, ws, stream)
         h_out.copy_(out, non_blocking=True)
 
     for i in range(args.warmup):
@@ -199,7 +204,7 @@ def run_ours(args, rank, world, local_rank):
         t = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_e2e = float(t.item())
-    e2e_value = KS_PER_STEP * args.steps * world / (ms_e2e / 1e3)
+    e2e_value = KS_PER_UNIT * B * args.steps * world / (ms_e2e / 1e3)
     h2d = (sets[0]["x"].numel() + sets[0]["y"].numel()) * 4
     d2h = out.numel() * 4
 
@@ -210,7 +215,7 @@ def run_ours(args, rank, world, local_rank):
             "metric": METRIC,
             "value": value,
             "unit": "key-switches/s",
-            "rotations_per_s": ROT_PER_STEP * args.steps * world / (ms / 1e3),
+            "rotations_per_s": ROT_PER_UNIT * B * args.steps * world / (ms / 1e3),
             "n_gpus": world,
             "steps": args.steps,
             "warmup": args.warmup,
@@ -221,18 +226,20 @@ def run_ours(args, rank, world, local_rank):
             "dtype": "u32",
             "data": "synthetic",
             "config": {"workload": "config 3: N=2^16, 36+12 primes < 2^30, dnum 3, level 35; "
-                                   "step = tensor + relin + rotate(1)",
+                                   f"step = batch of {B} independent units, each tensor + relin + "
+                                   "rotate(1) with its own keys",
                        "log_n": cfg.log_n, "n_q": cfg.n_q, "n_p": cfg.n_p, "dnum": cfg.dnum,
-                       "level": lvl, "key_switches_per_step": KS_PER_STEP,
-                       "l2": f"{N_SETS} rotating input/key sets (~{N_SETS * 150} MiB > 126 MB L2)",
+                       "level": lvl, "batch": B, "key_switches_per_step": KS_PER_UNIT * B,
+                       "l2": f"{N_SETS} rotating input/key sets (each > 126 MB L2)",
                        "parallelism": f"replicas x{world}"},
             "e2e": {"value": e2e_value, "unit": "key-switches/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": args.steps * LAUNCHES_PER_STEP,
+            "kernel_launches_note": "one launch per kernel covers the whole batch",
             "clocks": clk,
-            "roofline": roofline(cfg, dom_launches, dom_ms, clk),
-            "hbm_fraction_step": {"b_min_bytes_per_step": step_bytes_min(cfg),
-                                  "frac": step_bytes_min(cfg) / (ms_per_step / 1e3) / (HBM_PEAK_GBS * 1e9),
+            "roofline": roofline(cfg, dom_launches, dom_ms, clk, B),
+            "hbm_fraction_step": {"b_min_bytes_per_step": B * step_bytes_min(cfg),
+                                  "frac": B * step_bytes_min(cfg) / (ms_per_step / 1e3) / (HBM_PEAK_GBS * 1e9),
                                   "peak_gbs": HBM_PEAK_GBS, "peak_source": PEAK_SOURCE},
             "cpu_baseline": cpu,
         }
@@ -264,7 +271,7 @@ def alu_peak_tops(mhz: float) -> float:
 
 
 def ip_row_ops(cfg) -> float:
-    """Algorithmic int32 operations of one k_ip_row launch (one key switch), with the unit costs
+    """Algorithmic int32 operations of one key switch's share of a k_ip_row launch, with the unit costs
     of the op model: ChaCha12 block 608 (8 coefficients), 64-bit word reduction 8, NTT butterfly
     8, variable modular product 6, modular addition 2.  Units: beta*ext (digit, limb) pairs of N
     coefficients; the row pass (8 of log N stages) runs on the pairs outside their digit."""
@@ -280,11 +287,11 @@ def ip_row_ops(cfg) -> float:
     return chacha + a_red + ntt + macs
 
 
-def roofline(cfg, launches, total_ms, clk):
+def roofline(cfg, launches, total_ms, clk, batch):
     if not launches:
         return None
     avg_s = total_ms / launches / 1e3
-    achieved = ip_row_ops(cfg) / avg_s / 1e12
+    achieved = batch * ip_row_ops(cfg) / avg_s / 1e12
     peak = alu_peak_tops(SM_MAX_MHZ)
     return {"kernel": "k_ip_row (ModUp last NTT pass + ChaCha12 + key inner product)",
             "bound": "alu", "achieved": achieved, "peak": peak, "unit": "Tops (int32)",
@@ -355,9 +362,9 @@ def cpu_baseline(max_seconds: float = 20.0):
         if time.perf_counter() - t0 > max_seconds / 2 or k >= 8:
             break
     dt = time.perf_counter() - t0
-    return {"value": KS_PER_STEP * k / dt, "unit": "key-switches/s", "cores": _omp_threads(),
+    return {"value": KS_PER_UNIT * k / dt, "unit": "key-switches/s", "cores": _omp_threads(),
             "kind": "oracle",
-            "sample": f"{k} steps of config 3 (tensor + relin + rotate, 2 key switches each) "
+            "sample": f"{k} units of config 3 (tensor + relin + rotate, 2 key switches each) "
                       "on synthetic residues, plain C oracle with OpenMP over limbs"}
 
 
@@ -371,7 +378,7 @@ def run_reference(args, rank, world):
     for _ in range(args.steps):
         one_step()
     dt = time.perf_counter() - t0
-    value = KS_PER_STEP * args.steps / dt
+    value = KS_PER_UNIT * args.steps / dt
     cfg = W.CONFIGS[CONFIG_KEY]
     line = {
         "impl": "reference",
@@ -388,9 +395,9 @@ def run_reference(args, rank, world):
         "dtype": "u32",
         "data": "synthetic",
         "config": {"workload": "config 3: N=2^16, 36+12 primes < 2^30, dnum 3, level 35; "
-                               "step = tensor + relin + rotate(1)",
+                               "step = one unit: tensor + relin + rotate(1)",
                    "log_n": cfg.log_n, "n_q": cfg.n_q, "n_p": cfg.n_p, "dnum": cfg.dnum,
-                   "level": cfg.level, "key_switches_per_step": KS_PER_STEP},
+                   "level": cfg.level, "key_switches_per_step": KS_PER_UNIT},
         "cpu_baseline": {"kind": "oracle", "cores": _omp_threads(), "value": value,
                          "unit": "key-switches/s",
                          "sample": f"{args.steps} timed steps of config 3 on the host cores"},
@@ -407,6 +414,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=8, help="independent config-3 units per step")
     args = ap.parse_args()
     rank = _env_int("RANK", 0)
     world = _env_int("WORLD_SIZE", 1)

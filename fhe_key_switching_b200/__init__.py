@@ -54,6 +54,10 @@ _SIGS = {
     "ckks_rotate_hoisted": (_ci, [_vp, _vp, _ci, _ci, _u32p, ctypes.POINTER(ckks_evk), _vp, _vp,
                                   _sz, _vp]),
     "ckks_relin": (_ci, [_vp, _vp, _ci, ctypes.POINTER(ckks_evk), _vp, _vp, _sz, _vp]),
+    "ckks_keyswitch_batch": (_ci, [_vp, _ci, _vp, _ci, ctypes.POINTER(ckks_evk), _vp, _vp, _sz, _vp]),
+    "ckks_rotate_batch": (_ci, [_vp, _ci, _vp, _ci, _u32p, ctypes.POINTER(ckks_evk), _vp, _vp, _sz, _vp]),
+    "ckks_relin_batch": (_ci, [_vp, _ci, _vp, _ci, ctypes.POINTER(ckks_evk), _vp, _vp, _sz, _vp]),
+    "ckks_tensor_batch": (_ci, [_vp, _ci, _vp, _vp, _ci, _vp, _vp]),
     "ckks_tensor": (_ci, [_vp, _vp, _vp, _ci, _vp, _vp]),
     "ckks_chacha_expand": (_ci, [_vp, ctypes.POINTER(ctypes.c_uint8), _cu, _ci, _ci, _vp, _vp]),
     "ckks_workspace_bytes": (_sz, [_vp, _ci, _ci]),
@@ -232,6 +236,37 @@ def ckks_relin(ctx, d, level: int, evk: ckks_evk, out, ws, stream=None):
 
 def ckks_tensor(ctx, x, y, level: int, d, stream=None):
     _check(_L.ckks_tensor(ctx.handle, _ptr(x), _ptr(y), level, _ptr(d), _stream(stream)), "ckks_tensor")
+
+
+def _evk_array(evks):
+    n = len(evks)
+    return (ckks_evk * max(n, 1))(*evks)
+
+
+def ckks_keyswitch_batch(ctx, c, level: int, evks, out, ws, stream=None):
+    """Batch of len(evks) key switches: c [n][l+1][N] -> out [n][2][l+1][N]."""
+    _check(_L.ckks_keyswitch_batch(ctx.handle, len(evks), _ptr(c), level, _evk_array(evks), _ptr(out), _ptr(ws),
+                                   ws.numel() * ws.element_size(), _stream(stream)), "ckks_keyswitch_batch")
+
+
+def ckks_rotate_batch(ctx, ct, level: int, galois, evks, out, ws, stream=None):
+    """Batch of rotations: ct [n][2][l+1][N], galois and evks of n entries -> out [n][2][l+1][N]."""
+    n = len(galois)
+    ga = (ctypes.c_uint32 * max(n, 1))(*galois)
+    _check(_L.ckks_rotate_batch(ctx.handle, n, _ptr(ct), level, ga, _evk_array(evks), _ptr(out), _ptr(ws),
+                                ws.numel() * ws.element_size(), _stream(stream)), "ckks_rotate_batch")
+
+
+def ckks_relin_batch(ctx, d, level: int, evks, out, ws, stream=None):
+    """Batch of relinearisations: d [n][3][l+1][N] -> out [n][2][l+1][N]."""
+    _check(_L.ckks_relin_batch(ctx.handle, len(evks), _ptr(d), level, _evk_array(evks), _ptr(out), _ptr(ws),
+                               ws.numel() * ws.element_size(), _stream(stream)), "ckks_relin_batch")
+
+
+def ckks_tensor_batch(ctx, n: int, x, y, level: int, d, stream=None):
+    """Batch of tensor products: x, y [n][2][l+1][N] -> d [n][3][l+1][N]."""
+    _check(_L.ckks_tensor_batch(ctx.handle, n, _ptr(x), _ptr(y), level, _ptr(d), _stream(stream)),
+           "ckks_tensor_batch")
 
 
 def ckks_chacha_expand(ctx, seed: bytes, key_id: int, digit: int, limb: int, out, stream=None):

@@ -88,6 +88,8 @@ struct BconvArgs {
     int cfg_per_group;       // table config index = g * cfg_per_group + (n_in(g) - 1) (ModUp), or 0
     int cfg_stride;          // words per config in bmat = max_in * n_primes
     int g_base;              // logical group of blockIdx.y = 0 (a launch may cover a subset)
+    int nchunk;              // target chunks per item: blockIdx.z = item * nchunk + chunk
+    size_t y_item, out_item; // item strides (words)
 };
 
 constexpr int BCONV_THREADS = 256;
@@ -101,6 +103,9 @@ __global__ void __launch_bounds__(BCONV_THREADS)
 k_bconv(BconvArgs a) {
     extern __shared__ u32 smb[];          // [n_in + 1][T] constants (row n_in: [-D]_t), then half[n_in]
     const int g = a.g_base + blockIdx.y;
+    const int item = blockIdx.z / a.nchunk, chunk = blockIdx.z % a.nchunk;
+    const u32 *yb = a.y + item * a.y_item;
+    u32 *ob = a.out + item * a.out_item;
     const int n = 1 << a.log_n;
     const int n_in = (g == a.n_groups - 1) ? a.n_in_last : a.n_in_full;
     const int cfg = a.cfg_per_group ? g * a.cfg_per_group + (n_in - 1) : 0;
@@ -124,7 +129,7 @@ k_bconv(BconvArgs a) {
 #pragma unroll
     for (int i = 0; i < MAXIN; i++) {
         if (i < n_in) {
-            const uint2 t = reinterpret_cast<const uint2 *>(a.y + (size_t)(row0 + i) * n)[c2];
+            const uint2 t = reinterpret_cast<const uint2 *>(yb + (size_t)(row0 + i) * n)[c2];
             const u32 h = half[i];
             y0[i] = t.x; y1[i] = t.y;
             v0 += t.x > h ? 1u : 0u;
@@ -133,8 +138,8 @@ k_bconv(BconvArgs a) {
     }
     const int lo = a.map.skip_alpha > 0 ? g * a.map.skip_alpha : 0;
     const int hi = a.map.skip_alpha > 0 ? min(lo + a.map.skip_alpha, a.map.split) : 0;
-    const int k_end = min(T, (int)(blockIdx.z + 1) * BCONV_TCHUNK);
-    for (int kk = blockIdx.z * BCONV_TCHUNK; kk < k_end; kk++) {
+    const int k_end = min(T, (chunk + 1) * BCONV_TCHUNK);
+    for (int kk = chunk * BCONV_TCHUNK; kk < k_end; kk++) {
         if (kk >= lo && kk < hi) continue;
         const int t = kk < a.map.split ? a.map.lo_base + kk : a.map.hi_base + (kk - a.map.split);
         const PrimeInfo pi = a.pinfo[t];
@@ -167,6 +172,9 @@ __global__ void __launch_bounds__(BCONV_THREADS)
 k_bconv_n(BconvArgs a) {
     extern __shared__ __align__(16) u32 smc[];
     const int g = a.g_base + blockIdx.y;
+    const int item = blockIdx.z / a.nchunk, chunk = blockIdx.z % a.nchunk;
+    const u32 *yb = a.y + item * a.y_item;
+    u32 *ob = a.out + item * a.out_item;
     const int n = 1 << a.log_n;
     const int cfg = a.cfg_per_group ? g * a.cfg_per_group + (NIN - 1) : 0;
     const u32 *bm = a.bmat + (size_t)cfg * a.cfg_stride;
@@ -191,7 +199,7 @@ k_bconv_n(BconvArgs a) {
     u32 v0 = 0, v1 = 0;
 #pragma unroll
     for (int i = 0; i < NIN; i++) {
-        const uint2 t = reinterpret_cast<const uint2 *>(a.y + (size_t)(row0 + i) * n)[c2];
+        const uint2 t = reinterpret_cast<const uint2 *>(yb + (size_t)(row0 + i) * n)[c2];
         const u32 h = a.pinfo[p0 + i].half;
         y0[i] = t.x; y1[i] = t.y;
         v0 += t.x > h ? 1u : 0u;
@@ -200,7 +208,7 @@ k_bconv_n(BconvArgs a) {
     y0[NIN] = v0; y1[NIN] = v1;
     const int lo = a.map.skip_alpha > 0 ? g * a.map.skip_alpha : 0;
     const int hi = a.map.skip_alpha > 0 ? min(lo + a.map.skip_alpha, a.map.split) : 0;
-    const int k_beg = blockIdx.z * BCONV_TCHUNK;
+    const int k_beg = chunk * BCONV_TCHUNK;
     const int k_end = min(T, k_beg + BCONV_TCHUNK);
     for (int k4 = k_beg; k4 < k_end; k4 += 4) {
         u64 s0[4], s1[4];
@@ -224,7 +232,7 @@ k_bconv_n(BconvArgs a) {
             const PrimeInfo pi = a.pinfo[t];
             const uint2 r = make_uint2(reduce64(s0[m], pi.q, pi.r64, pi.r64p, pi.onep),
                                        reduce64(s1[m], pi.q, pi.r64, pi.r64p, pi.onep));
-            reinterpret_cast<uint2 *>(a.out + ((size_t)g * a.map.out_group_rows + a.map.out_k_base + kk) * n)[c2] = r;
+            reinterpret_cast<uint2 *>(ob + ((size_t)g * a.map.out_group_rows + a.map.out_k_base + kk) * n)[c2] = r;
         }
     }
 }
@@ -371,6 +379,9 @@ __global__ void k_tensor(const u32 *x, const u32 *y, u32 *d, const PrimeInfo *pi
     const size_t pl = (size_t)(level + 1) * n;
     const PrimeInfo pi = pinfo[i];
     const size_t off = (size_t)i * n;
+    x += blockIdx.z * 2 * pl;
+    y += blockIdx.z * 2 * pl;
+    d += blockIdx.z * 3 * pl;
     const uint4 x0 = reinterpret_cast<const uint4 *>(x + off)[c4];
     const uint4 x1 = reinterpret_cast<const uint4 *>(x + pl + off)[c4];
     const uint4 y0 = reinterpret_cast<const uint4 *>(y + off)[c4];
@@ -474,15 +485,17 @@ __device__ __forceinline__ void row_inv_regs(u32 (&x)[16], const tw_t *tw, u32 b
 struct IpRowArgs {
     const u32 *x;            // [beta][ext][N] ModUp column-pass output (non-digit limbs)
     const u32 *cdig;         // [l+1][N] input polynomial, evaluation domain
-    const u32 *b;            // [D][n_primes][N]
-    const u32 *a_stored;     // nullptr: regenerate
     u32 *acc;                // [2][ext][N]
+    size_t x_item, cdig_item, acc_item;        // item strides (words; 0 = shared)
     const tw_t *twf, *twi;
     const PrimeInfo *pinfo;
-    ChachaKey key;
-    u32 key_id;
     int log_n, level, n_q, n_primes, alpha, beta, ext;
-    u32 hoist_g, cdig_g;
+    // per item (blockIdx.z): the key and the rotation
+    const u32 *b[KS_MAXB];        // [D][n_primes][N]
+    const u32 *a_stored[KS_MAXB]; // nullptr: regenerate
+    ChachaKey key[KS_MAXB];
+    u32 key_id[KS_MAXB];
+    u32 hoist_g[KS_MAXB], cdig_g[KS_MAXB];
 };
 
 __global__ void __launch_bounds__(ROW_THREADS)
@@ -491,6 +504,15 @@ k_ip_row(IpRowArgs a) {
     const int n = 1 << a.log_n;
     const int na = a.level + 1;
     const int u = blockIdx.y;
+    const int item = blockIdx.z;
+    const u32 *xb = a.x + item * a.x_item;
+    const u32 *cdb = a.cdig + item * a.cdig_item;
+    u32 *accb = a.acc + item * a.acc_item;
+    const u32 *bkey = a.b[item];
+    const u32 *astore = a.a_stored[item];
+    const ChachaKey &key = a.key[item];
+    const u32 key_id = a.key_id[item];
+    const u32 hoist_g = a.hoist_g[item], cdig_g = a.cdig_g[item];
     const int t = u < na ? u : a.n_q + (u - na);
     const PrimeInfo pi = a.pinfo[t];
     const u32 q = pi.q, two_q = 2 * q;
@@ -501,7 +523,7 @@ k_ip_row(IpRowArgs a) {
     const int k0 = row * 256 + 16 * lo;              // first evaluation slot of this thread
     const tw_t *twf = a.twf + (size_t)t * n;
     // hoisted rotation: source row of this row under kappa_g
-    const int src_row = a.hoist_g ? (int)(automorph_src((u32)(row * 256), a.hoist_g, a.log_n) >> 8) : row;
+    const int src_row = hoist_g ? (int)(automorph_src((u32)(row * 256), hoist_g, a.log_n) >> 8) : row;
     u32 acc0[16], acc1[16];
 #pragma unroll
     for (int v = 0; v < 16; v++) acc0[v] = acc1[v] = 0;
@@ -509,8 +531,8 @@ k_ip_row(IpRowArgs a) {
         const bool in_digit = u < na && u >= j * a.alpha && u < min(j * a.alpha + a.alpha, na);
         u32 x[16];
         if (in_digit) {
-            const u32 *src = a.cdig + (size_t)u * n;
-            const u32 g = a.hoist_g ? a.hoist_g : a.cdig_g;
+            const u32 *src = cdb + (size_t)u * n;
+            const u32 g = hoist_g ? hoist_g : cdig_g;
             if (g) {
 #pragma unroll
                 for (int v = 0; v < 16; v++) x[v] = src[automorph_src((u32)(k0 + v), g, a.log_n)];
@@ -518,32 +540,32 @@ k_ip_row(IpRowArgs a) {
                 load16_vec(src + k0, x);
             }
         } else {
-            const u32 *src = a.x + ((size_t)j * a.ext + u) * n + (size_t)src_row * 256;
+            const u32 *src = xb + ((size_t)j * a.ext + u) * n + (size_t)src_row * 256;
 #pragma unroll
             for (int v = 0; v < 16; v++) x[v] = src[lo + 16 * v];
             row_fwd_regs(x, twf, R1 + (u32)src_row, lo, srow, q);
-            if (a.hoist_g) {            // permute inside the row: slot k takes source slot src(k)
+            if (hoist_g) {            // permute inside the row: slot k takes source slot src(k)
 #pragma unroll
                 for (int v = 0; v < 16; v++) srow[17 * lo + v] = x[v];
                 __syncwarp();
 #pragma unroll
                 for (int v = 0; v < 16; v++) {
-                    const u32 m = automorph_src((u32)(k0 + v), a.hoist_g, a.log_n) & 255u;
+                    const u32 m = automorph_src((u32)(k0 + v), hoist_g, a.log_n) & 255u;
                     x[v] = srow[m + (m >> 4)];
                 }
                 __syncwarp();
             }
         }
         u32 bv[16], av[16];
-        load16_vec(a.b + ((size_t)j * a.n_primes + t) * n + k0, bv);
-        if (a.a_stored) {
-            load16_vec(a.a_stored + ((size_t)j * a.n_primes + t) * n + k0, av);
+        load16_vec(bkey + ((size_t)j * a.n_primes + t) * n + k0, bv);
+        if (astore) {
+            load16_vec(astore + ((size_t)j * a.n_primes + t) * n + k0, av);
         } else {
             u32 h[8];
-            chacha_coeffs<false>(a.key, a.key_id, (u32)j, (u32)t, (u32)(k0 >> 3), pi, h);
+            chacha_coeffs<false>(key, key_id, (u32)j, (u32)t, (u32)(k0 >> 3), pi, h);
 #pragma unroll
             for (int v = 0; v < 8; v++) av[v] = h[v];
-            chacha_coeffs<false>(a.key, a.key_id, (u32)j, (u32)t, (u32)(k0 >> 3) + 1u, pi, h);
+            chacha_coeffs<false>(key, key_id, (u32)j, (u32)t, (u32)(k0 >> 3) + 1u, pi, h);
 #pragma unroll
             for (int v = 0; v < 8; v++) av[8 + v] = h[v];
         }
@@ -559,8 +581,8 @@ k_ip_row(IpRowArgs a) {
         acc0[v] = shoup_mul(acc0[v], pi.r64, pi.r64p, q);
         acc1[v] = shoup_mul(acc1[v], pi.r64, pi.r64p, q);
     }
-    u32 *o0 = a.acc + (size_t)u * n + (size_t)row * 256;
-    u32 *o1 = a.acc + ((size_t)a.ext + u) * n + (size_t)row * 256;
+    u32 *o0 = accb + (size_t)u * n + (size_t)row * 256;
+    u32 *o1 = accb + ((size_t)a.ext + u) * n + (size_t)row * 256;
 #pragma unroll
     for (int v = 0; v < 16; v++) { acc0[v] = csub(acc0[v], q); acc1[v] = csub(acc1[v], q); }
     store16_vec(o0 + 16 * lo, acc0);
@@ -577,18 +599,20 @@ struct RowCombineArgs {
     const u32 *acc;
     const u32 *add;
     u32 *out;                // [n_comp][l+1][N]
+    size_t conv_item, acc_item, add_item, out_item;   // item strides (words; 0 = shared)
     const tw_t *twf;
     const PrimeInfo *pinfo;
     const tw_t *pinv;
-    int log_n, level, ext, acc_comp_rows, add_comps;
-    u32 add_g;
+    int log_n, level, ext, acc_comp_rows, add_comps, n_comp;
+    u32 add_g[KS_MAXB];
 };
 
 __global__ void __launch_bounds__(ROW_THREADS)
 k_row_combine(RowCombineArgs a) {
     __shared__ u32 sm[16 * 272];
     const int n = 1 << a.log_n;
-    const int i = blockIdx.y, comp = blockIdx.z;
+    const int i = blockIdx.y, comp = blockIdx.z % a.n_comp, item = blockIdx.z / a.n_comp;
+    const u32 add_g = a.add_g[item];
     const int na = a.level + 1;
     const PrimeInfo pi = a.pinfo[i];
     const u32 q = pi.q;
@@ -597,26 +621,26 @@ k_row_combine(RowCombineArgs a) {
     const int k0 = row * 256 + 16 * lo;
     u32 *srow = sm + r * 272;
     u32 x[16];
-    const u32 *src = a.conv + ((size_t)comp * na + i) * n + (size_t)row * 256;
+    const u32 *src = a.conv + item * a.conv_item + ((size_t)comp * na + i) * n + (size_t)row * 256;
 #pragma unroll
     for (int v = 0; v < 16; v++) x[v] = src[lo + 16 * v];
     row_fwd_regs(x, a.twf + (size_t)i * n, (u32)(n >> 8) + (u32)row, lo, srow, q);
     u32 ac[16];
-    load16_vec(a.acc + ((size_t)comp * a.acc_comp_rows + i) * n + k0, ac);
+    load16_vec(a.acc + item * a.acc_item + ((size_t)comp * a.acc_comp_rows + i) * n + k0, ac);
     const tw_t w = a.pinv[i];
 #pragma unroll
     for (int v = 0; v < 16; v++) x[v] = csub(shoup_mul(ac[v] + q - x[v], w.x, w.y, q), q);
     if (comp < a.add_comps) {
-        const u32 *ad = a.add + ((size_t)comp * na + i) * n;
+        const u32 *ad = a.add + item * a.add_item + ((size_t)comp * na + i) * n;
         u32 y[16];
-        if (a.add_g) {
+        if (add_g) {
 #pragma unroll
-            for (int v = 0; v < 16; v++) y[v] = ad[automorph_src((u32)(k0 + v), a.add_g, a.log_n)];
+            for (int v = 0; v < 16; v++) y[v] = ad[automorph_src((u32)(k0 + v), add_g, a.log_n)];
         } else {
             load16_vec(ad + k0, y);
         }
 #pragma unroll
         for (int v = 0; v < 16; v++) x[v] = csub(x[v] + y[v], q);
     }
-    store16_vec(a.out + ((size_t)comp * na + i) * n + k0, x);
+    store16_vec(a.out + item * a.out_item + ((size_t)comp * na + i) * n + k0, x);
 }

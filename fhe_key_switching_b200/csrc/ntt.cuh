@@ -125,6 +125,10 @@ __device__ __forceinline__ u32 automorph_src(u32 k, u32 g, int log_n) {
     return __brev((e - 1u) >> 1) >> (32 - log_n);
 }
 
+// Batches: blockIdx.z selects an item; item z reads in + z*in_item and writes out + z*out_item
+// (strides in words).
+constexpr int KS_MAXB = 64;                 // items per launch
+
 struct NttArgs {
     const u32 *in;
     u32 *out;
@@ -133,7 +137,8 @@ struct NttArgs {
     const tw_t *scale;      // per-k output scale (inverse column pass), or nullptr
     JobMap map;
     int log_n;
-    u32 galois;             // inverse row pass: gather input through kappa_g (0 = none)
+    size_t in_item, out_item;
+    u32 galois[KS_MAXB];    // inverse row pass: gather item z's input through kappa_g (0 = none)
 };
 
 // ---------------------------------------------------------------- column pass (stages 0..r1-1)
@@ -165,8 +170,8 @@ k_ntt_col(NttArgs a) {
     const int lo = warp / cgroups;
     const int ccol = (warp % cgroups) * 32 + lane;          // column within block
     const int col = blockIdx.x * C::CPB + ccol;
-    const u32 *src = a.in + in_row * n;
-    u32 *dst = a.out + out_row * n;
+    const u32 *src = a.in + blockIdx.z * a.in_item + in_row * n;
+    u32 *dst = a.out + blockIdx.z * a.out_item + out_row * n;
     u32 x[16];
     if (FWD) {
 #pragma unroll
@@ -220,8 +225,9 @@ k_ntt_row(NttArgs a) {
     const int r = threadIdx.x >> 4, lo = threadIdx.x & 15;
     const int row = blockIdx.x * 16 + r;
     const u32 base = (u32)(n >> 8) + (u32)row;
-    const u32 *src = a.in + in_row * n;
-    u32 *dst = a.out + out_row * n + (size_t)row * 256;
+    const u32 *src = a.in + blockIdx.z * a.in_item + in_row * n;
+    u32 *dst = a.out + blockIdx.z * a.out_item + out_row * n + (size_t)row * 256;
+    const u32 galois = a.galois[blockIdx.z];
     u32 *srow = sm + r * 272;
     u32 x[16];
     if (FWD) {
@@ -245,10 +251,10 @@ k_ntt_row(NttArgs a) {
             reinterpret_cast<uint4 *>(dst + 16 * lo)[v] = o;
         }
     } else {
-        if (a.galois) {
+        if (galois) {
 #pragma unroll
             for (int u = 0; u < 16; u++)
-                x[u] = src[automorph_src((u32)(row * 256 + 16 * lo + u), a.galois, a.log_n)];
+                x[u] = src[automorph_src((u32)(row * 256 + 16 * lo + u), galois, a.log_n)];
         } else {
             const uint4 *s4 = reinterpret_cast<const uint4 *>(src + (size_t)row * 256 + 16 * lo);
 #pragma unroll

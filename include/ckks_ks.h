@@ -146,6 +146,21 @@ int ckks_relin(ckks_ctx *ctx, const uint32_t *d, int level, const ckks_evk *evk,
 int ckks_tensor(ckks_ctx *ctx, const uint32_t *x, const uint32_t *y, int level, uint32_t *d,
                 ckks_stream_t stream);
 
+/* Batches of independent operations at one level, executed by the same kernels as one launch
+ * per step (each launch covers all items, up to 64 at a time), which fills the GPU far better
+ * than one operation at a time.  Item z's operands are contiguous: c [n][l+1][N],
+ * ct/out [n][2][l+1][N], d [n][3][l+1][N], x, y [n][2][l+1][N]; keys and galois are host arrays
+ * of n entries (items may share a key).  Each item's result equals the corresponding single
+ * call bit for bit.  Workspace: ckks_workspace_bytes(ctx, level, n). */
+int ckks_keyswitch_batch(ckks_ctx *ctx, int n, const uint32_t *c, int level, const ckks_evk *keys,
+                         uint32_t *out, void *ws, size_t ws_bytes, ckks_stream_t stream);
+int ckks_rotate_batch(ckks_ctx *ctx, int n, const uint32_t *ct, int level, const uint32_t *galois,
+                      const ckks_evk *keys, uint32_t *out, void *ws, size_t ws_bytes, ckks_stream_t stream);
+int ckks_relin_batch(ckks_ctx *ctx, int n, const uint32_t *d, int level, const ckks_evk *keys, uint32_t *out,
+                     void *ws, size_t ws_bytes, ckks_stream_t stream);
+int ckks_tensor_batch(ckks_ctx *ctx, int n, const uint32_t *x, const uint32_t *y, int level, uint32_t *d,
+                      ckks_stream_t stream);
+
 /* The key's regenerated uniform half for one (digit, global limb): out [N] (device),
  * out[n] = w mod q_t with w = (x[2m] | x[2m+1] << 32), m = n mod 8, x = ChaCha12 block
  * (RFC 8439 state: key = seed as 8 LE words, counter = n/8, nonce = (key_id, digit, limb)). */
@@ -172,9 +187,9 @@ int ckks_chacha_expand(ckks_ctx *ctx, const uint8_t seed[32], uint32_t key_id, i
 int ckks_keyswitch_noalloc(ckks_ctx *ctx, const uint32_t *c, int level, const ckks_evk *evk,
                            uint32_t *out, ckks_stream_t stream);
 
-/* Workspace bytes for keyswitch/rotate/relin/modup/moddown at `level`
- * (n_rot > 1: rotate_hoisted with n_rot rotations). */
-size_t ckks_workspace_bytes(const ckks_ctx *ctx, int level, int n_rot);
+/* Workspace bytes for keyswitch/rotate/relin/modup/moddown at `level`; n > 1: a batch of n
+ * items, or rotate_hoisted with n rotations (batches run in chunks of 64, so n is capped at 64). */
+size_t ckks_workspace_bytes(const ckks_ctx *ctx, int level, int n);
 
 /* Waits for `stream` with a deadline (polling, no device-side wait): CKKS_OK when the
  * stream is idle and no CUDA error is pending, CKKS_ERR_TIMEOUT at the deadline,

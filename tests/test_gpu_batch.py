@@ -1,0 +1,103 @@
+"""Batched entry points: every item of a batch equals the single call (and so the oracle) bit for
+bit, including batches longer than one launch chunk and hoisted rotations spanning chunks."""
+import numpy as np
+import pytest
+
+import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+def _res(moduli, n, gen):
+    return torch.from_numpy(W.uniform_residues(moduli, n, gen)).cuda()
+
+
+def _setup(ks, key):
+    cfg = W.CONFIGS[key]
+    q, p = ks.ckks_gen_primes(cfg.log_n, cfg.n_q, cfg.n_p)
+    return cfg, q, p, ks.Context(cfg.log_n, q, p, cfg.dnum)
+
+
+@pytest.mark.parametrize("key,n", [("1", 5), ("2", 3), ("3", 2)])
+def test_batches_equal_single_calls(ks_lib, key, n):
+    ks = ks_lib
+    cfg, q, p, ctx = _setup(ks, key)
+    lvl, N = cfg.level, cfg.n
+    na = lvl + 1
+    gen = W.rng(cfg.seed, W.TAG_SYNTH, 900 + n)
+    nd = -(-cfg.n_q // cfg.alpha)
+    keys_t = [_res((q + p) * nd, N, gen).view(nd, len(q) + len(p), N) for _ in range(n)]
+    gs = [ks.galois_element(cfg.log_n, r) for r in (1, -1, 2, 3, -5, 7)[:n]]
+    evks = [ks.make_evk(keys_t[i], cfg.chacha_seed, gs[i]) for i in range(n)]
+    x = _res(q[:na] * 2 * n, N, gen).view(n, 2, na, N)
+    y = _res(q[:na] * 2 * n, N, gen).view(n, 2, na, N)
+    ws_b = ctx.workspace(lvl, n)
+    ws_1 = ctx.workspace(lvl)
+    # tensor
+    d = torch.empty((n, 3, na, N), dtype=torch.uint32, device="cuda")
+    ks.ckks_tensor_batch(ctx, n, x, y, lvl, d)
+    for i in range(n):
+        di = torch.empty((3, na, N), dtype=torch.uint32, device="cuda")
+        ks.ckks_tensor(ctx, x[i], y[i], lvl, di)
+        assert torch.equal(di, d[i])
+    # relin (items share one key), rotate, keyswitch
+    out = torch.empty((n, 2, na, N), dtype=torch.uint32, device="cuda")
+    one = torch.empty((2, na, N), dtype=torch.uint32, device="cuda")
+    ks.ckks_relin_batch(ctx, d, lvl, [evks[0]] * n, out, ws_b)
+    for i in range(n):
+        ks.ckks_relin(ctx, d[i], lvl, evks[0], one, ws_1)
+        assert torch.equal(one, out[i])
+    ks.ckks_rotate_batch(ctx, x, lvl, gs, evks, out, ws_b)
+    for i in range(n):
+        ks.ckks_rotate(ctx, x[i], lvl, gs[i], evks[i], one, ws_1)
+        assert torch.equal(one, out[i])
+    c = x[:, 1].contiguous()
+    ks.ckks_keyswitch_batch(ctx, c, lvl, evks, out, ws_b)
+    for i in range(n):
+        ks.ckks_keyswitch(ctx, c[i], lvl, evks[i], one, ws_1)
+        assert torch.equal(one, out[i])
+
+
+def test_rotate_batch_longer_than_a_chunk(ks_lib):
+    """70 rotations at N=2^12 (two launch chunks of at most 64 items)."""
+    ks = ks_lib
+    cfg, q, p, ctx = _setup(ks, "1b")
+    lvl, N, na, n = cfg.level, cfg.n, cfg.level + 1, 70
+    gen = W.rng(cfg.seed, W.TAG_SYNTH, 77)
+    nd = -(-cfg.n_q // cfg.alpha)
+    kt = _res((q + p) * nd, N, gen).view(nd, len(q) + len(p), N)
+    gs = [ks.galois_element(cfg.log_n, r) for r in range(1, n + 1)]
+    evks = [ks.make_evk(kt, cfg.chacha_seed, g) for g in gs]
+    ct = _res(q[:na] * 2 * n, N, gen).view(n, 2, na, N)
+    out = torch.empty((n, 2, na, N), dtype=torch.uint32, device="cuda")
+    ks.ckks_rotate_batch(ctx, ct, lvl, gs, evks, out, ctx.workspace(lvl, n))
+    one = torch.empty((2, na, N), dtype=torch.uint32, device="cuda")
+    ws1 = ctx.workspace(lvl)
+    for i in (0, 63, 64, 69):
+        ks.ckks_rotate(ctx, ct[i], lvl, gs[i], evks[i], one, ws1)
+        assert torch.equal(one, out[i])
+
+
+def test_hoisted_across_chunks_matches_oracle(ks_lib, oracle_mod):
+    """Hoisted rotations spanning two chunks equal the oracle (sampled rotations)."""
+    from oracle.scenario import Scenario
+    ks = ks_lib
+    cfg = W.CONFIGS["1b"]
+    sc = Scenario(cfg)
+    q, p = ks.ckks_gen_primes(cfg.log_n, cfg.n_q, cfg.n_p)
+    ctx = ks.Context(cfg.log_n, q, p, cfg.dnum)
+    lvl, n = cfg.level, 66
+    _, ct = sc.ciphertext(0)
+    steps = list(range(1, n + 1))
+    gs = [sc.galois(r) for r in steps]
+    keys_np = {g: sc.key(g) for g in gs}
+    keys_t = {g: torch.from_numpy(keys_np[g]).cuda() for g in gs}
+    evks = [ks.make_evk(keys_t[g], cfg.chacha_seed, g) for g in gs]
+    out = torch.empty((n, 2, lvl + 1, cfg.n), dtype=torch.uint32, device="cuda")
+    ks.ckks_rotate_hoisted(ctx, torch.from_numpy(ct).cuda(), lvl, gs, evks, out, ctx.workspace(lvl, n))
+    got = out.cpu().numpy()
+    for i in (0, 40, 64, 65):
+        want = sc.ctx.rotate(ct, lvl, cfg.alpha, gs[i], keys_np[gs[i]], cfg.chacha_seed, gs[i])
+        assert np.array_equal(got[i], want)
