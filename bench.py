@@ -48,6 +48,28 @@ def _env_int(name, default):
         return default
 
 
+def rank_env():
+    """(rank, world, local_rank) from the torchrun environment (1 process when absent)."""
+    return _env_int("RANK", 0), _env_int("WORLD_SIZE", 1), _env_int("LOCAL_RANK", 0)
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Max of a per-rank float over all ranks (the job's time is its slowest rank's)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: int, world: int, ms_max: float) -> float:
+    """Whole-job throughput: every rank processes its own units (weak scaling, replicas); the
+    job takes the slowest rank's time."""
+    return units_per_rank * world / (ms_max / 1e3)
+
+
 class ClockSampler:
     """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
 
@@ -166,13 +188,9 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     clk = clocks.stop()
     dom_launches, dom_ms = ks.ckks_prof_end(ctx)
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     ms_per_step = ms / args.steps
-    value = KS_PER_UNIT * B * args.steps * world / (ms / 1e3)
+    value = job_throughput(KS_PER_UNIT * B * args.steps, world, ms)
 
     # end to end: pinned host inputs copied in, result copied out, every step
     h_x = [s["x"].cpu().pin_memory() for s in sets]
@@ -199,12 +217,8 @@ def run_ours(args, rank, world, local_rank):
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    ms_e2e = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t.item())
-    e2e_value = KS_PER_UNIT * B * args.steps * world / (ms_e2e / 1e3)
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e_value = job_throughput(KS_PER_UNIT * B * args.steps, world, ms_e2e)
     h2d = (sets[0]["x"].numel() + sets[0]["y"].numel()) * 4
     d2h = out.numel() * 4
 
@@ -215,7 +229,7 @@ def run_ours(args, rank, world, local_rank):
             "metric": METRIC,
             "value": value,
             "unit": "key-switches/s",
-            "rotations_per_s": ROT_PER_UNIT * B * args.steps * world / (ms / 1e3),
+            "rotations_per_s": job_throughput(ROT_PER_UNIT * B * args.steps, world, ms),
             "n_gpus": world,
             "steps": args.steps,
             "warmup": args.warmup,
@@ -416,9 +430,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=8, help="independent config-3 units per step")
     args = ap.parse_args()
-    rank = _env_int("RANK", 0)
-    world = _env_int("WORLD_SIZE", 1)
-    local_rank = _env_int("LOCAL_RANK", 0)
+    rank, world, local_rank = rank_env()
     if args.impl == "reference":
         if args.steps > 3:
             args.steps = 3          # each oracle step is seconds of CPU work
