@@ -309,14 +309,16 @@ def roofline(cfg, launches, total_ms, clk, batch):
     peak = alu_peak_tops(SM_MAX_MHZ)
     return {"kernel": "k_ip_row (ModUp last NTT pass + ChaCha12 + key inner product)",
             "bound": "alu", "achieved": achieved, "peak": peak, "unit": "Tops (int32)",
-            "frac": achieved / peak, "traffic": IP_ROW_TRAFFIC, "launches": launches,
+            "frac": achieved / peak,
+            "traffic": None if IP_ROW_TRAFFIC_PER_UNIT is None else IP_ROW_TRAFFIC_PER_UNIT * batch,
+            "launches": launches,
             "avg_launch_us": avg_s * 1e6,
             "peak_source": f"derived: {N_SM} SMs x 128 int32 lanes x {SM_MAX_MHZ:.0f} MHz"}
 
 
-# DRAM bytes (read + write) of one k_ip_row launch from an ncu capture of the current kernel;
-# None when the kernel changed after the capture.
-IP_ROW_TRAFFIC = None
+# DRAM bytes (read + write) per unit of a k_ip_row launch, from an ncu capture of the current
+# kernel (scaled by the units a launch covers); None when the kernel changed after the capture.
+IP_ROW_TRAFFIC_PER_UNIT = 966.96e6 / 8   # bytes: ncu dram__bytes_read 782.29 MB + write 184.67 MB, one 8-unit launch
 
 
 def step_bytes_min(cfg) -> int:
