@@ -89,12 +89,13 @@ struct BconvArgs {
     int cfg_stride;          // words per config in bmat = max_in * n_primes
     int g_base;              // logical group of blockIdx.y = 0 (a launch may cover a subset)
     int nchunk;              // target chunks per item: blockIdx.z = item * nchunk + chunk
+    int tchunk;              // targets per chunk (a multiple of 4)
     size_t y_item, out_item; // item strides (words)
 };
 
 constexpr int BCONV_THREADS = 256;
 constexpr int BCONV_MAX_IN = 64;
-constexpr int BCONV_TCHUNK = 12;      // targets per block (blockIdx.z splits the target list)
+constexpr int BCONV_TCHUNK = 12;      // targets per block for small launches (see BconvArgs::tchunk)
 
 // MAXIN: compile-time bound on the group's input count (inputs live in registers).
 // Each thread converts 2 consecutive coefficients.
@@ -138,8 +139,8 @@ k_bconv(BconvArgs a) {
     }
     const int lo = a.map.skip_alpha > 0 ? g * a.map.skip_alpha : 0;
     const int hi = a.map.skip_alpha > 0 ? min(lo + a.map.skip_alpha, a.map.split) : 0;
-    const int k_end = min(T, (chunk + 1) * BCONV_TCHUNK);
-    for (int kk = chunk * BCONV_TCHUNK; kk < k_end; kk++) {
+    const int k_end = min(T, (chunk + 1) * a.tchunk);
+    for (int kk = chunk * a.tchunk; kk < k_end; kk++) {
         if (kk >= lo && kk < hi) continue;
         const int t = kk < a.map.split ? a.map.lo_base + kk : a.map.hi_base + (kk - a.map.split);
         const PrimeInfo pi = a.pinfo[t];
@@ -208,8 +209,8 @@ k_bconv_n(BconvArgs a) {
     y0[NIN] = v0; y1[NIN] = v1;
     const int lo = a.map.skip_alpha > 0 ? g * a.map.skip_alpha : 0;
     const int hi = a.map.skip_alpha > 0 ? min(lo + a.map.skip_alpha, a.map.split) : 0;
-    const int k_beg = chunk * BCONV_TCHUNK;
-    const int k_end = min(T, k_beg + BCONV_TCHUNK);
+    const int k_beg = chunk * a.tchunk;
+    const int k_end = min(T, k_beg + a.tchunk);
     for (int k4 = k_beg; k4 < k_end; k4 += 4) {
         u64 s0[4], s1[4];
 #pragma unroll
