@@ -148,9 +148,14 @@ def run_ours(args, rank, world, local_rank):
         y = residues(q[:na] * 2 * B, 10 * s + 2).view(B, 2, na, n)
         b_rel = residues(mods * nd * B, 10 * s + 3).view(B, nd, len(mods), n)
         b_rot = residues(mods * nd * B, 10 * s + 4).view(B, nd, len(mods), n)
-        sets.append(dict(x=x, y=y, b_rel=b_rel, b_rot=b_rot,
-                         k_rel=[ks.make_evk(b_rel[i], cfg.chacha_seed, 0) for i in range(B)],
-                         k_rot=[ks.make_evk(b_rot[i], cfg.chacha_seed, g) for i in range(B)]))
+        # --stored-a (ablation): the keys carry a stored a half read from HBM instead of ChaCha12
+        a_rel = residues(mods * nd * B, 10 * s + 5).view(B, nd, len(mods), n) if args.stored_a else None
+        a_rot = residues(mods * nd * B, 10 * s + 6).view(B, nd, len(mods), n) if args.stored_a else None
+        sets.append(dict(x=x, y=y, b_rel=b_rel, b_rot=b_rot, a_rel=a_rel, a_rot=a_rot,
+                         k_rel=[ks.make_evk(b_rel[i], cfg.chacha_seed, 0,
+                                            a=a_rel[i] if args.stored_a else None) for i in range(B)],
+                         k_rot=[ks.make_evk(b_rot[i], cfg.chacha_seed, g,
+                                            a=a_rot[i] if args.stored_a else None) for i in range(B)]))
     d = torch.empty((B, 3, na, n), dtype=torch.uint32, device=dev)
     r = torch.empty((B, 2, na, n), dtype=torch.uint32, device=dev)
     out = torch.empty((B, 2, na, n), dtype=torch.uint32, device=dev)
@@ -244,6 +249,7 @@ def run_ours(args, rank, world, local_rank):
                                    "rotate(1) with its own keys",
                        "log_n": cfg.log_n, "n_q": cfg.n_q, "n_p": cfg.n_p, "dnum": cfg.dnum,
                        "level": lvl, "batch": B, "key_switches_per_step": KS_PER_UNIT * B,
+                       "key_a_half": "stored (ablation)" if args.stored_a else "regenerated by ChaCha12",
                        "l2": f"{N_SETS} rotating input/key sets (each > 126 MB L2)",
                        "parallelism": f"replicas x{world}"},
             "e2e": {"value": e2e_value, "unit": "key-switches/s", "h2d_bytes_per_step": h2d,
@@ -335,6 +341,86 @@ def step_bytes_min(cfg) -> int:
 # kernels launched by one step: tensor (1) + 2 key switches x 10 (ModUp 4, inner product with
 # the last ModUp and first ModDown NTT passes 2, ModDown 4 including the fused combine)
 LAUNCHES_PER_STEP = 1 + 2 * 10
+
+
+def run_workload(args, local_rank):
+    """Informational throughput of configs 4 and 5 (not the benchmark's headline line):
+    config 4 = 32 hoisted rotations of one ciphertext at level 24 (one ModUp, 32 keys);
+    config 5 = 64 pairs, each tensor + relin + rotate by 2^(i mod 15), level 20, dnum 4
+    (one relinearisation key, 15 rotation keys, all as batched calls)."""
+    import torch
+    import fhe_key_switching_b200 as ks
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    key = str(args.workload)
+    cfg = W.CONFIGS[key]
+    n, lvl = cfg.n, cfg.level
+    na = lvl + 1
+    q, p = ks.ckks_gen_primes(cfg.log_n, cfg.n_q, cfg.n_p)
+    ctx = ks.Context(cfg.log_n, q, p, cfg.dnum)
+    nd = -(-cfg.n_q // cfg.alpha)
+    mods = q + p
+    gen = W.rng(cfg.seed, W.TAG_SYNTH, 7)
+
+    def res(moduli):
+        return torch.from_numpy(W.uniform_residues(moduli, n, gen)).to(dev)
+
+    steps_g = sorted(set(cfg.rot_steps), key=cfg.rot_steps.index)
+    gal = {r: ks.galois_element(cfg.log_n, r) for r in steps_g}
+    keys_t = {r: res(mods * nd).view(nd, len(mods), n) for r in steps_g}
+    evk = {r: ks.make_evk(keys_t[r], cfg.chacha_seed, gal[r]) for r in steps_g}
+    stream = torch.cuda.current_stream(dev)
+    if key == "4":
+        cts = [res(q[:na] * 2).view(2, na, n) for _ in range(N_SETS)]
+        R = len(cfg.rot_steps)
+        gs = [gal[r] for r in cfg.rot_steps]
+        ev = [evk[r] for r in cfg.rot_steps]
+        out = torch.empty((R, 2, na, n), dtype=torch.uint32, device=dev)
+        ws = ctx.workspace(lvl, R, device=dev)
+
+        def step(i):
+            ks.ckks_rotate_hoisted(ctx, cts[i % N_SETS], lvl, gs, ev, out, ws, stream)
+        ks_per_step, rot_per_step = R, R
+    elif key == "5":
+        P_ = cfg.n_pairs
+        xs = [res(q[:na] * 2 * P_).view(P_, 2, na, n) for _ in range(2)]
+        ys = [res(q[:na] * 2 * P_).view(P_, 2, na, n) for _ in range(2)]
+        b_rel = res(mods * nd).view(nd, len(mods), n)
+        k_rel = ks.make_evk(b_rel, cfg.chacha_seed, 0)
+        d = torch.empty((P_, 3, na, n), dtype=torch.uint32, device=dev)
+        r1 = torch.empty((P_, 2, na, n), dtype=torch.uint32, device=dev)
+        out = torch.empty((P_, 2, na, n), dtype=torch.uint32, device=dev)
+        ws = ctx.workspace(lvl, P_, device=dev)
+        gs = [gal[r] for r in cfg.rot_steps]
+        ev = [evk[r] for r in cfg.rot_steps]
+
+        def step(i):
+            ks.ckks_tensor_batch(ctx, P_, xs[i % 2], ys[i % 2], lvl, d, stream)
+            ks.ckks_relin_batch(ctx, d, lvl, [k_rel] * P_, r1, ws, stream)
+            ks.ckks_rotate_batch(ctx, r1, lvl, gs, ev, out, ws, stream)
+        ks_per_step, rot_per_step = 2 * P_, P_
+    else:
+        raise SystemExit(f"--workload {key}: use 3 (default), 4 or 5")
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    print(json.dumps({"workload": f"config {key}", "informational": True,
+                      "key_switches_per_s": ks_per_step * args.steps / (ms / 1e3),
+                      "rotations_per_s": rot_per_step * args.steps / (ms / 1e3),
+                      "ms_per_step": ms / args.steps, "steps": args.steps, "warmup": args.warmup,
+                      "key_switches_per_step": ks_per_step, "clocks": clk}), flush=True)
 
 
 def _oracle_sample():
@@ -431,6 +517,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=8, help="independent config-3 units per step")
+    ap.add_argument("--workload", default="3", help="3 (benchmark line), or 4 / 5 (informational)")
+    ap.add_argument("--stored-a", action="store_true",
+                    help="ablation: keys with a stored a half (read from HBM) instead of ChaCha12")
     args = ap.parse_args()
     rank, world, local_rank = rank_env()
     if args.impl == "reference":
@@ -438,6 +527,9 @@ def main():
             args.steps = 3          # each oracle step is seconds of CPU work
         args.warmup = min(args.warmup, 1)
         run_reference(args, rank, world)
+        return
+    if str(args.workload) != "3":
+        run_workload(args, local_rank)
         return
     run_ours(args, rank, world, local_rank)
 
