@@ -164,13 +164,22 @@ k_bconv(BconvArgs a) {
     }
 }
 
-// Exact-count variant: NIN inputs known at compile time; each thread converts 2 consecutive
-// coefficients for 4 targets at a time (8 independent 64-bit sums).  Constants are staged as
-// [NIN + 1][T4] with T4 = T rounded up to 4 (row NIN holds [-D]_t, multiplied by the count v
-// of negative representatives), so one 128-bit shared load gives 4 targets' constants.
+// Exact-count variant: NIN inputs known at compile time; each thread converts BCONV_CPT = 4
+// consecutive coefficients for 4 targets at a time (16 independent 64-bit sums).  Staged in
+// shared memory: the constants as [NIN + 1][T4] words with T4 = T rounded up to 4 (row NIN
+// holds [-D]_t, multiplied by the count v of negative representatives), so one 128-bit load
+// gives 4 targets' constants, then each target's (t, [2^32]_t, its Shoup companion,
+// floor(2^32/t)) as one 128-bit record.
+// Output is lazily reduced, in [0, 4t): every consumer is a forward NTT, whose butterflies take
+// inputs in [0, 4t) and whose output is canonical.
+constexpr int BCONV_CPT = 4;
+
+__host__ __device__ constexpr size_t bconv_n_smem_words(int nin, int t4) { return (size_t)(nin + 5) * t4; }
+
 template <int NIN>
 __global__ void __launch_bounds__(BCONV_THREADS)
 k_bconv_n(BconvArgs a) {
+    constexpr int CPT = BCONV_CPT;
     extern __shared__ __align__(16) u32 smc[];
     const int g = a.g_base + blockIdx.y;
     const int item = blockIdx.z / a.nchunk, chunk = blockIdx.z % a.nchunk;
@@ -193,47 +202,60 @@ k_bconv_n(BconvArgs a) {
         }
         smc[idx] = val;
     }
+    uint4 *sq = reinterpret_cast<uint4 *>(smc + (NIN + 1) * T4);
+    for (int kk = threadIdx.x; kk < T4; kk += blockDim.x) {
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (kk < T) {
+            const int t = kk < a.map.split ? a.map.lo_base + kk : a.map.hi_base + (kk - a.map.split);
+            const PrimeInfo pi = a.pinfo[t];
+            v = make_uint4(pi.q, pi.r64, pi.r64p, pi.onep);
+        }
+        sq[kk] = v;
+    }
     __syncthreads();
-    const int c2 = blockIdx.x * blockDim.x + threadIdx.x;   // coefficient pair
-    if (2 * c2 >= n) return;
-    u32 y0[NIN + 1], y1[NIN + 1];
-    u32 v0 = 0, v1 = 0;
+    const int cv = blockIdx.x * blockDim.x + threadIdx.x;   // coefficients CPT cv .. CPT cv + 3
+    if (CPT * cv >= n) return;
+    u32 y[CPT][NIN + 1];
+    u32 v[CPT] = {0, 0, 0, 0};
 #pragma unroll
     for (int i = 0; i < NIN; i++) {
-        const uint2 t = reinterpret_cast<const uint2 *>(yb + (size_t)(row0 + i) * n)[c2];
         const u32 h = a.pinfo[p0 + i].half;
-        y0[i] = t.x; y1[i] = t.y;
-        v0 += t.x > h ? 1u : 0u;
-        v1 += t.y > h ? 1u : 0u;
+        const uint4 w = reinterpret_cast<const uint4 *>(yb + (size_t)(row0 + i) * n)[cv];
+        const u32 t[CPT] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int c = 0; c < CPT; c++) { y[c][i] = t[c]; v[c] += t[c] > h ? 1u : 0u; }
     }
-    y0[NIN] = v0; y1[NIN] = v1;
+#pragma unroll
+    for (int c = 0; c < CPT; c++) y[c][NIN] = v[c];
     const int lo = a.map.skip_alpha > 0 ? g * a.map.skip_alpha : 0;
     const int hi = a.map.skip_alpha > 0 ? min(lo + a.map.skip_alpha, a.map.split) : 0;
     const int k_beg = chunk * a.tchunk;
     const int k_end = min(T, k_beg + a.tchunk);
     for (int k4 = k_beg; k4 < k_end; k4 += 4) {
-        u64 s0[4], s1[4];
+        u64 s[CPT][4];
 #pragma unroll
-        for (int m = 0; m < 4; m++) s0[m] = s1[m] = 0;
+        for (int c = 0; c < CPT; c++)
+#pragma unroll
+            for (int m = 0; m < 4; m++) s[c][m] = 0;
 #pragma unroll
         for (int i = 0; i <= NIN; i++) {
             const uint4 b4 = *reinterpret_cast<const uint4 *>(smc + i * T4 + k4);
             const u32 bb[4] = {b4.x, b4.y, b4.z, b4.w};
 #pragma unroll
-            for (int m = 0; m < 4; m++) {
-                s0[m] += (u64)y0[i] * bb[m];
-                s1[m] += (u64)y1[i] * bb[m];
-            }
+            for (int m = 0; m < 4; m++)
+#pragma unroll
+                for (int c = 0; c < CPT; c++) s[c][m] += (u64)y[c][i] * bb[m];
         }
 #pragma unroll
         for (int m = 0; m < 4; m++) {
             const int kk = k4 + m;
             if (kk >= k_end || (kk >= lo && kk < hi)) continue;
-            const int t = kk < a.map.split ? a.map.lo_base + kk : a.map.hi_base + (kk - a.map.split);
-            const PrimeInfo pi = a.pinfo[t];
-            const uint2 r = make_uint2(reduce64(s0[m], pi.q, pi.r64, pi.r64p, pi.onep),
-                                       reduce64(s1[m], pi.q, pi.r64, pi.r64p, pi.onep));
-            reinterpret_cast<uint2 *>(ob + ((size_t)g * a.map.out_group_rows + a.map.out_k_base + kk) * n)[c2] = r;
+            const uint4 pq = sq[kk];
+            u32 r[CPT];
+#pragma unroll
+            for (int c = 0; c < CPT; c++) r[c] = reduce64_lazy(s[c][m], pq.x, pq.y, pq.z, pq.w);
+            u32 *dst = ob + ((size_t)g * a.map.out_group_rows + a.map.out_k_base + kk) * n;
+            reinterpret_cast<uint4 *>(dst)[cv] = make_uint4(r[0], r[1], r[2], r[3]);
         }
     }
 }
