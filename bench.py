@@ -159,45 +159,90 @@ def run_ours(args, rank, world, local_rank):
     d = torch.empty((B, 3, na, n), dtype=torch.uint32, device=dev)
     r = torch.empty((B, 2, na, n), dtype=torch.uint32, device=dev)
     out = torch.empty((B, 2, na, n), dtype=torch.uint32, device=dev)
-    ws = ctx.workspace(lvl, B, device=dev)
-    stream = torch.cuda.current_stream(dev)
-    gal = [g] * B
+    # the batch runs as S sub-batches of B/S units, one per CUDA stream, so that one sub-batch's
+    # ALU-bound kernels overlap another's memory-bound ones
+    S = args.streams if args.streams is not None else (2 if B % 2 == 0 else 1)
+    if S < 1 or B % S:
+        raise SystemExit(f"--streams {S} must divide --batch {B}")
+    Bs = B // S
+    main = torch.cuda.current_stream(dev)
+    streams = [main] + [torch.cuda.Stream(dev) for _ in range(S - 1)]
+    wss = [ctx.workspace(lvl, Bs, device=dev) for _ in range(S)]
+    gal = [g] * Bs
 
-    def step(i):
+    def sub(si):
+        return slice(si * Bs, (si + 1) * Bs)
+
+    def step_on(si, st, x, y, stream):
+        z = sub(si)
+        ks.ckks_tensor_batch(ctx, Bs, x[z], y[z], lvl, d[z], stream)
+        ks.ckks_relin_batch(ctx, d[z], lvl, st["k_rel"][z], r[z], wss[si], stream)
+        ks.ckks_rotate_batch(ctx, r[z], lvl, gal, st["k_rot"][z], out[z], wss[si], stream)
+
+    def step(i, n_streams=S):
         st = sets[i % N_SETS]
-        ks.ckks_tensor_batch(ctx, B, st["x"], st["y"], lvl, d, stream)
-        ks.ckks_relin_batch(ctx, d, lvl, st["k_rel"], r, ws, stream)
-        ks.ckks_rotate_batch(ctx, r, lvl, gal, st["k_rot"], out, ws, stream)
+        if n_streams == 1:          # the same work, every sub-batch on the main stream in turn
+            for si in range(S):
+                step_on(si, st, st["x"], st["y"], main)
+            return
+        for si in range(S):
+            step_on(si, st, st["x"], st["y"], streams[si])
+
+    def fork():
+        ev = torch.cuda.Event()
+        ev.record(main)
+        for s_ in streams[1:]:
+            s_.wait_event(ev)
+
+    def join():
+        for s_ in streams[1:]:
+            ev = torch.cuda.Event()
+            ev.record(s_)
+            main.wait_event(ev)
 
     def barrier():
         if world > 1:
             dist.barrier()
 
+    def timed(fn, steps):
+        """Device time of `steps` calls of fn (ms, max over ranks), events on the main stream."""
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(main)
+        fork()
+        for i in range(steps):
+            fn(i)
+        join()
+        e1.record(main)
+        torch.cuda.synchronize()
+        barrier()
+        return max_over_ranks(e0.elapsed_time(e1), world, dev)
+
+    fork()
     for i in range(args.warmup):
         step(i)
+    join()
     torch.cuda.synchronize()
     barrier()
     clocks = ClockSampler(local_rank)
     clocks.start()
     time.sleep(0.3)
-    torch.cuda.synchronize()
-    barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    # the dominant kernel's launches are bracketed by events on the launching stream
-    ks.ckks_prof_begin(ctx, DOMINANT, KS_PER_UNIT * args.steps)
-    e0.record(stream)
-    for i in range(args.steps):
-        step(i)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    clk = clocks.stop()
+    # the dominant kernel's launches inside the timed region (overlapped with the other streams)
+    ks.ckks_prof_begin(ctx, DOMINANT, KS_PER_UNIT * S * args.steps)
+    ms = timed(step, args.steps)
+    dom_launches_ov, dom_ms_ov = ks.ckks_prof_end(ctx)
+    # the dominant kernel alone: the same steps with every launch on the main stream, so that
+    # each launch's events bracket that kernel only
+    ks.ckks_prof_begin(ctx, DOMINANT, KS_PER_UNIT * S * args.steps)
+    ms_single = timed(lambda i: step(i, 1), args.steps)
     dom_launches, dom_ms = ks.ckks_prof_end(ctx)
-    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    clk = clocks.stop()
     ms_per_step = ms / args.steps
     value = job_throughput(KS_PER_UNIT * B * args.steps, world, ms)
 
-    # end to end: pinned host inputs copied in, result copied out, every step
+    # end to end: pinned host inputs copied in, result copied out, every step; each stream
+    # copies its own sub-batch
     h_x = [s["x"].cpu().pin_memory() for s in sets]
     h_y = [s["y"].cpu().pin_memory() for s in sets]
     h_out = torch.empty((B, 2, na, n), dtype=torch.uint32).pin_memory()
@@ -205,24 +250,20 @@ def run_ours(args, rank, world, local_rank):
 
     def step_e2e(i):
         st = sets[i % N_SETS]
-        dx.copy_(h_x[i % N_SETS], non_blocking=True)
-        dy.copy_(h_y[i % N_SETS], non_blocking=True)
-        ks.ckks_tensor_batch(ctx, B, dx, dy, lvl, d, stream)
-        ks.ckks_relin_batch(ctx, d, lvl, st["k_rel"], r, ws, stream)
-        ks.ckks_rotate_batch(ctx, r, lvl, gal, st["k_rot"], out, ws, stream)
-        h_out.copy_(out, non_blocking=True)
+        for si in range(S):
+            z = sub(si)
+            with torch.cuda.stream(streams[si]):
+                dx[z].copy_(h_x[i % N_SETS][z], non_blocking=True)
+                dy[z].copy_(h_y[i % N_SETS][z], non_blocking=True)
+            step_on(si, st, dx, dy, streams[si])
+            with torch.cuda.stream(streams[si]):
+                h_out[z].copy_(out[z], non_blocking=True)
 
+    fork()
     for i in range(args.warmup):
         step_e2e(i)
-    torch.cuda.synchronize()
-    barrier()
-    e0.record(stream)
-    for i in range(args.steps):
-        step_e2e(i)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    ms_e2e = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    join()
+    ms_e2e = timed(step_e2e, args.steps)
     e2e_value = job_throughput(KS_PER_UNIT * B * args.steps, world, ms_e2e)
     h2d = (sets[0]["x"].numel() + sets[0]["y"].numel()) * 4
     d2h = out.numel() * 4
@@ -247,6 +288,7 @@ def run_ours(args, rank, world, local_rank):
             "config": {"workload": "config 3: N=2^16, 36+12 primes < 2^30, dnum 3, level 35; "
                                    f"step = batch of {B} independent units, each tensor + relin + "
                                    "rotate(1) with its own keys",
+                       "streams": f"{S} CUDA streams x {Bs} units",
                        "log_n": cfg.log_n, "n_q": cfg.n_q, "n_p": cfg.n_p, "dnum": cfg.dnum,
                        "level": lvl, "batch": B, "key_switches_per_step": KS_PER_UNIT * B,
                        "key_a_half": "stored (ablation)" if args.stored_a else "regenerated by ChaCha12",
@@ -254,10 +296,11 @@ def run_ours(args, rank, world, local_rank):
                        "parallelism": f"replicas x{world}"},
             "e2e": {"value": e2e_value, "unit": "key-switches/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            "gpu_launches": args.steps * LAUNCHES_PER_STEP,
+            "gpu_launches": args.steps * LAUNCHES_PER_STEP * S,
             "kernel_launches_note": "one launch per kernel covers the whole batch",
             "clocks": clk,
-            "roofline": roofline(cfg, dom_launches, dom_ms, clk, B),
+            "roofline": roofline(cfg, dom_launches, dom_ms, clk, Bs, ms_single / args.steps,
+                                 dom_launches_ov, dom_ms_ov),
             "hbm_fraction_step": {"b_min_bytes_per_step": B * step_bytes_min(cfg),
                                   "frac": B * step_bytes_min(cfg) / (ms_per_step / 1e3) / (HBM_PEAK_GBS * 1e9),
                                   "peak_gbs": HBM_PEAK_GBS, "peak_source": PEAK_SOURCE},
@@ -307,24 +350,37 @@ def ip_row_ops(cfg) -> float:
     return chacha + a_red + ntt + macs
 
 
-def roofline(cfg, launches, total_ms, clk, batch):
+def roofline(cfg, launches, total_ms, clk, batch, single_step_ms, launches_ov, total_ms_ov):
+    """The dominant kernel against the int32 ALU issue peak.  `launches`/`total_ms`: its launches
+    in a single-stream pass of the timed steps (each launch's events bracket that kernel only);
+    `launches_ov`/`total_ms_ov`: the same kernel inside the timed multi-stream region, where its
+    events also span the other streams' concurrent kernels."""
     if not launches:
         return None
     avg_s = total_ms / launches / 1e3
     achieved = batch * ip_row_ops(cfg) / avg_s / 1e12
     peak = alu_peak_tops(SM_MAX_MHZ)
-    return {"kernel": "k_ip_row (ModUp last NTT pass + ChaCha12 + key inner product)",
-            "bound": "alu", "achieved": achieved, "peak": peak, "unit": "Tops (int32)",
-            "frac": achieved / peak,
-            "traffic": None if IP_ROW_TRAFFIC_PER_UNIT is None else IP_ROW_TRAFFIC_PER_UNIT * batch,
-            "launches": launches,
-            "avg_launch_us": avg_s * 1e6,
-            "peak_source": f"derived: {N_SM} SMs x 128 int32 lanes x {SM_MAX_MHZ:.0f} MHz"}
+    out = {"kernel": "k_ip_row (ModUp last NTT pass + ChaCha12 + key inner product)",
+           "bound": "alu", "achieved": achieved, "peak": peak, "unit": "Tops (int32)",
+           "frac": achieved / peak,
+           "traffic": None if IP_ROW_TRAFFIC_PER_UNIT is None else IP_ROW_TRAFFIC_PER_UNIT * batch,
+           "units_per_launch": batch,
+           "launches": launches,
+           "avg_launch_us": avg_s * 1e6,
+           "timed_in": "single-stream pass of the timed steps, right after the timed region "
+                       f"({single_step_ms:.3f} ms per step)",
+           "peak_source": f"derived: {N_SM} SMs x 128 int32 lanes x {SM_MAX_MHZ:.0f} MHz"}
+    if launches_ov:
+        out["in_timed_region"] = {"launches": launches_ov,
+                                  "avg_launch_us": total_ms_ov / launches_ov * 1e3,
+                                  "note": "overlapped with the other streams' kernels"}
+    return out
 
 
-# DRAM bytes (read + write) per unit of a k_ip_row launch, from an ncu capture of the current
-# kernel (scaled by the units a launch covers); None when the kernel changed after the capture.
-IP_ROW_TRAFFIC_PER_UNIT = 966.96e6 / 8   # bytes: ncu dram__bytes_read 782.29 MB + write 184.67 MB, one 8-unit launch
+# DRAM bytes (read + write) per unit of a k_ip_row launch, from an ncu launch list of this
+# benchmark (4-unit launches; mean of 20: dram__bytes_read 392.07 MB + write 79.28 MB), scaled
+# by the units a launch covers; None when the kernel changed after the capture.
+IP_ROW_TRAFFIC_PER_UNIT = 471.35e6 / 4
 
 
 def step_bytes_min(cfg) -> int:
@@ -518,6 +574,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=8, help="independent config-3 units per step")
     ap.add_argument("--workload", default="3", help="3 (benchmark line), or 4 / 5 (informational)")
+    ap.add_argument("--streams", type=int, default=None,
+                    help="CUDA streams the batch is split over, each running batch/streams units "
+                         "(default 2 for an even batch, else 1)")
     ap.add_argument("--stored-a", action="store_true",
                     help="ablation: keys with a stored a half (read from HBM) instead of ChaCha12")
     args = ap.parse_args()
