@@ -61,6 +61,7 @@ def lib():
                                          ctypes.POINTER(u32p), u8p, u32p, u32p]),
             "or_relin": (None, [vp, u32p, ci, ci, u32p, u32p, u8p, cu, u32p]),
             "or_tensor": (None, [vp, u32p, u32p, ci, u32p]),
+            "or_rescale": (None, [vp, u32p, ci, ci, u32p]),
             "or_signed_to_eval": (None, [vp, i64p, ci, u32p]),
             "or_keygen": (None, [vp, ci, i64p, u32p, i64p, u8p, cu, u32p, u32p]),
             "or_encrypt": (None, [vp, i64p, i64p, i64p, u32p, ci, u32p]),
@@ -264,6 +265,16 @@ class Ctx:
         sp, _keep = _u8(seed)
         ap = _u32(np.ascontiguousarray(a_stored, dtype=np.uint32)) if a_stored is not None else None
         lib().or_relin(self._h, _u32(d), level, alpha, _u32(b), ap, sp, key_id, _u32(out))
+        return out
+
+    def rescale(self, ct, level):
+        """Rescale by q_level: [n_comp][level+1][N] -> [n_comp][level][N] (evaluation domain)."""
+        ct = np.ascontiguousarray(ct, dtype=np.uint32)
+        if ct.ndim == 2:
+            ct = ct[None]
+        assert level >= 1 and ct.shape[1:] == (level + 1, self.n)
+        out = np.empty((ct.shape[0], level, self.n), dtype=np.uint32)
+        lib().or_rescale(self._h, _u32(ct), ct.shape[0], level, _u32(out))
         return out
 
     def tensor(self, x, y, level):

@@ -538,6 +538,41 @@ void or_tensor(const or_ctx *c, const u32 *x, const u32 *y, int level, u32 *d) {
     }
 }
 
+/* Rescaling by the last active prime (full-RNS CKKS, Cheon, Han, Kim, Kim, Song, SAC 2018,
+ * the RNS rescale: the pages name no rescale of their own).  For each component, with C the
+ * integer polynomial whose residues are the component's limbs 0..l:
+ *   out = (C - [C]_{q_l}) / q_l   reduced modulo q_0 .. q_{l-1},
+ * where [C]_{q_l} is the centred residue of C modulo q_l, in (-q_l/2, q_l/2] (the same
+ * centred lift the base conversion uses).  The division is exact, so per limb
+ *   out_i = (c_i - [C]_{q_l} mod q_i) * q_l^-1  (mod q_i).
+ * [C]_{q_l} is a coefficient-domain quantity: limb l is brought to coefficients by the inverse
+ * NTT, lifted, reduced modulo q_i and brought back by the forward NTT of prime q_i.
+ * ct: [n_comp][l+1][N] (evaluation domain); out: [n_comp][l][N].  level >= 1. */
+void or_rescale(const or_ctx *c, const u32 *ct, int n_comp, int level, u32 *out) {
+    int n = c->n, na = level + 1;
+    u64 ql = c->mod[level];
+    u32 *last = (u32 *)malloc(sizeof(u32) * (size_t)n);
+    for (int comp = 0; comp < n_comp; comp++) {
+        const u32 *cc = ct + (size_t)comp * na * n;
+        memcpy(last, cc + (size_t)level * n, sizeof(u32) * (size_t)n);
+        or_ntt_inv_limb(c, level, last);
+#pragma omp parallel for
+        for (int i = 0; i < level; i++) {
+            u64 q = c->mod[i];
+            u64 ql_inv = invmod(ql % q, q);
+            u32 *o = out + ((size_t)comp * level + i) * n;
+            for (int m = 0; m < n; m++) {
+                i64 v = last[m] > (ql - 1) / 2 ? (i64)last[m] - (i64)ql : (i64)last[m];
+                o[m] = (u32)smod(v, q);
+            }
+            or_ntt_fwd_limb(c, i, o);
+            const u32 *ci = cc + (size_t)i * n;
+            for (int m = 0; m < n; m++) o[m] = (u32)mulmod((ci[m] + q - o[m]) % q, ql_inv, q);
+        }
+    }
+    free(last);
+}
+
 /* ------------------------------------------------------------------ keys, encryption
  * Signed coefficient vector -> evaluation-domain limb t. */
 void or_signed_to_eval(const or_ctx *c, const i64 *v, int t, u32 *out) {
