@@ -59,6 +59,8 @@ _SIGS = {
     "ckks_relin_batch": (_ci, [_vp, _ci, _vp, _ci, ctypes.POINTER(ckks_evk), _vp, _vp, _sz, _vp]),
     "ckks_tensor_batch": (_ci, [_vp, _ci, _vp, _vp, _ci, _vp, _vp]),
     "ckks_tensor": (_ci, [_vp, _vp, _vp, _ci, _vp, _vp]),
+    "ckks_rescale": (_ci, [_vp, _vp, _ci, _vp, _vp, _sz, _vp]),
+    "ckks_rescale_batch": (_ci, [_vp, _ci, _vp, _ci, _vp, _vp, _sz, _vp]),
     "ckks_chacha_expand": (_ci, [_vp, ctypes.POINTER(ctypes.c_uint8), _cu, _ci, _ci, _vp, _vp]),
     "ckks_workspace_bytes": (_sz, [_vp, _ci, _ci]),
     "ckks_sync_status": (_ci, [_vp, _vp, _ci]),
@@ -269,6 +271,18 @@ def ckks_tensor_batch(ctx, n: int, x, y, level: int, d, stream=None):
            "ckks_tensor_batch")
 
 
+def ckks_rescale(ctx, ct, level: int, out, ws, stream=None):
+    """Rescale by q_level: ct [2][l+1][N] -> out [2][l][N]."""
+    _check(_L.ckks_rescale(ctx.handle, _ptr(ct), level, _ptr(out), _ptr(ws), ws.numel() * ws.element_size(),
+                           _stream(stream)), "ckks_rescale")
+
+
+def ckks_rescale_batch(ctx, n: int, ct, level: int, out, ws, stream=None):
+    """Batch of rescales: ct [n][2][l+1][N] -> out [n][2][l][N]."""
+    _check(_L.ckks_rescale_batch(ctx.handle, n, _ptr(ct), level, _ptr(out), _ptr(ws),
+                                 ws.numel() * ws.element_size(), _stream(stream)), "ckks_rescale_batch")
+
+
 def ckks_chacha_expand(ctx, seed: bytes, key_id: int, digit: int, limb: int, out, stream=None):
     sb = (ctypes.c_uint8 * 32).from_buffer_copy(seed)
     _check(_L.ckks_chacha_expand(ctx.handle, sb, key_id, digit, limb, _ptr(out), _stream(stream)),
@@ -295,3 +309,9 @@ def galois_element(log_n: int, r: int) -> int:
     """Galois element of a rotation by r slots: 5^r mod 2N (r < 0: 5^(N/2+r))."""
     n = 1 << log_n
     return pow(5, r % (n // 2), 2 * n)
+
+
+def conjugation_element(log_n: int) -> int:
+    """Galois element of complex conjugation of the slots: 2N - 1 (X -> X^-1); its key has
+    key_id 2N - 1 and it runs through ckks_rotate like any rotation."""
+    return (2 << log_n) - 1

@@ -138,6 +138,10 @@ struct NttArgs {
     JobMap map;
     int log_n;
     size_t in_item, out_item;
+    // forward column pass only, lift_q != 0: every job of group g reads the group's single
+    // input row (in_group_rows * g + in_k_base), a canonical residue y mod lift_q, and
+    // transforms its centred lift (y - lift_q if y > lift_half) reduced mod the job's prime
+    u32 lift_q, lift_half;
     u32 galois[KS_MAXB];    // inverse row pass: gather item z's input through kappa_g (0 = none)
 };
 
@@ -170,12 +174,17 @@ k_ntt_col(NttArgs a) {
     const int lo = warp / cgroups;
     const int ccol = (warp % cgroups) * 32 + lane;          // column within block
     const int col = blockIdx.x * C::CPB + ccol;
-    const u32 *src = a.in + blockIdx.z * a.in_item + in_row * n;
+    const u32 *src = a.in + blockIdx.z * a.in_item + (FWD && a.lift_q ? in_row - k : in_row) * n;
     u32 *dst = a.out + blockIdx.z * a.out_item + out_row * n;
     u32 x[16];
     if (FWD) {
 #pragma unroll
         for (int u = 0; u < 16; u++) x[u] = src[(size_t)(lo + C::LOS * u) * 256 + col];
+        if (a.lift_q) {
+            // y - lift_q + 2q lies in (2q - lift_q/2, 2q), inside the butterflies' [0, 4q) input
+#pragma unroll
+            for (int u = 0; u < 16; u++) x[u] = x[u] > a.lift_half ? x[u] + two_q - a.lift_q : x[u];
+        }
         fwd_top4(x, tw, 1u, q, two_q);
 #pragma unroll
         for (int u = 0; u < 16; u++) sm[(lo + C::LOS * u) * C::CPB + ccol] = x[u];

@@ -161,6 +161,23 @@ int ckks_relin_batch(ckks_ctx *ctx, int n, const uint32_t *d, int level, const c
 int ckks_tensor_batch(ckks_ctx *ctx, int n, const uint32_t *x, const uint32_t *y, int level, uint32_t *d,
                       ckks_stream_t stream);
 
+/* Rescale by the last active prime q_l (the RNS rescale of full-RNS CKKS, Cheon, Han, Kim,
+ * Kim, Song, SAC 2018; the Perseus pages name no rescale of their own, and it follows the
+ * tensor product and relinearisation of a multiplication):
+ *   ct [2][l+1][N] at level l -> out [2][l][N] at level l-1, evaluation domain, canonical;
+ *   per component with integer polynomial C over q_0..q_l, out = (C - [C]_{q_l}) / q_l mod
+ *   q_0..q_{l-1}, with the centred residue [C]_{q_l} in (-q_l/2, q_l/2] (rounding to nearest);
+ *   limb by limb: out_i = (c_i - NTT_i(lift(iNTT_l(c_l)))) [q_l^-1]_{q_i}.
+ * The plaintext scale is divided by q_l.  level >= 1.  Batched: ct [n][2][l+1][N],
+ * out [n][2][l][N].  Workspace: ckks_workspace_bytes(ctx, level, n).  out must not overlap ct
+ * (CKKS_ERR_ARG).  Errors as for the other calls: CKKS_ERR_ARG for a null pointer, n < 0 or
+ * level < 1; CKKS_ERR_UNSUPPORTED for a level above the chain; CKKS_ERR_ALIGN for pointers not
+ * 16-byte aligned; CKKS_ERR_WORKSPACE for a short workspace. */
+int ckks_rescale(ckks_ctx *ctx, const uint32_t *ct, int level, uint32_t *out, void *ws, size_t ws_bytes,
+                 ckks_stream_t stream);
+int ckks_rescale_batch(ckks_ctx *ctx, int n, const uint32_t *ct, int level, uint32_t *out, void *ws,
+                       size_t ws_bytes, ckks_stream_t stream);
+
 /* The key's regenerated uniform half for one (digit, global limb): out [N] (device),
  * out[n] = w mod q_t with w = (x[2m] | x[2m+1] << 32), m = n mod 8, x = ChaCha12 block
  * (RFC 8439 state: key = seed as 8 LE words, counter = n/8, nonce = (key_id, digit, limb)). */
