@@ -400,17 +400,19 @@ LAUNCHES_PER_STEP = 1 + 2 * 10
 
 
 def run_workload(args, local_rank):
-    """Informational throughput of configs 4 and 5 (not the benchmark's headline line):
-    config 4 = 32 hoisted rotations of one ciphertext at level 24 (one ModUp, 32 keys);
-    config 5 = 64 pairs, each tensor + relin + rotate by 2^(i mod 15), level 20, dnum 4
-    (one relinearisation key, 15 rotation keys, all as batched calls)."""
+    """Informational throughput (not the benchmark's headline line):
+    4 = 32 hoisted rotations of one ciphertext at level 24 (one ModUp, 32 keys);
+    5 = 64 pairs, each tensor + relin + rotate by 2^(i mod 15), level 20, dnum 4
+        (one relinearisation key, 15 rotation keys, all as batched calls);
+    5r = the same with a rescale after the relinearisation (rotation at level 19);
+    rescale = 64 rescales of level-35 ciphertexts at N=2^16 (config 3's chain) per step."""
     import torch
     import fhe_key_switching_b200 as ks
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     key = str(args.workload)
-    cfg = W.CONFIGS[key]
+    cfg = W.CONFIGS[{"5r": "5", "rescale": "3"}.get(key, key)]
     n, lvl = cfg.n, cfg.level
     na = lvl + 1
     q, p = ks.ckks_gen_primes(cfg.log_n, cfg.n_q, cfg.n_p)
@@ -456,8 +458,37 @@ def run_workload(args, local_rank):
             ks.ckks_relin_batch(ctx, d, lvl, [k_rel] * P_, r1, ws, stream)
             ks.ckks_rotate_batch(ctx, r1, lvl, gs, ev, out, ws, stream)
         ks_per_step, rot_per_step = 2 * P_, P_
+    elif key == "5r":
+        P_ = cfg.n_pairs
+        xs = [res(q[:na] * 2 * P_).view(P_, 2, na, n) for _ in range(2)]
+        ys = [res(q[:na] * 2 * P_).view(P_, 2, na, n) for _ in range(2)]
+        b_rel = res(mods * nd).view(nd, len(mods), n)
+        k_rel = ks.make_evk(b_rel, cfg.chacha_seed, 0)
+        d = torch.empty((P_, 3, na, n), dtype=torch.uint32, device=dev)
+        r1 = torch.empty((P_, 2, na, n), dtype=torch.uint32, device=dev)
+        r2 = torch.empty((P_, 2, lvl, n), dtype=torch.uint32, device=dev)
+        out = torch.empty((P_, 2, lvl, n), dtype=torch.uint32, device=dev)
+        ws = ctx.workspace(lvl, P_, device=dev)
+        gs = [gal[r] for r in cfg.rot_steps]
+        ev = [evk[r] for r in cfg.rot_steps]
+
+        def step(i):
+            ks.ckks_tensor_batch(ctx, P_, xs[i % 2], ys[i % 2], lvl, d, stream)
+            ks.ckks_relin_batch(ctx, d, lvl, [k_rel] * P_, r1, ws, stream)
+            ks.ckks_rescale_batch(ctx, P_, r1, lvl, r2, ws, stream)
+            ks.ckks_rotate_batch(ctx, r2, lvl - 1, gs, ev, out, ws, stream)
+        ks_per_step, rot_per_step = 2 * P_, P_
+    elif key == "rescale":
+        R = 64
+        cts = [res(q[:na] * 2 * R).view(R, 2, na, n) for _ in range(N_SETS)]
+        out = torch.empty((R, 2, lvl, n), dtype=torch.uint32, device=dev)
+        ws = ctx.workspace(lvl, R, device=dev)
+
+        def step(i):
+            ks.ckks_rescale_batch(ctx, R, cts[i % N_SETS], lvl, out, ws, stream)
+        ks_per_step, rot_per_step = 0, 0
     else:
-        raise SystemExit(f"--workload {key}: use 3 (default), 4 or 5")
+        raise SystemExit(f"--workload {key}: use 3 (default), 4, 5, 5r or rescale")
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
@@ -472,6 +503,17 @@ def run_workload(args, local_rank):
     torch.cuda.synchronize()
     clk = clocks.stop()
     ms = e0.elapsed_time(e1)
+    if key == "rescale":
+        # compulsory bytes per rescale: read 2(l+1) limbs, write 2l limbs
+        b_min = (2 * na + 2 * lvl) * n * 4
+        per_s = R * args.steps / (ms / 1e3)
+        print(json.dumps({"workload": f"rescale: N=2^{cfg.log_n}, level {lvl} -> {lvl - 1}, {R} per step",
+                          "informational": True, "rescales_per_s": per_s, "ms_per_step": ms / args.steps,
+                          "steps": args.steps, "warmup": args.warmup,
+                          "hbm": {"b_min_bytes_per_rescale": b_min, "achieved_gbs": b_min * per_s / 1e9,
+                                  "peak_gbs": HBM_PEAK_GBS, "frac": b_min * per_s / 1e9 / HBM_PEAK_GBS},
+                          "clocks": clk}), flush=True)
+        return
     print(json.dumps({"workload": f"config {key}", "informational": True,
                       "key_switches_per_s": ks_per_step * args.steps / (ms / 1e3),
                       "rotations_per_s": rot_per_step * args.steps / (ms / 1e3),
@@ -573,7 +615,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=8, help="independent config-3 units per step")
-    ap.add_argument("--workload", default="3", help="3 (benchmark line), or 4 / 5 (informational)")
+    ap.add_argument("--workload", default="3",
+                    help="3 (benchmark line), or 4 / 5 / 5r / rescale (informational lines)")
     ap.add_argument("--streams", type=int, default=None,
                     help="CUDA streams the batch is split over, each running batch/streams units "
                          "(default 2 for an even batch, else 1)")
