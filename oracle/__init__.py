@@ -277,6 +277,62 @@ class Ctx:
         lib().or_rescale(self._h, _u32(ct), ct.shape[0], level, _u32(out))
         return out
 
+    def bsgs(self, ct, level, alpha, baby_g, baby_keys, giant_g, giant_keys, pt, seed):
+        """Baby-step giant-step linear transform with double hoisting.
+
+        Computes sum_j rot_{G_j}( sum_k pt[j][k] * rot_{B_k}(ct) ) where the baby rotations are
+        hoisted (one ModUp of c1) and kept in the extended basis PQ, the plaintext products are
+        summed there, and one ModDown per giant step follows (double hoisting: Bossuat, Mouchet,
+        Troncoso-Pastoriza, Hubaux, "Efficient Bootstrapping for Approximate Homomorphic
+        Encryption with Non-Sparse Keys", Eurocrypt 2021, Sec. 6; the BSGS split is Halevi and
+        Shoup's).  Then each giant partial is rotated (a full single rotation; identity for
+        G_j = 1) and the partials are added.  In PQ the baby term for B_k is
+            X_k = (acc0_k + P kappa_{B_k}(c0), acc1_k),  acc_k = IP(kappa_{B_k}(ModUp(c1)), key_k),
+        with P c0 zero on the special limbs; for B_k = 1 (no rotation) X_k = (P c0, P c1).
+        baby_keys[k], giant_keys[j]: (b, key_id), ignored where the Galois element is 1.
+        pt: [n_giant][n_baby][ext][N] canonical evaluation-domain plaintexts over q_0..q_l, p_*.
+        Returns [2][l+1][N]."""
+        na, n, npr = level + 1, self.n, self.n_p
+        ext = na + npr
+        ct = np.ascontiguousarray(ct, dtype=np.uint32).reshape(2, na, n)
+        pt = np.asarray(pt)
+        assert pt.shape == (len(giant_g), len(baby_g), ext, n)
+        mods = np.array(self.q[:na] + self.p, dtype=np.uint64)[:, None]
+        P = 1
+        for p in self.p:
+            P *= p
+        p_mod_q = np.array([P % q for q in self.q[:na]], dtype=np.uint64)[:, None]
+        dt = None
+        X = []
+        for k, g in enumerate(baby_g):
+            x = np.zeros((2, ext, n), dtype=np.uint64)
+            if g == 1:
+                for comp in range(2):
+                    x[comp, :na] = (ct[comp].astype(np.uint64) * p_mod_q) % mods[:na]
+            else:
+                if dt is None:
+                    dt = self.modup(ct[1], level, alpha)
+                b, key_id = baby_keys[k]
+                acc0, acc1 = self.inner_product(self.automorph_eval(dt, g), level, alpha, b, seed, key_id)
+                rc0 = self.automorph_eval(ct[0], g).astype(np.uint64)
+                x[0] = acc0
+                x[0, :na] = (x[0, :na] + rc0 * p_mod_q) % mods[:na]
+                x[1] = acc1
+            X.append(x)
+        out = np.zeros((2, na, n), dtype=np.uint64)
+        for j, g in enumerate(giant_g):
+            v = np.zeros((2, ext, n), dtype=np.uint64)
+            for k in range(len(baby_g)):
+                pk = pt[j, k].astype(np.uint64)
+                for comp in range(2):
+                    v[comp] = (v[comp] + (pk * X[k][comp]) % mods) % mods
+            part = np.stack([self.moddown(v[comp].astype(np.uint32), level) for comp in range(2)])
+            if g != 1:
+                b, key_id = giant_keys[j]
+                part = self.rotate(part, level, alpha, g, b, seed, key_id)
+            out = (out + part) % mods[:na]
+        return out.astype(np.uint32)
+
     def tensor(self, x, y, level):
         x = np.ascontiguousarray(x, dtype=np.uint32)
         y = np.ascontiguousarray(y, dtype=np.uint32)
