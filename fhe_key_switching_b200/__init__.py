@@ -60,6 +60,9 @@ _SIGS = {
     "ckks_tensor_batch": (_ci, [_vp, _ci, _vp, _vp, _ci, _vp, _vp]),
     "ckks_tensor": (_ci, [_vp, _vp, _vp, _ci, _vp, _vp]),
     "ckks_rescale": (_ci, [_vp, _vp, _ci, _vp, _vp, _sz, _vp]),
+    "ckks_bsgs_workspace_bytes": (_sz, [_vp, _ci, _ci, _ci]),
+    "ckks_bsgs": (_ci, [_vp, _vp, _ci, _ci, _u32p, ctypes.POINTER(ckks_evk), _ci, _u32p, ctypes.POINTER(ckks_evk),
+                        _vp, _vp, _vp, _sz, _vp]),
     "ckks_rescale_batch": (_ci, [_vp, _ci, _vp, _ci, _vp, _vp, _sz, _vp]),
     "ckks_chacha_expand": (_ci, [_vp, ctypes.POINTER(ctypes.c_uint8), _cu, _ci, _ci, _vp, _vp]),
     "ckks_workspace_bytes": (_sz, [_vp, _ci, _ci]),
@@ -281,6 +284,28 @@ def ckks_rescale_batch(ctx, n: int, ct, level: int, out, ws, stream=None):
     """Batch of rescales: ct [n][2][l+1][N] -> out [n][2][l][N]."""
     _check(_L.ckks_rescale_batch(ctx.handle, n, _ptr(ct), level, _ptr(out), _ptr(ws),
                                  ws.numel() * ws.element_size(), _stream(stream)), "ckks_rescale_batch")
+
+
+def ckks_bsgs_workspace(ctx, level: int, n_baby: int, n_giant: int, device=None):
+    import torch
+    nb = int(_L.ckks_bsgs_workspace_bytes(ctx.handle, level, n_baby, n_giant))
+    if nb == 0:
+        raise ValueError("ckks_bsgs_workspace_bytes: arguments out of range")
+    return torch.empty(nb, dtype=torch.uint8,
+                       device=device or torch.device("cuda", torch.cuda.current_device()))
+
+
+def ckks_bsgs(ctx, ct, level: int, baby_galois, baby_evks, giant_galois, giant_evks, pt, out, ws, stream=None):
+    """Baby-step giant-step transform: out = sum_j rot_Gj(sum_k pt[j][k] * rot_Bk(ct)).
+    baby_evks / giant_evks: one ckks_evk per step (None where the Galois element is 1)."""
+    nb, ng = len(baby_galois), len(giant_galois)
+    empty = ckks_evk()
+    bk = (ckks_evk * nb)(*[e if e is not None else empty for e in baby_evks])
+    gk = (ckks_evk * ng)(*[e if e is not None else empty for e in giant_evks])
+    bg = (ctypes.c_uint32 * nb)(*baby_galois)
+    gg = (ctypes.c_uint32 * ng)(*giant_galois)
+    _check(_L.ckks_bsgs(ctx.handle, _ptr(ct), level, nb, bg, bk, ng, gg, gk, _ptr(pt), _ptr(out), _ptr(ws),
+                        ws.numel() * ws.element_size(), _stream(stream)), "ckks_bsgs")
 
 
 def ckks_chacha_expand(ctx, seed: bytes, key_id: int, digit: int, limb: int, out, stream=None):

@@ -667,3 +667,112 @@ k_row_combine(RowCombineArgs a) {
     }
     store16_vec(a.out + item * a.out_item + ((size_t)comp * na + i) * n + k0, x);
 }
+
+// ---------------------------------------------------------------- baby-step giant-step transform
+// Plaintext-diagonal sums of a baby-step giant-step linear transform with double hoisting
+// (Bossuat, Mouchet, Troncoso-Pastoriza, Hubaux, Eurocrypt 2021, Sec. 6), in the extended
+// basis PQ before any ModDown:
+//   V_j[comp][u] = sum_k pt[j][k][u] * X_k[comp][u]   (mod t, t the prime of extended row u),
+// X_k = (acc0_k + [P]_t kappa_{g_k}(c0), acc1_k) for a rotated baby, whose accumulators come
+// from the hoisted inner product (the P c0 term only on rows u <= l, where P is invertible),
+// and X_k = ([P]_t c0, [P]_t c1) on rows u <= l, 0 on the special rows, for the identity baby.
+// One thread per coefficient of one extended row; a launch covers babies k0 .. k0+kc-1 (their
+// X in registers) and every giant step, carrying partial sums in V between launches.
+constexpr int BSGS_KC = 16;
+constexpr int BSGS_THREADS = 256;
+
+struct BsgsArgs {
+    const u32 *acc;          // baby accumulators: item z at acc + z * acc_item, [2][ext][N]
+    size_t acc_item;
+    const u32 *ct;           // input ciphertext [2][l+1][N]
+    const u32 *pt;           // plaintexts [n_giant][n_baby][ext][N], canonical
+    u32 *v;                  // giant sums: item j at v + j * v_item, [2][ext][N]
+    size_t v_item;
+    const PrimeInfo *pinfo;
+    const tw_t *pmod;        // [n_q]: [P]_{q_i} and its Shoup companion
+    int log_n, level, n_q, ext, n_baby, n_giant, k0, kc;
+    int item_of[KS_MAXB];    // baby k -> accumulator item, -1 for the identity baby
+    u32 galois[KS_MAXB];     // baby k's Galois element
+};
+
+__global__ void __launch_bounds__(BSGS_THREADS)
+k_bsgs_combine(BsgsArgs a) {
+    const int n = 1 << a.log_n;
+    const int m = blockIdx.x * blockDim.x + threadIdx.x;
+    if (m >= n) return;
+    const int u = blockIdx.y;
+    const int na = a.level + 1;
+    const int t = u < na ? u : a.n_q + (u - na);
+    const PrimeInfo pi = a.pinfo[t];
+    const u32 q = pi.q;
+    const tw_t pm = u < na ? a.pmod[u] : make_uint2(0u, 0u);
+    const u32 *c0 = a.ct + (size_t)u * n;
+    const u32 *c1 = a.ct + ((size_t)na + u) * n;
+    u32 x0[BSGS_KC], x1[BSGS_KC];
+#pragma unroll
+    for (int kk = 0; kk < BSGS_KC; kk++) {
+        x0[kk] = x1[kk] = 0;
+        if (kk < a.kc) {
+            const int k = a.k0 + kk;
+            const int z = a.item_of[k];
+            if (z < 0) {
+                if (u < na) {
+                    x0[kk] = csub(shoup_mul(c0[m], pm.x, pm.y, q), q);
+                    x1[kk] = csub(shoup_mul(c1[m], pm.x, pm.y, q), q);
+                }
+            } else {
+                const u32 *ac = a.acc + (size_t)z * a.acc_item;
+                u32 v0 = ac[(size_t)u * n + m];
+                if (u < na) {
+                    const u32 rc0 = c0[automorph_src((u32)m, a.galois[k], a.log_n)];
+                    v0 = csub(v0 + csub(shoup_mul(rc0, pm.x, pm.y, q), q), q);
+                }
+                x0[kk] = v0;
+                x1[kk] = ac[((size_t)a.ext + u) * n + m];
+            }
+        }
+    }
+    const size_t plane = (size_t)a.ext * n;          // one plaintext
+    for (int j = 0; j < a.n_giant; j++) {
+        u32 *vj = a.v + (size_t)j * a.v_item;
+        // a canonical carry plus 16 products of two values below q < 2^30 stays below 2^64
+        u64 s0 = a.k0 ? vj[(size_t)u * n + m] : 0u;
+        u64 s1 = a.k0 ? vj[((size_t)a.ext + u) * n + m] : 0u;
+        const u32 *pj = a.pt + ((size_t)j * a.n_baby + a.k0) * plane + (size_t)u * n + m;
+#pragma unroll
+        for (int kk = 0; kk < BSGS_KC; kk++) {
+            if (kk < a.kc) {
+                const u64 p = __ldg(pj + (size_t)kk * plane);
+                s0 += p * x0[kk];
+                s1 += p * x1[kk];
+            }
+        }
+        vj[(size_t)u * n + m] = reduce64(s0, q, pi.r64, pi.r64p, pi.onep);
+        vj[((size_t)a.ext + u) * n + m] = reduce64(s1, q, pi.r64, pi.r64p, pi.onep);
+    }
+}
+
+// out[r] = sum_s src_s[r] (mod q_(r mod (l+1))) over 2(l+1) rows [2][l+1][N]; 4 coefficients
+// per thread.
+struct SumArgs {
+    const u32 *src[KS_MAXB];
+    int n_src;
+    u32 *out;
+    const PrimeInfo *pinfo;
+    int log_n, level;
+};
+
+__global__ void __launch_bounds__(256)
+k_sum_parts(SumArgs a) {
+    const int n = 1 << a.log_n;
+    const int c4 = blockIdx.x * blockDim.x + threadIdx.x;
+    if (4 * c4 >= n) return;
+    const int r = blockIdx.y;
+    const u32 q = a.pinfo[r % (a.level + 1)].q;
+    uint4 s = make_uint4(0u, 0u, 0u, 0u);
+    for (int i = 0; i < a.n_src; i++) {
+        const uint4 v = reinterpret_cast<const uint4 *>(a.src[i] + (size_t)r * n)[c4];
+        s.x = csub(s.x + v.x, q); s.y = csub(s.y + v.y, q); s.z = csub(s.z + v.z, q); s.w = csub(s.w + v.w, q);
+    }
+    reinterpret_cast<uint4 *>(a.out + (size_t)r * n)[c4] = s;
+}

@@ -178,6 +178,33 @@ int ckks_rescale(ckks_ctx *ctx, const uint32_t *ct, int level, uint32_t *out, vo
 int ckks_rescale_batch(ckks_ctx *ctx, int n, const uint32_t *ct, int level, uint32_t *out, void *ws,
                        size_t ws_bytes, ckks_stream_t stream);
 
+/* Baby-step giant-step linear transform with double hoisting (Bossuat, Mouchet,
+ * Troncoso-Pastoriza, Hubaux, "Efficient Bootstrapping for Approximate Homomorphic Encryption
+ * with Non-Sparse Keys", Eurocrypt 2021, Sec. 6; the split into baby and giant steps is Halevi
+ * and Shoup's).  The Perseus pages do not describe it; it is the linear-transform step that the
+ * hoisted rotation keys of a CoeffToSlot level serve.
+ *   out = sum_j rot_{G_j}( sum_k pt[j][k] * rot_{B_k}(ct) )
+ * computed as: one ModUp of c1; for every baby k with B_k != 1 the hoisted inner product with
+ * kappa_{B_k} applied to the extended digits, kept in the extended basis PQ as
+ * X_k = (acc0_k + P kappa_{B_k}(c0), acc1_k) (X_k = (P c0, P c1) for B_k = 1); for every giant j
+ * the sum V_j = sum_k pt[j][k] X_k in PQ and one ModDown of it; then each partial rotated by
+ * ckks_rotate's path (none for G_j = 1) and the partials added.
+ *   ct, out: [2][l+1][N] (device, evaluation domain; out must not overlap ct);
+ *   baby_galois[n_baby], giant_galois[n_giant]: host arrays of odd elements in (0, 2N), 1 meaning
+ *     no rotation; baby_keys, giant_keys: host arrays of the same lengths (entries for element 1
+ *     are not read);
+ *   pt: [n_giant][n_baby][ext][N] (device) canonical evaluation-domain plaintexts over the
+ *     extended basis q_0..q_l, p_0..p_{k-1}, ext = l+1+k (the caller pre-rotates the diagonal of
+ *     index (j, k) by -G_j in the slots, as usual for baby-step giant-step);
+ *   1 <= n_baby, n_giant <= 64; workspace: ckks_bsgs_workspace_bytes(ctx, level, n_baby, n_giant)
+ *     (0 for arguments out of range).
+ * Errors: CKKS_ERR_ARG (null pointer, counts out of range, even Galois element, overlap),
+ * CKKS_ERR_UNSUPPORTED (level), CKKS_ERR_ALIGN, CKKS_ERR_WORKSPACE. */
+size_t ckks_bsgs_workspace_bytes(ckks_ctx *ctx, int level, int n_baby, int n_giant);
+int ckks_bsgs(ckks_ctx *ctx, const uint32_t *ct, int level, int n_baby, const uint32_t *baby_galois,
+              const ckks_evk *baby_keys, int n_giant, const uint32_t *giant_galois, const ckks_evk *giant_keys,
+              const uint32_t *pt, uint32_t *out, void *ws, size_t ws_bytes, ckks_stream_t stream);
+
 /* The key's regenerated uniform half for one (digit, global limb): out [N] (device),
  * out[n] = w mod q_t with w = (x[2m] | x[2m+1] << 32), m = n mod 8, x = ChaCha12 block
  * (RFC 8439 state: key = seed as 8 LE words, counter = n/8, nonce = (key_id, digit, limb)). */
