@@ -405,14 +405,16 @@ def run_workload(args, local_rank):
     5 = 64 pairs, each tensor + relin + rotate by 2^(i mod 15), level 20, dnum 4
         (one relinearisation key, 15 rotation keys, all as batched calls);
     5r = the same with a rescale after the relinearisation (rotation at level 19);
-    rescale = 64 rescales of level-35 ciphertexts at N=2^16 (config 3's chain) per step."""
+    rescale = 64 rescales of level-35 ciphertexts at N=2^16 (config 3's chain) per step;
+    bsgs = one baby-step giant-step transform with config 4's 32 keys (baby steps 0..15, giant
+        steps 16 j for j = 0..17: 288 plaintext diagonals over the extended basis, level 24)."""
     import torch
     import fhe_key_switching_b200 as ks
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     key = str(args.workload)
-    cfg = W.CONFIGS[{"5r": "5", "rescale": "3"}.get(key, key)]
+    cfg = W.CONFIGS[{"5r": "5", "rescale": "3", "bsgs": "4"}.get(key, key)]
     n, lvl = cfg.n, cfg.level
     na = lvl + 1
     q, p = ks.ckks_gen_primes(cfg.log_n, cfg.n_q, cfg.n_p)
@@ -487,8 +489,25 @@ def run_workload(args, local_rank):
         def step(i):
             ks.ckks_rescale_batch(ctx, R, cts[i % N_SETS], lvl, out, ws, stream)
         ks_per_step, rot_per_step = 0, 0
+    elif key == "bsgs":
+        n1, n2 = 16, 18
+        baby = [1] + [ks.galois_element(cfg.log_n, k) for k in range(1, n1)]
+        giant = [1] + [ks.galois_element(cfg.log_n, n1 * j) for j in range(1, n2)]
+        gk = {g: ks.make_evk(res(mods * nd).view(nd, len(mods), n), cfg.chacha_seed, g)
+              for g in baby + giant if g != 1}
+        ext = na + cfg.n_p
+        pt = res((q[:na] + p) * n2 * n1).view(n2, n1, ext, n)
+        cts = [res(q[:na] * 2).view(2, na, n) for _ in range(N_SETS)]
+        out = torch.empty((2, na, n), dtype=torch.uint32, device=dev)
+        ws = ks.ckks_bsgs_workspace(ctx, lvl, n1, n2, device=dev)
+        bk = [gk.get(g) for g in baby]
+        gkk = [gk.get(g) for g in giant]
+
+        def step(i):
+            ks.ckks_bsgs(ctx, cts[i % N_SETS], lvl, baby, bk, giant, gkk, pt, out, ws, stream)
+        ks_per_step, rot_per_step = (n1 - 1) + (n2 - 1), (n1 - 1) + (n2 - 1)
     else:
-        raise SystemExit(f"--workload {key}: use 3 (default), 4, 5, 5r or rescale")
+        raise SystemExit(f"--workload {key}: use 3 (default), 4, 5, 5r, rescale or bsgs")
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
@@ -496,6 +515,8 @@ def run_workload(args, local_rank):
     clocks.start()
     time.sleep(0.3)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if key == "bsgs":
+        ks.ckks_prof_begin(ctx, "bsgs_combine", args.steps)
     e0.record(stream)
     for i in range(args.steps):
         step(i)
@@ -503,6 +524,23 @@ def run_workload(args, local_rank):
     torch.cuda.synchronize()
     clk = clocks.stop()
     ms = e0.elapsed_time(e1)
+    if key == "bsgs":
+        launches, comb_ms = ks.ckks_prof_end(ctx)
+        # compulsory bytes of one combine launch: every plaintext once, the 15 rotated babies'
+        # accumulators and the input ciphertext once, the 18 giant sums written once
+        b_comb = (n2 * n1 * ext + (n1 - 1) * 2 * ext + 2 * na + n2 * 2 * ext) * n * 4
+        comb_s = comb_ms / max(launches, 1) / 1e3
+        print(json.dumps({"workload": f"bsgs: config 4 keys, {n1} baby x {n2} giant steps, level {lvl}",
+                          "informational": True, "transforms_per_s": args.steps / (ms / 1e3),
+                          "ms_per_step": ms / args.steps, "steps": args.steps, "warmup": args.warmup,
+                          "rotations_per_transform": ks_per_step,
+                          "combine_kernel": {"avg_launch_us": comb_s * 1e6, "launches": launches,
+                                             "bytes_per_launch": b_comb, "achieved_gbs": b_comb / comb_s / 1e9,
+                                             "peak_gbs": HBM_PEAK_GBS,
+                                             "frac": b_comb / comb_s / 1e9 / HBM_PEAK_GBS,
+                                             "share_of_step": comb_s * 1e3 / (ms / args.steps)},
+                          "clocks": clk}), flush=True)
+        return
     if key == "rescale":
         # compulsory bytes per rescale: read 2(l+1) limbs, write 2l limbs
         b_min = (2 * na + 2 * lvl) * n * 4
@@ -616,7 +654,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=8, help="independent config-3 units per step")
     ap.add_argument("--workload", default="3",
-                    help="3 (benchmark line), or 4 / 5 / 5r / rescale (informational lines)")
+                    help="3 (benchmark line), or 4 / 5 / 5r / rescale / bsgs (informational lines)")
     ap.add_argument("--streams", type=int, default=None,
                     help="CUDA streams the batch is split over, each running batch/streams units "
                          "(default 2 for an even batch, else 1)")

@@ -676,8 +676,8 @@ k_row_combine(RowCombineArgs a) {
 // X_k = (acc0_k + [P]_t kappa_{g_k}(c0), acc1_k) for a rotated baby, whose accumulators come
 // from the hoisted inner product (the P c0 term only on rows u <= l, where P is invertible),
 // and X_k = ([P]_t c0, [P]_t c1) on rows u <= l, 0 on the special rows, for the identity baby.
-// One thread per coefficient of one extended row; a launch covers babies k0 .. k0+kc-1 (their
-// X in registers) and every giant step, carrying partial sums in V between launches.
+// A thread covers 2 coefficients of one extended row; a launch covers babies k0 .. k0+kc-1
+// (their X in registers) and every giant step, carrying partial sums in V between launches.
 constexpr int BSGS_KC = 16;
 constexpr int BSGS_THREADS = 256;
 
@@ -697,58 +697,89 @@ struct BsgsArgs {
 
 __global__ void __launch_bounds__(BSGS_THREADS)
 k_bsgs_combine(BsgsArgs a) {
+    // 2 consecutive coefficients per thread (64-bit loads), two giant steps per iteration, so
+    // that each thread keeps 2 x 16 plaintext loads in flight against HBM latency
     const int n = 1 << a.log_n;
-    const int m = blockIdx.x * blockDim.x + threadIdx.x;
-    if (m >= n) return;
+    const int c2 = blockIdx.x * blockDim.x + threadIdx.x;
+    if (2 * c2 >= n) return;
     const int u = blockIdx.y;
     const int na = a.level + 1;
     const int t = u < na ? u : a.n_q + (u - na);
     const PrimeInfo pi = a.pinfo[t];
     const u32 q = pi.q;
     const tw_t pm = u < na ? a.pmod[u] : make_uint2(0u, 0u);
-    const u32 *c0 = a.ct + (size_t)u * n;
-    const u32 *c1 = a.ct + ((size_t)na + u) * n;
-    u32 x0[BSGS_KC], x1[BSGS_KC];
+    const size_t r0 = (size_t)u * n, r1 = ((size_t)a.ext + u) * n;     // component rows in [2][ext]
+    u32 x0[BSGS_KC][2], x1[BSGS_KC][2];
 #pragma unroll
     for (int kk = 0; kk < BSGS_KC; kk++) {
-        x0[kk] = x1[kk] = 0;
+        x0[kk][0] = x0[kk][1] = x1[kk][0] = x1[kk][1] = 0;
         if (kk < a.kc) {
             const int k = a.k0 + kk;
             const int z = a.item_of[k];
             if (z < 0) {
                 if (u < na) {
-                    x0[kk] = csub(shoup_mul(c0[m], pm.x, pm.y, q), q);
-                    x1[kk] = csub(shoup_mul(c1[m], pm.x, pm.y, q), q);
+                    const uint2 v0 = reinterpret_cast<const uint2 *>(a.ct + (size_t)u * n)[c2];
+                    const uint2 v1 = reinterpret_cast<const uint2 *>(a.ct + ((size_t)na + u) * n)[c2];
+                    x0[kk][0] = csub(shoup_mul(v0.x, pm.x, pm.y, q), q);
+                    x0[kk][1] = csub(shoup_mul(v0.y, pm.x, pm.y, q), q);
+                    x1[kk][0] = csub(shoup_mul(v1.x, pm.x, pm.y, q), q);
+                    x1[kk][1] = csub(shoup_mul(v1.y, pm.x, pm.y, q), q);
                 }
             } else {
                 const u32 *ac = a.acc + (size_t)z * a.acc_item;
-                u32 v0 = ac[(size_t)u * n + m];
+                const uint2 v0 = reinterpret_cast<const uint2 *>(ac + r0)[c2];
+                const uint2 v1 = reinterpret_cast<const uint2 *>(ac + r1)[c2];
+                u32 e0 = v0.x, e1 = v0.y;
                 if (u < na) {
-                    const u32 rc0 = c0[automorph_src((u32)m, a.galois[k], a.log_n)];
-                    v0 = csub(v0 + csub(shoup_mul(rc0, pm.x, pm.y, q), q), q);
+                    const u32 *c0 = a.ct + (size_t)u * n;
+                    const u32 g = a.galois[k];
+                    e0 = csub(e0 + csub(shoup_mul(c0[automorph_src((u32)(2 * c2), g, a.log_n)], pm.x, pm.y, q), q), q);
+                    e1 = csub(e1 + csub(shoup_mul(c0[automorph_src((u32)(2 * c2 + 1), g, a.log_n)], pm.x, pm.y, q), q), q);
                 }
-                x0[kk] = v0;
-                x1[kk] = ac[((size_t)a.ext + u) * n + m];
+                x0[kk][0] = e0; x0[kk][1] = e1;
+                x1[kk][0] = v1.x; x1[kk][1] = v1.y;
             }
         }
     }
     const size_t plane = (size_t)a.ext * n;          // one plaintext
-    for (int j = 0; j < a.n_giant; j++) {
-        u32 *vj = a.v + (size_t)j * a.v_item;
+    for (int j = 0; j < a.n_giant; j += 2) {
+        const bool two = j + 1 < a.n_giant;
         // a canonical carry plus 16 products of two values below q < 2^30 stays below 2^64
-        u64 s0 = a.k0 ? vj[(size_t)u * n + m] : 0u;
-        u64 s1 = a.k0 ? vj[((size_t)a.ext + u) * n + m] : 0u;
-        const u32 *pj = a.pt + ((size_t)j * a.n_baby + a.k0) * plane + (size_t)u * n + m;
+        u64 s[2][2][2];                              // [giant][component][coefficient]
+#pragma unroll
+        for (int h = 0; h < 2; h++) {
+            const u32 *vj = a.v + (size_t)(j + h) * a.v_item;
+            if (a.k0 && (h == 0 || two)) {
+                const uint2 w0 = reinterpret_cast<const uint2 *>(vj + r0)[c2];
+                const uint2 w1 = reinterpret_cast<const uint2 *>(vj + r1)[c2];
+                s[h][0][0] = w0.x; s[h][0][1] = w0.y; s[h][1][0] = w1.x; s[h][1][1] = w1.y;
+            } else {
+                s[h][0][0] = s[h][0][1] = s[h][1][0] = s[h][1][1] = 0;
+            }
+        }
+        const u32 *pj = a.pt + ((size_t)j * a.n_baby + a.k0) * plane + (size_t)u * n;
+        const size_t pnext = (size_t)a.n_baby * plane;    // the next giant's plaintexts
 #pragma unroll
         for (int kk = 0; kk < BSGS_KC; kk++) {
             if (kk < a.kc) {
-                const u64 p = __ldg(pj + (size_t)kk * plane);
-                s0 += p * x0[kk];
-                s1 += p * x1[kk];
+                const uint2 p0 = __ldg(reinterpret_cast<const uint2 *>(pj + (size_t)kk * plane) + c2);
+                const uint2 p1 = two ? __ldg(reinterpret_cast<const uint2 *>(pj + pnext + (size_t)kk * plane) + c2)
+                                     : make_uint2(0u, 0u);
+                s[0][0][0] += (u64)p0.x * x0[kk][0]; s[0][0][1] += (u64)p0.y * x0[kk][1];
+                s[0][1][0] += (u64)p0.x * x1[kk][0]; s[0][1][1] += (u64)p0.y * x1[kk][1];
+                s[1][0][0] += (u64)p1.x * x0[kk][0]; s[1][0][1] += (u64)p1.y * x0[kk][1];
+                s[1][1][0] += (u64)p1.x * x1[kk][0]; s[1][1][1] += (u64)p1.y * x1[kk][1];
             }
         }
-        vj[(size_t)u * n + m] = reduce64(s0, q, pi.r64, pi.r64p, pi.onep);
-        vj[((size_t)a.ext + u) * n + m] = reduce64(s1, q, pi.r64, pi.r64p, pi.onep);
+#pragma unroll
+        for (int h = 0; h < 2; h++) {
+            if (h == 1 && !two) break;
+            u32 *vj = a.v + (size_t)(j + h) * a.v_item;
+            reinterpret_cast<uint2 *>(vj + r0)[c2] =
+                make_uint2(reduce64(s[h][0][0], q, pi.r64, pi.r64p, pi.onep), reduce64(s[h][0][1], q, pi.r64, pi.r64p, pi.onep));
+            reinterpret_cast<uint2 *>(vj + r1)[c2] =
+                make_uint2(reduce64(s[h][1][0], q, pi.r64, pi.r64p, pi.onep), reduce64(s[h][1][1], q, pi.r64, pi.r64p, pi.onep));
+        }
     }
 }
 
