@@ -678,6 +678,7 @@ k_row_combine(RowCombineArgs a) {
 // and X_k = ([P]_t c0, [P]_t c1) on rows u <= l, 0 on the special rows, for the identity baby.
 // A thread covers 2 coefficients of one extended row; a launch covers babies k0 .. k0+kc-1
 // (their X in registers) and every giant step, carrying partial sums in V between launches.
+// n must be a multiple of 512 (true for every supported N).
 constexpr int BSGS_KC = 16;
 constexpr int BSGS_THREADS = 256;
 
@@ -691,17 +692,73 @@ struct BsgsArgs {
     const PrimeInfo *pinfo;
     const tw_t *pmod;        // [n_q]: [P]_{q_i} and its Shoup companion
     int log_n, level, n_q, ext, n_baby, n_giant, k0, kc;
+    int *err;                // device error word: CKKS_DEV_ERR_WAIT is or-ed in when a wait expires
     int item_of[KS_MAXB];    // baby k -> accumulator item, -1 for the identity baby
     u32 galois[KS_MAXB];     // baby k's Galois element
 };
 
+// ---- bulk asynchronous copies into shared memory, completed on an mbarrier (sm_90+ PTX)
+__device__ __forceinline__ u32 smem_addr(const void *p) { return (u32)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(u64 *bar, u32 count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(u64 *bar, u32 bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+                 : "memory");
+}
+
+// global -> this CTA's shared memory, `bytes` a multiple of 16, both addresses 16-byte aligned
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, u32 bytes, u64 *bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(u64 *bar, u32 phase) {
+    u32 ok;
+    asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(smem_addr(bar)), "r"(phase) : "memory");
+    return ok != 0;
+}
+
+constexpr int CKKS_DEV_ERR_WAIT = 1;              // a bounded device wait expired
+constexpr u64 MBAR_WAIT_NS = 1000000000ull;       // wait bound: 1 s of the global timer
+constexpr u32 MBAR_WAIT_TRIES = 1u << 30;         // backstop on the number of try_wait rounds
+
+__device__ __forceinline__ u64 global_ns() {
+    u64 t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Waits for `phase` of `bar`; false when MBAR_WAIT_NS (or the round backstop) expires.
+__device__ __forceinline__ bool mbar_wait_bounded(u64 *bar, u32 phase) {
+    if (mbar_try_wait(bar, phase)) return true;
+    const u64 t0 = global_ns();
+    for (u32 i = 0; i < MBAR_WAIT_TRIES; i++) {
+        if (mbar_try_wait(bar, phase)) return true;
+        if (global_ns() - t0 > MBAR_WAIT_NS) return false;
+    }
+    return false;
+}
+
+// The plaintexts stream through shared memory: a block covers 512 coefficients (2 per thread)
+// of one extended row, and stage s holds one giant step's kc plaintext chunks of 2 KB, loaded
+// by one thread with bulk copies on the stage's mbarrier, BSGS_STAGES giant steps ahead of
+// the computation.  The babies' terms X stay in registers.
+constexpr int BSGS_STAGES = 3;
+constexpr int BSGS_CHUNK = 2 * BSGS_THREADS;                 // coefficients per block
+constexpr size_t BSGS_SMEM = (size_t)BSGS_STAGES * BSGS_KC * BSGS_CHUNK * sizeof(u32);
+
 __global__ void __launch_bounds__(BSGS_THREADS)
 k_bsgs_combine(BsgsArgs a) {
-    // 2 consecutive coefficients per thread (64-bit loads), two giant steps per iteration, so
-    // that each thread keeps 2 x 16 plaintext loads in flight against HBM latency
+    extern __shared__ __align__(128) u32 sp[];               // [stage][kk][BSGS_CHUNK]
+    __shared__ __align__(8) u64 full[BSGS_STAGES];
     const int n = 1 << a.log_n;
-    const int c2 = blockIdx.x * blockDim.x + threadIdx.x;
-    if (2 * c2 >= n) return;
+    const int tid = threadIdx.x;
+    const int c2 = blockIdx.x * BSGS_THREADS + tid;          // coefficient pair of this thread
     const int u = blockIdx.y;
     const int na = a.level + 1;
     const int t = u < na ? u : a.n_q + (u - na);
@@ -709,6 +766,26 @@ k_bsgs_combine(BsgsArgs a) {
     const u32 q = pi.q;
     const tw_t pm = u < na ? a.pmod[u] : make_uint2(0u, 0u);
     const size_t r0 = (size_t)u * n, r1 = ((size_t)a.ext + u) * n;     // component rows in [2][ext]
+    const size_t plane = (size_t)a.ext * n;                  // one plaintext
+    const u32 stage_bytes = (u32)(a.kc * BSGS_CHUNK * sizeof(u32));
+    const u32 *pbase = a.pt + (size_t)a.k0 * plane + r0 + (size_t)blockIdx.x * BSGS_CHUNK;
+    if (tid == 0) {
+        for (int st = 0; st < BSGS_STAGES; st++) mbar_init(&full[st], 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    // thread 0: giant step j's plaintext chunks into stage j % BSGS_STAGES
+    auto issue = [&](int j) {
+        const int st = j % BSGS_STAGES;
+        mbar_expect_tx(&full[st], stage_bytes);
+        const u32 *src = pbase + (size_t)j * a.n_baby * plane;
+        for (int kk = 0; kk < a.kc; kk++)
+            bulk_load(sp + ((size_t)st * BSGS_KC + kk) * BSGS_CHUNK, src + (size_t)kk * plane,
+                      BSGS_CHUNK * sizeof(u32), &full[st]);
+    };
+    if (tid == 0)
+        for (int j = 0; j < BSGS_STAGES && j < a.n_giant; j++) issue(j);
+    // the babies' terms for this thread's two coefficients (overlaps the first copies)
     u32 x0[BSGS_KC][2], x1[BSGS_KC][2];
 #pragma unroll
     for (int kk = 0; kk < BSGS_KC; kk++) {
@@ -741,45 +818,41 @@ k_bsgs_combine(BsgsArgs a) {
             }
         }
     }
-    const size_t plane = (size_t)a.ext * n;          // one plaintext
-    for (int j = 0; j < a.n_giant; j += 2) {
-        const bool two = j + 1 < a.n_giant;
-        // a canonical carry plus 16 products of two values below q < 2^30 stays below 2^64
-        u64 s[2][2][2];                              // [giant][component][coefficient]
-#pragma unroll
-        for (int h = 0; h < 2; h++) {
-            const u32 *vj = a.v + (size_t)(j + h) * a.v_item;
-            if (a.k0 && (h == 0 || two)) {
-                const uint2 w0 = reinterpret_cast<const uint2 *>(vj + r0)[c2];
-                const uint2 w1 = reinterpret_cast<const uint2 *>(vj + r1)[c2];
-                s[h][0][0] = w0.x; s[h][0][1] = w0.y; s[h][1][0] = w1.x; s[h][1][1] = w1.y;
-            } else {
-                s[h][0][0] = s[h][0][1] = s[h][1][0] = s[h][1][1] = 0;
+    for (int j = 0; j < a.n_giant; j++) {
+        const int st = j % BSGS_STAGES;
+        const bool expired = !mbar_wait_bounded(&full[st], (u32)(j / BSGS_STAGES) & 1u);
+        if (__syncthreads_or(expired)) {
+            // leave together: record the failure, let this block's copies in flight land
+            if (tid == 0) {
+                atomicOr(a.err, CKKS_DEV_ERR_WAIT);
+                for (int jj = j; jj < j + BSGS_STAGES && jj < a.n_giant; jj++)
+                    (void)mbar_wait_bounded(&full[jj % BSGS_STAGES], (u32)(jj / BSGS_STAGES) & 1u);
             }
+            return;
         }
-        const u32 *pj = a.pt + ((size_t)j * a.n_baby + a.k0) * plane + (size_t)u * n;
-        const size_t pnext = (size_t)a.n_baby * plane;    // the next giant's plaintexts
+        u32 *vj = a.v + (size_t)j * a.v_item;
+        // a canonical carry plus 16 products of two values below q < 2^30 stays below 2^64
+        u64 s00 = 0, s01 = 0, s10 = 0, s11 = 0;              // [component][coefficient]
+        if (a.k0) {
+            const uint2 w0 = reinterpret_cast<const uint2 *>(vj + r0)[c2];
+            const uint2 w1 = reinterpret_cast<const uint2 *>(vj + r1)[c2];
+            s00 = w0.x; s01 = w0.y; s10 = w1.x; s11 = w1.y;
+        }
+        const uint2 *ps = reinterpret_cast<const uint2 *>(sp + (size_t)st * BSGS_KC * BSGS_CHUNK) + tid;
 #pragma unroll
         for (int kk = 0; kk < BSGS_KC; kk++) {
             if (kk < a.kc) {
-                const uint2 p0 = __ldg(reinterpret_cast<const uint2 *>(pj + (size_t)kk * plane) + c2);
-                const uint2 p1 = two ? __ldg(reinterpret_cast<const uint2 *>(pj + pnext + (size_t)kk * plane) + c2)
-                                     : make_uint2(0u, 0u);
-                s[0][0][0] += (u64)p0.x * x0[kk][0]; s[0][0][1] += (u64)p0.y * x0[kk][1];
-                s[0][1][0] += (u64)p0.x * x1[kk][0]; s[0][1][1] += (u64)p0.y * x1[kk][1];
-                s[1][0][0] += (u64)p1.x * x0[kk][0]; s[1][0][1] += (u64)p1.y * x0[kk][1];
-                s[1][1][0] += (u64)p1.x * x1[kk][0]; s[1][1][1] += (u64)p1.y * x1[kk][1];
+                const uint2 p = ps[(size_t)kk * (BSGS_CHUNK / 2)];
+                s00 += (u64)p.x * x0[kk][0]; s01 += (u64)p.y * x0[kk][1];
+                s10 += (u64)p.x * x1[kk][0]; s11 += (u64)p.y * x1[kk][1];
             }
         }
-#pragma unroll
-        for (int h = 0; h < 2; h++) {
-            if (h == 1 && !two) break;
-            u32 *vj = a.v + (size_t)(j + h) * a.v_item;
-            reinterpret_cast<uint2 *>(vj + r0)[c2] =
-                make_uint2(reduce64(s[h][0][0], q, pi.r64, pi.r64p, pi.onep), reduce64(s[h][0][1], q, pi.r64, pi.r64p, pi.onep));
-            reinterpret_cast<uint2 *>(vj + r1)[c2] =
-                make_uint2(reduce64(s[h][1][0], q, pi.r64, pi.r64p, pi.onep), reduce64(s[h][1][1], q, pi.r64, pi.r64p, pi.onep));
-        }
+        reinterpret_cast<uint2 *>(vj + r0)[c2] =
+            make_uint2(reduce64(s00, q, pi.r64, pi.r64p, pi.onep), reduce64(s01, q, pi.r64, pi.r64p, pi.onep));
+        reinterpret_cast<uint2 *>(vj + r1)[c2] =
+            make_uint2(reduce64(s10, q, pi.r64, pi.r64p, pi.onep), reduce64(s11, q, pi.r64, pi.r64p, pi.onep));
+        __syncthreads();                                     // stage st fully read
+        if (tid == 0 && j + BSGS_STAGES < a.n_giant) issue(j + BSGS_STAGES);
     }
 }
 

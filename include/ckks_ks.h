@@ -237,12 +237,16 @@ size_t ckks_workspace_bytes(const ckks_ctx *ctx, int level, int n);
 
 /* Waits for `stream` with a deadline (polling, no device-side wait): CKKS_OK when the
  * stream is idle and no CUDA error is pending, CKKS_ERR_TIMEOUT at the deadline,
- * CKKS_ERR_CUDA on an asynchronous error. */
+ * CKKS_ERR_CUDA on an asynchronous error.  With a context, it then reads (and clears) the
+ * context's device error word: kernels whose waits are bounded (the shared-memory pipeline of
+ * ckks_bsgs) record an expired wait there and return early, and ckks_sync_status reports it as
+ * CKKS_ERR_TIMEOUT; the results of the calls since the previous check are then invalid, and the
+ * context stays usable. */
 int ckks_sync_status(ckks_ctx *ctx, ckks_stream_t stream, int timeout_ms);
 
 /* Kernel timing.  Between ckks_prof_begin and ckks_prof_end, every launch of the kernel named
  * `kernel` ("ip_row", "bconv", "ntt_col_fwd", "ntt_col_inv", "ntt_row_fwd", "ntt_row_inv",
- * "row_combine", "tensor") made through `ctx` is bracketed by CUDA events recorded on its
+ * "row_combine", "tensor", "bsgs_combine") made through `ctx` is bracketed by CUDA events recorded on its
  * launching stream; up to max_launches launches are recorded (the events are created by
  * ckks_prof_begin, outside any timed region).  ckks_prof_end synchronises on the last event and
  * returns the number of recorded launches and their summed device time in milliseconds.
