@@ -407,14 +407,16 @@ def run_workload(args, local_rank):
     5r = the same with a rescale after the relinearisation (rotation at level 19);
     rescale = 64 rescales of level-35 ciphertexts at N=2^16 (config 3's chain) per step;
     bsgs = one baby-step giant-step transform with config 4's 32 keys (baby steps 0..15, giant
-        steps 16 j for j = 0..17: 288 plaintext diagonals over the extended basis, level 24)."""
+        steps 16 j for j = 0..17: 288 plaintext diagonals over the extended basis, level 24);
+    bsgs2 = the same transform shape on config 2's chain (N=2^14, level 11), a smaller case
+        whose plaintexts (302 MB) still exceed L2, for profiling."""
     import torch
     import fhe_key_switching_b200 as ks
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     key = str(args.workload)
-    cfg = W.CONFIGS[{"5r": "5", "rescale": "3", "bsgs": "4"}.get(key, key)]
+    cfg = W.CONFIGS[{"5r": "5", "rescale": "3", "bsgs": "4", "bsgs2": "2"}.get(key, key)]
     n, lvl = cfg.n, cfg.level
     na = lvl + 1
     q, p = ks.ckks_gen_primes(cfg.log_n, cfg.n_q, cfg.n_p)
@@ -489,7 +491,7 @@ def run_workload(args, local_rank):
         def step(i):
             ks.ckks_rescale_batch(ctx, R, cts[i % N_SETS], lvl, out, ws, stream)
         ks_per_step, rot_per_step = 0, 0
-    elif key == "bsgs":
+    elif key in ("bsgs", "bsgs2"):
         n1, n2 = 16, 18
         baby = [1] + [ks.galois_element(cfg.log_n, k) for k in range(1, n1)]
         giant = [1] + [ks.galois_element(cfg.log_n, n1 * j) for j in range(1, n2)]
@@ -515,7 +517,7 @@ def run_workload(args, local_rank):
     clocks.start()
     time.sleep(0.3)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if key == "bsgs":
+    if key in ("bsgs", "bsgs2"):
         ks.ckks_prof_begin(ctx, "bsgs_combine", args.steps)
     e0.record(stream)
     for i in range(args.steps):
@@ -524,13 +526,14 @@ def run_workload(args, local_rank):
     torch.cuda.synchronize()
     clk = clocks.stop()
     ms = e0.elapsed_time(e1)
-    if key == "bsgs":
+    if key in ("bsgs", "bsgs2"):
         launches, comb_ms = ks.ckks_prof_end(ctx)
         # compulsory bytes of one combine launch: every plaintext once, the 15 rotated babies'
         # accumulators and the input ciphertext once, the 18 giant sums written once
         b_comb = (n2 * n1 * ext + (n1 - 1) * 2 * ext + 2 * na + n2 * 2 * ext) * n * 4
         comb_s = comb_ms / max(launches, 1) / 1e3
-        print(json.dumps({"workload": f"bsgs: config 4 keys, {n1} baby x {n2} giant steps, level {lvl}",
+        print(json.dumps({"workload": f"bsgs: config {cfg.key} chain, N=2^{cfg.log_n}, {n1} baby x {n2} giant "
+                                      f"steps, level {lvl}",
                           "informational": True, "transforms_per_s": args.steps / (ms / 1e3),
                           "ms_per_step": ms / args.steps, "steps": args.steps, "warmup": args.warmup,
                           "rotations_per_transform": ks_per_step,
@@ -654,7 +657,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=8, help="independent config-3 units per step")
     ap.add_argument("--workload", default="3",
-                    help="3 (benchmark line), or 4 / 5 / 5r / rescale / bsgs (informational lines)")
+                    help="3 (benchmark line), or 4 / 5 / 5r / rescale / bsgs / bsgs2 (informational lines)")
     ap.add_argument("--streams", type=int, default=None,
                     help="CUDA streams the batch is split over, each running batch/streams units "
                          "(default 2 for an even batch, else 1)")

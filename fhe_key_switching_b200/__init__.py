@@ -67,6 +67,7 @@ _SIGS = {
     "ckks_chacha_expand": (_ci, [_vp, ctypes.POINTER(ctypes.c_uint8), _cu, _ci, _ci, _vp, _vp]),
     "ckks_workspace_bytes": (_sz, [_vp, _ci, _ci]),
     "ckks_sync_status": (_ci, [_vp, _vp, _ci]),
+    "ckks_selftest_wait_expiry": (_ci, [_vp, _vp]),
     "ckks_keyswitch_noalloc": (_ci, [_vp, _vp, _ci, ctypes.POINTER(ckks_evk), _vp, _vp]),
     "ckks_prof_begin": (_ci, [_vp, ctypes.c_char_p, _ci]),
     "ckks_prof_end": (_ci, [_vp, ctypes.POINTER(_ci), ctypes.POINTER(ctypes.c_double)]),
@@ -316,6 +317,10 @@ def ckks_chacha_expand(ctx, seed: bytes, key_id: int, digit: int, limb: int, out
 
 def ckks_sync_status(ctx, stream=None, timeout_ms: int = 10000) -> int:
     return int(_L.ckks_sync_status(ctx.handle if ctx is not None else None, _stream(stream), timeout_ms))
+
+
+def ckks_selftest_wait_expiry(ctx, stream=None):
+    _check(_L.ckks_selftest_wait_expiry(ctx.handle, _stream(stream)), "ckks_selftest_wait_expiry")
 
 
 def ckks_prof_begin(ctx, kernel: str, max_launches: int):

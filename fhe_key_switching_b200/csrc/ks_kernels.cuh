@@ -744,6 +744,20 @@ __device__ __forceinline__ bool mbar_wait_bounded(u64 *bar, u32 phase) {
     return false;
 }
 
+// Self-test of the bounded-wait failure path: one block waits on an mbarrier that expects two
+// arrivals and receives one, so the wait expires after MBAR_WAIT_NS and the error word is set.
+// No copy is involved and nothing else waits on this block.
+__global__ void k_wait_expiry_probe(int *err) {
+    __shared__ __align__(8) u64 bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 2);
+        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(&bar)) : "memory");
+    }
+    __syncthreads();
+    const bool expired = !mbar_wait_bounded(&bar, 0u);
+    if (threadIdx.x == 0 && expired) atomicOr(err, CKKS_DEV_ERR_WAIT);
+}
+
 // The plaintexts stream through shared memory: a block covers 512 coefficients (2 per thread)
 // of one extended row, and stage s holds one giant step's kc plaintext chunks of 2 KB, loaded
 // by one thread with bulk copies on the stage's mbarrier, BSGS_STAGES giant steps ahead of

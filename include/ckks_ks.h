@@ -244,6 +244,13 @@ size_t ckks_workspace_bytes(const ckks_ctx *ctx, int level, int n);
  * context stays usable. */
 int ckks_sync_status(ckks_ctx *ctx, ckks_stream_t stream, int timeout_ms);
 
+/* Self-test of the failure path of bounded device waits (no counterpart in the pages):
+ * launches one block that waits on an mbarrier that never completes, so its bounded wait
+ * expires after about one second and sets the context's device error word; the next
+ * ckks_sync_status on `stream` returns CKKS_ERR_TIMEOUT and clears it, and the context stays
+ * usable.  Nothing faults or hangs. */
+int ckks_selftest_wait_expiry(ckks_ctx *ctx, ckks_stream_t stream);
+
 /* Kernel timing.  Between ckks_prof_begin and ckks_prof_end, every launch of the kernel named
  * `kernel` ("ip_row", "bconv", "ntt_col_fwd", "ntt_col_inv", "ntt_row_fwd", "ntt_row_inv",
  * "row_combine", "tensor", "bsgs_combine") made through `ctx` is bracketed by CUDA events recorded on its
