@@ -21,6 +21,7 @@ cores instead, on a bounded sample of the same workload.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -151,10 +152,12 @@ def run_ours(args, rank, world, local_rank):
         # --stored-a (ablation): the keys carry a stored a half read from HBM instead of ChaCha12
         a_rel = residues(mods * nd * B, 10 * s + 5).view(B, nd, len(mods), n) if args.stored_a else None
         a_rot = residues(mods * nd * B, 10 * s + 6).view(B, nd, len(mods), n) if args.stored_a else None
+        # every unit has its own key pair: its own seed (so its own regenerated a half) and b half
+        seeds = [hashlib.sha256(cfg.chacha_seed + bytes([s, i])).digest() for i in range(B)]
         sets.append(dict(x=x, y=y, b_rel=b_rel, b_rot=b_rot, a_rel=a_rel, a_rot=a_rot,
-                         k_rel=[ks.make_evk(b_rel[i], cfg.chacha_seed, 0,
+                         k_rel=[ks.make_evk(b_rel[i], seeds[i], 0,
                                             a=a_rel[i] if args.stored_a else None) for i in range(B)],
-                         k_rot=[ks.make_evk(b_rot[i], cfg.chacha_seed, g,
+                         k_rot=[ks.make_evk(b_rot[i], seeds[i], g,
                                             a=a_rot[i] if args.stored_a else None) for i in range(B)]))
     d = torch.empty((B, 3, na, n), dtype=torch.uint32, device=dev)
     r = torch.empty((B, 2, na, n), dtype=torch.uint32, device=dev)

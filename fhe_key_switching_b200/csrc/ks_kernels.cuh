@@ -495,8 +495,8 @@ __device__ __forceinline__ void row_inv_regs(u32 (&x)[16], const tw_t *tw, u32 b
     inv_top4(x, tw, base, q, two_q);
 }
 
-// Key inner product fused with the last forward NTT pass of ModUp.  Block (16 rows, u): for
-// every active digit j, the extended digit dt_j[u] is completed in registers (forward row
+// Key inner product fused with the last forward NTT pass of ModUp.  Block (16 rows, u, group):
+// for every active digit j, the extended digit dt_j[u] is completed in registers (forward row
 // pass of the column-pass output x[j][u], or the input polynomial itself for u inside digit
 // j), the key's a half for (digit j, limb t) is regenerated by ChaCha12 for the same 16
 // slots, and
@@ -504,7 +504,15 @@ __device__ __forceinline__ void row_inv_regs(u32 (&x)[16], const tw_t *tw, u32 b
 // Rotations: hoist_g != 0 reads every dt_j[u] through kappa_{hoist_g} (hoisted rotation:
 // the source row is transformed, then permuted inside the row); cdig_g != 0 reads only the
 // input polynomial's digit limbs through kappa_{cdig_g} (single rotation).
+// Items whose a half is the same (same seed and key id, regenerated) form a group of up to
+// IP_GROUP_MAX: its block regenerates a_j once for all active digits into shared memory and
+// then runs the group's items one after another, each with its own b half, inputs and
+// rotation.  A group of one keeps the keystream in registers.
 // Output: acc rows, canonical evaluation values.
+constexpr int IP_GROUP_MAX = 8;
+constexpr int IP_GROUP_MAX_BETA = 4;             // digits whose a half fits the shared buffer
+constexpr size_t IP_GROUP_SMEM = (size_t)IP_GROUP_MAX_BETA * 16 * ROW_THREADS * sizeof(u32);
+
 struct IpRowArgs {
     const u32 *x;            // [beta][ext][N] ModUp column-pass output (non-digit limbs)
     const u32 *cdig;         // [l+1][N] input polynomial, evaluation domain
@@ -513,29 +521,24 @@ struct IpRowArgs {
     const tw_t *twf, *twi;
     const PrimeInfo *pinfo;
     int log_n, level, n_q, n_primes, alpha, beta, ext;
-    // per item (blockIdx.z): the key and the rotation
+    // per item: the key and the rotation
     const u32 *b[KS_MAXB];        // [D][n_primes][N]
     const u32 *a_stored[KS_MAXB]; // nullptr: regenerate
     ChachaKey key[KS_MAXB];
     u32 key_id[KS_MAXB];
     u32 hoist_g[KS_MAXB], cdig_g[KS_MAXB];
+    // groups (blockIdx.z): items grp_item[grp_first[g] .. grp_first[g] + grp_count[g] - 1]
+    int grp_first[KS_MAXB], grp_count[KS_MAXB], grp_item[KS_MAXB];
 };
 
 __global__ void __launch_bounds__(ROW_THREADS)
 k_ip_row(IpRowArgs a) {
     __shared__ u32 sm[16 * 272];
+    extern __shared__ u32 sa[];                      // shared a half: [digit][16][ROW_THREADS]
     const int n = 1 << a.log_n;
     const int na = a.level + 1;
     const int u = blockIdx.y;
-    const int item = blockIdx.z;
-    const u32 *xb = a.x + item * a.x_item;
-    const u32 *cdb = a.cdig + item * a.cdig_item;
-    u32 *accb = a.acc + item * a.acc_item;
-    const u32 *bkey = a.b[item];
-    const u32 *astore = a.a_stored[item];
-    const ChachaKey &key = a.key[item];
-    const u32 key_id = a.key_id[item];
-    const u32 hoist_g = a.hoist_g[item], cdig_g = a.cdig_g[item];
+    const int g0 = a.grp_first[blockIdx.z], gcnt = a.grp_count[blockIdx.z];
     const int t = u < na ? u : a.n_q + (u - na);
     const PrimeInfo pi = a.pinfo[t];
     const u32 q = pi.q, two_q = 2 * q;
@@ -545,71 +548,94 @@ k_ip_row(IpRowArgs a) {
     u32 *srow = sm + r * 272;
     const int k0 = row * 256 + 16 * lo;              // first evaluation slot of this thread
     const tw_t *twf = a.twf + (size_t)t * n;
-    // hoisted rotation: source row of this row under kappa_g
-    const int src_row = hoist_g ? (int)(automorph_src((u32)(row * 256), hoist_g, a.log_n) >> 8) : row;
-    u32 acc0[16], acc1[16];
-#pragma unroll
-    for (int v = 0; v < 16; v++) acc0[v] = acc1[v] = 0;
-    for (int j = 0; j < a.beta; j++) {
-        const bool in_digit = u < na && u >= j * a.alpha && u < min(j * a.alpha + a.alpha, na);
-        u32 x[16];
-        if (in_digit) {
-            const u32 *src = cdb + (size_t)u * n;
-            const u32 g = hoist_g ? hoist_g : cdig_g;
-            if (g) {
-#pragma unroll
-                for (int v = 0; v < 16; v++) x[v] = src[automorph_src((u32)(k0 + v), g, a.log_n)];
-            } else {
-                load16_vec(src + k0, x);
-            }
-        } else {
-            const u32 *src = xb + ((size_t)j * a.ext + u) * n + (size_t)src_row * 256;
-#pragma unroll
-            for (int v = 0; v < 16; v++) x[v] = src[lo + 16 * v];
-            row_fwd_regs(x, twf, R1 + (u32)src_row, lo, srow, q);
-            if (hoist_g) {            // permute inside the row: slot k takes source slot src(k)
-#pragma unroll
-                for (int v = 0; v < 16; v++) srow[17 * lo + v] = x[v];
-                __syncwarp();
-#pragma unroll
-                for (int v = 0; v < 16; v++) {
-                    const u32 m = automorph_src((u32)(k0 + v), hoist_g, a.log_n) & 255u;
-                    x[v] = srow[m + (m >> 4)];
-                }
-                __syncwarp();
-            }
-        }
-        u32 bv[16], av[16];
-        load16_vec(bkey + ((size_t)j * a.n_primes + t) * n + k0, bv);
-        if (astore) {
-            load16_vec(astore + ((size_t)j * a.n_primes + t) * n + k0, av);
-        } else {
+    if (gcnt > 1) {                                  // the group's shared a half, once per digit
+        const int item = a.grp_item[g0];
+        for (int j = 0; j < a.beta; j++) {
             u32 h[8];
-            chacha_coeffs<false>(key, key_id, (u32)j, (u32)t, (u32)(k0 >> 3), pi, h);
+            u32 *dst = sa + (size_t)j * 16 * ROW_THREADS + threadIdx.x;
+            chacha_coeffs<false>(a.key[item], a.key_id[item], (u32)j, (u32)t, (u32)(k0 >> 3), pi, h);
 #pragma unroll
-            for (int v = 0; v < 8; v++) av[v] = h[v];
-            chacha_coeffs<false>(key, key_id, (u32)j, (u32)t, (u32)(k0 >> 3) + 1u, pi, h);
+            for (int v = 0; v < 8; v++) dst[v * ROW_THREADS] = h[v];
+            chacha_coeffs<false>(a.key[item], a.key_id[item], (u32)j, (u32)t, (u32)(k0 >> 3) + 1u, pi, h);
 #pragma unroll
-            for (int v = 0; v < 8; v++) av[8 + v] = h[v];
+            for (int v = 0; v < 8; v++) dst[(8 + v) * ROW_THREADS] = h[v];
         }
+        __syncthreads();
+    }
+    for (int it = 0; it < gcnt; it++) {
+        const int item = a.grp_item[g0 + it];
+        const u32 *xb = a.x + item * a.x_item;
+        const u32 *cdb = a.cdig + item * a.cdig_item;
+        u32 *accb = a.acc + item * a.acc_item;
+        const u32 *bkey = a.b[item];
+        const u32 *astore = a.a_stored[item];
+        const u32 hoist_g = a.hoist_g[item], cdig_g = a.cdig_g[item];
+        // hoisted rotation: source row of this row under kappa_g
+        const int src_row = hoist_g ? (int)(automorph_src((u32)(row * 256), hoist_g, a.log_n) >> 8) : row;
+        u32 acc0[16], acc1[16];
+#pragma unroll
+        for (int v = 0; v < 16; v++) acc0[v] = acc1[v] = 0;
+        for (int j = 0; j < a.beta; j++) {
+            const bool in_digit = u < na && u >= j * a.alpha && u < min(j * a.alpha + a.alpha, na);
+            u32 x[16];
+            if (in_digit) {
+                const u32 *src = cdb + (size_t)u * n;
+                const u32 g = hoist_g ? hoist_g : cdig_g;
+                if (g) {
+#pragma unroll
+                    for (int v = 0; v < 16; v++) x[v] = src[automorph_src((u32)(k0 + v), g, a.log_n)];
+                } else {
+                    load16_vec(src + k0, x);
+                }
+            } else {
+                const u32 *src = xb + ((size_t)j * a.ext + u) * n + (size_t)src_row * 256;
+#pragma unroll
+                for (int v = 0; v < 16; v++) x[v] = src[lo + 16 * v];
+                row_fwd_regs(x, twf, R1 + (u32)src_row, lo, srow, q);
+                if (hoist_g) {        // permute inside the row: slot k takes source slot src(k)
+#pragma unroll
+                    for (int v = 0; v < 16; v++) srow[17 * lo + v] = x[v];
+                    __syncwarp();
+#pragma unroll
+                    for (int v = 0; v < 16; v++) {
+                        const u32 m = automorph_src((u32)(k0 + v), hoist_g, a.log_n) & 255u;
+                        x[v] = srow[m + (m >> 4)];
+                    }
+                    __syncwarp();
+                }
+            }
+            u32 bv[16], av[16];
+            load16_vec(bkey + ((size_t)j * a.n_primes + t) * n + k0, bv);
+            if (gcnt > 1) {
+                const u32 *src = sa + (size_t)j * 16 * ROW_THREADS + threadIdx.x;
+#pragma unroll
+                for (int v = 0; v < 16; v++) av[v] = src[v * ROW_THREADS];
+            } else if (astore) {
+                load16_vec(astore + ((size_t)j * a.n_primes + t) * n + k0, av);
+            } else {
+                u32 h[8];
+                chacha_coeffs<false>(a.key[item], a.key_id[item], (u32)j, (u32)t, (u32)(k0 >> 3), pi, h);
+#pragma unroll
+                for (int v = 0; v < 8; v++) av[v] = h[v];
+                chacha_coeffs<false>(a.key[item], a.key_id[item], (u32)j, (u32)t, (u32)(k0 >> 3) + 1u, pi, h);
+#pragma unroll
+                for (int v = 0; v < 8; v++) av[8 + v] = h[v];
+            }
+#pragma unroll
+            for (int v = 0; v < 16; v++) {
+                acc0[v] = csub(acc0[v] + mont_mul(x[v], bv[v], q, pi.qinv), two_q);
+                acc1[v] = csub(acc1[v] + mont_mul(x[v], av[v], q, pi.qinv), two_q);
+            }
+        }
+        // undo the Montgomery factor 2^-32
 #pragma unroll
         for (int v = 0; v < 16; v++) {
-            acc0[v] = csub(acc0[v] + mont_mul(x[v], bv[v], q, pi.qinv), two_q);
-            acc1[v] = csub(acc1[v] + mont_mul(x[v], av[v], q, pi.qinv), two_q);
+            acc0[v] = csub(shoup_mul(acc0[v], pi.r64, pi.r64p, q), q);
+            acc1[v] = csub(shoup_mul(acc1[v], pi.r64, pi.r64p, q), q);
         }
+        store16_vec(accb + (size_t)u * n + (size_t)row * 256 + 16 * lo, acc0);
+        store16_vec(accb + ((size_t)a.ext + u) * n + (size_t)row * 256 + 16 * lo, acc1);
     }
-    // undo the Montgomery factor 2^-32
-#pragma unroll
-    for (int v = 0; v < 16; v++) {
-        acc0[v] = shoup_mul(acc0[v], pi.r64, pi.r64p, q);
-        acc1[v] = shoup_mul(acc1[v], pi.r64, pi.r64p, q);
-    }
-    u32 *o0 = accb + (size_t)u * n + (size_t)row * 256;
-    u32 *o1 = accb + ((size_t)a.ext + u) * n + (size_t)row * 256;
-#pragma unroll
-    for (int v = 0; v < 16; v++) { acc0[v] = csub(acc0[v], q); acc1[v] = csub(acc1[v], q); }
-    store16_vec(o0 + 16 * lo, acc0);
-    store16_vec(o1 + 16 * lo, acc1);
 }
 
 // Last forward NTT pass of ModDown's converted limbs fused with the combine:

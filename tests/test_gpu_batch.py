@@ -101,3 +101,33 @@ def test_hoisted_across_chunks_matches_oracle(ks_lib, oracle_mod):
     for i in (0, 40, 64, 65):
         want = sc.ctx.rotate(ct, lvl, cfg.alpha, gs[i], keys_np[gs[i]], cfg.chacha_seed, gs[i])
         assert np.array_equal(got[i], want)
+
+
+def test_shared_key_groups(ks_lib):
+    """Items whose a half is the same (same seed and key id) share one regenerated keystream in
+    groups of up to 8; items with another seed, or a stored a half, do not.  Every item equals
+    the single call (which regenerates the keystream in registers)."""
+    ks = ks_lib
+    cfg, q, p, ctx = _setup(ks, "2")
+    lvl, N = cfg.level, cfg.n
+    na = lvl + 1
+    gen = W.rng(cfg.seed, W.TAG_SYNTH, 4242)
+    nd = -(-cfg.n_q // cfg.alpha)
+    shape = (nd, len(q) + len(p), N)
+    b1, b2, b3, b4, a4 = (_res((q + p) * nd, N, gen).view(*shape) for _ in range(5))
+    s1, s2 = bytes(range(32)), bytes(range(1, 33))
+    kid = 77
+    A = ks.make_evk(b1, s1, kid)            # shares its a half with A2 (same seed and key id)
+    A2 = ks.make_evk(b2, s1, kid)
+    Bk = ks.make_evk(b3, s2, kid)
+    S = ks.make_evk(b4, s1, kid, a=a4)      # stored a half: never grouped
+    n = 21
+    evks = [[A, A2, Bk][i % 3] for i in range(n - 1)] + [S]
+    c = _res(q[:na] * n, N, gen).view(n, na, N)
+    out = torch.empty((n, 2, na, N), dtype=torch.uint32, device="cuda")
+    one = torch.empty((2, na, N), dtype=torch.uint32, device="cuda")
+    ks.ckks_keyswitch_batch(ctx, c, lvl, evks, out, ctx.workspace(lvl, n))
+    ws_1 = ctx.workspace(lvl)
+    for i in range(n):
+        ks.ckks_keyswitch(ctx, c[i], lvl, evks[i], one, ws_1)
+        assert torch.equal(one, out[i]), i
