@@ -166,7 +166,8 @@ def ckks_ctx_create(log_n: int, q, p, dnum: int) -> Context:
 
 def make_evk(b, seed: bytes, key_id: int, a=None) -> ckks_evk:
     """Key-switching key record: b (and optionally a stored a) are CUDA tensors
-    [D][n_q+n_p][N]; the caller keeps them alive while the record is used."""
+    [D][n_q+n_p][N].  The record holds references to them, so their device memory stays
+    allocated for as long as the record exists (the C struct itself only carries pointers)."""
     k = ckks_evk()
     k.b = _ptr(b)
     k.a = _ptr(a) if a is not None else None
@@ -174,6 +175,7 @@ def make_evk(b, seed: bytes, key_id: int, a=None) -> ckks_evk:
         raise ValueError("seed must be 32 bytes")
     ctypes.memmove(k.seed, seed, 32)
     k.key_id = key_id
+    k._tensors = (b, a)
     return k
 
 

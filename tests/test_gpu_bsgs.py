@@ -79,6 +79,34 @@ def test_bsgs_parity_small(ks_lib):
     assert np.array_equal(got, want)
 
 
+def test_bsgs_parity_two_primes_per_digit(ks_lib):
+    """Config 1: dnum 2 (two primes per digit) and a single special prime."""
+    s = setup_for(ks_lib, "1")
+    lvl = s.cfg.level
+    baby = [1, s.sc.galois(1)]
+    giant = [1, s.sc.galois(2)]
+    _, ct = s.sc.ciphertext(0)
+    got, want = s.run(baby, giant, s.rand_pt(lvl, 2, 2, 15), ct, lvl)
+    assert np.array_equal(got, want)
+
+
+def test_evk_keeps_its_tensors_alive(ks_lib):
+    """A key record made from a temporary tensor keeps that device memory allocated."""
+    import gc
+    ks = ks_lib
+    s = setup_for(ks_lib, "1")
+    lvl, g = s.cfg.level, s.sc.galois(1)
+    b = s.sc.key(g)
+    evk = ks.make_evk(_dev(b), s.cfg.chacha_seed, g)      # no other reference to the tensor
+    gc.collect()
+    junk = [torch.full((b.size,), 7, dtype=torch.int32, device="cuda") for _ in range(4)]
+    _, ct = s.sc.ciphertext(0)
+    out = torch.empty((2, lvl + 1, s.cfg.n), dtype=torch.uint32, device="cuda")
+    ks.ckks_rotate(s.ctx, _dev(ct), lvl, g, evk, out, s.ctx.workspace(lvl))
+    assert np.array_equal(_host(out), s.sc.ctx.rotate(ct, lvl, s.cfg.alpha, g, b, s.cfg.chacha_seed, g))
+    del junk
+
+
 def test_bsgs_parity_identity_in_the_middle(ks_lib):
     """Identity steps at any position (the giant rotations then run as two batches)."""
     s = setup_for(ks_lib, "2")

@@ -207,7 +207,7 @@ def test_stored_a_ablation_parity(ks_lib):
     assert np.array_equal(_host(out), s.sc.ctx.rotate(ct, lvl, s.cfg.alpha, g, b, s.cfg.chacha_seed, g))
 
 
-@pytest.mark.parametrize("key,steps", [("1b", (1, -1, 3)), ("2", W.CONFIGS["2"].rot_steps)])
+@pytest.mark.parametrize("key,steps", [("1", (1, -1, 2)), ("1b", (1, -1, 3)), ("2", W.CONFIGS["2"].rot_steps)])
 def test_hoisted_parity(ks_lib, key, steps):
     ks = ks_lib
     s = setup_for(ks, key)
