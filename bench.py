@@ -381,9 +381,9 @@ def roofline(cfg, launches, total_ms, clk, batch, single_step_ms, launches_ov, t
 
 
 # DRAM bytes (read + write) per unit of a k_ip_row launch, from an ncu launch list of this
-# benchmark (4-unit launches; mean of 20: dram__bytes_read 392.07 MB + write 79.28 MB), scaled
+# benchmark (4-unit launches; mean of 20: dram__bytes_read 392.51 MB + write 78.97 MB), scaled
 # by the units a launch covers; None when the kernel changed after the capture.
-IP_ROW_TRAFFIC_PER_UNIT = 471.35e6 / 4
+IP_ROW_TRAFFIC_PER_UNIT = 471.48e6 / 4
 
 
 def step_bytes_min(cfg) -> int:
