@@ -288,15 +288,7 @@ def run_ours(args, rank, world, local_rank):
             "vs_baseline": None,
             "dtype": "u32",
             "data": "synthetic",
-            "config": {"workload": "config 3: N=2^16, 36+12 primes < 2^30, dnum 3, level 35; "
-                                   f"step = batch of {B} independent units, each tensor + relin + "
-                                   "rotate(1) with its own keys",
-                       "streams": f"{S} CUDA streams x {Bs} units",
-                       "log_n": cfg.log_n, "n_q": cfg.n_q, "n_p": cfg.n_p, "dnum": cfg.dnum,
-                       "level": lvl, "batch": B, "key_switches_per_step": KS_PER_UNIT * B,
-                       "key_a_half": "stored (ablation)" if args.stored_a else "regenerated by ChaCha12",
-                       "l2": f"{N_SETS} rotating input/key sets (each > 126 MB L2)",
-                       "parallelism": f"replicas x{world}"},
+            "config": workload_config(cfg, B, world, args.stored_a, f"{S} CUDA streams x {Bs} units"),
             "e2e": {"value": e2e_value, "unit": "key-switches/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": args.steps * LAUNCHES_PER_STEP * S,
@@ -612,6 +604,21 @@ def cpu_baseline(max_seconds: float = 20.0):
                       "on synthetic residues, plain C oracle with OpenMP over limbs"}
 
 
+def workload_config(cfg, batch: int, world: int, stored_a: bool = False, streams: str | None = None) -> dict:
+    """The benchmark workload, the same for both arms."""
+    c = {"workload": "config 3: N=2^16, 36+12 primes < 2^30, dnum 3, level 35; "
+                     f"step = batch of {batch} independent units, each tensor + relin + "
+                     "rotate(1) with its own keys",
+         "log_n": cfg.log_n, "n_q": cfg.n_q, "n_p": cfg.n_p, "dnum": cfg.dnum,
+         "level": cfg.level, "batch": batch, "key_switches_per_step": KS_PER_UNIT * batch,
+         "key_a_half": "stored (ablation)" if stored_a else "regenerated by ChaCha12",
+         "l2": f"{N_SETS} rotating input/key sets (each > 126 MB L2)",
+         "parallelism": f"replicas x{world}"}
+    if streams:
+        c["streams"] = streams
+    return c
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return
@@ -638,13 +645,13 @@ def run_reference(args, rank, world):
         "vs_baseline": None,
         "dtype": "u32",
         "data": "synthetic",
-        "config": {"workload": "config 3: N=2^16, 36+12 primes < 2^30, dnum 3, level 35; "
-                               "step = one unit: tensor + relin + rotate(1)",
-                   "log_n": cfg.log_n, "n_q": cfg.n_q, "n_p": cfg.n_p, "dnum": cfg.dnum,
-                   "level": cfg.level, "key_switches_per_step": KS_PER_UNIT},
+        "config": workload_config(cfg, args.batch, world),
         "cpu_baseline": {"kind": "oracle", "cores": _omp_threads(), "value": value,
                          "unit": "key-switches/s",
-                         "sample": f"{args.steps} timed steps of config 3 on the host cores"},
+                         "sample": f"{args.steps} timed steps, each a bounded sample of the workload: "
+                                   f"1 of its {args.batch} units (tensor + relin + rotate, "
+                                   f"{KS_PER_UNIT} key switches) on synthetic residues, plain C oracle "
+                                   "with OpenMP over limbs on the host cores"},
         "e2e": {"value": value, "unit": "key-switches/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
