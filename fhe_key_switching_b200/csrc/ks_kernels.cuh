@@ -160,7 +160,7 @@ k_bconv(BconvArgs a) {
         }
         const uint2 r = make_uint2(reduce64(s0, pi.q, pi.r64, pi.r64p, pi.onep),
                                    reduce64(s1, pi.q, pi.r64, pi.r64p, pi.onep));
-        reinterpret_cast<uint2 *>(a.out + ((size_t)g * a.map.out_group_rows + a.map.out_k_base + kk) * n)[c2] = r;
+        reinterpret_cast<uint2 *>(ob + ((size_t)g * a.map.out_group_rows + a.map.out_k_base + kk) * n)[c2] = r;
     }
 }
 
@@ -344,52 +344,6 @@ k_inner_product(IpArgs a) {
     o0[1] = make_uint4(r0[4], r0[5], r0[6], r0[7]);
     o1[0] = make_uint4(r1[0], r1[1], r1[2], r1[3]);
     o1[1] = make_uint4(r1[4], r1[5], r1[6], r1[7]);
-}
-
-// ---------------------------------------------------------------- ModDown combine
-// out_c[i] = (acc_c[i] - conv_c[i]) [P^-1]_{q_i} + add_c[i]   (mod q_i), c = 0, 1.
-// add: nullptr, or [2][l+1][N] rows (relinearisation), or component 0 only gathered through
-// kappa_{add_g} (rotation, add0_only).
-struct CombineArgs {
-    const u32 *acc;          // [2][ext][N]  (Q rows 0..l of each component used)
-    const u32 *conv;         // [2][l+1][N]
-    const u32 *add;          // see above
-    u32 *out;                // [2][l+1][N]
-    const PrimeInfo *pinfo;
-    const tw_t *pinv;        // [n_q] (P^-1 mod q_i, Shoup)
-    int log_n, level, ext;
-    int add_comps;           // 0, 1 (component 0 only) or 2
-    u32 add_g;               // gather add through kappa_g
-};
-
-__global__ void k_moddown_combine(CombineArgs a) {
-    const int n = 1 << a.log_n;
-    const int c4 = blockIdx.x * blockDim.x + threadIdx.x;    // 4 coefficients each
-    if (c4 >= n / 4) return;
-    const int i = blockIdx.y, comp = blockIdx.z;
-    const int na = a.level + 1;
-    const PrimeInfo pi = a.pinfo[i];
-    const u32 q = pi.q;
-    const tw_t w = a.pinv[i];
-    const uint4 av = reinterpret_cast<const uint4 *>(a.acc + ((size_t)comp * a.ext + i) * n)[c4];
-    const uint4 cv = reinterpret_cast<const uint4 *>(a.conv + ((size_t)comp * na + i) * n)[c4];
-    u32 r[4] = {av.x + q - cv.x, av.y + q - cv.y, av.z + q - cv.z, av.w + q - cv.w};
-#pragma unroll
-    for (int m = 0; m < 4; m++) r[m] = csub(shoup_mul(r[m], w.x, w.y, q), q);
-    if (comp < a.add_comps) {
-        const u32 *src = a.add + ((size_t)comp * na + i) * n;
-        u32 ad[4];
-        if (a.add_g) {
-#pragma unroll
-            for (int m = 0; m < 4; m++) ad[m] = src[automorph_src((u32)(4 * c4 + m), a.add_g, a.log_n)];
-        } else {
-            const uint4 t = reinterpret_cast<const uint4 *>(src)[c4];
-            ad[0] = t.x; ad[1] = t.y; ad[2] = t.z; ad[3] = t.w;
-        }
-#pragma unroll
-        for (int m = 0; m < 4; m++) r[m] = csub(r[m] + ad[m], q);
-    }
-    reinterpret_cast<uint4 *>(a.out + ((size_t)comp * na + i) * n)[c4] = make_uint4(r[0], r[1], r[2], r[3]);
 }
 
 // ---------------------------------------------------------------- tensor product

@@ -287,6 +287,31 @@ def test_extreme_dnum(ks_lib, oracle_mod, dnum):
         assert np.array_equal(_host(out), octx.moddown(acc, level))
 
 
+def test_extreme_dnum_batch(ks_lib, oracle_mod):
+    """dnum = 1: both base conversions use the generic kernel (digit of 36 primes, 24 special
+    primes).  A batch of 3 key switches with distinct keys equals the single calls, and item 0
+    equals the oracle."""
+    ks = ks_lib
+    log_n, n_q, n_p, dnum = 12, 36, 24, 1
+    q, p = ks.ckks_gen_primes(log_n, n_q, n_p)
+    octx = oracle_mod.Ctx(log_n, n_q, n_p)
+    ctx = ks.Context(log_n, q, p, dnum)
+    n, items = 1 << log_n, 3
+    seed = bytes(range(32))
+    for level in (35, 17):
+        keys = [_rand_limbs(q + p, n, 40 + 3 * level + i).reshape(1, n_q + n_p, n) for i in range(items)]
+        evks = [ks.make_evk(_dev(k), seed, 3 + 2 * i) for i, k in enumerate(keys)]
+        c = np.stack([_rand_limbs(q[: level + 1], n, 60 + 3 * level + i) for i in range(items)])
+        out = torch.empty((items, 2, level + 1, n), dtype=torch.uint32, device="cuda")
+        ks.ckks_keyswitch_batch(ctx, _dev(c), level, evks, out, ctx.workspace(level, items))
+        got = _host(out)
+        one = torch.empty((2, level + 1, n), dtype=torch.uint32, device="cuda")
+        for i in range(items):
+            ks.ckks_keyswitch(ctx, _dev(c[i]), level, evks[i], one, ctx.workspace(level))
+            assert np.array_equal(_host(one), got[i]), (level, i)
+        assert np.array_equal(got[0], octx.keyswitch(c[0], level, n_q, keys[0], seed, 3))
+
+
 def test_error_codes(ks_lib):
     ks = ks_lib
     s = setup_for(ks, "1")
