@@ -1,7 +1,7 @@
-"""Benchmark: RNS-CKKS hybrid key switching at N=2^16 (config 3) on B200.
+"""Benchmark: RNS-CKKS hybrid key switching at N=2^16, full level, on B200.
 
 One step = one pass of the whole key-switching path over one batch of B independent units
-of config 3 (default B = 8), each unit
+of the N=2^16 full-level workload (`n16-full`; default B = 8), each unit
   d   = tensor(x, y)            (ct x ct product, 36 limbs)
   r   = relin(d)                (key switch #1: ModUp, ChaCha12 inner product, ModDown)
   out = rotate(r, g = 5)        (automorphism + key switch #2)
@@ -35,7 +35,7 @@ if ROOT not in sys.path:
 
 import workloads as W  # noqa: E402
 
-CONFIG_KEY = "3"
+CONFIG_KEY = "n16-full"
 METRIC = "key-switches/s (rotations/s) at N=2^16, 32-bit RNS; % of HBM roofline"
 KS_PER_UNIT = 2          # relin + rotation
 ROT_PER_UNIT = 1
@@ -396,22 +396,25 @@ LAUNCHES_PER_STEP = 1 + 2 * 10
 
 def run_workload(args, local_rank):
     """Informational throughput (not the benchmark's headline line):
-    4 = 32 hoisted rotations of one ciphertext at level 24 (one ModUp, 32 keys);
-    5 = 64 pairs, each tensor + relin + rotate by 2^(i mod 15), level 20, dnum 4
+    n16-bsgs32 = 32 hoisted rotations of one ciphertext at level 24 (one ModUp, 32 keys);
+    n16-stream64 = 64 pairs, each tensor + relin + rotate by 2^(i mod 15), level 20, dnum 4
         (one relinearisation key, 15 rotation keys, all as batched calls);
-    5r = the same with a rescale after the relinearisation (rotation at level 19);
-    rescale = 64 rescales of level-35 ciphertexts at N=2^16 (config 3's chain) per step;
-    bsgs = one baby-step giant-step transform with config 4's 32 keys (baby steps 0..15, giant
-        steps 16 j for j = 0..17: 288 plaintext diagonals over the extended basis, level 24);
-    bsgs2 = the same transform shape on config 2's chain (N=2^14, level 11), a smaller case
-        whose plaintexts (302 MB) still exceed L2, for profiling."""
+    n16-stream64-rescale = the same with a rescale after the relinearisation (rotation at
+        level 19);
+    rescale = 64 rescales of level-35 ciphertexts on the N=2^16 full-level chain per step;
+    bsgs = one baby-step giant-step transform with n16-bsgs32's 32 keys (baby steps 0..15,
+        giant steps 16 j for j = 0..17: 288 plaintext diagonals over the extended basis,
+        level 24);
+    bsgs-n14 = the same transform shape on the N=2^14 chain (level 11), a smaller case whose
+        plaintexts (302 MB) still exceed L2, for profiling."""
     import torch
     import fhe_key_switching_b200 as ks
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     key = str(args.workload)
-    cfg = W.CONFIGS[{"5r": "5", "rescale": "3", "bsgs": "4", "bsgs2": "2"}.get(key, key)]
+    cfg = W.CONFIGS[{"n16-stream64-rescale": "n16-stream64", "rescale": "n16-full", "bsgs": "n16-bsgs32",
+                     "bsgs-n14": "n14-hoisted8"}.get(key, key)]
     n, lvl = cfg.n, cfg.level
     na = lvl + 1
     q, p = ks.ckks_gen_primes(cfg.log_n, cfg.n_q, cfg.n_p)
@@ -428,7 +431,7 @@ def run_workload(args, local_rank):
     keys_t = {r: res(mods * nd).view(nd, len(mods), n) for r in steps_g}
     evk = {r: ks.make_evk(keys_t[r], cfg.chacha_seed, gal[r]) for r in steps_g}
     stream = torch.cuda.current_stream(dev)
-    if key == "4":
+    if key == "n16-bsgs32":
         cts = [res(q[:na] * 2).view(2, na, n) for _ in range(N_SETS)]
         R = len(cfg.rot_steps)
         gs = [gal[r] for r in cfg.rot_steps]
@@ -439,7 +442,7 @@ def run_workload(args, local_rank):
         def step(i):
             ks.ckks_rotate_hoisted(ctx, cts[i % N_SETS], lvl, gs, ev, out, ws, stream)
         ks_per_step, rot_per_step = R, R
-    elif key == "5":
+    elif key == "n16-stream64":
         P_ = cfg.n_pairs
         xs = [res(q[:na] * 2 * P_).view(P_, 2, na, n) for _ in range(2)]
         ys = [res(q[:na] * 2 * P_).view(P_, 2, na, n) for _ in range(2)]
@@ -457,7 +460,7 @@ def run_workload(args, local_rank):
             ks.ckks_relin_batch(ctx, d, lvl, [k_rel] * P_, r1, ws, stream)
             ks.ckks_rotate_batch(ctx, r1, lvl, gs, ev, out, ws, stream)
         ks_per_step, rot_per_step = 2 * P_, P_
-    elif key == "5r":
+    elif key == "n16-stream64-rescale":
         P_ = cfg.n_pairs
         xs = [res(q[:na] * 2 * P_).view(P_, 2, na, n) for _ in range(2)]
         ys = [res(q[:na] * 2 * P_).view(P_, 2, na, n) for _ in range(2)]
@@ -486,7 +489,7 @@ def run_workload(args, local_rank):
         def step(i):
             ks.ckks_rescale_batch(ctx, R, cts[i % N_SETS], lvl, out, ws, stream)
         ks_per_step, rot_per_step = 0, 0
-    elif key in ("bsgs", "bsgs2"):
+    elif key in ("bsgs", "bsgs-n14"):
         n1, n2 = 16, 18
         baby = [1] + [ks.galois_element(cfg.log_n, k) for k in range(1, n1)]
         giant = [1] + [ks.galois_element(cfg.log_n, n1 * j) for j in range(1, n2)]
@@ -504,7 +507,8 @@ def run_workload(args, local_rank):
             ks.ckks_bsgs(ctx, cts[i % N_SETS], lvl, baby, bk, giant, gkk, pt, out, ws, stream)
         ks_per_step, rot_per_step = (n1 - 1) + (n2 - 1), (n1 - 1) + (n2 - 1)
     else:
-        raise SystemExit(f"--workload {key}: use 3 (default), 4, 5, 5r, rescale or bsgs")
+        raise SystemExit(f"--workload {key}: use n16-full (default), n16-bsgs32, n16-stream64, "
+                         "n16-stream64-rescale, rescale, bsgs or bsgs-n14")
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
@@ -512,7 +516,7 @@ def run_workload(args, local_rank):
     clocks.start()
     time.sleep(0.3)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if key in ("bsgs", "bsgs2"):
+    if key in ("bsgs", "bsgs-n14"):
         ks.ckks_prof_begin(ctx, "bsgs_combine", args.steps)
     e0.record(stream)
     for i in range(args.steps):
@@ -521,13 +525,13 @@ def run_workload(args, local_rank):
     torch.cuda.synchronize()
     clk = clocks.stop()
     ms = e0.elapsed_time(e1)
-    if key in ("bsgs", "bsgs2"):
+    if key in ("bsgs", "bsgs-n14"):
         launches, comb_ms = ks.ckks_prof_end(ctx)
         # compulsory bytes of one combine launch: every plaintext once, the 15 rotated babies'
         # accumulators and the input ciphertext once, the 18 giant sums written once
         b_comb = (n2 * n1 * ext + (n1 - 1) * 2 * ext + 2 * na + n2 * 2 * ext) * n * 4
         comb_s = comb_ms / max(launches, 1) / 1e3
-        print(json.dumps({"workload": f"bsgs: config {cfg.key} chain, N=2^{cfg.log_n}, {n1} baby x {n2} giant "
+        print(json.dumps({"workload": f"bsgs: {cfg.key} chain, N=2^{cfg.log_n}, {n1} baby x {n2} giant "
                                       f"steps, level {lvl}",
                           "informational": True, "transforms_per_s": args.steps / (ms / 1e3),
                           "ms_per_step": ms / args.steps, "steps": args.steps, "warmup": args.warmup,
@@ -550,7 +554,7 @@ def run_workload(args, local_rank):
                                   "peak_gbs": HBM_PEAK_GBS, "frac": b_min * per_s / 1e9 / HBM_PEAK_GBS},
                           "clocks": clk}), flush=True)
         return
-    print(json.dumps({"workload": f"config {key}", "informational": True,
+    print(json.dumps({"workload": key, "informational": True,
                       "key_switches_per_s": ks_per_step * args.steps / (ms / 1e3),
                       "rotations_per_s": rot_per_step * args.steps / (ms / 1e3),
                       "ms_per_step": ms / args.steps, "steps": args.steps, "warmup": args.warmup,
@@ -558,7 +562,7 @@ def run_workload(args, local_rank):
 
 
 def _oracle_sample():
-    """Bounded CPU sample of the same step: one relinearisation and one rotation at config 3,
+    """Bounded CPU sample of the same step: one relinearisation and one rotation of n16-full,
     timed on the oracle with synthetic residues (cost is data independent)."""
     import numpy as np
     import oracle
@@ -600,13 +604,14 @@ def cpu_baseline(max_seconds: float = 20.0):
     dt = time.perf_counter() - t0
     return {"value": KS_PER_UNIT * k / dt, "unit": "key-switches/s", "cores": _omp_threads(),
             "kind": "oracle",
-            "sample": f"{k} units of config 3 (tensor + relin + rotate, 2 key switches each) "
+            "sample": f"{k} units of the N=2^16 full-level workload (tensor + relin + rotate, "
+                      "2 key switches each) "
                       "on synthetic residues, plain C oracle with OpenMP over limbs"}
 
 
 def workload_config(cfg, batch: int, world: int, stored_a: bool = False, streams: str | None = None) -> dict:
     """The benchmark workload, the same for both arms."""
-    c = {"workload": "config 3: N=2^16, 36+12 primes < 2^30, dnum 3, level 35; "
+    c = {"workload": "n16-full: N=2^16, 36+12 primes < 2^30, dnum 3, level 35; "
                      f"step = batch of {batch} independent units, each tensor + relin + "
                      "rotate(1) with its own keys",
          "log_n": cfg.log_n, "n_q": cfg.n_q, "n_p": cfg.n_p, "dnum": cfg.dnum,
@@ -665,9 +670,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--batch", type=int, default=8, help="independent config-3 units per step")
-    ap.add_argument("--workload", default="3",
-                    help="3 (benchmark line), or 4 / 5 / 5r / rescale / bsgs / bsgs2 (informational lines)")
+    ap.add_argument("--batch", type=int, default=8, help="independent n16-full units per step")
+    ap.add_argument("--workload", default=CONFIG_KEY,
+                    help="n16-full (benchmark line), or n16-bsgs32 / n16-stream64 / n16-stream64-rescale / "
+                         "rescale / bsgs / bsgs-n14 (informational lines)")
     ap.add_argument("--streams", type=int, default=None,
                     help="CUDA streams the batch is split over, each running batch/streams units "
                          "(default 2 for an even batch, else 1)")
@@ -681,7 +687,7 @@ def main():
         args.warmup = min(args.warmup, 1)
         run_reference(args, rank, world)
         return
-    if str(args.workload) != "3":
+    if str(args.workload) != CONFIG_KEY:
         run_workload(args, local_rank)
         return
     run_ours(args, rank, world, local_rank)

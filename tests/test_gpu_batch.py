@@ -20,7 +20,7 @@ def _setup(ks, key):
     return cfg, q, p, ks.Context(cfg.log_n, q, p, cfg.dnum)
 
 
-@pytest.mark.parametrize("key,n", [("1", 5), ("2", 3), ("3", 2)])
+@pytest.mark.parametrize("key,n", [("n12-dnum2", 5), ("n14-hoisted8", 3), ("n16-full", 2)])
 def test_batches_equal_single_calls(ks_lib, key, n):
     ks = ks_lib
     cfg, q, p, ctx = _setup(ks, key)
@@ -63,7 +63,7 @@ def test_batches_equal_single_calls(ks_lib, key, n):
 def test_rotate_batch_longer_than_a_chunk(ks_lib):
     """70 rotations at N=2^12 (two launch chunks of at most 64 items)."""
     ks = ks_lib
-    cfg, q, p, ctx = _setup(ks, "1b")
+    cfg, q, p, ctx = _setup(ks, "n12-dnum4")
     lvl, N, na, n = cfg.level, cfg.n, cfg.level + 1, 70
     gen = W.rng(cfg.seed, W.TAG_SYNTH, 77)
     nd = -(-cfg.n_q // cfg.alpha)
@@ -84,7 +84,7 @@ def test_hoisted_across_chunks_matches_oracle(ks_lib, oracle_mod):
     """Hoisted rotations spanning two chunks equal the oracle (sampled rotations)."""
     from oracle.scenario import Scenario
     ks = ks_lib
-    cfg = W.CONFIGS["1b"]
+    cfg = W.CONFIGS["n12-dnum4"]
     sc = Scenario(cfg)
     q, p = ks.ckks_gen_primes(cfg.log_n, cfg.n_q, cfg.n_p)
     ctx = ks.Context(cfg.log_n, q, p, cfg.dnum)
@@ -108,7 +108,7 @@ def test_shared_key_groups(ks_lib):
     groups of up to 8; items with another seed, or a stored a half, do not.  Every item equals
     the single call (which regenerates the keystream in registers)."""
     ks = ks_lib
-    cfg, q, p, ctx = _setup(ks, "2")
+    cfg, q, p, ctx = _setup(ks, "n14-hoisted8")
     lvl, N = cfg.level, cfg.n
     na = lvl + 1
     gen = W.rng(cfg.seed, W.TAG_SYNTH, 4242)

@@ -70,7 +70,7 @@ def setup_for(ks, key):
 
 
 def test_bsgs_parity_small(ks_lib):
-    s = setup_for(ks_lib, "1b")
+    s = setup_for(ks_lib, "n12-dnum4")
     lvl = s.cfg.level
     baby = [1] + [s.sc.galois(k) for k in (1, 2, 3)]
     giant = [1, s.sc.galois(4), s.sc.galois(8)]
@@ -80,8 +80,8 @@ def test_bsgs_parity_small(ks_lib):
 
 
 def test_bsgs_parity_two_primes_per_digit(ks_lib):
-    """Config 1: dnum 2 (two primes per digit) and a single special prime."""
-    s = setup_for(ks_lib, "1")
+    """n12-dnum2: dnum 2 (two primes per digit) and a single special prime."""
+    s = setup_for(ks_lib, "n12-dnum2")
     lvl = s.cfg.level
     baby = [1, s.sc.galois(1)]
     giant = [1, s.sc.galois(2)]
@@ -94,7 +94,7 @@ def test_evk_keeps_its_tensors_alive(ks_lib):
     """A key record made from a temporary tensor keeps that device memory allocated."""
     import gc
     ks = ks_lib
-    s = setup_for(ks_lib, "1")
+    s = setup_for(ks_lib, "n12-dnum2")
     lvl, g = s.cfg.level, s.sc.galois(1)
     b = s.sc.key(g)
     evk = ks.make_evk(_dev(b), s.cfg.chacha_seed, g)      # no other reference to the tensor
@@ -109,7 +109,7 @@ def test_evk_keeps_its_tensors_alive(ks_lib):
 
 def test_bsgs_parity_identity_in_the_middle(ks_lib):
     """Identity steps at any position (the giant rotations then run as two batches)."""
-    s = setup_for(ks_lib, "2")
+    s = setup_for(ks_lib, "n14-hoisted8")
     lvl = s.cfg.level
     baby = [s.sc.galois(1), s.sc.galois(2), 1, s.sc.galois(3)]
     giant = [s.sc.galois(4), 1, s.sc.galois(8)]
@@ -120,7 +120,7 @@ def test_bsgs_parity_identity_in_the_middle(ks_lib):
 
 def test_bsgs_parity_more_than_16_babies(ks_lib):
     """20 baby steps: the plaintext sums run in two launches, carrying partial sums."""
-    s = setup_for(ks_lib, "1b")
+    s = setup_for(ks_lib, "n12-dnum4")
     lvl = s.cfg.level
     baby = [1] + [s.sc.galois(k) for k in range(1, 20)]
     giant = [1, s.sc.galois(20)]
@@ -132,7 +132,7 @@ def test_bsgs_parity_more_than_16_babies(ks_lib):
 def test_bsgs_decode(ks_lib):
     """Encoded diagonals: the GPU result decodes to sum_i d_i * rot_i(z)."""
     from oracle import encode
-    s = setup_for(ks_lib, "2")
+    s = setup_for(ks_lib, "n14-hoisted8")
     sc, ctx, lvl, n = s.sc, s.sc.ctx, s.cfg.level, s.cfg.n
     z, ct = sc.ciphertext(0)
     n1, n2 = 4, 3
@@ -150,10 +150,10 @@ def test_bsgs_decode(ks_lib):
 
 
 @pytest.mark.slow
-def test_bsgs_parity_config4_full(ks_lib):
-    """Config 4's 32 rotation keys as one transform: baby steps 0..15, giant steps 16 j for
+def test_bsgs_parity_n16_bsgs32_full(ks_lib):
+    """n16-bsgs32's 32 rotation keys as one transform: baby steps 0..15, giant steps 16 j for
     j = 0..17 (288 diagonals), level 24, random plaintexts over the extended basis."""
-    s = setup_for(ks_lib, "4")
+    s = setup_for(ks_lib, "n16-bsgs32")
     lvl = s.cfg.level
     baby = [1] + [s.sc.galois(k) for k in range(1, 16)]
     giant = [1] + [s.sc.galois(16 * j) for j in range(1, 18)]
@@ -164,7 +164,7 @@ def test_bsgs_parity_config4_full(ks_lib):
 
 def test_bsgs_errors(ks_lib):
     ks = ks_lib
-    s = setup_for(ks, "1")
+    s = setup_for(ks, "n12-dnum2")
     lvl, n = s.cfg.level, s.cfg.n
     ct = torch.zeros((2, lvl + 1, n), dtype=torch.uint32, device="cuda")
     out = torch.empty_like(ct)

@@ -15,7 +15,7 @@ torch = pytest.importorskip("torch")
 def test_wait_expiry_is_reported_and_context_survives(ks_lib):
     from oracle.scenario import Scenario
     ks = ks_lib
-    cfg = W.CONFIGS["1"]
+    cfg = W.CONFIGS["n12-dnum2"]
     sc = Scenario(cfg)
     q, p = ks.ckks_gen_primes(cfg.log_n, cfg.n_q, cfg.n_p)
     ctx = ks.Context(cfg.log_n, q, p, cfg.dnum)

@@ -93,7 +93,7 @@ def test_ntt_parity(ks_lib, oracle_mod, log_n):
 
 def test_automorph_parity(ks_lib, oracle_mod):
     ks = ks_lib
-    s = setup_for(ks, "2")
+    s = setup_for(ks, "n14-hoisted8")
     n = s.cfg.n
     a = _rand_limbs(s.sc.ctx.q[:3], n, 3)
     out = torch.empty_like(_dev(a))
@@ -104,7 +104,7 @@ def test_automorph_parity(ks_lib, oracle_mod):
 
 def test_chacha_expand_parity(ks_lib):
     ks = ks_lib
-    s = setup_for(ks, "3")
+    s = setup_for(ks, "n16-full")
     out = torch.empty(s.cfg.n, dtype=torch.uint32, device="cuda")
     for (kid, j, t) in [(0, 0, 0), (5, 2, 47), (2**32 - 1, 1, 36)]:
         ks.ckks_chacha_expand(s.ctx, s.cfg.chacha_seed, kid, j, t, out)
@@ -113,7 +113,7 @@ def test_chacha_expand_parity(ks_lib):
 
 # ----------------------------------------------------------------------------- steps
 
-@pytest.mark.parametrize("key,level", [("1", 3), ("1", 0), ("1b", 2), ("2", 11), ("2", 6), ("3", 35), ("4", 24), ("5", 20)])
+@pytest.mark.parametrize("key,level", [("n12-dnum2", 3), ("n12-dnum2", 0), ("n12-dnum4", 2), ("n14-hoisted8", 11), ("n14-hoisted8", 6), ("n16-full", 35), ("n16-bsgs32", 24), ("n16-stream64", 20)])
 def test_modup_parity(ks_lib, key, level):
     ks = ks_lib
     s = setup_for(ks, key)
@@ -127,7 +127,7 @@ def test_modup_parity(ks_lib, key, level):
     assert np.array_equal(_host(dt), s.sc.ctx.modup(c, level, s.cfg.alpha))
 
 
-@pytest.mark.parametrize("key,level", [("1", 3), ("2", 11), ("2", 4), ("3", 35), ("5", 20)])
+@pytest.mark.parametrize("key,level", [("n12-dnum2", 3), ("n14-hoisted8", 11), ("n14-hoisted8", 4), ("n16-full", 35), ("n16-stream64", 20)])
 def test_inner_product_parity(ks_lib, key, level):
     ks = ks_lib
     s = setup_for(ks, key)
@@ -146,7 +146,7 @@ def test_inner_product_parity(ks_lib, key, level):
         assert np.array_equal(got[0], a0) and np.array_equal(got[1], a1)
 
 
-@pytest.mark.parametrize("key,level", [("1", 3), ("2", 11), ("3", 35), ("3", 0), ("5", 20)])
+@pytest.mark.parametrize("key,level", [("n12-dnum2", 3), ("n14-hoisted8", 11), ("n16-full", 35), ("n16-full", 0), ("n16-stream64", 20)])
 def test_moddown_parity(ks_lib, key, level):
     ks = ks_lib
     s = setup_for(ks, key)
@@ -161,7 +161,7 @@ def test_moddown_parity(ks_lib, key, level):
 
 def test_tensor_parity(ks_lib):
     ks = ks_lib
-    s = setup_for(ks, "2")
+    s = setup_for(ks, "n14-hoisted8")
     _, x = s.sc.ciphertext(0)
     _, y = s.sc.ciphertext(1)
     d = torch.empty((3,) + x.shape[1:], dtype=torch.uint32, device="cuda")
@@ -171,7 +171,7 @@ def test_tensor_parity(ks_lib):
 
 # ----------------------------------------------------------------------------- composites
 
-@pytest.mark.parametrize("key", ["1", "1b", "2", "3"])
+@pytest.mark.parametrize("key", ["n12-dnum2", "n12-dnum4", "n14-hoisted8", "n16-full"])
 def test_rotate_relin_parity(ks_lib, key):
     ks = ks_lib
     s = setup_for(ks, key)
@@ -197,7 +197,7 @@ def test_rotate_relin_parity(ks_lib, key):
 
 def test_stored_a_ablation_parity(ks_lib):
     ks = ks_lib
-    s = setup_for(ks, "2")
+    s = setup_for(ks, "n14-hoisted8")
     lvl = s.cfg.level
     _, ct = s.sc.ciphertext(0)
     g = s.sc.galois(1)
@@ -207,7 +207,7 @@ def test_stored_a_ablation_parity(ks_lib):
     assert np.array_equal(_host(out), s.sc.ctx.rotate(ct, lvl, s.cfg.alpha, g, b, s.cfg.chacha_seed, g))
 
 
-@pytest.mark.parametrize("key,steps", [("1", (1, -1, 2)), ("1b", (1, -1, 3)), ("2", W.CONFIGS["2"].rot_steps)])
+@pytest.mark.parametrize("key,steps", [("n12-dnum2", (1, -1, 2)), ("n12-dnum4", (1, -1, 3)), ("n14-hoisted8", W.CONFIGS["n14-hoisted8"].rot_steps)])
 def test_hoisted_parity(ks_lib, key, steps):
     ks = ks_lib
     s = setup_for(ks, key)
@@ -221,11 +221,11 @@ def test_hoisted_parity(ks_lib, key, steps):
     assert np.array_equal(_host(out), want)
 
 
-def test_config4_hoisted_sampled(ks_lib):
-    """Config 4 (32 hoisted rotations at level 24, dnum 4): the GPU runs the full batch of 32;
+def test_n16_bsgs32_hoisted_sampled(ks_lib):
+    """n16-bsgs32 (32 hoisted rotations at level 24, dnum 4): the GPU runs the full batch of 32;
     the oracle recomputes a sample of 3 rotations (each output depends only on its own key)."""
     ks = ks_lib
-    s = setup_for(ks, "4")
+    s = setup_for(ks, "n16-bsgs32")
     cfg, lvl = s.cfg, s.cfg.level
     _, ct = s.sc.ciphertext(0)
     gs = [s.sc.galois(r) for r in cfg.rot_steps]
@@ -238,11 +238,11 @@ def test_config4_hoisted_sampled(ks_lib):
         assert np.array_equal(got[i], want)
 
 
-def test_config5_pipeline_sampled(ks_lib):
-    """Config 5 (tensor + relin + rotate by 2^(i mod 15) at level 20, dnum 4) on a sample of
+def test_n16_stream64_pipeline_sampled(ks_lib):
+    """n16-stream64 (tensor + relin + rotate by 2^(i mod 15) at level 20, dnum 4) on a sample of
     pairs; every pair is independent."""
     ks = ks_lib
-    s = setup_for(ks, "5")
+    s = setup_for(ks, "n16-stream64")
     cfg, lvl = s.cfg, s.cfg.level
     ws = s.ctx.workspace(lvl)
     na = lvl + 1
@@ -314,7 +314,7 @@ def test_extreme_dnum_batch(ks_lib, oracle_mod):
 
 def test_error_codes(ks_lib):
     ks = ks_lib
-    s = setup_for(ks, "1")
+    s = setup_for(ks, "n12-dnum2")
     lvl, n = s.cfg.level, s.cfg.n
     ct = torch.zeros((2, lvl + 1, n), dtype=torch.uint32, device="cuda")
     out = torch.empty_like(ct)

@@ -49,7 +49,7 @@ def setup_for(ks, key):
     return _S[key]
 
 
-@pytest.mark.parametrize("key,level", [("1", 3), ("1", 1), ("2", 11), ("2", 5), ("3", 35), ("3", 1), ("5", 20)])
+@pytest.mark.parametrize("key,level", [("n12-dnum2", 3), ("n12-dnum2", 1), ("n14-hoisted8", 11), ("n14-hoisted8", 5), ("n16-full", 35), ("n16-full", 1), ("n16-stream64", 20)])
 def test_rescale_parity(ks_lib, key, level):
     ks = ks_lib
     s = setup_for(ks, key)
@@ -60,7 +60,7 @@ def test_rescale_parity(ks_lib, key, level):
     assert np.array_equal(_host(out), s.sc.ctx.rescale(ct, level))
 
 
-@pytest.mark.parametrize("key,level,n", [("2", 11, 3), ("1", 2, 66)])
+@pytest.mark.parametrize("key,level,n", [("n14-hoisted8", 11, 3), ("n12-dnum2", 2, 66)])
 def test_rescale_batch_parity(ks_lib, key, level, n):
     """Every item equals the oracle; 66 items cross the 64-item launch chunk."""
     ks = ks_lib
@@ -74,7 +74,7 @@ def test_rescale_batch_parity(ks_lib, key, level, n):
         assert np.array_equal(got[z], s.sc.ctx.rescale(ct[z], level)), z
 
 
-@pytest.mark.parametrize("key", ["1b", "2"])
+@pytest.mark.parametrize("key", ["n12-dnum4", "n14-hoisted8"])
 def test_mul_relin_rescale_chain(ks_lib, key):
     """tensor -> relin -> rescale on the GPU equals the oracle chain and decodes to z1*z2."""
     ks = ks_lib
@@ -98,7 +98,7 @@ def test_mul_relin_rescale_chain(ks_lib, key):
     assert np.abs(s.sc.decrypt_slots(got, level=lvl - 1, scale=scale) - z1 * z2).max() < 2.0 ** -9
 
 
-@pytest.mark.parametrize("key", ["1b", "2", "3"])
+@pytest.mark.parametrize("key", ["n12-dnum4", "n14-hoisted8", "n16-full"])
 def test_conjugation_parity(ks_lib, key):
     ks = ks_lib
     s = setup_for(ks, key)
@@ -111,14 +111,14 @@ def test_conjugation_parity(ks_lib, key):
     ks.ckks_rotate(s.ctx, _dev(ct), lvl, g, evk, out, s.ctx.workspace(lvl))
     got = _host(out)
     assert np.array_equal(got, s.sc.ctx.rotate(ct, lvl, s.cfg.alpha, g, b, s.cfg.chacha_seed, g))
-    if key != "3":
+    if key != "n16-full":
         assert np.abs(s.sc.decrypt_slots(got) - np.conj(z)).max() < 2.0 ** -9.5
 
 
 def test_conjugation_in_hoisted_batch(ks_lib):
     """Conjugation hoisted together with rotations equals the single calls."""
     ks = ks_lib
-    s = setup_for(ks, "2")
+    s = setup_for(ks, "n14-hoisted8")
     lvl, n = s.cfg.level, s.cfg.n
     gs = [s.sc.galois(1), ks.conjugation_element(s.cfg.log_n), s.sc.galois(-2)]
     keys = [s.evk(g) for g in gs]
@@ -134,7 +134,7 @@ def test_conjugation_in_hoisted_batch(ks_lib):
 
 def test_rescale_errors(ks_lib):
     ks = ks_lib
-    s = setup_for(ks, "1")
+    s = setup_for(ks, "n12-dnum2")
     lvl, n = s.cfg.level, s.cfg.n
     ct = torch.zeros((2, lvl + 1, n), dtype=torch.uint32, device="cuda")
     out = torch.empty((2, lvl, n), dtype=torch.uint32, device="cuda")

@@ -30,7 +30,7 @@ def _ones(ctx, level, n_giant, n_baby, at):
 
 @pytest.fixture(scope="module")
 def sc1b():
-    return Scenario(W.CONFIGS["1b"])
+    return Scenario(W.CONFIGS["n12-dnum4"])
 
 
 def _keys(sc, gs):
@@ -64,9 +64,9 @@ def test_bsgs_single_diagonal_is_rotation(sc1b, j, k):
 
 
 def test_bsgs_decode():
-    """A 12-diagonal transform (baby 0..3, giant 0, 4, 8) on config 2 decodes to
+    """A 12-diagonal transform (baby 0..3, giant 0, 4, 8) on n14-hoisted8 decodes to
     sum_i d_i * rot_i(z); the plaintexts are the diagonals pre-rotated by -G_j."""
-    sc = Scenario(W.CONFIGS["2"])
+    sc = Scenario(W.CONFIGS["n14-hoisted8"])
     ctx, lvl, n = sc.ctx, sc.level, sc.n
     z, ct = sc.ciphertext(0)
     n1, n2 = 4, 3
@@ -85,7 +85,7 @@ def test_bsgs_decode():
     want = sum(d[i] * np.roll(z, -i) for i in range(n1 * n2))
     err = np.abs(sc.decrypt_slots(out, scale=sc.scale * scale_p) - want).max()
     # each of the 12 terms carries one rotation's key-switching noise (max about 2^-10.3 at
-    # config 2); their sum stays below 2^-7.5, while a misplaced diagonal errs by order 1
+    # n14-hoisted8); their sum stays below 2^-7.5, while a misplaced diagonal errs by order 1
     assert err < 2.0 ** -7.5
     # the same plaintexts without the -G_j pre-rotation give a different transform
     assert np.abs(sc.decrypt_slots(out, scale=sc.scale * scale_p)

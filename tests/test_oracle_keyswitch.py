@@ -3,7 +3,8 @@ the tensor product: decryption identities and decoding against the plaintext slo
 
 Decoding tolerances come from the key-switching noise model
   std(slot error) ~ sqrt(N) * sqrt(N) * sigma * sqrt(beta) * (D_j / P) / Delta,
-which gives max errors of about 2^-10 at configs 1b and 2 and about 2^-8 at N=2^16 (config 3);
+which gives max errors of about 2^-10 at n12-dnum4 and n14-hoisted8 and about 2^-8 at N=2^16
+(n16-full);
 a wrong sign, term or index anywhere in the pipeline gives errors of order 1 or larger.
 """
 import numpy as np
@@ -21,7 +22,7 @@ def _noise(ctx, vals, level):
 
 @pytest.fixture(scope="module")
 def sc1b():
-    return Scenario(W.CONFIGS["1b"])
+    return Scenario(W.CONFIGS["n12-dnum4"])
 
 
 def test_keyswitch_identity(sc1b):
@@ -60,7 +61,7 @@ def test_stored_a_equals_regenerated(sc1b):
     assert np.array_equal(o1, o2)
 
 
-@pytest.mark.parametrize("key,tol", [("1b", 2.0 ** -9.5), ("2", 2.0 ** -9.5)])
+@pytest.mark.parametrize("key,tol", [("n12-dnum4", 2.0 ** -9.5), ("n14-hoisted8", 2.0 ** -9.5)])
 def test_rotations_decode(key, tol):
     sc = Scenario(W.CONFIGS[key])
     z, ct = sc.ciphertext(0)
@@ -70,7 +71,7 @@ def test_rotations_decode(key, tol):
         assert np.abs(sc.decrypt_slots(out) - np.roll(z, -r)).max() < tol
 
 
-@pytest.mark.parametrize("key", ["1b", "2"])
+@pytest.mark.parametrize("key", ["n12-dnum4", "n14-hoisted8"])
 def test_hoisted_decode_and_equals_single(key):
     """With centred fast base conversion, BConv(-x) = -BConv(x) coefficient-wise, and kappa_g
     only permutes coefficients with sign changes, so ModUp commutes with kappa_g: hoisted and
@@ -88,7 +89,7 @@ def test_hoisted_decode_and_equals_single(key):
         assert np.array_equal(single, out[i])
 
 
-@pytest.mark.parametrize("key", ["1b", "2"])
+@pytest.mark.parametrize("key", ["n12-dnum4", "n14-hoisted8"])
 def test_tensor_relin_decode(key):
     sc = Scenario(W.CONFIGS[key])
     z1, x = sc.ciphertext(0)
@@ -100,10 +101,10 @@ def test_tensor_relin_decode(key):
     assert np.abs(sc.decrypt_slots(out, scale=sc.scale ** 2) - z1 * z2).max() < 2.0 ** -9.5
 
 
-def test_config1_dnum2_noise_is_large():
-    """Config 1 (dnum=2, one special prime): P ~ 2^30 << D_j ~ 2^60, so the output is bit-exact
+def test_n12_dnum2_noise_is_large():
+    """n12-dnum2 (dnum=2, one special prime): P ~ 2^30 << D_j ~ 2^60, so the output is bit-exact
     material only; its decode error is far above 2^-10 (recorded, not a failure)."""
-    sc = Scenario(W.CONFIGS["1"])
+    sc = Scenario(W.CONFIGS["n12-dnum2"])
     z, ct = sc.ciphertext(0)
     g = sc.galois(1)
     out = sc.ctx.rotate(ct, sc.level, sc.alpha, g, sc.key(g), sc.seed_bytes, g)
@@ -111,8 +112,8 @@ def test_config1_dnum2_noise_is_large():
 
 
 @pytest.mark.slow
-def test_config3_rotation_relin_decode():
-    sc = Scenario(W.CONFIGS["3"])
+def test_n16_full_rotation_relin_decode():
+    sc = Scenario(W.CONFIGS["n16-full"])
     z1, x = sc.ciphertext(0)
     g = sc.galois(1)
     out = sc.ctx.rotate(x, sc.level, sc.alpha, g, sc.key(g), sc.seed_bytes, g)

@@ -26,7 +26,7 @@ def _coef_ints(ctx, limbs, n_limbs):
 
 @pytest.fixture(scope="module")
 def sc1b():
-    return Scenario(W.CONFIGS["1b"])
+    return Scenario(W.CONFIGS["n12-dnum4"])
 
 
 @pytest.mark.parametrize("level", [3, 2, 1])
@@ -67,7 +67,7 @@ def test_rescale_centred_not_unsigned(sc1b):
         assert not got[i, 1:].any()
 
 
-@pytest.mark.parametrize("key,tol", [("1b", 2.0 ** -9), ("2", 2.0 ** -13)])
+@pytest.mark.parametrize("key,tol", [("n12-dnum4", 2.0 ** -9), ("n14-hoisted8", 2.0 ** -13)])
 def test_tensor_relin_rescale_decode(key, tol):
     sc = Scenario(W.CONFIGS[key])
     ctx, lvl = sc.ctx, sc.level
@@ -83,7 +83,7 @@ def test_tensor_relin_rescale_decode(key, tol):
     assert np.abs(sc.decrypt_slots(out, level=lvl - 1, scale=sc.scale ** 2) - z1 * z2).max() > 0.1
 
 
-@pytest.mark.parametrize("key", ["1b", "2"])
+@pytest.mark.parametrize("key", ["n12-dnum4", "n14-hoisted8"])
 def test_conjugation_decode(key):
     sc = Scenario(W.CONFIGS[key])
     g = 2 * sc.n - 1

@@ -23,7 +23,7 @@ def _residues(moduli, n, gen):
     return torch.from_numpy(W.uniform_residues(moduli, n, gen)).cuda()
 
 
-@pytest.mark.parametrize("key", ["1", "2"])
+@pytest.mark.parametrize("key", ["n12-dnum2", "n14-hoisted8"])
 def test_noalloc_matches_keyswitch_twice(ks_lib, key):
     ks = ks_lib
     cfg = W.CONFIGS[key]
@@ -48,7 +48,7 @@ def test_noalloc_matches_keyswitch_twice(ks_lib, key):
 
 def test_noalloc_rejects_oversized(ks_lib):
     ks = ks_lib
-    cfg = W.CONFIGS["3"]
+    cfg = W.CONFIGS["n16-full"]
     q, p = ks.ckks_gen_primes(cfg.log_n, cfg.n_q, cfg.n_p)
     ctx = ks.Context(cfg.log_n, q, p, cfg.dnum)
     assert ctx.workspace_bytes(cfg.level) > ks.NOALLOC_SCRATCH_BYTES

@@ -6,20 +6,20 @@ errors, encryption randomness, message slots, synthetic residues).  It holds non
 method's arithmetic: no modular reduction of method data, no NTT, no key derivation.  Both the
 oracle and the CUDA library compute everything else on their own.
 
-Configurations (the parameter sets of the key-switching workloads):
+Workloads (named by ring size and shape):
 
-* ``1``  -- N=2^12, 4 ciphertext primes + 1 special prime, dnum=2, h=64, scale 2^25,
+* ``n12-dnum2``    -- N=2^12, 4 ciphertext primes + 1 special prime, dnum=2, h=64, scale 2^25,
   one rotation by 1 and one relinearisation.
-* ``1b`` -- config 1's chain with dnum=4 (one prime per digit).  With dnum=2 and a single
-  special prime P ~ 2^30 is far below the digit modulus ~ 2^60, so config 1 cannot decrypt to
-  2^-10; 1b carries the decode-accuracy check on the same chain.
-* ``2``  -- N=2^14, 12 + 4 primes, dnum=3, scale 2^28; 8 hoisted rotations (+-1, +-2, +-4, +-8)
-  and one ct x ct multiply then relinearisation.
-* ``3``  -- N=2^16, 36 + 12 primes, dnum=3, h=192, scale 2^28; a single rotation and a single
-  relinearisation at full level.
-* ``4``  -- N=2^16 (config 3's chain) at level 24 with dnum=4: 32 hoisted rotations of one
+* ``n12-dnum4``    -- the same chain with dnum=4 (one prime per digit).  With dnum=2 a single
+  special prime P ~ 2^30 is far below the digit modulus ~ 2^60, so n12-dnum2 cannot decrypt
+  to 2^-10; n12-dnum4 carries the decode-accuracy check on the same chain.
+* ``n14-hoisted8`` -- N=2^14, 12 + 4 primes, dnum=3, scale 2^28; 8 hoisted rotations
+  (+-1, +-2, +-4, +-8) and one ct x ct multiply then relinearisation.
+* ``n16-full``     -- N=2^16, 36 + 12 primes, dnum=3, h=192, scale 2^28; a single rotation and a
+  single relinearisation at full level (35).
+* ``n16-bsgs32``   -- the N=2^16 chain at level 24 with dnum=4: 32 hoisted rotations of one
   ciphertext, baby steps 1..16 and giant steps 16*k for k=2..17 (32 distinct keys).
-* ``5``  -- N=2^16 (config 3's chain) at level 20 with dnum=4: 64 independent ct x ct tensor
+* ``n16-stream64`` -- the N=2^16 chain at level 20 with dnum=4: 64 independent ct x ct tensor
   products, each relinearised and then rotated by 2^(i mod 15); slots Gaussian sigma=1
   clipped to [-4, 4].
 """
@@ -45,9 +45,9 @@ class Config:
     slots: str            # "uniform" or "gauss_clip4"
     rot_steps: tuple = ()          # rotation steps (slot shift r; negative = right)
     hoisted: bool = False          # rotations share one ModUp
-    n_pairs: int = 0               # config 5: number of independent ct x ct pairs
+    n_pairs: int = 0               # number of independent ct x ct pairs (n16-stream64)
     relin: bool = True
-    seed: int = 0                  # RNG seed = 1000 + config index
+    seed: int = 0                  # RNG seed of the workload's draws
 
     @property
     def n(self) -> int:
@@ -63,27 +63,27 @@ class Config:
         return chacha_seed(self.key)
 
 
-def _c5_steps() -> tuple:
+def _stream_steps() -> tuple:
     return tuple(1 << (i % 15) for i in range(64))
 
 
 CONFIGS = {
-    "1": Config("1", 12, 4, 1, 2, 3, 64, 3.2, 25, "uniform", rot_steps=(1,), seed=1001),
-    "1b": Config("1b", 12, 4, 1, 4, 3, 64, 3.2, 25, "uniform", rot_steps=(1,), seed=1011),
-    "2": Config("2", 14, 12, 4, 3, 11, 192, 3.2, 28, "uniform",
-                rot_steps=(1, -1, 2, -2, 4, -4, 8, -8), hoisted=True, seed=1002),
-    "3": Config("3", 16, 36, 12, 3, 35, 192, 3.2, 28, "uniform", rot_steps=(1,), seed=1003),
-    "4": Config("4", 16, 36, 12, 4, 24, 192, 3.2, 28, "uniform",
-                rot_steps=tuple(range(1, 17)) + tuple(16 * k for k in range(2, 18)),
-                hoisted=True, relin=False, seed=1004),
-    "5": Config("5", 16, 36, 12, 4, 20, 192, 3.2, 28, "gauss_clip4",
-                rot_steps=_c5_steps(), n_pairs=64, seed=1005),
+    "n12-dnum2": Config("n12-dnum2", 12, 4, 1, 2, 3, 64, 3.2, 25, "uniform", rot_steps=(1,), seed=1001),
+    "n12-dnum4": Config("n12-dnum4", 12, 4, 1, 4, 3, 64, 3.2, 25, "uniform", rot_steps=(1,), seed=1011),
+    "n14-hoisted8": Config("n14-hoisted8", 14, 12, 4, 3, 11, 192, 3.2, 28, "uniform",
+                           rot_steps=(1, -1, 2, -2, 4, -4, 8, -8), hoisted=True, seed=1002),
+    "n16-full": Config("n16-full", 16, 36, 12, 3, 35, 192, 3.2, 28, "uniform", rot_steps=(1,), seed=1003),
+    "n16-bsgs32": Config("n16-bsgs32", 16, 36, 12, 4, 24, 192, 3.2, 28, "uniform",
+                         rot_steps=tuple(range(1, 17)) + tuple(16 * k for k in range(2, 18)),
+                         hoisted=True, relin=False, seed=1004),
+    "n16-stream64": Config("n16-stream64", 16, 36, 12, 4, 20, 192, 3.2, 28, "gauss_clip4",
+                           rot_steps=_stream_steps(), n_pairs=64, seed=1005),
 }
 
 
 def chacha_seed(key: str) -> bytes:
-    """32-byte key-expansion seed: SHA-256 of the ASCII string ``fhe-ks-evk/config<c>``."""
-    return hashlib.sha256(f"fhe-ks-evk/config{key}".encode("ascii")).digest()
+    """32-byte key-expansion seed: SHA-256 of the ASCII string ``fhe-ks-evk/<workload name>``."""
+    return hashlib.sha256(f"fhe-ks-evk/{key}".encode("ascii")).digest()
 
 
 def rng(seed: int, *tags: int) -> np.random.Generator:
