@@ -131,3 +131,48 @@ def test_shared_key_groups(ks_lib):
     for i in range(n):
         ks.ckks_keyswitch(ctx, c[i], lvl, evks[i], one, ws_1)
         assert torch.equal(one, out[i]), i
+
+
+@pytest.mark.slow
+def test_bench_launch_configuration(ks_lib, oracle_mod):
+    """The launch configuration the benchmark times: n16-full, 4 units per batched call, every
+    unit with its own seed and b half; tensor -> relin -> rotate(1).  Every item equals the
+    single calls; items 0 and 3 equal the oracle (sampled: the oracle takes seconds per unit)."""
+    import hashlib
+    ks = ks_lib
+    cfg, q, p, ctx = _setup(ks, "n16-full")
+    lvl, N = cfg.level, cfg.n
+    na, B = lvl + 1, 4
+    gen = W.rng(cfg.seed, W.TAG_SYNTH, 777)
+    nd = -(-cfg.n_q // cfg.alpha)
+    g = ks.galois_element(cfg.log_n, 1)
+    b_rel = [_res((q + p) * nd, N, gen).view(nd, len(q) + len(p), N) for _ in range(B)]
+    b_rot = [_res((q + p) * nd, N, gen).view(nd, len(q) + len(p), N) for _ in range(B)]
+    seeds = [hashlib.sha256(cfg.chacha_seed + bytes([0, i])).digest() for i in range(B)]
+    k_rel = [ks.make_evk(b_rel[i], seeds[i], 0) for i in range(B)]
+    k_rot = [ks.make_evk(b_rot[i], seeds[i], g) for i in range(B)]
+    x = _res(q[:na] * 2 * B, N, gen).view(B, 2, na, N)
+    y = _res(q[:na] * 2 * B, N, gen).view(B, 2, na, N)
+    d = torch.empty((B, 3, na, N), dtype=torch.uint32, device="cuda")
+    r = torch.empty((B, 2, na, N), dtype=torch.uint32, device="cuda")
+    out = torch.empty((B, 2, na, N), dtype=torch.uint32, device="cuda")
+    ws = ctx.workspace(lvl, B)
+    ks.ckks_tensor_batch(ctx, B, x, y, lvl, d)
+    ks.ckks_relin_batch(ctx, d, lvl, k_rel, r, ws)
+    ks.ckks_rotate_batch(ctx, r, lvl, [g] * B, k_rot, out, ws)
+    torch.cuda.synchronize()
+    one_d = torch.empty((3, na, N), dtype=torch.uint32, device="cuda")
+    one_r = torch.empty((2, na, N), dtype=torch.uint32, device="cuda")
+    one_o = torch.empty((2, na, N), dtype=torch.uint32, device="cuda")
+    ws1 = ctx.workspace(lvl)
+    for i in range(B):
+        ks.ckks_tensor(ctx, x[i], y[i], lvl, one_d)
+        ks.ckks_relin(ctx, one_d, lvl, k_rel[i], one_r, ws1)
+        ks.ckks_rotate(ctx, one_r, lvl, g, k_rot[i], one_o, ws1)
+        assert torch.equal(one_o, out[i]), i
+    octx = oracle_mod.Ctx(cfg.log_n, cfg.n_q, cfg.n_p)
+    for i in (0, B - 1):
+        xi, yi = x[i].cpu().numpy(), y[i].cpu().numpy()
+        rel = octx.relin(octx.tensor(xi, yi, lvl), lvl, cfg.alpha, b_rel[i].cpu().numpy(), seeds[i], 0)
+        want = octx.rotate(rel, lvl, cfg.alpha, g, b_rot[i].cpu().numpy(), seeds[i], g)
+        assert np.array_equal(out[i].cpu().numpy(), want), i
