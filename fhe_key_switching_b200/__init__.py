@@ -17,8 +17,8 @@ LIB_PATH = os.path.join(_HERE, "_build", "libckks_ks.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"CUDA library {LIB_PATH} is not built; run `python -m fhe_key_switching_b200.build` "
-        "(nvcc, sm_100a) first")
+        f"CUDA library {LIB_PATH} is not built; run `python fhe_key_switching_b200/build.py` "
+        "(nvcc, sm_100a) or `python __graft_entry__.py` first")
 
 _L = ctypes.CDLL(LIB_PATH)
 

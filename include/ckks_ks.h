@@ -24,7 +24,11 @@
  *    psi^N = -1, brv the log_n-bit reversal.  Ciphertexts are [2][l+1][N], the tensor
  *    product is [3][l+1][N]; all in the evaluation domain.
  *  - Device pointers must be 16-byte aligned.  Outputs must not alias inputs unless the
- *    entry point says so.  The caller owns every buffer and the stream.
+ *    entry point says so, and the workspace must not overlap either; the key-switching, rescale
+ *    and baby-step giant-step entry points check this and return CKKS_ERR_ARG.  The caller owns
+ *    every buffer and the stream.
+ *  - A context belongs to the device that was current when it was created; every entry point
+ *    that takes a context returns CKKS_ERR_ARG when another device is current.
  *  - Every call is asynchronous on `stream`; nothing synchronises the device, nothing
  *    allocates device memory except ckks_ctx_create.  The workspace `ws` is caller-owned
  *    device memory of at least ckks_workspace_bytes(...) bytes; calls on different streams
@@ -220,8 +224,11 @@ int ckks_chacha_expand(ckks_ctx *ctx, const uint8_t seed[32], uint32_t key_id, i
  * library until the process exits) instead of a caller buffer.
  *  - Returns CKKS_ERR_WORKSPACE when ckks_workspace_bytes(ctx, level, 1) exceeds that size
  *    (N=2^12 and N=2^14 parameter sets fit; N=2^16 with 36+12 primes does not).
- *  - The first call on a device looks up the array's device address (once per device, with
- *    that device current) and should come before any stream capture on that device.
+ *  - ckks_ctx_create looks up the array's device address on the context's device and keeps it
+ *    in the context, so the entry point itself makes no set-up call.  A device reset
+ *    invalidates the address together with the context's tables: create a new context after it.
+ *    Like every entry point, it returns CKKS_ERR_ARG when the current device is not the
+ *    context's.
  *  - Every call on a device shares the one array: calls that may overlap on the GPU (different
  *    streams, or different host threads) race on it; serialise them.  Nothing in the array
  *    needs to start at zero, so the previous call's contents are harmless.

@@ -12,9 +12,9 @@ Kim-Song, SAC 2018) and hybrid key switching (Han-Ki, CT-RSA 2020).
 
 Parity status: every function here is pinned by ``tests/test_oracle_*.py`` against brute force,
 closed forms, Python big-integer restatements, an independent ChaCha20 (OpenSSL through
-``cryptography``) and the RFC 8439 block vector, and by decryption identities.  The one
-exception is the 12-round count itself, which has no published ChaCha12-IETF vector on hand:
-it is pinned only structurally (same round function as the pinned 20-round core).
+``cryptography``) and the RFC 8439 block vector, and by decryption identities.  The 12-round
+count is pinned by the published reduced-round test vectors (ChaCha12 and ChaCha8 with an
+all-zero key and IV, ``tests/golden/chacha_vectors.txt``), beside the 20-round RFC vectors.
 """
 from __future__ import annotations
 

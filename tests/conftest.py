@@ -13,11 +13,21 @@ def pytest_configure(config):
     config.addinivalue_line("markers", "slow: oracle work at N=2^16 (seconds)")
 
 
+def build_library():
+    """Builds the CUDA library in-tree (nvcc cross-compiles for sm_100a without a GPU).  The build
+    script is loaded by path, since importing the package needs the built library."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_ckks_ks_build", os.path.join(ROOT, "fhe_key_switching_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod.build()
+
+
 @pytest.fixture(scope="session")
 def ks_lib():
-    """The CUDA library, built in-tree (nvcc cross-compiles for sm_100a without a GPU)."""
-    from fhe_key_switching_b200 import build as _build
-    _build.build()
+    """The CUDA library, built in-tree."""
+    build_library()
     import fhe_key_switching_b200 as ks
     return ks
 
