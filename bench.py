@@ -36,6 +36,9 @@ if ROOT not in sys.path:
 import workloads as W  # noqa: E402
 
 CONFIG_KEY = "n16-full"
+# workloads whose step is a batch of independent (tensor, relin, rotate) units: the benchmark line
+# (n16-full) and informational lines on the N=2^12 chains
+UNIT_WORKLOADS = ("n16-full", "n12-dnum2", "n12-dnum4")
 METRIC = "key-switches/s (rotations/s) at N=2^16, 32-bit RNS; % of HBM roofline"
 KS_PER_UNIT = 2          # relin + rotation
 ROT_PER_UNIT = 1
@@ -129,7 +132,8 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
-    cfg = W.CONFIGS[CONFIG_KEY]
+    cfg = W.CONFIGS[args.workload]
+    headline = args.workload == CONFIG_KEY
     n, lvl = cfg.n, cfg.level
     na = lvl + 1
     q, p = ks.ckks_gen_primes(cfg.log_n, cfg.n_q, cfg.n_p)
@@ -304,11 +308,14 @@ def run_ours(args, rank, world, local_rank):
     h2d = (sets[0]["x"].numel() + sets[0]["y"].numel()) * 4
     d2h = out.numel() * 4
 
-    cpu = cpu_baseline() if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
+    # the integer peaks of this GPU, measured now (a fraction of a second), for both rooflines
+    peaks = measure_int_peaks(ks, dev)
+    um = unit_model(cfg, lvl)
+    cpu = cpu_baseline(args.workload) if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
 
     if rank == 0:
         line = {
-            "metric": METRIC,
+            "metric": METRIC if headline else f"key-switches/s on {cfg.key} (informational)",
             "value": value,
             "unit": "key-switches/s",
             "rotations_per_s": job_throughput(ROT_PER_UNIT * B * args.steps, world, ms),
@@ -330,12 +337,18 @@ def run_ours(args, rank, world, local_rank):
             "kernel_launches_note": "one launch per kernel covers the whole batch",
             "clocks": clk,
             "roofline": roofline(cfg, dom_launches, dom_ms, clk, Bs, ms_single / args.steps,
-                                 dom_launches_ov, dom_ms_ov),
+                                 dom_launches_ov, dom_ms_ov, peaks),
+            "path_roofline": dict(path_roofline(B * um["ops"], B * um["chacha_blocks"], B * um["bytes"],
+                                                ms_per_step / 1e3, peaks),
+                                  per="one step (the whole batch)"),
+            "int_peaks": int_peaks_summary(peaks),
             "hbm_fraction_step": {"b_min_bytes_per_step": B * step_bytes_min(cfg),
                                   "frac": B * step_bytes_min(cfg) / (ms_per_step / 1e3) / (HBM_PEAK_GBS * 1e9),
                                   "peak_gbs": HBM_PEAK_GBS, "peak_source": PEAK_SOURCE},
             "cpu_baseline": cpu,
         }
+        if not headline:
+            line["informational"] = True
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
@@ -359,8 +372,91 @@ N_SM = 148
 
 
 def alu_peak_tops(mhz: float) -> float:
-    """int32 issue peak: 148 SMs x 4 sub-partitions x 32 lanes x 1 instruction/clock."""
+    """int32 issue ceiling, derived: 148 SMs x 4 sub-partitions x 32 lanes x 1 instruction/clock.
+    Context only; the rooflines use the measured rates of `measure_int_peaks`."""
     return N_SM * 4 * 32 * mhz * 1e6 / 1e12
+
+
+# ----------------------------------------------------------------------------- op model
+# Algorithmic int32 operations of the path, with the unit costs of the op model: NTT butterfly 8
+# (Shoup product 4, two lazy additions 2 + 2), constant modular product 4, modular addition 2,
+# 32x32->64 multiply-add 2, 64->32 reduction 8, ChaCha12 block 608 (6 double rounds x 8
+# quarter-rounds x 12 add/xor/rotate, plus 32 for the feed-forward and set-up; it yields 8
+# coefficients), reduction of a 64-bit keystream word 8.
+BFLY, CMUL, MADD, MAC, RED, CHACHA_BLOCK, AREDUCE = 8, 4, 2, 2, 8, 608, 8
+
+
+def limb_ntt_ops(log_n: int) -> int:
+    """One length-N negacyclic NTT (or inverse) of one limb: N/2 log N butterflies."""
+    return (1 << log_n) // 2 * log_n * BFLY
+
+
+def digit_sizes(cfg, level: int) -> list:
+    na = level + 1
+    return [min(cfg.alpha, na - lo) for lo in range(0, na, cfg.alpha)]
+
+
+def modup_ops(cfg, level: int) -> int:
+    """Inverse NTT of the l+1 limbs; per digit j (alpha_j primes) the base conversion onto the
+    ext - alpha_j other limbs (alpha_j multiply-adds and one reduction per output) and their NTTs."""
+    n, na = cfg.n, level + 1
+    ext = na + cfg.n_p
+    ds = digit_sizes(cfg, level)
+    ntt = limb_ntt_ops(cfg.log_n)
+    return na * ntt + sum((ext - a) * n * (a * MAC + RED) for a in ds) + sum(ext - a for a in ds) * ntt
+
+
+def chacha_blocks(cfg, level: int) -> int:
+    """ChaCha12 blocks that regenerate the a half of one key switch: beta * ext limbs of N/8."""
+    na = level + 1
+    return len(digit_sizes(cfg, level)) * (na + cfg.n_p) * cfg.n // 8
+
+
+def ip_ops(cfg, level: int) -> int:
+    """Key inner product: two multiply-adds per (digit, limb, coefficient), one reduction per
+    accumulator word; plus the keystream's blocks and word reductions."""
+    n, na = cfg.n, level + 1
+    ext = na + cfg.n_p
+    beta = len(digit_sizes(cfg, level))
+    return (2 * beta * ext * n * MAC + 2 * ext * n * RED
+            + chacha_blocks(cfg, level) * CHACHA_BLOCK + beta * ext * n * AREDUCE)
+
+
+def moddown_ops(cfg, level: int, comps: int = 2) -> int:
+    """Per component: inverse NTT of the k special limbs, base conversion P -> q_0..q_l, NTT of
+    the l+1 converted limbs, (acc - conv) P^-1 (one product, one subtraction)."""
+    n, na, k = cfg.n, level + 1, cfg.n_p
+    ntt = limb_ntt_ops(cfg.log_n)
+    return comps * (k * ntt + na * n * (k * MAC + RED) + na * ntt + na * n * (CMUL + MADD))
+
+
+def keyswitch_ops(cfg, level: int) -> int:
+    """One hybrid key switch (about 2.3 G at N=2^16, 36+12 primes, dnum 3, level 35)."""
+    return modup_ops(cfg, level) + ip_ops(cfg, level) + moddown_ops(cfg, level)
+
+
+def tensor_ops(cfg, level: int) -> int:
+    """ct x ct: four products, one addition, three reductions per coefficient and limb."""
+    return (level + 1) * cfg.n * (4 * MAC + 3 * RED)
+
+
+def rescale_ops(cfg, level: int) -> int:
+    """Per component: inverse NTT of limb l, NTT of its lift mod q_0..q_{l-1}, (c - conv) q_l^-1."""
+    ntt = limb_ntt_ops(cfg.log_n)
+    return 2 * (ntt + level * ntt + level * cfg.n * (CMUL + MADD))
+
+
+def key_limbs(cfg, level: int) -> int:
+    """Limbs of a key's b half one key switch reads: beta active digits x ext limbs."""
+    return len(digit_sizes(cfg, level)) * (level + 1 + cfg.n_p)
+
+
+def unit_model(cfg, level: int) -> dict:
+    """One unit of the benchmark step (tensor, relinearisation, rotation): op-model int32 operations,
+    ChaCha12 blocks and compulsory HBM bytes."""
+    na, n = level + 1, cfg.n
+    ops = tensor_ops(cfg, level) + 2 * keyswitch_ops(cfg, level) + 3 * na * n * MADD
+    return {"ops": ops, "chacha_blocks": 2 * chacha_blocks(cfg, level), "bytes": step_bytes_min(cfg, level)}
 
 
 def ip_row_ops(cfg) -> float:
@@ -380,26 +476,109 @@ def ip_row_ops(cfg) -> float:
     return chacha + a_red + ntt + macs
 
 
-def roofline(cfg, launches, total_ms, clk, batch, single_step_ms, launches_ov, total_ms_ov):
-    """The dominant kernel against the int32 ALU issue peak.  `launches`/`total_ms`: its launches
-    in a single-stream pass of the timed steps (each launch's events bracket that kernel only);
-    `launches_ov`/`total_ms_ov`: the same kernel inside the timed multi-stream region, where its
-    events also span the other streams' concurrent kernels."""
+# ----------------------------------------------------------------------------- measured int peaks
+# Probes of ckks_int_probe (include/ckks_ks.h) and the iterations that make one launch last a few ms.
+INT_PROBES = {"iadd": (0, 12288), "lop3": (1, 12288), "shf": (2, 12288), "imad": (3, 12288),
+              "imad_hi": (4, 12288), "imad_wide": (5, 12288), "mix_lop3_imad": (6, 12288), "chacha12": (7, 1024)}
+# the probes whose instruction any int32 operation of the op model can be issued as
+GENERAL_PROBES = ("iadd", "lop3", "shf", "imad", "mix_lop3_imad")
+
+
+def measure_int_peaks(ks, dev, reps: int = 3) -> dict:
+    """Runs every probe `reps` times (after one warm-up launch) on all SMs and keeps the fastest:
+    operations per second, per SM per clock (with the SM clock sampled meanwhile)."""
+    import torch
+    n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    blocks = n_sms * 6
+    sink = torch.empty(blocks * 256, dtype=torch.uint32, device=dev)
+    clocks = ClockSampler(dev.index or 0)
+    clocks.start()
+    time.sleep(0.2)
+    res = {}
+    for name, (op, iters) in INT_PROBES.items():
+        ks.ckks_int_probe(op, blocks, iters, sink)                 # warm-up
+        best = None
+        for _ in range(reps):
+            ms, ops = ks.ckks_int_probe(op, blocks, iters, sink)
+            best = ms if best is None else min(best, ms)
+        res[name] = {"ops_per_s": ops / (best / 1e3), "ms": best}
+    clk = clocks.stop()
+    mhz = clk.get("sm_mhz") or SM_MAX_MHZ
+    for r in res.values():
+        r["per_sm_per_clk"] = r["ops_per_s"] / (n_sms * mhz * 1e6)
+    best_name = max(GENERAL_PROBES, key=lambda k: res[k]["ops_per_s"])
+    return {"probes": res, "sm_mhz": mhz, "clocks": clk, "n_sms": n_sms,
+            "int_tops": res[best_name]["ops_per_s"] / 1e12, "int_probe": best_name,
+            "chacha_tops": res["chacha12"]["ops_per_s"] / 1e12,
+            "source": f"measured live: ckks_int_probe, {blocks} blocks x 256 threads, 8 chains per thread, "
+                      f"best of {reps}; int32 peak = fastest general probe ({best_name}); ChaCha12 peak = "
+                      "the library's block function at 608 ops per block"}
+
+
+def int_peaks_summary(peaks: dict) -> dict:
+    """Compact record of the measured probes for the JSON line."""
+    return {"sm_mhz": peaks["sm_mhz"], "int_tops": peaks["int_tops"], "int_probe": peaks["int_probe"],
+            "chacha12_tops": peaks["chacha_tops"],
+            "per_sm_per_clk": {k: round(v["per_sm_per_clk"], 2) for k, v in peaks["probes"].items()},
+            "derived_issue_tops": alu_peak_tops(peaks["sm_mhz"])}
+
+
+def _derived_peaks() -> dict:
+    t = alu_peak_tops(SM_MAX_MHZ)
+    return {"int_tops": t, "chacha_tops": t, "int_probe": None,
+            "source": f"derived: {N_SM} SMs x 128 int32 lanes x {SM_MAX_MHZ:.0f} MHz (no measurement)"}
+
+
+def int_time_s(ops: float, blocks: float, peaks: dict) -> float:
+    """Time the op model's operations need at the measured peaks: every operation at the fastest
+    general int32 rate, and the ChaCha12 blocks no faster than the measured ChaCha12 rate."""
+    return max(ops / (peaks["int_tops"] * 1e12), blocks * CHACHA_BLOCK / (peaks["chacha_tops"] * 1e12))
+
+
+def path_roofline(ops: float, blocks: float, nbytes: float, t_meas_s: float, peaks: dict) -> dict:
+    """The whole path against the slower of its two floors: T_hbm = compulsory bytes / measured HBM
+    bandwidth, T_int = op-model int32 operations at the measured integer peaks; frac = max / T."""
+    t_int = int_time_s(ops, blocks, peaks)
+    t_hbm = nbytes / (HBM_PEAK_GBS * 1e9)
+    t_floor = max(t_int, t_hbm)
+    return {"bound": "alu" if t_int >= t_hbm else "hbm", "frac": t_floor / t_meas_s,
+            "t_measured_us": t_meas_s * 1e6, "t_int_us": t_int * 1e6, "t_hbm_us": t_hbm * 1e6,
+            "int32_ops": ops, "chacha12_blocks": blocks, "hbm_bytes": nbytes,
+            "int_peak_tops": peaks["int_tops"], "chacha12_peak_tops": peaks["chacha_tops"],
+            "hbm_peak_gbs": HBM_PEAK_GBS, "hbm_frac": t_hbm / t_meas_s,
+            "int_frac_at_general_peak": ops / (peaks["int_tops"] * 1e12) / t_meas_s,
+            "peak_source": f"int: {peaks['source']}; hbm: {PEAK_SOURCE} (MEASURED_PEAKS.json copy)"
+                           if PEAK_SOURCE == "measured" else f"int: {peaks['source']}; hbm: fallback 6650 GB/s"}
+
+
+def roofline(cfg, launches, total_ms, clk, batch, single_step_ms, launches_ov, total_ms_ov, peaks=None):
+    """The dominant kernel against its integer floor: achieved = algorithmic int32 operations per
+    launch / average launch time; peak = the rate the measured peaks allow for this kernel's mix
+    (its ChaCha12 blocks at the measured ChaCha12 rate, everything at the fastest general rate).
+    `launches`/`total_ms`: its launches in a single-stream pass of the timed steps (each launch's
+    events bracket that kernel only); `launches_ov`/`total_ms_ov`: the same kernel inside the timed
+    multi-stream region, where its events also span the other streams' concurrent kernels."""
     if not launches:
         return None
+    peaks = peaks or _derived_peaks()
     avg_s = total_ms / launches / 1e3
-    achieved = batch * ip_row_ops(cfg) / avg_s / 1e12
-    peak = alu_peak_tops(SM_MAX_MHZ)
+    ops = batch * ip_row_ops(cfg)
+    blocks = batch * chacha_blocks(cfg, cfg.level)
+    t_floor = int_time_s(ops, blocks, peaks)
+    achieved = ops / avg_s / 1e12
+    peak = ops / t_floor / 1e12
+    traffic = ip_row_traffic_per_unit()
     out = {"kernel": "k_ip_row (ModUp last NTT pass + ChaCha12 + key inner product)",
            "bound": "alu", "achieved": achieved, "peak": peak, "unit": "Tops (int32)",
            "frac": achieved / peak,
-           "traffic": None if IP_ROW_TRAFFIC_PER_UNIT is None else IP_ROW_TRAFFIC_PER_UNIT * batch,
+           "traffic": None if traffic is None else traffic * batch,
            "units_per_launch": batch,
            "launches": launches,
            "avg_launch_us": avg_s * 1e6,
            "timed_in": "single-stream pass of the timed steps, right after the timed region "
                        f"({single_step_ms:.3f} ms per step)",
-           "peak_source": f"derived: {N_SM} SMs x 128 int32 lanes x {SM_MAX_MHZ:.0f} MHz"}
+           "peak_source": peaks["source"],
+           "frac_of_derived_issue_peak": achieved / alu_peak_tops(SM_MAX_MHZ)}
     if launches_ov:
         out["in_timed_region"] = {"launches": launches_ov,
                                   "avg_launch_us": total_ms_ov / launches_ov * 1e3,
@@ -407,19 +586,35 @@ def roofline(cfg, launches, total_ms, clk, batch, single_step_ms, launches_ov, t
     return out
 
 
-# DRAM bytes (read + write) per unit of a k_ip_row launch, from an ncu launch list of this
-# benchmark (4-unit launches; mean of 20: dram__bytes_read 392.51 MB + write 78.97 MB), scaled
-# by the units a launch covers; None when the kernel changed after the capture.
-IP_ROW_TRAFFIC_PER_UNIT = 471.48e6 / 4
+# DRAM bytes (read + write) per unit of a k_ip_row launch from an ncu capture, valid only for the
+# kernel sources it was taken on (sha-256 prefix of the device-code headers): after any change to
+# them the figure is reported as null until a new capture replaces it.
+IP_ROW_TRAFFIC = {"sources_sha16": None, "bytes_per_unit": None,
+                  "capture": "profiles/keyswitch_n16_full_launches.md"}
+KERNEL_HEADERS = ("modarith.cuh", "chacha.cuh", "ntt.cuh", "ks_kernels.cuh")
 
 
-def step_bytes_min(cfg) -> int:
-    """Compulsory HBM bytes of one step: inputs, the keys' stored b halves and outputs of the
+def kernel_sources_sha16() -> str:
+    h = hashlib.sha256()
+    for name in KERNEL_HEADERS:
+        with open(os.path.join(ROOT, "fhe_key_switching_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ip_row_traffic_per_unit():
+    if IP_ROW_TRAFFIC["sources_sha16"] != kernel_sources_sha16():
+        return None
+    return IP_ROW_TRAFFIC["bytes_per_unit"]
+
+
+def step_bytes_min(cfg, level: int | None = None) -> int:
+    """Compulsory HBM bytes of one unit: inputs, the keys' stored b halves and outputs of the
     tensor product (4 -> 3 polys), the relinearisation (3 polys + key -> 2) and the rotation
     (2 polys + key -> 2); the a halves are regenerated, intermediates are not counted."""
-    na = cfg.level + 1
-    nd = -(-cfg.n_q // cfg.alpha)
-    key = nd * (cfg.n_q + cfg.n_p)
+    level = cfg.level if level is None else level
+    na = level + 1
+    key = key_limbs(cfg, level)
     limbs = (4 + 3) * na + (3 * na + key + 2 * na) + (2 * na + key + 2 * na)
     return limbs * cfg.n * 4
 
@@ -430,7 +625,11 @@ LAUNCHES_PER_STEP = 1 + 2 * 10
 
 
 def run_workload(args, local_rank):
-    """Informational throughput (not the benchmark's headline line):
+    """Informational throughput (not the benchmark's headline line), each with its path roofline
+    (op-model int32 operations and compulsory bytes against the measured peaks) and the oracle
+    timed on a bounded sample of the same step:
+    n14-hoisted8 = 8 units, each 8 hoisted rotations (+-1, +-2, +-4, +-8) of one ciphertext, then a
+        tensor product and relinearisation with a second ciphertext (level 11, dnum 3);
     n16-bsgs32 = 32 hoisted rotations of one ciphertext at level 24 (one ModUp, 32 keys);
     n16-stream64 = 64 pairs, each tensor + relin + rotate by 2^(i mod 15), level 20, dnum 4
         (one relinearisation key, 15 rotation keys, all as batched calls);
@@ -448,15 +647,18 @@ def run_workload(args, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     key = str(args.workload)
-    cfg = W.CONFIGS[{"n16-stream64-rescale": "n16-stream64", "rescale": "n16-full", "bsgs": "n16-bsgs32",
-                     "bsgs-n14": "n14-hoisted8"}.get(key, key)]
+    if key not in INFO_WORKLOADS:
+        raise SystemExit(f"--workload {key}: use one of {', '.join(UNIT_WORKLOADS + INFO_WORKLOADS)}")
+    cfg = W.CONFIGS[INFO_WORKLOADS[key]]
     n, lvl = cfg.n, cfg.level
     na = lvl + 1
+    ext = na + cfg.n_p
     q, p = ks.ckks_gen_primes(cfg.log_n, cfg.n_q, cfg.n_p)
     ctx = ks.Context(cfg.log_n, q, p, cfg.dnum)
     nd = -(-cfg.n_q // cfg.alpha)
     mods = q + p
     gen = W.rng(cfg.seed, W.TAG_SYNTH, 7)
+    limb = n * 4
 
     def res(moduli):
         return torch.from_numpy(W.uniform_residues(moduli, n, gen)).to(dev)
@@ -466,7 +668,33 @@ def run_workload(args, local_rank):
     keys_t = {r: res(mods * nd).view(nd, len(mods), n) for r in steps_g}
     evk = {r: ks.make_evk(keys_t[r], cfg.chacha_seed, gal[r]) for r in steps_g}
     stream = torch.cuda.current_stream(dev)
-    if key == "n16-bsgs32":
+    ksw, kl = keyswitch_ops(cfg, lvl), key_limbs(cfg, lvl) * limb
+    extra = {}
+    if key == "n14-hoisted8":
+        U, R = 8, len(cfg.rot_steps)
+        cts = [res(q[:na] * 2 * U).view(U, 2, na, n) for _ in range(N_SETS)]
+        ys = [res(q[:na] * 2 * U).view(U, 2, na, n) for _ in range(N_SETS)]
+        k_rel = ks.make_evk(res(mods * nd).view(nd, len(mods), n), cfg.chacha_seed, 0)
+        gs = [gal[r] for r in cfg.rot_steps]
+        ev = [evk[r] for r in cfg.rot_steps]
+        rot = torch.empty((U, R, 2, na, n), dtype=torch.uint32, device=dev)
+        d = torch.empty((U, 3, na, n), dtype=torch.uint32, device=dev)
+        rl = torch.empty((U, 2, na, n), dtype=torch.uint32, device=dev)
+        ws_h = [ctx.workspace(lvl, R, device=dev) for _ in range(U)]
+        ws_b = ctx.workspace(lvl, U, device=dev)
+
+        def step(i):
+            x, y = cts[i % N_SETS], ys[i % N_SETS]
+            for u in range(U):
+                ks.ckks_rotate_hoisted(ctx, x[u], lvl, gs, ev, rot[u], ws_h[u], stream)
+            ks.ckks_tensor_batch(ctx, U, x, y, lvl, d, stream)
+            ks.ckks_relin_batch(ctx, d, lvl, [k_rel] * U, rl, ws_b, stream)
+        ks_per_step, rot_per_step = U * (R + 1), U * R
+        ops = U * (modup_ops(cfg, lvl) + R * (ip_ops(cfg, lvl) + moddown_ops(cfg, lvl) + na * n * MADD)
+                   + tensor_ops(cfg, lvl) + ksw + 2 * na * n * MADD)
+        blocks = U * (R + 1) * chacha_blocks(cfg, lvl)
+        nbytes = U * (2 * na * limb + R * 2 * na * limb + 7 * na * limb + 5 * na * limb) + (R + 1) * kl
+    elif key == "n16-bsgs32":
         cts = [res(q[:na] * 2).view(2, na, n) for _ in range(N_SETS)]
         R = len(cfg.rot_steps)
         gs = [gal[r] for r in cfg.rot_steps]
@@ -477,15 +705,21 @@ def run_workload(args, local_rank):
         def step(i):
             ks.ckks_rotate_hoisted(ctx, cts[i % N_SETS], lvl, gs, ev, out, ws, stream)
         ks_per_step, rot_per_step = R, R
-    elif key == "n16-stream64":
+        ops = modup_ops(cfg, lvl) + R * (ip_ops(cfg, lvl) + moddown_ops(cfg, lvl) + na * n * MADD)
+        blocks = R * chacha_blocks(cfg, lvl)
+        nbytes = 2 * na * limb + R * (kl + 2 * na * limb)
+    elif key in ("n16-stream64", "n16-stream64-rescale"):
+        rs = key.endswith("rescale")
         P_ = cfg.n_pairs
+        lr = lvl - 1 if rs else lvl               # the rotation's level
         xs = [res(q[:na] * 2 * P_).view(P_, 2, na, n) for _ in range(2)]
         ys = [res(q[:na] * 2 * P_).view(P_, 2, na, n) for _ in range(2)]
         b_rel = res(mods * nd).view(nd, len(mods), n)
         k_rel = ks.make_evk(b_rel, cfg.chacha_seed, 0)
         d = torch.empty((P_, 3, na, n), dtype=torch.uint32, device=dev)
         r1 = torch.empty((P_, 2, na, n), dtype=torch.uint32, device=dev)
-        out = torch.empty((P_, 2, na, n), dtype=torch.uint32, device=dev)
+        r2 = torch.empty((P_, 2, lr + 1, n), dtype=torch.uint32, device=dev) if rs else r1
+        out = torch.empty((P_, 2, lr + 1, n), dtype=torch.uint32, device=dev)
         ws = ctx.workspace(lvl, P_, device=dev)
         gs = [gal[r] for r in cfg.rot_steps]
         ev = [evk[r] for r in cfg.rot_steps]
@@ -493,28 +727,17 @@ def run_workload(args, local_rank):
         def step(i):
             ks.ckks_tensor_batch(ctx, P_, xs[i % 2], ys[i % 2], lvl, d, stream)
             ks.ckks_relin_batch(ctx, d, lvl, [k_rel] * P_, r1, ws, stream)
-            ks.ckks_rotate_batch(ctx, r1, lvl, gs, ev, out, ws, stream)
+            if rs:
+                ks.ckks_rescale_batch(ctx, P_, r1, lvl, r2, ws, stream)
+            ks.ckks_rotate_batch(ctx, r2, lr, gs, ev, out, ws, stream)
         ks_per_step, rot_per_step = 2 * P_, P_
-    elif key == "n16-stream64-rescale":
-        P_ = cfg.n_pairs
-        xs = [res(q[:na] * 2 * P_).view(P_, 2, na, n) for _ in range(2)]
-        ys = [res(q[:na] * 2 * P_).view(P_, 2, na, n) for _ in range(2)]
-        b_rel = res(mods * nd).view(nd, len(mods), n)
-        k_rel = ks.make_evk(b_rel, cfg.chacha_seed, 0)
-        d = torch.empty((P_, 3, na, n), dtype=torch.uint32, device=dev)
-        r1 = torch.empty((P_, 2, na, n), dtype=torch.uint32, device=dev)
-        r2 = torch.empty((P_, 2, lvl, n), dtype=torch.uint32, device=dev)
-        out = torch.empty((P_, 2, lvl, n), dtype=torch.uint32, device=dev)
-        ws = ctx.workspace(lvl, P_, device=dev)
-        gs = [gal[r] for r in cfg.rot_steps]
-        ev = [evk[r] for r in cfg.rot_steps]
-
-        def step(i):
-            ks.ckks_tensor_batch(ctx, P_, xs[i % 2], ys[i % 2], lvl, d, stream)
-            ks.ckks_relin_batch(ctx, d, lvl, [k_rel] * P_, r1, ws, stream)
-            ks.ckks_rescale_batch(ctx, P_, r1, lvl, r2, ws, stream)
-            ks.ckks_rotate_batch(ctx, r2, lvl - 1, gs, ev, out, ws, stream)
-        ks_per_step, rot_per_step = 2 * P_, P_
+        nr = lr + 1
+        ops = P_ * (tensor_ops(cfg, lvl) + ksw + 2 * na * n * MADD + keyswitch_ops(cfg, lr) + nr * n * MADD
+                    + (rescale_ops(cfg, lvl) if rs else 0))
+        blocks = P_ * (chacha_blocks(cfg, lvl) + chacha_blocks(cfg, lr))
+        # per call, each key once (one relinearisation key, 15 rotation keys)
+        nbytes = (P_ * (7 * na + 3 * na + 2 * na + (2 * na + 2 * nr if rs else 0) + 2 * nr + 2 * nr) * limb
+                  + kl + len(steps_g) * key_limbs(cfg, lr) * limb)
     elif key == "rescale":
         R = 64
         cts = [res(q[:na] * 2 * R).view(R, 2, na, n) for _ in range(N_SETS)]
@@ -524,13 +747,14 @@ def run_workload(args, local_rank):
         def step(i):
             ks.ckks_rescale_batch(ctx, R, cts[i % N_SETS], lvl, out, ws, stream)
         ks_per_step, rot_per_step = 0, 0
-    elif key in ("bsgs", "bsgs-n14"):
+        ops, blocks = R * rescale_ops(cfg, lvl), 0
+        nbytes = R * (2 * na + 2 * lvl) * limb
+    else:                                          # bsgs, bsgs-n14
         n1, n2 = 16, 18
         baby = [1] + [ks.galois_element(cfg.log_n, k) for k in range(1, n1)]
         giant = [1] + [ks.galois_element(cfg.log_n, n1 * j) for j in range(1, n2)]
         gk = {g: ks.make_evk(res(mods * nd).view(nd, len(mods), n), cfg.chacha_seed, g)
               for g in baby + giant if g != 1}
-        ext = na + cfg.n_p
         pt = res((q[:na] + p) * n2 * n1).view(n2, n1, ext, n)
         cts = [res(q[:na] * 2).view(2, na, n) for _ in range(N_SETS)]
         out = torch.empty((2, na, n), dtype=torch.uint32, device=dev)
@@ -541,9 +765,14 @@ def run_workload(args, local_rank):
         def step(i):
             ks.ckks_bsgs(ctx, cts[i % N_SETS], lvl, baby, bk, giant, gkk, pt, out, ws, stream)
         ks_per_step, rot_per_step = (n1 - 1) + (n2 - 1), (n1 - 1) + (n2 - 1)
-    else:
-        raise SystemExit(f"--workload {key}: use n16-full (default), n16-bsgs32, n16-stream64, "
-                         "n16-stream64-rescale, rescale, bsgs or bsgs-n14")
+        # one ModUp, 15 hoisted inner products, the plaintext sums (two multiply-adds and a
+        # reduction share per term), 18 ModDowns, 17 giant rotations, the sum of 18 partials
+        ops = (modup_ops(cfg, lvl) + (n1 - 1) * ip_ops(cfg, lvl) + n2 * n1 * 2 * ext * n * MAC
+               + n2 * 2 * ext * n * RED + n2 * moddown_ops(cfg, lvl) + (n2 - 1) * (ksw + na * n * MADD)
+               + n2 * 2 * na * n * MADD)
+        blocks = (n1 - 1 + n2 - 1) * chacha_blocks(cfg, lvl)
+        nbytes = (n2 * n1 * ext + 2 * na + 2 * na) * limb + (n1 - 1 + n2 - 1) * kl
+        b_comb = (n2 * n1 * ext + (n1 - 1) * 2 * ext + 2 * na + n2 * 2 * ext) * limb
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
@@ -551,7 +780,8 @@ def run_workload(args, local_rank):
     clocks.start()
     time.sleep(0.3)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if key in ("bsgs", "bsgs-n14"):
+    is_bsgs = key in ("bsgs", "bsgs-n14")
+    if is_bsgs:
         ks.ckks_prof_begin(ctx, "bsgs_combine", args.steps)
     e0.record(stream)
     for i in range(args.steps):
@@ -560,49 +790,147 @@ def run_workload(args, local_rank):
     torch.cuda.synchronize()
     clk = clocks.stop()
     ms = e0.elapsed_time(e1)
-    if key in ("bsgs", "bsgs-n14"):
+    if is_bsgs:
         launches, comb_ms = ks.ckks_prof_end(ctx)
-        # compulsory bytes of one combine launch: every plaintext once, the 15 rotated babies'
-        # accumulators and the input ciphertext once, the 18 giant sums written once
-        b_comb = (n2 * n1 * ext + (n1 - 1) * 2 * ext + 2 * na + n2 * 2 * ext) * n * 4
         comb_s = comb_ms / max(launches, 1) / 1e3
-        print(json.dumps({"workload": f"bsgs: {cfg.key} chain, N=2^{cfg.log_n}, {n1} baby x {n2} giant "
-                                      f"steps, level {lvl}",
-                          "informational": True, "transforms_per_s": args.steps / (ms / 1e3),
-                          "ms_per_step": ms / args.steps, "steps": args.steps, "warmup": args.warmup,
-                          "rotations_per_transform": ks_per_step,
-                          "combine_kernel": {"avg_launch_us": comb_s * 1e6, "launches": launches,
-                                             "bytes_per_launch": b_comb, "achieved_gbs": b_comb / comb_s / 1e9,
-                                             "peak_gbs": HBM_PEAK_GBS,
-                                             "frac": b_comb / comb_s / 1e9 / HBM_PEAK_GBS,
-                                             "share_of_step": comb_s * 1e3 / (ms / args.steps)},
-                          "clocks": clk}), flush=True)
-        return
+        extra["combine_kernel"] = {"avg_launch_us": comb_s * 1e6, "launches": launches,
+                                   "bytes_per_launch": b_comb, "achieved_gbs": b_comb / comb_s / 1e9,
+                                   "peak_gbs": HBM_PEAK_GBS, "frac": b_comb / comb_s / 1e9 / HBM_PEAK_GBS,
+                                   "share_of_step": comb_s * 1e3 / (ms / args.steps)}
+    peaks = measure_int_peaks(ks, dev)
+    t_step = ms / args.steps / 1e3
+    line = {"workload": key, "informational": True, "config": INFO_DESCRIPTIONS[key],
+            "ms_per_step": ms / args.steps, "steps": args.steps, "warmup": args.warmup}
     if key == "rescale":
-        # compulsory bytes per rescale: read 2(l+1) limbs, write 2l limbs
-        b_min = (2 * na + 2 * lvl) * n * 4
-        per_s = R * args.steps / (ms / 1e3)
-        print(json.dumps({"workload": f"rescale: N=2^{cfg.log_n}, level {lvl} -> {lvl - 1}, {R} per step",
-                          "informational": True, "rescales_per_s": per_s, "ms_per_step": ms / args.steps,
-                          "steps": args.steps, "warmup": args.warmup,
-                          "hbm": {"b_min_bytes_per_rescale": b_min, "achieved_gbs": b_min * per_s / 1e9,
-                                  "peak_gbs": HBM_PEAK_GBS, "frac": b_min * per_s / 1e9 / HBM_PEAK_GBS},
-                          "clocks": clk}), flush=True)
-        return
-    print(json.dumps({"workload": key, "informational": True,
-                      "key_switches_per_s": ks_per_step * args.steps / (ms / 1e3),
-                      "rotations_per_s": rot_per_step * args.steps / (ms / 1e3),
-                      "ms_per_step": ms / args.steps, "steps": args.steps, "warmup": args.warmup,
-                      "key_switches_per_step": ks_per_step, "clocks": clk}), flush=True)
+        line["rescales_per_s"] = R / t_step
+    elif is_bsgs:
+        line["transforms_per_s"] = 1 / t_step
+        line["rotations_per_transform"] = rot_per_step
+    if ks_per_step:
+        line["key_switches_per_s"] = ks_per_step / t_step
+        line["rotations_per_s"] = rot_per_step / t_step
+        line["key_switches_per_step"] = ks_per_step
+    line["path_roofline"] = dict(path_roofline(ops, blocks, nbytes, t_step, peaks), per="one step")
+    line.update(extra)
+    line["int_peaks"] = int_peaks_summary(peaks)
+    line["clocks"] = clk
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = info_cpu_baseline(key)
+    print(json.dumps(line), flush=True)
 
 
-def _oracle_sample():
-    """Bounded CPU sample of the same step: one relinearisation and one rotation of n16-full,
-    timed on the oracle with synthetic residues (cost is data independent)."""
+INFO_WORKLOADS = {"n14-hoisted8": "n14-hoisted8", "n16-bsgs32": "n16-bsgs32", "n16-stream64": "n16-stream64",
+                  "n16-stream64-rescale": "n16-stream64", "rescale": "n16-full", "bsgs": "n16-bsgs32",
+                  "bsgs-n14": "n14-hoisted8"}
+INFO_DESCRIPTIONS = {
+    "n14-hoisted8": "N=2^14, 12+4 primes, dnum 3, level 11; step = 8 units, each 8 hoisted rotations "
+                    "(+-1, +-2, +-4, +-8) + tensor + relin",
+    "n16-bsgs32": "N=2^16, 36+12 primes, dnum 4, level 24; step = 32 hoisted rotations of one ciphertext",
+    "n16-stream64": "N=2^16, 36+12 primes, dnum 4, level 20; step = 64 pairs, each tensor + relin + "
+                    "rotate by 2^(i mod 15)",
+    "n16-stream64-rescale": "as n16-stream64 with a rescale after the relinearisation (rotation at level 19)",
+    "rescale": "N=2^16, 36+12 primes, level 35 -> 34; step = 64 rescales",
+    "bsgs": "N=2^16, 36+12 primes, dnum 4, level 24; step = one 16 baby x 18 giant step transform "
+            "(288 plaintext diagonals)",
+    "bsgs-n14": "N=2^14, 12+4 primes, dnum 3, level 11; step = one 16 baby x 18 giant step transform",
+}
+
+
+def info_cpu_baseline(key: str, max_seconds: float = 8.0):
+    """The oracle on a bounded sample of an informational line's step (synthetic residues; the cost
+    is data independent), in the line's own unit."""
     import numpy as np
     import oracle
 
-    cfg = W.CONFIGS[CONFIG_KEY]
+    cfg = W.CONFIGS[INFO_WORKLOADS[key]]
+    n, lvl = cfg.n, cfg.level
+    na = lvl + 1
+    octx = oracle.Ctx(cfg.log_n, cfg.n_q, cfg.n_p)
+    nd = -(-cfg.n_q // cfg.alpha)
+    gen = W.rng(cfg.seed, W.TAG_SYNTH, 98)
+    ct = W.uniform_residues(octx.q[:na] * 2, n, gen).reshape(2, na, n)
+    b = W.uniform_residues(octx.mod * nd, n, gen).reshape(nd, len(octx.mod), n)
+    seed = cfg.chacha_seed
+    if key == "bsgs":
+        return None                 # the oracle's plaintext sums take minutes at N=2^16
+    if key == "n14-hoisted8":
+        gs = [octx.galois(r) for r in cfg.rot_steps]
+        y = W.uniform_residues(octx.q[:na] * 2, n, gen).reshape(2, na, n)
+
+        def fn():
+            octx.rotate_hoisted(ct, lvl, cfg.alpha, gs, [b] * len(gs), [seed] * len(gs), gs)
+            octx.relin(octx.tensor(ct, y, lvl), lvl, cfg.alpha, b, seed, 0)
+        units, unit, what = len(gs) + 1, "key-switches/s", "one unit (8 hoisted rotations + tensor + relin)"
+    elif key == "n16-bsgs32":
+        gs = [octx.galois(r) for r in cfg.rot_steps[:2]]
+
+        def fn():
+            octx.rotate_hoisted(ct, lvl, cfg.alpha, gs, [b] * 2, [seed] * 2, gs)
+        units, unit, what = 2, "rotations/s", "2 of the 32 hoisted rotations (one ModUp)"
+    elif key in ("n16-stream64", "n16-stream64-rescale"):
+        y = W.uniform_residues(octx.q[:na] * 2, n, gen).reshape(2, na, n)
+        g = octx.galois(1)
+
+        def fn():
+            r = octx.relin(octx.tensor(ct, y, lvl), lvl, cfg.alpha, b, seed, 0)
+            lv = lvl
+            if key.endswith("rescale"):
+                r, lv = octx.rescale(r, lvl), lvl - 1
+            octx.rotate(r, lv, cfg.alpha, g, b, seed, g)
+        units, unit, what = 2, "key-switches/s", "one pair of the 64"
+    elif key == "rescale":
+        def fn():
+            octx.rescale(ct, lvl)
+        units, unit, what = 1, "rescales/s", "one of the 64 rescales"
+    else:                           # bsgs-n14
+        n1, n2 = 16, 18
+        ext = na + cfg.n_p
+        baby = [1] + [octx.galois(k) for k in range(1, n1)]
+        giant = [1] + [octx.galois(n1 * j) for j in range(1, n2)]
+        pt = W.uniform_residues((octx.q[:na] + octx.p) * n1 * n2, n, gen).reshape(n2, n1, ext, n)
+        kb = [None] + [(b, g) for g in baby[1:]]
+        kg = [None] + [(b, g) for g in giant[1:]]
+
+        def fn():
+            octx.bsgs(ct, lvl, cfg.alpha, baby, kb, giant, kg, pt, seed)
+        units, unit, what = 1, "transforms/s", "one whole transform"
+    fn()
+    t0 = time.perf_counter()
+    k = 0
+    while True:
+        fn()
+        k += 1
+        if time.perf_counter() - t0 > max_seconds / 2 or k >= 16:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": units * k / dt, "unit": unit, "cores": _omp_threads(), "kind": "oracle",
+            "sample": f"{k} x {what} of {key} on synthetic residues, plain C oracle with OpenMP over limbs"}
+
+
+def run_int_peaks(local_rank):
+    """Informational line: the integer probes of ckks_int_probe, as operations per second and per
+    SM per clock at the sampled SM clock."""
+    import torch
+    import fhe_key_switching_b200 as ks
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    peaks = measure_int_peaks(ks, dev, reps=5)
+    print(json.dumps({"informational": True, "int_peaks": {
+        k: {"tops": v["ops_per_s"] / 1e12, "per_sm_per_clk": v["per_sm_per_clk"], "ms": v["ms"]}
+        for k, v in peaks["probes"].items()},
+        "sm_mhz": peaks["sm_mhz"], "n_sms": peaks["n_sms"], "int_tops": peaks["int_tops"],
+        "int_probe": peaks["int_probe"], "chacha12_tops": peaks["chacha_tops"],
+        "derived_issue_tops": alu_peak_tops(peaks["sm_mhz"]), "source": peaks["source"],
+        "clocks": peaks["clocks"]}), flush=True)
+
+
+def _oracle_sample(key: str = CONFIG_KEY):
+    """Bounded CPU sample of the same step: one unit (tensor, relinearisation, rotation) of the
+    workload, timed on the oracle with synthetic residues (cost is data independent)."""
+    import numpy as np
+    import oracle
+
+    cfg = W.CONFIGS[key]
     ctx = oracle.Ctx(cfg.log_n, cfg.n_q, cfg.n_p)
     n, lvl = cfg.n, cfg.level
     na = lvl + 1
@@ -626,8 +954,8 @@ def _omp_threads():
     return int(v) if v and v.isdigit() else (os.cpu_count() or 1)
 
 
-def cpu_baseline(max_seconds: float = 20.0):
-    one_step = _oracle_sample()
+def cpu_baseline(key: str = CONFIG_KEY, max_seconds: float = 20.0):
+    one_step = _oracle_sample(key)
     one_step()                              # warm (tables, page faults)
     t0 = time.perf_counter()
     k = 0
@@ -639,15 +967,14 @@ def cpu_baseline(max_seconds: float = 20.0):
     dt = time.perf_counter() - t0
     return {"value": KS_PER_UNIT * k / dt, "unit": "key-switches/s", "cores": _omp_threads(),
             "kind": "oracle",
-            "sample": f"{k} units of the N=2^16 full-level workload (tensor + relin + rotate, "
-                      "2 key switches each) "
+            "sample": f"{k} units of the {key} workload (tensor + relin + rotate, 2 key switches each) "
                       "on synthetic residues, plain C oracle with OpenMP over limbs"}
 
 
 def workload_config(cfg, batch: int, world: int, stored_a: bool = False, streams: str | None = None) -> dict:
     """The benchmark workload, the same for both arms."""
-    c = {"workload": "n16-full: N=2^16, 36+12 primes < 2^30, dnum 3, level 35; "
-                     f"step = batch of {batch} independent units, each tensor + relin + "
+    c = {"workload": f"{cfg.key}: N=2^{cfg.log_n}, {cfg.n_q}+{cfg.n_p} primes < 2^30, dnum {cfg.dnum}, "
+                     f"level {cfg.level}; step = batch of {batch} independent units, each tensor + relin + "
                      "rotate(1) with its own keys",
          "log_n": cfg.log_n, "n_q": cfg.n_q, "n_p": cfg.n_p, "dnum": cfg.dnum,
          "level": cfg.level, "batch": batch, "key_switches_per_step": KS_PER_UNIT * batch,
@@ -705,27 +1032,36 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--batch", type=int, default=8, help="independent n16-full units per step")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="independent units per step (default 8 for n16-full, 64 for the N=2^12 lines)")
     ap.add_argument("--workload", default=CONFIG_KEY,
-                    help="n16-full (benchmark line), or n16-bsgs32 / n16-stream64 / n16-stream64-rescale / "
-                         "rescale / bsgs / bsgs-n14 (informational lines)")
+                    help="n16-full (benchmark line), or n12-dnum2 / n12-dnum4 / n14-hoisted8 / n16-bsgs32 / "
+                         "n16-stream64 / n16-stream64-rescale / rescale / bsgs / bsgs-n14 (informational lines)")
     ap.add_argument("--streams", type=int, default=None,
                     help="CUDA streams the batch is split over, each running batch/streams units "
                          "(default 2 for an even batch, else 1)")
     ap.add_argument("--graph", action="store_true",
                     help="time one CUDA graph replay per step instead of eager launches (pays at small "
                          "batches; at 2 streams x 4 units the other stream already hides launch gaps)")
+    ap.add_argument("--int-peaks", action="store_true",
+                    help="measure this GPU's integer throughput per instruction class (ckks_int_probe) and "
+                         "print it as one JSON line")
     ap.add_argument("--stored-a", action="store_true",
                     help="ablation: keys with a stored a half (read from HBM) instead of ChaCha12")
     args = ap.parse_args()
     rank, world, local_rank = rank_env()
+    if args.batch is None:
+        args.batch = 8 if args.workload == CONFIG_KEY or args.impl == "reference" else 64
     if args.impl == "reference":
         if args.steps > 3:
             args.steps = 3          # each oracle step is seconds of CPU work
         args.warmup = min(args.warmup, 1)
         run_reference(args, rank, world)
         return
-    if str(args.workload) != CONFIG_KEY:
+    if args.int_peaks:
+        run_int_peaks(local_rank)
+        return
+    if str(args.workload) not in UNIT_WORKLOADS:
         run_workload(args, local_rank)
         return
     run_ours(args, rank, world, local_rank)

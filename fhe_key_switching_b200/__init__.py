@@ -71,6 +71,8 @@ _SIGS = {
     "ckks_keyswitch_noalloc": (_ci, [_vp, _vp, _ci, ctypes.POINTER(ckks_evk), _vp, _vp]),
     "ckks_prof_begin": (_ci, [_vp, ctypes.c_char_p, _ci]),
     "ckks_prof_end": (_ci, [_vp, ctypes.POINTER(_ci), ctypes.POINTER(ctypes.c_double)]),
+    "ckks_int_probe": (_ci, [_ci, _ci, _ci, _vp, _vp, ctypes.POINTER(ctypes.c_float),
+                             ctypes.POINTER(ctypes.c_double)]),
     "ckks_last_error": (ctypes.c_char_p, []),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -335,6 +337,19 @@ def ckks_prof_end(ctx):
     ms = ctypes.c_double()
     _check(_L.ckks_prof_end(ctx.handle, ctypes.byref(n), ctypes.byref(ms)), "ckks_prof_end")
     return n.value, ms.value
+
+
+def ckks_int_probe(op: int, blocks: int, iters: int, sink, stream=None):
+    """One integer-throughput probe launch (a measurement aid): returns (elapsed ms, operations).
+    sink: CUDA uint32 tensor of blocks * 256 words."""
+    if sink.numel() < blocks * 256:
+        raise ValueError("sink must hold blocks * 256 words")
+    ms = ctypes.c_float()
+    ops = ctypes.c_double()
+    code = _L.ckks_int_probe(op, blocks, iters, _ptr(sink), _stream(stream), ctypes.byref(ms), ctypes.byref(ops))
+    if code != CKKS_OK:
+        raise CkksError(code, "ckks_int_probe")
+    return ms.value, ops.value
 
 
 def galois_element(log_n: int, r: int) -> int:

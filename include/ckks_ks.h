@@ -268,6 +268,25 @@ int ckks_selftest_wait_expiry(ckks_ctx *ctx, ckks_stream_t stream);
 int ckks_prof_begin(ckks_ctx *ctx, const char *kernel, int max_launches);
 int ckks_prof_end(ckks_ctx *ctx, int *launches, double *total_ms);
 
+/* Integer throughput probe (a measurement aid; the pages have no counterpart).  Launches one
+ * kernel of `blocks` blocks x 256 threads on `stream`, each thread running 8 independent
+ * dependency chains of the operation `op` for `iters` iterations, and waits for it.
+ *   CKKS_PROBE_IADD       add.u32              CKKS_PROBE_IMAD       mad.lo.u32
+ *   CKKS_PROBE_LOP3       lop3.b32             CKKS_PROBE_IMAD_HI    mad.hi.u32
+ *   CKKS_PROBE_SHF        shf.l.wrap.b32       CKKS_PROBE_IMAD_WIDE  mad.wide.u32 (64-bit sum)
+ *   CKKS_PROBE_MIX        alternating lop3.b32 and mad.lo.u32
+ *   CKKS_PROBE_CHACHA12   the library's ChaCha12 block function, counted as 608 int32
+ *                         operations per block (the op model's unit cost)
+ * sink: device, blocks * 256 words (written, 16-byte aligned).  *ms: the launch's elapsed time
+ * (CUDA events on `stream`); *ops: the operations it executed.  Returns CKKS_ERR_ARG for a bad
+ * argument, CKKS_ERR_CUDA when the launch fails.  Synchronous; not for use inside a capture. */
+enum {
+    CKKS_PROBE_IADD = 0, CKKS_PROBE_LOP3, CKKS_PROBE_SHF, CKKS_PROBE_IMAD, CKKS_PROBE_IMAD_HI,
+    CKKS_PROBE_IMAD_WIDE, CKKS_PROBE_MIX, CKKS_PROBE_CHACHA12, CKKS_PROBE_COUNT
+};
+int ckks_int_probe(int op, int blocks, int iters, uint32_t *sink, ckks_stream_t stream, float *ms,
+                   double *ops);
+
 /* Message of the last error on this thread ("" if none). */
 const char *ckks_last_error(void);
 

@@ -16,8 +16,60 @@ def test_roofline_record_has_the_contract_keys():
     assert math.isclose(r["frac"], r["achieved"] / r["peak"])
     # achieved = algorithmic ops per launch / average launch time
     assert math.isclose(r["achieved"], 4 * bench.ip_row_ops(cfg) / 235e-6 / 1e12)
-    assert math.isclose(r["traffic"], 4 * bench.IP_ROW_TRAFFIC_PER_UNIT)
+    t = bench.ip_row_traffic_per_unit()
+    assert r["traffic"] == (None if t is None else 4 * t)
     assert bench.roofline(cfg, 0, 0.0, clk, 4, 2.75, 0, 0.0) is None
+
+
+def test_traffic_figure_is_tied_to_the_kernel_sources(monkeypatch):
+    """A DRAM figure taken on other kernel sources is never reported."""
+    monkeypatch.setitem(bench.IP_ROW_TRAFFIC, "sources_sha16", "0" * 16)
+    monkeypatch.setitem(bench.IP_ROW_TRAFFIC, "bytes_per_unit", 1.0e8)
+    assert bench.ip_row_traffic_per_unit() is None
+    monkeypatch.setitem(bench.IP_ROW_TRAFFIC, "sources_sha16", bench.kernel_sources_sha16())
+    assert bench.ip_row_traffic_per_unit() == 1.0e8
+
+
+def test_kernel_roofline_uses_the_measured_peaks():
+    """With measured peaks the kernel's floor is the slower of all operations at the general int32
+    rate and its ChaCha12 blocks at the measured ChaCha12 rate."""
+    cfg = W.CONFIGS[bench.CONFIG_KEY]
+    clk = {"sm_mhz": 1965.0}
+    peaks = {"int_tops": 30.0, "chacha_tops": 15.0, "int_probe": "mix_lop3_imad", "source": "test"}
+    r = bench.roofline(cfg, 10, 10 * 0.2, clk, 4, 2.5, 0, 0.0, peaks)
+    ops, blocks = 4 * bench.ip_row_ops(cfg), 4 * bench.chacha_blocks(cfg, cfg.level)
+    t_floor = max(ops / 30e12, blocks * 608 / 15e12)
+    assert math.isclose(r["peak"], ops / t_floor / 1e12)
+    assert math.isclose(r["frac"], t_floor / 200e-6)
+
+
+def test_path_op_model_matches_the_unit_costs():
+    """Per key switch at N=2^16, 36+12 primes, dnum 3, level 35: ModUp 0.83 G, ChaCha12 + inner
+    product 0.88 G, ModDown 0.58 G, 2.29 G in all; 144 (digit, limb) pairs of N/8 ChaCha12 blocks."""
+    cfg = W.CONFIGS[bench.CONFIG_KEY]
+    n, log_n = cfg.n, cfg.log_n
+    ntt = n // 2 * log_n * 8
+    assert bench.limb_ntt_ops(log_n) == ntt
+    assert bench.chacha_blocks(cfg, 35) == 3 * 48 * n // 8
+    # 36 inverse NTTs; per digit 36 targets x (12 multiply-adds + 1 reduction) and 36 NTTs
+    assert bench.modup_ops(cfg, 35) == 36 * ntt + 3 * 36 * n * (12 * 2 + 8) + 108 * ntt
+    # two components of 12 inverse NTTs, 36 x (12 multiply-adds + reduction), 36 NTTs, 36 combines
+    assert bench.moddown_ops(cfg, 35) == 2 * (12 * ntt + 36 * n * (12 * 2 + 8) + 36 * ntt + 36 * n * 6)
+    assert 2.2e9 < bench.keyswitch_ops(cfg, 35) < 2.4e9
+    # at level 20 with dnum 4 (alpha 9): digits of 9, 9, 3 primes
+    c5 = W.CONFIGS["n16-stream64"]
+    assert bench.digit_sizes(c5, 20) == [9, 9, 3]
+    assert bench.key_limbs(c5, 20) == 3 * 33
+
+
+def test_path_roofline_takes_the_slower_floor():
+    peaks = {"int_tops": 20.0, "chacha_tops": 10.0, "source": "test"}
+    r = bench.path_roofline(2e9, 1e6, 1e8, 1e-3, peaks)
+    t_int = max(2e9 / 20e12, 1e6 * 608 / 10e12)
+    t_hbm = 1e8 / (bench.HBM_PEAK_GBS * 1e9)
+    assert r["bound"] == ("alu" if t_int >= t_hbm else "hbm")
+    assert math.isclose(r["frac"], max(t_int, t_hbm) / 1e-3)
+    assert math.isclose(r["hbm_frac"], t_hbm / 1e-3)
 
 
 def test_alu_peak_and_op_model():

@@ -176,3 +176,43 @@ def test_bench_launch_configuration(ks_lib, oracle_mod):
         rel = octx.relin(octx.tensor(xi, yi, lvl), lvl, cfg.alpha, b_rel[i].cpu().numpy(), seeds[i], 0)
         want = octx.rotate(rel, lvl, cfg.alpha, g, b_rot[i].cpu().numpy(), seeds[i], g)
         assert np.array_equal(out[i].cpu().numpy(), want), i
+
+
+@pytest.mark.slow
+def test_n16_stream64_shared_keystream_batches(ks_lib, oracle_mod):
+    """The n16-stream64 line's launch configuration (N=2^16, level 20, dnum 4, so beta = 3):
+    ckks_relin_batch over 64 items with one relinearisation key, whose items form 8 groups of 8
+    that share one regenerated a half, and ckks_rotate_batch over 64 items with the 15 keys of
+    steps 2^(i mod 15), groups of 4 or 5 items.  Sampled items (the first and last of the batch,
+    and items inside a group) equal the oracle bit for bit."""
+    ks = ks_lib
+    cfg, q, p, ctx = _setup(ks, "n16-stream64")
+    lvl, N = cfg.level, cfg.n
+    na, P = lvl + 1, cfg.n_pairs
+    gen = W.rng(cfg.seed, W.TAG_SYNTH, 6464)
+    nd = -(-cfg.n_q // cfg.alpha)
+    shape = (nd, len(q) + len(p), N)
+    b_rel = W.uniform_residues((q + p) * nd, N, gen).reshape(shape)
+    steps = sorted(set(cfg.rot_steps), key=cfg.rot_steps.index)
+    gal = {r: ks.galois_element(cfg.log_n, r) for r in steps}
+    b_rot = {r: W.uniform_residues((q + p) * nd, N, gen).reshape(shape) for r in steps}
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    k_rel = ks.make_evk(dev(b_rel), cfg.chacha_seed, 0)
+    k_rot = {r: ks.make_evk(dev(b_rot[r]), cfg.chacha_seed, gal[r]) for r in steps}
+    d = W.uniform_residues(q[:na] * 3 * P, N, gen).reshape(P, 3, na, N)
+    ws = ctx.workspace(lvl, P)
+    r1 = torch.empty((P, 2, na, N), dtype=torch.uint32, device="cuda")
+    out = torch.empty_like(r1)
+    ks.ckks_relin_batch(ctx, dev(d), lvl, [k_rel] * P, r1, ws)
+    ks.ckks_rotate_batch(ctx, r1, lvl, [gal[r] for r in cfg.rot_steps], [k_rot[r] for r in cfg.rot_steps],
+                         out, ws)
+    torch.cuda.synchronize()
+    got_r, got_o = r1.cpu().numpy(), out.cpu().numpy()
+    octx = oracle_mod.Ctx(cfg.log_n, cfg.n_q, cfg.n_p)
+    for i in (0, 13, 63):           # 13: inside the relinearisation group of items 8..15
+        want = octx.relin(d[i], lvl, cfg.alpha, b_rel, cfg.chacha_seed, 0)
+        assert np.array_equal(got_r[i], want), ("relin", i)
+    for i in (0, 17, 63):           # 17: step 4's group is items 2, 17, 32, 47, 62
+        r = cfg.rot_steps[i]
+        want = octx.rotate(got_r[i], lvl, cfg.alpha, gal[r], b_rot[r], cfg.chacha_seed, gal[r])
+        assert np.array_equal(got_o[i], want), ("rotate", i)
