@@ -138,6 +138,7 @@ def run_ours(args, rank, world, local_rank):
     na = lvl + 1
     q, p = ks.ckks_gen_primes(cfg.log_n, cfg.n_q, cfg.n_p)
     ctx = ks.Context(cfg.log_n, q, p, cfg.dnum)
+    set_bconv(ks, ctx, args)
     g = ks.galois_element(cfg.log_n, cfg.rot_steps[0])
     nd = -(-cfg.n_q // cfg.alpha)
     mods = q + p
@@ -329,6 +330,7 @@ def run_ours(args, rank, world, local_rank):
             "dtype": "u32",
             "data": "synthetic",
             "config": dict(workload_config(cfg, B, world, args.stored_a, f"{S} CUDA streams x {Bs} units"),
+                           base_conversion=BCONV_ENGINES[args.bconv],
                            launch="one CUDA graph replay per step (captured per input set)" if graphs
                            else "eager launches"),
             "e2e": {"value": e2e_value, "unit": "key-switches/s", "h2d_bytes_per_step": h2d,
@@ -655,6 +657,7 @@ def run_workload(args, local_rank):
     ext = na + cfg.n_p
     q, p = ks.ckks_gen_primes(cfg.log_n, cfg.n_q, cfg.n_p)
     ctx = ks.Context(cfg.log_n, q, p, cfg.dnum)
+    set_bconv(ks, ctx, args)
     nd = -(-cfg.n_q // cfg.alpha)
     mods = q + p
     gen = W.rng(cfg.seed, W.TAG_SYNTH, 7)
@@ -800,6 +803,7 @@ def run_workload(args, local_rank):
     peaks = measure_int_peaks(ks, dev)
     t_step = ms / args.steps / 1e3
     line = {"workload": key, "informational": True, "config": INFO_DESCRIPTIONS[key],
+            "base_conversion": BCONV_ENGINES[args.bconv],
             "ms_per_step": ms / args.steps, "steps": args.steps, "warmup": args.warmup}
     if key == "rescale":
         line["rescales_per_s"] = R / t_step
@@ -905,6 +909,14 @@ def info_cpu_baseline(key: str, max_seconds: float = 8.0):
     dt = time.perf_counter() - t0
     return {"value": units * k / dt, "unit": unit, "cores": _omp_threads(), "kind": "oracle",
             "sample": f"{k} x {what} of {key} on synthetic residues, plain C oracle with OpenMP over limbs"}
+
+
+BCONV_ENGINES = {"cuda": "CUDA cores (32x32->64-bit multiply-adds)",
+                 "tensor": "tensor cores (8-bit split, tcgen05.mma kind::i8)"}
+
+
+def set_bconv(ks, ctx, args):
+    ks.ckks_set_bconv_mode(ctx, ks.CKKS_BCONV_TENSOR if args.bconv == "tensor" else ks.CKKS_BCONV_CUDA_CORES)
 
 
 def run_int_peaks(local_rank):
@@ -1043,6 +1055,9 @@ def main():
     ap.add_argument("--graph", action="store_true",
                     help="time one CUDA graph replay per step instead of eager launches (pays at small "
                          "batches; at 2 streams x 4 units the other stream already hides launch gaps)")
+    ap.add_argument("--bconv", default="cuda", choices=sorted(BCONV_ENGINES),
+                    help="base-conversion engine: cuda (CUDA cores, default) or tensor (8-bit split on the "
+                         "tensor cores); the output bits are the same")
     ap.add_argument("--int-peaks", action="store_true",
                     help="measure this GPU's integer throughput per instruction class (ckks_int_probe) and "
                          "print it as one JSON line")

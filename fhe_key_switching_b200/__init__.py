@@ -71,6 +71,7 @@ _SIGS = {
     "ckks_keyswitch_noalloc": (_ci, [_vp, _vp, _ci, ctypes.POINTER(ckks_evk), _vp, _vp]),
     "ckks_prof_begin": (_ci, [_vp, ctypes.c_char_p, _ci]),
     "ckks_prof_end": (_ci, [_vp, ctypes.POINTER(_ci), ctypes.POINTER(ctypes.c_double)]),
+    "ckks_set_bconv_mode": (_ci, [_vp, _ci]),
     "ckks_int_probe": (_ci, [_ci, _ci, _ci, _vp, _vp, ctypes.POINTER(ctypes.c_float),
                              ctypes.POINTER(ctypes.c_double)]),
     "ckks_last_error": (ctypes.c_char_p, []),
@@ -337,6 +338,15 @@ def ckks_prof_end(ctx):
     ms = ctypes.c_double()
     _check(_L.ckks_prof_end(ctx.handle, ctypes.byref(n), ctypes.byref(ms)), "ckks_prof_end")
     return n.value, ms.value
+
+
+CKKS_BCONV_CUDA_CORES, CKKS_BCONV_TENSOR = 0, 1
+
+
+def ckks_set_bconv_mode(ctx, mode: int):
+    """Base-conversion engine of later calls on ctx: CKKS_BCONV_CUDA_CORES (default) or
+    CKKS_BCONV_TENSOR (8-bit contraction on the tensor cores); same output bits either way."""
+    _check(_L.ckks_set_bconv_mode(ctx.handle, mode), "ckks_set_bconv_mode")
 
 
 def ckks_int_probe(op: int, blocks: int, iters: int, sink, stream=None):

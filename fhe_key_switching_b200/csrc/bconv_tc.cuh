@@ -1,0 +1,223 @@
+// bconv_tc.cuh -- fast base conversion as an 8-bit integer contraction on the tensor cores
+// (tcgen05.mma kind::i8, accumulators in tensor memory).
+//
+// The conversion of one group (a ModUp digit or the ModDown special primes) is
+//   out_t[n] = sum_i y_i[n] [D/r_i]_t + v[n] [-D]_t   (mod t),   v[n] = #{i : y_i[n] > (r_i-1)/2},
+// the centred fast base conversion (Cheon, Han, Kim, Kim, Song, SAC 2018) that k_bconv_n computes
+// with 64-bit multiply-adds.  Here it is split into bytes so that it becomes an exact u8 x u8 ->
+// s32 matrix product:
+//   A[n][k] = byte a of y_i[n] for k = 4i + a (i < n_in), A[n][4 n_in] = v[n], 0 beyond;
+//   B'[k][t] = [[D/r_i]_t 2^(8a)]_t for k = 4i + a, B'[4 n_in][t] = [-D]_t;
+//   B[k][4u + c] = byte c of B'[k][t_u]   (4 columns per target t_u);
+//   G[n][4u + c] = sum_k A[n][k] B[k][4u + c]  <  64 * 255 * 255 < 2^22  (exact in s32);
+//   out_t[n] = sum_c G[n][4u + c] 2^(8c) = s1 + s2 2^16 (mod t) with s1 = G0 + 2^8 G1 and
+//   s2 = G2 + 2^8 G3, both below 2^31, reduced with one Shoup product by [2^16]_t = 2^16.
+// Since sum_k A[n][k] B'[k][t] = sum_i y_i [D/r_i]_t + v [-D]_t exactly as integers modulo t,
+// the result is the same residue as k_bconv_n's; like it, it is left lazily in [0, 4t), which
+// the forward NTT that always follows accepts.
+//
+// Tile: M = 128 coefficients (one per tensor-memory lane), K = 64 bytes (n_in <= 15), N = 4 x
+// (targets of the chunk), at most 128 columns.  A CTA of 128 threads (4 warps) stages the
+// chunk's B once, then loops over coefficient tiles: every thread transposes its coefficient's
+// n_in inputs into one A row in shared memory, thread 0 issues the two K = 32 MMAs and commits
+// them to an mbarrier, and every thread reads its row's accumulators back (tcgen05.ld), combines
+// them and stores its targets' outputs (one coalesced 128-byte row segment per warp and target).
+// Both operands are K-major without swizzle: core matrices of 8 rows x 16 bytes, stored
+// [16-byte K chunk][row][16 bytes], so the leading-dimension offset (next K chunk) is
+// rows x 16 bytes and the stride-dimension offset (next 8 rows) is 128 bytes.
+#pragma once
+#include "ntt.cuh"
+
+constexpr int TC_M = 128;                 // coefficients per tile = tensor-memory lanes
+constexpr int TC_K = 64;                  // K bytes (two MMAs of K = 32)
+constexpr int TC_MAX_IN = 15;             // 4 * 15 + 1 = 61 <= 64
+constexpr int TC_MAX_T = 32;              // targets per chunk: N = 4 T <= 128 columns
+constexpr int TC_THREADS = 128;
+constexpr int TC_TILES = 4;               // coefficient tiles per CTA
+constexpr int TC_COLS = 128;              // tensor-memory columns a CTA allocates
+// Dynamic shared memory per CTA: A (8 KB) + B (<= 8 KB) + target records, padded so that at most
+// 4 CTAs share an SM (4 x 128 columns = all 512 columns of tensor memory: no CTA waits in alloc;
+// 5 x 53 KB would exceed the SM's 228 KB).
+constexpr size_t TC_SMEM = 52 * 1024;
+constexpr int TC_A_BYTES = 4 * TC_M * 16;  // [4 K chunks][128 rows][16 B]
+
+struct BconvTcArgs {
+    const u32 *y;            // input rows
+    u32 *out;                // output rows
+    const uint4 *tb;         // per (config, global prime t): [4 columns c][4 K chunks] x 16 bytes
+    const PrimeInfo *pinfo;
+    JobMap map;              // targets: per_group, split, bases, out rows, skip_alpha
+    int n_primes, log_n;
+    int in_row0, in_group_rows, in_prime0, in_prime_step;
+    int n_in_full, n_in_last, n_groups, cfg_per_group, g_base;
+    int nchunk, tchunk;      // target chunks per item (blockIdx.z = item * nchunk + chunk)
+    size_t y_item, out_item;
+    int *err;                // device error word: CKKS_DEV_ERR_WAIT when a wait expires
+};
+
+__device__ __forceinline__ u32 tc_smem_u32(const void *p) { return (u32)__cvta_generic_to_shared(p); }
+
+// K-major, no swizzle: start address, leading-dimension byte offset (next 16-byte K chunk),
+// stride-dimension byte offset (next 8 rows), descriptor version 1, layout type 0.
+__device__ __forceinline__ u64 tc_smem_desc(u32 addr, u32 lbo, u32 sbo) {
+    return (u64)((addr >> 4) & 0x3FFFu) | ((u64)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((u64)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+
+// Instruction descriptor of kind::i8: s32 accumulator, unsigned 8-bit A and B, both K-major,
+// N >> 3 at bit 17, M >> 4 at bit 24.
+__host__ __device__ constexpr u32 tc_idesc(int m, int n) {
+    return (2u << 4) | ((u32)(n >> 3) << 17) | ((u32)(m >> 4) << 24);
+}
+
+__device__ __forceinline__ void tc_mma(u32 d_tmem, u64 adesc, u64 bdesc, u32 idesc, u32 accumulate) {
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}"
+                 ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate) : "memory");
+}
+
+__device__ __forceinline__ void tc_commit(u64 *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 ::"r"(tc_smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void tc_ld16(u32 taddr, u32 (&r)[16]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+                 "%12, %13, %14, %15}, [%16];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                   "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+                   "=r"(r[14]), "=r"(r[15])
+                 : "r"(taddr));
+}
+
+__device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// Included by ks_kernels.cuh after the mbarrier helpers (mbar_init, mbar_wait_bounded,
+// CKKS_DEV_ERR_WAIT), which the kernel below uses.
+constexpr int TC_REC_OFF = TC_A_BYTES + 4 * (4 * TC_MAX_T) * 16;   // per-target records after A and B
+
+__global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
+    extern __shared__ __align__(1024) unsigned char tc_sm[];
+    __shared__ __align__(8) u64 bar;
+    __shared__ u32 tmem_base;
+    __shared__ u32 half_s[TC_MAX_IN];
+    unsigned char *As = tc_sm;                                    // [4 K chunks][128 rows][16 B]
+    unsigned char *Bs = tc_sm + TC_A_BYTES;                       // [4 K chunks][N rows][16 B]
+    uint4 *trec = reinterpret_cast<uint4 *>(tc_sm + TC_REC_OFF);  // per target: (t, 2t, Shoup(2^16), row)
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int g = a.g_base + blockIdx.y;
+    const int item = blockIdx.z / a.nchunk, chunk = blockIdx.z % a.nchunk;
+    const int n = 1 << a.log_n;
+    const int n_in = (g == a.n_groups - 1) ? a.n_in_last : a.n_in_full;
+    const int cfg = a.cfg_per_group ? g * a.cfg_per_group + (n_in - 1) : 0;
+    const int T = a.map.per_group;
+    const int lo = a.map.skip_alpha > 0 ? g * a.map.skip_alpha : 0;
+    const int hi = a.map.skip_alpha > 0 ? min(lo + a.map.skip_alpha, a.map.split) : 0;
+    const int u0 = chunk * a.tchunk;
+    const int Tc = min(a.tchunk, T - (hi - lo) - u0);             // targets of this chunk
+    if (Tc <= 0) return;                                          // (uniform: before any barrier)
+    const int N = (4 * Tc + 15) & ~15;
+    auto target_pos = [&](int u) { const int idx = u0 + u; return idx < lo ? idx : idx + (hi - lo); };
+    auto prime_of = [&](int kk) { return kk < a.map.split ? a.map.lo_base + kk : a.map.hi_base + (kk - a.map.split); };
+    const int p0 = a.in_prime0 + g * a.in_prime_step;
+    for (int i = tid; i < n_in; i += TC_THREADS) half_s[i] = a.pinfo[p0 + i].half;
+    for (int u = tid; u < Tc; u += TC_THREADS) {
+        const int kk = target_pos(u);
+        const u32 q = a.pinfo[prime_of(kk)].q;
+        trec[u] = make_uint4(q, 2u * q, (u32)((1ull << 48) / q), (u32)kk);
+    }
+    for (int idx = tid; idx < 4 * N; idx += TC_THREADS) {        // B: (K chunk, column) -> 16 bytes
+        const int kc = idx / N, col = idx - kc * N;
+        const int u = col >> 2, c = col & 3;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (u < Tc) v = a.tb[((size_t)cfg * a.n_primes + prime_of(target_pos(u))) * 16 + c * 4 + kc];
+        reinterpret_cast<uint4 *>(Bs)[(size_t)kc * N + col] = v;
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(tc_smem_u32(&tmem_base)), "r"(TC_COLS) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (tid == 0) {
+        mbar_init(&bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    tc_fence_async_smem();                                        // B visible to the tensor cores
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const u32 tmem = tmem_base;
+    const u32 taddr = tmem + ((u32)(warp * 32) << 16);            // this warp's 32 lanes
+    const u32 idesc = tc_idesc(TC_M, N);
+    const u32 a_base = tc_smem_u32(As), b_base = tc_smem_u32(Bs);
+    const u32 *yb = a.y + item * a.y_item + (size_t)(a.in_row0 + g * a.in_group_rows) * n;
+    u32 *ob = a.out + item * a.out_item + ((size_t)g * a.map.out_group_rows + a.map.out_k_base) * n;
+    int failed_phase = -1;
+    for (int tile = 0; tile < TC_TILES; tile++) {
+        const int nc = (blockIdx.x * TC_TILES + tile) * TC_M + tid;   // this thread's coefficient
+        u32 w[16];
+        u32 vcount = 0;
+#pragma unroll
+        for (int i = 0; i < 16; i++) {
+            u32 val = 0;
+            if (i < n_in) {
+                val = yb[(size_t)i * n + nc];
+                vcount += val > half_s[i] ? 1u : 0u;
+            } else if (i == n_in) {
+                val = vcount;
+            }
+            w[i] = val;
+        }
+        uint4 *arow = reinterpret_cast<uint4 *>(As) + tid;
+#pragma unroll
+        for (int kc = 0; kc < 4; kc++)
+            arow[kc * TC_M] = make_uint4(w[4 * kc], w[4 * kc + 1], w[4 * kc + 2], w[4 * kc + 3]);
+        tc_fence_async_smem();                                    // A visible to the tensor cores
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int s = 0; s < 2; s++)
+                tc_mma(tmem, tc_smem_desc(a_base + (u32)(2 * s * TC_M * 16), TC_M * 16, 128),
+                       tc_smem_desc(b_base + (u32)(2 * s * N * 16), (u32)N * 16, 128), idesc, (u32)s);
+            tc_commit(&bar);
+        }
+        const bool expired = !mbar_wait_bounded(&bar, (u32)(tile & 1));
+        if (__syncthreads_or(expired)) {                          // leave together
+            failed_phase = tile & 1;
+            break;
+        }
+        tc_fence_after();
+        for (int c0 = 0; c0 < 4 * Tc; c0 += 16) {
+            u32 r[16];
+            tc_ld16(taddr + (u32)c0, r);
+            tc_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                const int u = (c0 >> 2) + j;
+                if (u < Tc) {
+                    const uint4 rec = trec[u];
+                    const u32 s1 = r[4 * j] + (r[4 * j + 1] << 8);
+                    const u32 s2 = r[4 * j + 2] + (r[4 * j + 3] << 8);
+                    ob[(size_t)rec.w * n + nc] = shoup_mul(s2, 65536u, rec.z, rec.x) + csub(s1, rec.y);
+                }
+            }
+        }
+        tc_fence_before();                                        // reads done before the next MMA
+    }
+    if (failed_phase >= 0) {
+        // record the failure and give the MMA in flight a second bounded wait before freeing its
+        // tensor memory
+        if (tid == 0) atomicOr(a.err, CKKS_DEV_ERR_WAIT);
+        (void)mbar_wait_bounded(&bar, (u32)failed_phase);
+    }
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TC_COLS) : "memory");
+    }
+}

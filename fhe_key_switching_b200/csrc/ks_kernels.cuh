@@ -825,3 +825,6 @@ k_sum_parts(SumArgs a) {
     }
     reinterpret_cast<uint4 *>(a.out + (size_t)r * n)[c4] = s;
 }
+
+// ---------------------------------------------------------------- base conversion on the tensor cores
+#include "bconv_tc.cuh"

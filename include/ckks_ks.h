@@ -209,6 +209,18 @@ int ckks_bsgs(ckks_ctx *ctx, const uint32_t *ct, int level, int n_baby, const ui
               const ckks_evk *baby_keys, int n_giant, const uint32_t *giant_galois, const ckks_evk *giant_keys,
               const uint32_t *pt, uint32_t *out, void *ws, size_t ws_bytes, ckks_stream_t stream);
 
+/* Base-conversion engine (the results are the same residues either way; the bits of every
+ * entry point's output are identical):
+ *  CKKS_BCONV_CUDA_CORES (default): 32 x 32 -> 64-bit multiply-adds on the CUDA cores;
+ *  CKKS_BCONV_TENSOR: the conversion as an exact 8-bit contraction on the tensor cores
+ *    (tcgen05.mma kind::i8, sm_100a): inputs and constants split into bytes, 4 byte columns per
+ *    target summed with shifts 0, 8, 16, 24 in the epilogue.  Groups of more than 15 primes
+ *    still use the CUDA cores.
+ * The mode applies to later calls on the context; it is not synchronised with calls in flight
+ * from other threads.  CKKS_ERR_ARG for an unknown mode. */
+enum { CKKS_BCONV_CUDA_CORES = 0, CKKS_BCONV_TENSOR = 1 };
+int ckks_set_bconv_mode(ckks_ctx *ctx, int mode);
+
 /* The key's regenerated uniform half for one (digit, global limb): out [N] (device),
  * out[n] = w mod q_t with w = (x[2m] | x[2m+1] << 32), m = n mod 8, x = ChaCha12 block
  * (RFC 8439 state: key = seed as 8 LE words, counter = n/8, nonce = (key_id, digit, limb)). */

@@ -45,23 +45,27 @@ def _prod_mod(ms, m) -> int:
     return r
 
 
-def _setup(ks, oracle_mod, key):
+def _setup(ks, oracle_mod, key, mode):
     cfg = W.CONFIGS[key]
     q, p = ks.ckks_gen_primes(cfg.log_n, cfg.n_q, cfg.n_p)
     octx = oracle_mod.Ctx(cfg.log_n, cfg.n_q, cfg.n_p)
     assert octx.q == q and octx.p == p
-    return cfg, octx, ks.Context(cfg.log_n, q, p, cfg.dnum)
+    ctx = ks.Context(cfg.log_n, q, p, cfg.dnum)
+    ks.ckks_set_bconv_mode(ctx, ks.CKKS_BCONV_TENSOR if mode == "tensor" else ks.CKKS_BCONV_CUDA_CORES)
+    return cfg, octx, ctx
 
 
 CASES = [("n12-dnum2", 3), ("n14-hoisted8", 11), ("n14-hoisted8", 6), ("n16-full", 35)]
+MODES = ["cuda_cores", "tensor"]       # the base-conversion engine (same bits either way)
 
 
 @pytest.mark.gpu
+@pytest.mark.parametrize("mode", MODES)
 @pytest.mark.parametrize("key,level", CASES)
-def test_modup_threshold(ks_lib, oracle_mod, key, level):
+def test_modup_threshold(ks_lib, oracle_mod, key, level, mode):
     """ModUp: y_i = iNTT(c_i) (D_j/q_i)^-1 lands on the thresholds, so c_i = NTT(y_i (D_j/q_i))."""
     ks = ks_lib
-    cfg, octx, ctx = _setup(ks, oracle_mod, key)
+    cfg, octx, ctx = _setup(ks, oracle_mod, key, mode)
     n, na, alpha = cfg.n, level + 1, cfg.alpha
     gen = W.rng(cfg.seed, W.TAG_SYNTH, 5150 + level)
     coef = np.empty((na, n), dtype=np.uint32)
@@ -79,11 +83,12 @@ def test_modup_threshold(ks_lib, oracle_mod, key, level):
 
 
 @pytest.mark.gpu
+@pytest.mark.parametrize("mode", MODES)
 @pytest.mark.parametrize("key,level", CASES)
-def test_moddown_threshold(ks_lib, oracle_mod, key, level):
+def test_moddown_threshold(ks_lib, oracle_mod, key, level, mode):
     """ModDown: the special limbs' y_i = iNTT(acc_{p_i}) (P/p_i)^-1 land on the thresholds."""
     ks = ks_lib
-    cfg, octx, ctx = _setup(ks, oracle_mod, key)
+    cfg, octx, ctx = _setup(ks, oracle_mod, key, mode)
     n, na, k = cfg.n, level + 1, cfg.n_p
     gen = W.rng(cfg.seed, W.TAG_SYNTH, 6150 + level)
     acc = W.uniform_residues(octx.q[:na] + octx.p, n, gen)
@@ -99,11 +104,12 @@ def test_moddown_threshold(ks_lib, oracle_mod, key, level):
 
 
 @pytest.mark.gpu
+@pytest.mark.parametrize("mode", MODES)
 @pytest.mark.parametrize("key,level", CASES)
-def test_rescale_threshold(ks_lib, oracle_mod, key, level):
+def test_rescale_threshold(ks_lib, oracle_mod, key, level, mode):
     """Rescale: limb l of both components holds (q_l -+ 1)/2, 0 and q_l - 1 as coefficients."""
     ks = ks_lib
-    cfg, octx, ctx = _setup(ks, oracle_mod, key)
+    cfg, octx, ctx = _setup(ks, oracle_mod, key, mode)
     n, na = cfg.n, level + 1
     gen = W.rng(cfg.seed, W.TAG_SYNTH, 7150 + level)
     ct = W.uniform_residues(octx.q[:na] * 2, n, gen).reshape(2, na, n)
