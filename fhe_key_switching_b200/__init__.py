@@ -72,6 +72,7 @@ _SIGS = {
     "ckks_prof_begin": (_ci, [_vp, ctypes.c_char_p, _ci]),
     "ckks_prof_end": (_ci, [_vp, ctypes.POINTER(_ci), ctypes.POINTER(ctypes.c_double)]),
     "ckks_set_bconv_mode": (_ci, [_vp, _ci]),
+    "ckks_modraise": (_ci, [_vp, _vp, _ci, _vp, _vp, _sz, _vp]),
     "ckks_int_probe": (_ci, [_ci, _ci, _ci, _vp, _vp, ctypes.POINTER(ctypes.c_float),
                              ctypes.POINTER(ctypes.c_double)]),
     "ckks_last_error": (ctypes.c_char_p, []),
@@ -338,6 +339,12 @@ def ckks_prof_end(ctx):
     ms = ctypes.c_double()
     _check(_L.ckks_prof_end(ctx.handle, ctypes.byref(n), ctypes.byref(ms)), "ckks_prof_end")
     return n.value, ms.value
+
+
+def ckks_modraise(ctx, ct, level: int, out, ws, stream=None):
+    """ModRaise: ct [2][1][N] at level 0 -> out [2][level+1][N] (centred lift of the q_0 residues)."""
+    _check(_L.ckks_modraise(ctx.handle, _ptr(ct), level, _ptr(out), _ptr(ws), ws.numel() * ws.element_size(),
+                            _stream(stream)), "ckks_modraise")
 
 
 CKKS_BCONV_CUDA_CORES, CKKS_BCONV_TENSOR = 0, 1

@@ -209,6 +209,17 @@ int ckks_bsgs(ckks_ctx *ctx, const uint32_t *ct, int level, int n_baby, const ui
               const ckks_evk *baby_keys, int n_giant, const uint32_t *giant_galois, const ckks_evk *giant_keys,
               const uint32_t *pt, uint32_t *out, void *ws, size_t ws_bytes, ckks_stream_t stream);
 
+/* ModRaise, the first step of CKKS bootstrapping (Cheon, Han, Kim, Kim, Song, Eurocrypt 2018;
+ * the pages give no construction): a ciphertext at level 0, ct [2][1][N] (evaluation domain mod
+ * q_0), is read as integer polynomials with centred coefficients in (-q_0/2, q_0/2] and reduced
+ * into q_0..q_level: out [2][level+1][N], evaluation domain, canonical.  Per component: inverse
+ * NTT mod q_0, centred lift, NTT in every limb.  It decrypts to m + q_0 I with a small integer
+ * polynomial I, which the bootstrapping's modular reduction then removes.
+ * Workspace: 2 N words (ws_bytes >= 8 N).  out must not overlap ct, and ws neither
+ * (CKKS_ERR_ARG); other errors as for the key-switching calls. */
+int ckks_modraise(ckks_ctx *ctx, const uint32_t *ct, int level, uint32_t *out, void *ws, size_t ws_bytes,
+                  ckks_stream_t stream);
+
 /* Base-conversion engine (the results are the same residues either way; the bits of every
  * entry point's output are identical):
  *  CKKS_BCONV_CUDA_CORES (default): 32 x 32 -> 64-bit multiply-adds on the CUDA cores;

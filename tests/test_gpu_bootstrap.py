@@ -1,0 +1,85 @@
+"""The linear parts of bootstrapping on the GPU against the oracle, bit for bit.
+
+ModRaise (ckks_modraise) and the DFT levels of CoeffToSlot and SlotToCoeff, each level one
+baby-step giant-step transform (ckks_bsgs, double hoisting) with the level's slot diagonals
+encoded by the oracle at scale q_level, followed by one rescale (ckks_rescale).  Every level's
+output equals the oracle's; the last one also decodes to the numpy map (the oracle's own pin in
+tests/test_oracle_dft.py)."""
+import numpy as np
+import pytest
+
+import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+def _dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.uint32)).cuda()
+
+
+def _host(t):
+    torch.cuda.synchronize()
+    return t.cpu().numpy()
+
+
+@pytest.mark.parametrize("key,level", [("n12-dnum4", 3), ("n14-hoisted8", 11), ("n16-full", 35)])
+def test_modraise_parity(ks_lib, oracle_mod, key, level):
+    from oracle import bootstrap as bt
+    ks = ks_lib
+    cfg = W.CONFIGS[key]
+    q, p = ks.ckks_gen_primes(cfg.log_n, cfg.n_q, cfg.n_p)
+    octx = oracle_mod.Ctx(cfg.log_n, cfg.n_q, cfg.n_p)
+    ctx = ks.Context(cfg.log_n, q, p, cfg.dnum)
+    ct = W.uniform_residues([q[0]] * 2, cfg.n, W.rng(cfg.seed, W.TAG_SYNTH, 9100)).reshape(2, 1, cfg.n)
+    out = torch.empty((2, level + 1, cfg.n), dtype=torch.uint32, device="cuda")
+    ws = torch.empty(2 * cfg.n, dtype=torch.uint32, device="cuda")
+    ks.ckks_modraise(ctx, _dev(ct), level, out, ws)
+    assert np.array_equal(_host(out), bt.modraise(octx, ct, level))
+
+
+@pytest.mark.parametrize("direction", ["coeff_to_slot", "slot_to_coeff"])
+@pytest.mark.parametrize("key,levels,n1", [("n12-dnum4", 3, 4), ("n14-hoisted8", 3, 8)])
+def test_dft_levels_parity(ks_lib, oracle_mod, key, levels, n1, direction):
+    from oracle import bootstrap as bt
+    from oracle.scenario import Scenario
+    ks = ks_lib
+    cfg = W.CONFIGS[key]
+    sc = Scenario(cfg)
+    octx, log_n, ns = sc.ctx, cfg.log_n, cfg.n // 2
+    q, p = ks.ckks_gen_primes(cfg.log_n, cfg.n_q, cfg.n_p)
+    ctx = ks.Context(cfg.log_n, q, p, cfg.dnum)
+    inverse = direction == "coeff_to_slot"
+    z, ct = sc.ciphertext(0)
+    if not inverse:
+        z = z / 4.0
+        ct = sc.encrypt_slots(z, 0)
+    lvl = cfg.level
+    keys, evks = {}, {}
+    g_ct = _dev(ct)
+    for lens in bt.split_levels(log_n, levels, inverse):
+        babies, giants, pt = bt.bsgs_plan(bt.level_diagonals(log_n, lens, inverse), ns, n1)
+        for s in babies + giants:
+            g = bt.galois_of_shift(octx, s)
+            if g != 1 and g not in keys:
+                keys[g] = sc.key(g)
+                evks[g] = ks.make_evk(_dev(keys[g]), cfg.chacha_seed, g)
+        enc = bt.encode_plan(octx, pt, lvl, float(octx.q[lvl]))
+        want = bt.linear_level(octx, ct, lvl, cfg.alpha, babies, giants, enc, keys, cfg.chacha_seed)
+        bg = [bt.galois_of_shift(octx, s) for s in babies]
+        gg = [bt.galois_of_shift(octx, s) for s in giants]
+        na = lvl + 1
+        mid = torch.empty((2, na, cfg.n), dtype=torch.uint32, device="cuda")
+        ws = ks.ckks_bsgs_workspace(ctx, lvl, len(bg), len(gg))
+        ks.ckks_bsgs(ctx, g_ct, lvl, bg, [evks.get(g) for g in bg], gg, [evks.get(g) for g in gg], _dev(enc),
+                     mid, ws)
+        g_next = torch.empty((2, lvl, cfg.n), dtype=torch.uint32, device="cuda")
+        ks.ckks_rescale(ctx, mid, lvl, g_next, ctx.workspace(lvl))
+        assert ks.ckks_sync_status(ctx, None, 10000) == ks.CKKS_OK
+        assert np.array_equal(_host(g_next), want), (direction, lvl)
+        ct, g_ct, lvl = want, g_next, lvl - 1
+    got = sc.decrypt_slots(_host(g_ct), lvl)
+    ref = bt.coeff_to_slot(z, log_n, levels) if inverse else bt.slot_to_coeff(z, log_n, levels)
+    err = np.max(np.abs(got - ref))
+    assert err < (2.0 ** -8 if inverse else 2.0 ** -9 * np.max(np.abs(ref))), err
