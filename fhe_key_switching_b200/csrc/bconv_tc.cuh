@@ -156,9 +156,9 @@ __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
     const u32 *yb = a.y + item * a.y_item + (size_t)(a.in_row0 + g * a.in_group_rows) * n;
     u32 *ob = a.out + item * a.out_item + ((size_t)g * a.map.out_group_rows + a.map.out_k_base) * n;
     int failed_phase = -1;
-    for (int tile = 0; tile < TC_TILES; tile++) {
-        const int nc = (blockIdx.x * TC_TILES + tile) * TC_M + tid;   // this thread's coefficient
-        u32 w[16];
+    // this thread's A row of tile `tile`: its coefficient's n_in inputs, the count v, zeros
+    auto load_row = [&](int tile, u32 (&w)[16]) {
+        const int nc = (blockIdx.x * TC_TILES + tile) * TC_M + tid;
         u32 vcount = 0;
 #pragma unroll
         for (int i = 0; i < 16; i++) {
@@ -171,6 +171,11 @@ __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
             }
             w[i] = val;
         }
+    };
+    u32 w[16];
+    load_row(0, w);
+    for (int tile = 0; tile < TC_TILES; tile++) {
+        const int nc = (blockIdx.x * TC_TILES + tile) * TC_M + tid;   // this thread's coefficient
         uint4 *arow = reinterpret_cast<uint4 *>(As) + tid;
 #pragma unroll
         for (int kc = 0; kc < 4; kc++)
@@ -186,6 +191,8 @@ __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
                        tc_smem_desc(b_base + (u32)(2 * s * N * 16), (u32)N * 16, 128), idesc, (u32)s);
             tc_commit(&bar);
         }
+        // the next tile's inputs load while the tensor cores and this tile's epilogue run
+        if (tile + 1 < TC_TILES) load_row(tile + 1, w);
         const bool expired = !mbar_wait_bounded(&bar, (u32)(tile & 1));
         if (__syncthreads_or(expired)) {                          // leave together
             failed_phase = tile & 1;
