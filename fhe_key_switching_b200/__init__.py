@@ -73,6 +73,8 @@ _SIGS = {
     "ckks_prof_end": (_ci, [_vp, ctypes.POINTER(_ci), ctypes.POINTER(ctypes.c_double)]),
     "ckks_set_bconv_mode": (_ci, [_vp, _ci]),
     "ckks_modraise": (_ci, [_vp, _vp, _ci, _vp, _vp, _sz, _vp]),
+    "ckks_encode": (_ci, [_vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double), ctypes.c_double,
+                          _ci, _ci, _vp, _vp, _sz, _vp]),
     "ckks_int_probe": (_ci, [_ci, _ci, _ci, _vp, _vp, ctypes.POINTER(ctypes.c_float),
                              ctypes.POINTER(ctypes.c_double)]),
     "ckks_last_error": (ctypes.c_char_p, []),
@@ -339,6 +341,18 @@ def ckks_prof_end(ctx):
     ms = ctypes.c_double()
     _check(_L.ckks_prof_end(ctx.handle, ctypes.byref(n), ctypes.byref(ms)), "ckks_prof_end")
     return n.value, ms.value
+
+
+def ckks_encode(ctx, slots, scale: float, level: int, out, ws, with_special: bool = False, stream=None):
+    """CKKS encoding of N/2 complex slots (a host sequence of complex numbers) at `scale` into out
+    [(level+1) (+ n_p)][N] (CUDA uint32, evaluation domain); ws: CUDA buffer of >= 8 N bytes."""
+    n = len(slots)
+    if n != ctx.n // 2:
+        raise ValueError(f"expected N/2 = {ctx.n // 2} slots, got {n}")
+    re = (ctypes.c_double * n)(*[complex(v).real for v in slots])
+    im = (ctypes.c_double * n)(*[complex(v).imag for v in slots])
+    _check(_L.ckks_encode(ctx.handle, re, im, float(scale), level, 1 if with_special else 0, _ptr(out), _ptr(ws),
+                          ws.numel() * ws.element_size(), _stream(stream)), "ckks_encode")
 
 
 def ckks_modraise(ctx, ct, level: int, out, ws, stream=None):

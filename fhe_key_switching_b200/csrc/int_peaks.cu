@@ -82,41 +82,41 @@ __global__ void __launch_bounds__(PROBE_THREADS) k_int_probe(u32 *sink, int iter
             for (int i = 0; i < 16; i++) acc ^= o[i];
         }
         sink[tid] = acc;
-        return;
-    }
-    for (int it = 0; it < iters; it++) {
+    } else {
+        for (int it = 0; it < iters; it++) {
 #pragma unroll
-        for (int r = 0; r < PROBE_UNROLL; r++) {
+            for (int r = 0; r < PROBE_UNROLL; r++) {
 #pragma unroll
-            for (int k = 0; k < PROBE_CHAINS; k++) {
-                if (OP == CKKS_PROBE_IADD) {
-                    a[k] = op_add(a[k], b[k]);
-                    b[k] = op_add(b[k], a[k]);
-                } else if (OP == CKKS_PROBE_LOP3) {
-                    a[k] = op_lop3<0x96>(a[k], b[k], c[k]);     // a ^ b ^ c
-                    b[k] = op_lop3<0xE8>(b[k], c[k], a[k]);     // majority(b, c, a)
-                } else if (OP == CKKS_PROBE_SHF) {
-                    a[k] = op_shf<7>(a[k], b[k]);
-                    b[k] = op_shf<13>(b[k], a[k]);
-                } else if (OP == CKKS_PROBE_IMAD) {
-                    a[k] = op_mad(a[k], b[k], c[k]);
-                    b[k] = op_mad(b[k], a[k], c[k]);
-                } else if (OP == CKKS_PROBE_IMAD_HI) {
-                    a[k] = op_madhi(a[k], b[k], c[k]);
-                    b[k] = op_madhi(b[k], a[k], c[k]);
-                } else if (OP == CKKS_PROBE_IMAD_WIDE) {
-                    w[k] = op_madwide((u32)w[k], c[k], w[k]);
-                } else if (OP == CKKS_PROBE_MIX) {              // one logic op and one multiply-add
-                    a[k] = op_lop3<0x96>(a[k], b[k], c[k]);
-                    b[k] = op_mad(b[k], a[k], c[k]);
+                for (int k = 0; k < PROBE_CHAINS; k++) {
+                    if (OP == CKKS_PROBE_IADD) {
+                        a[k] = op_add(a[k], b[k]);
+                        b[k] = op_add(b[k], a[k]);
+                    } else if (OP == CKKS_PROBE_LOP3) {
+                        a[k] = op_lop3<0x96>(a[k], b[k], c[k]);     // a ^ b ^ c
+                        b[k] = op_lop3<0xE8>(b[k], c[k], a[k]);     // majority(b, c, a)
+                    } else if (OP == CKKS_PROBE_SHF) {
+                        a[k] = op_shf<7>(a[k], b[k]);
+                        b[k] = op_shf<13>(b[k], a[k]);
+                    } else if (OP == CKKS_PROBE_IMAD) {
+                        a[k] = op_mad(a[k], b[k], c[k]);
+                        b[k] = op_mad(b[k], a[k], c[k]);
+                    } else if (OP == CKKS_PROBE_IMAD_HI) {
+                        a[k] = op_madhi(a[k], b[k], c[k]);
+                        b[k] = op_madhi(b[k], a[k], c[k]);
+                    } else if (OP == CKKS_PROBE_IMAD_WIDE) {
+                        w[k] = op_madwide((u32)w[k], c[k], w[k]);
+                    } else if (OP == CKKS_PROBE_MIX) {              // one logic op and one multiply-add
+                        a[k] = op_lop3<0x96>(a[k], b[k], c[k]);
+                        b[k] = op_mad(b[k], a[k], c[k]);
+                    }
                 }
             }
         }
-    }
-    u32 s = 0;
+        u32 s = 0;
 #pragma unroll
-    for (int k = 0; k < PROBE_CHAINS; k++) s ^= a[k] ^ b[k] ^ (u32)w[k] ^ (u32)(w[k] >> 32);
-    sink[tid] = s;
+        for (int k = 0; k < PROBE_CHAINS; k++) s ^= a[k] ^ b[k] ^ (u32)w[k] ^ (u32)(w[k] >> 32);
+        sink[tid] = s;
+    }
 }
 
 }  // namespace

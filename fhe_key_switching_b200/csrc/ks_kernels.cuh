@@ -337,6 +337,21 @@ __global__ void k_automorph(const u32 *in, u32 *out, int log_n, u32 g) {
     out[off + k] = in[off + automorph_src((u32)k, g, log_n)];
 }
 
+// Signed integer coefficients into RNS rows: out[row][k] = m[k] mod t (canonical), the rows
+// mapped to primes like an NTT job map (the forward NTT follows).
+__global__ void k_encode_rns(const long long *m, u32 *out, const PrimeInfo *pinfo, JobMap map, int log_n) {
+    const int n = 1 << log_n;
+    const int k = blockIdx.x * blockDim.x + threadIdx.x;
+    if (k >= n) return;
+    int prime, kk;
+    size_t in_row, out_row;
+    if (!map_job(map, blockIdx.y, prime, in_row, out_row, kk)) return;
+    const long long q = pinfo[prime].q;
+    long long r = m[k] % q;
+    if (r < 0) r += q;
+    out[out_row * n + k] = (u32)r;
+}
+
 // digit limbs of the extended output: dtilde[j][u] = c[u] for u inside digit j
 __global__ void k_copy_digit_limbs(const u32 *c, u32 *dt, int log_n, int level, int alpha, int ext) {
     const int n = 1 << log_n;

@@ -209,6 +209,22 @@ int ckks_bsgs(ckks_ctx *ctx, const uint32_t *ct, int level, int n_baby, const ui
               const ckks_evk *baby_keys, int n_giant, const uint32_t *giant_galois, const ckks_evk *giant_keys,
               const uint32_t *pt, uint32_t *out, void *ws, size_t ws_bytes, ckks_stream_t stream);
 
+/* CKKS encoding of N/2 complex slots into a plaintext (the pages give no encoder; this is the
+ * canonical embedding of full-RNS CKKS): m is the real integer polynomial with
+ * m(zeta^(5^j)) ~ scale * z_j, zeta = exp(i pi / N), j < N/2, computed on the host in double
+ * precision by the inverse of the slot DFT (radix-2 stages, then bit reversal) and rounded half
+ * away from zero; then reduced into q_0..q_level (and p_0..p_(k-1) when with_special != 0, the
+ * extended basis that ckks_bsgs's plaintexts use) and transformed to the evaluation domain on the
+ * GPU.  re, im: host arrays of N/2 doubles (the call copies them before returning);
+ * out: device [(level+1) (+ n_p)][N], canonical; ws: device, >= 8 N bytes (the coefficients);
+ * scale > 0.  The caller keeps |scale * t| well below 2^62 and below half the basis' modulus.
+ * Integer coefficients are decided in double precision, so another correct encoder may differ by
+ * one in a rare coefficient whose scaled value lies within rounding error of a half-integer.
+ * Errors: CKKS_ERR_ARG (null, scale, overlap), CKKS_ERR_UNSUPPORTED (level), CKKS_ERR_ALIGN,
+ * CKKS_ERR_WORKSPACE, CKKS_ERR_CUDA. */
+int ckks_encode(ckks_ctx *ctx, const double *re, const double *im, double scale, int level, int with_special,
+                uint32_t *out, void *ws, size_t ws_bytes, ckks_stream_t stream);
+
 /* ModRaise, the first step of CKKS bootstrapping (Cheon, Han, Kim, Kim, Song, Eurocrypt 2018;
  * the pages give no construction): a ciphertext at level 0, ct [2][1][N] (evaluation domain mod
  * q_0), is read as integer polynomials with centred coefficients in (-q_0/2, q_0/2] and reduced
