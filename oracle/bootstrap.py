@@ -6,9 +6,9 @@ TEST INFRASTRUCTURE ONLY (tests, smoke check).  Shares no code with the CUDA lib
 Bootstrapping (Cheon, Han, Kim, Kim, Song, Eurocrypt 2018; the linear maps in the form of Chen,
 Chillotti, Song, Eurocrypt 2019) moves a ciphertext's coefficients into its slots (CoeffToSlot),
 reduces them modulo q_0 slot-wise (EvalMod), and moves them back (SlotToCoeff).  The Perseus
-pages put bootstrap placement at the centre of their stack and EncryptedLLM's summary quotes
-22-27 ms per bootstrap; neither page gives the construction, which is restated here from its
-definition:
+write-up (ai4snews, Interpretation) puts bootstrap placement at the centre of its stack, and the
+summary of EncryptedLLM (lpnh.cn page, Results) quotes 22-27 ms per bootstrap; no page gives the
+construction, which is restated here from its definition:
 
   Decoding evaluates the plaintext m (degree < N, real coefficients) at the slot roots
   w_j = zeta^(5^j mod 2N), zeta = exp(i pi / N), j < n = N/2.  Since w_j^n = i, with

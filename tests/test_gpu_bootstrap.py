@@ -42,6 +42,17 @@ def test_modraise_parity(ks_lib, oracle_mod, key, level):
 @pytest.mark.parametrize("direction", ["coeff_to_slot", "slot_to_coeff"])
 @pytest.mark.parametrize("key,levels,n1", [("n12-dnum4", 3, 4), ("n14-hoisted8", 3, 8)])
 def test_dft_levels_parity(ks_lib, oracle_mod, key, levels, n1, direction):
+    _dft_levels(ks_lib, key, levels, n1, direction)
+
+
+@pytest.mark.slow
+def test_dft_levels_parity_n16(ks_lib, oracle_mod):
+    """CoeffToSlot on the N=2^16 chain (level 24, dnum 4): 15 stages in 3 levels of 5, 63
+    diagonals per level in 8 baby x 8 giant steps."""
+    _dft_levels(ks_lib, "n16-bsgs32", 3, 8, "coeff_to_slot")
+
+
+def _dft_levels(ks_lib, key, levels, n1, direction):
     from oracle import bootstrap as bt
     from oracle.scenario import Scenario
     ks = ks_lib
