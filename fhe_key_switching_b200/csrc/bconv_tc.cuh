@@ -33,13 +33,14 @@ constexpr int TC_K = 64;                  // K bytes (two MMAs of K = 32)
 constexpr int TC_MAX_IN = 15;             // 4 * 15 + 1 = 61 <= 64
 constexpr int TC_MAX_T = 32;              // targets per chunk: N = 4 T <= 128 columns
 constexpr int TC_THREADS = 128;
-constexpr int TC_TILES = 4;               // coefficient tiles per CTA
+constexpr int TC_TILES = 16;              // coefficient tiles per CTA
+constexpr int TC_STAGES = 3;              // A ring: the inputs of two tiles ahead are in flight
 constexpr int TC_COLS = 128;              // tensor-memory columns a CTA allocates
-// Dynamic shared memory per CTA: A (8 KB) + B (<= 8 KB) + target records, padded so that at most
-// 4 CTAs share an SM (4 x 128 columns = all 512 columns of tensor memory: no CTA waits in alloc;
-// 5 x 53 KB would exceed the SM's 228 KB).
+// Dynamic shared memory per CTA: the A ring (3 x 8 KB) + B (<= 8 KB) + target records, padded so
+// that at most 4 CTAs share an SM (4 x 128 columns = all 512 columns of tensor memory: no CTA
+// waits in alloc; 5 x 53 KB would exceed the SM's 228 KB).
 constexpr size_t TC_SMEM = 52 * 1024;
-constexpr int TC_A_BYTES = 4 * TC_M * 16;  // [4 K chunks][128 rows][16 B]
+constexpr int TC_A_BYTES = 4 * TC_M * 16;  // one A stage: [4 K chunks][128 rows][16 B]
 
 struct BconvTcArgs {
     const u32 *y;            // input rows
@@ -95,17 +96,26 @@ __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence:
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
+// 4-byte asynchronous copy global -> shared (completed by cp.async.wait_group)
+__device__ __forceinline__ void tc_cp_async4(void *dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(tc_smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void tc_cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void tc_cp_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void tc_cp_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
 // Included by ks_kernels.cuh after the mbarrier helpers (mbar_init, mbar_wait_bounded,
 // CKKS_DEV_ERR_WAIT), which the kernel below uses.
-constexpr int TC_REC_OFF = TC_A_BYTES + 4 * (4 * TC_MAX_T) * 16;   // per-target records after A and B
+constexpr int TC_B_OFF = TC_STAGES * TC_A_BYTES;                          // B after the A ring
+constexpr int TC_REC_OFF = TC_B_OFF + 4 * (4 * TC_MAX_T) * 16;            // per-target records after B
+static_assert(TC_REC_OFF + TC_MAX_T * 16 <= (int)TC_SMEM, "tensor-core conversion: shared memory");
 
 __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
     extern __shared__ __align__(1024) unsigned char tc_sm[];
     __shared__ __align__(8) u64 bar;
     __shared__ u32 tmem_base;
     __shared__ u32 half_s[TC_MAX_IN];
-    unsigned char *As = tc_sm;                                    // [4 K chunks][128 rows][16 B]
-    unsigned char *Bs = tc_sm + TC_A_BYTES;                       // [4 K chunks][N rows][16 B]
+    unsigned char *Bs = tc_sm + TC_B_OFF;                         // [4 K chunks][N rows][16 B]
     uint4 *trec = reinterpret_cast<uint4 *>(tc_sm + TC_REC_OFF);  // per target: (t, 2t, Shoup(2^16), row)
     const int tid = threadIdx.x, warp = tid >> 5;
     const int g = a.g_base + blockIdx.y;
@@ -123,11 +133,33 @@ __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
     auto target_pos = [&](int u) { const int idx = u0 + u; return idx < lo ? idx : idx + (hi - lo); };
     auto prime_of = [&](int kk) { return kk < a.map.split ? a.map.lo_base + kk : a.map.hi_base + (kk - a.map.split); };
     const int p0 = a.in_prime0 + g * a.in_prime_step;
+    const u32 *yb = a.y + item * a.y_item + (size_t)(a.in_row0 + g * a.in_group_rows) * n;
+    u32 *ob = a.out + item * a.out_item + ((size_t)g * a.map.out_group_rows + a.map.out_k_base) * n;
+    auto a_stage = [&](int tile) { return tc_sm + (size_t)(tile % TC_STAGES) * TC_A_BYTES; };
+    // tile `tile`'s inputs: 4-byte copies straight into this thread's A row (word i of the row,
+    // i.e. K chunk i / 4, word i % 4), one commit group per tile (possibly empty)
+    auto issue_loads = [&](int tile) {
+        if (tile < TC_TILES) {
+            const int nc = (blockIdx.x * TC_TILES + tile) * TC_M + tid;
+            unsigned char *row = a_stage(tile) + (size_t)tid * 16;
+            for (int i = 0; i < n_in; i++) tc_cp_async4(row + (i >> 2) * (TC_M * 16) + (i & 3) * 4, yb + (size_t)i * n + nc);
+        }
+        tc_cp_commit();
+    };
+    issue_loads(0);
+    issue_loads(1);
+    // words n_in + 1 .. 15 of every row stay zero (the copies never write them)
+    for (int st = 0; st < TC_STAGES; st++) {
+        u32 *row = reinterpret_cast<u32 *>(tc_sm + (size_t)st * TC_A_BYTES + (size_t)tid * 16);
+        for (int i = n_in + 1; i < 16; i++) row[(i >> 2) * (TC_M * 4) + (i & 3)] = 0u;
+    }
     for (int i = tid; i < n_in; i += TC_THREADS) half_s[i] = a.pinfo[p0 + i].half;
     for (int u = tid; u < Tc; u += TC_THREADS) {
         const int kk = target_pos(u);
-        const u32 q = a.pinfo[prime_of(kk)].q;
-        trec[u] = make_uint4(q, 2u * q, (u32)((1ull << 48) / q), (u32)kk);
+        const PrimeInfo pi = a.pinfo[prime_of(kk)];
+        // floor(2^48 / t) = 2^16 floor(2^32 / t) + floor(2^16 [2^32]_t / t), the last term being
+        // the Shoup companion of [2^32]_t shifted right by 16
+        trec[u] = make_uint4(pi.q, 2u * pi.q, (pi.onep << 16) + (pi.r64p >> 16), (u32)kk);
     }
     for (int idx = tid; idx < 4 * N; idx += TC_THREADS) {        // B: (K chunk, column) -> 16 bytes
         const int kc = idx / N, col = idx - kc * N;
@@ -145,55 +177,40 @@ __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
         mbar_init(&bar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    tc_fence_async_smem();                                        // B visible to the tensor cores
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const u32 tmem = tmem_base;
     const u32 taddr = tmem + ((u32)(warp * 32) << 16);            // this warp's 32 lanes
     const u32 idesc = tc_idesc(TC_M, N);
-    const u32 a_base = tc_smem_u32(As), b_base = tc_smem_u32(Bs);
-    const u32 *yb = a.y + item * a.y_item + (size_t)(a.in_row0 + g * a.in_group_rows) * n;
-    u32 *ob = a.out + item * a.out_item + ((size_t)g * a.map.out_group_rows + a.map.out_k_base) * n;
+    const u32 b_base = tc_smem_u32(Bs);
     int failed_phase = -1;
-    // this thread's A row of tile `tile`: its coefficient's n_in inputs, the count v, zeros
-    auto load_row = [&](int tile, u32 (&w)[16]) {
-        const int nc = (blockIdx.x * TC_TILES + tile) * TC_M + tid;
-        u32 vcount = 0;
-#pragma unroll
-        for (int i = 0; i < 16; i++) {
-            u32 val = 0;
-            if (i < n_in) {
-                val = yb[(size_t)i * n + nc];
-                vcount += val > half_s[i] ? 1u : 0u;
-            } else if (i == n_in) {
-                val = vcount;
-            }
-            w[i] = val;
-        }
-    };
-    u32 w[16];
-    load_row(0, w);
     for (int tile = 0; tile < TC_TILES; tile++) {
         const int nc = (blockIdx.x * TC_TILES + tile) * TC_M + tid;   // this thread's coefficient
-        uint4 *arow = reinterpret_cast<uint4 *>(As) + tid;
+        tc_cp_wait1();                                            // this tile's copies have landed
+        {   // the count v of negative representatives goes into word n_in of the row
+            u32 *row = reinterpret_cast<u32 *>(a_stage(tile) + (size_t)tid * 16);
+            u32 vcount = 0;
 #pragma unroll
-        for (int kc = 0; kc < 4; kc++)
-            arow[kc * TC_M] = make_uint4(w[4 * kc], w[4 * kc + 1], w[4 * kc + 2], w[4 * kc + 3]);
-        tc_fence_async_smem();                                    // A visible to the tensor cores
+            for (int i = 0; i < TC_MAX_IN; i++)
+                if (i < n_in) vcount += row[(i >> 2) * (TC_M * 4) + (i & 3)] > half_s[i] ? 1u : 0u;
+            row[(n_in >> 2) * (TC_M * 4) + (n_in & 3)] = vcount;
+        }
+        tc_fence_async_smem();                                    // A and B visible to the tensor cores
         tc_fence_before();
         __syncthreads();
+        bool expired = false;
         if (tid == 0) {
             tc_fence_after();
+            const u32 a_base = tc_smem_u32(a_stage(tile));
 #pragma unroll
             for (int s = 0; s < 2; s++)
                 tc_mma(tmem, tc_smem_desc(a_base + (u32)(2 * s * TC_M * 16), TC_M * 16, 128),
                        tc_smem_desc(b_base + (u32)(2 * s * N * 16), (u32)N * 16, 128), idesc, (u32)s);
             tc_commit(&bar);
         }
-        // the next tile's inputs load while the tensor cores and this tile's epilogue run
-        if (tile + 1 < TC_TILES) load_row(tile + 1, w);
-        const bool expired = !mbar_wait_bounded(&bar, (u32)(tile & 1));
+        issue_loads(tile + 2);                                    // into the stage of tile - 1 (its MMA is done)
+        if (tid == 0) expired = !mbar_wait_bounded(&bar, (u32)(tile & 1));
         if (__syncthreads_or(expired)) {                          // leave together
             failed_phase = tile & 1;
             break;
@@ -216,11 +233,14 @@ __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
         }
         tc_fence_before();                                        // reads done before the next MMA
     }
+    tc_cp_wait0();                                                // no copy outlives the block
     if (failed_phase >= 0) {
         // record the failure and give the MMA in flight a second bounded wait before freeing its
         // tensor memory
-        if (tid == 0) atomicOr(a.err, CKKS_DEV_ERR_WAIT);
-        (void)mbar_wait_bounded(&bar, (u32)failed_phase);
+        if (tid == 0) {
+            atomicOr(a.err, CKKS_DEV_ERR_WAIT);
+            (void)mbar_wait_bounded(&bar, (u32)failed_phase);
+        }
     }
     __syncthreads();
     if (warp == 0) {
