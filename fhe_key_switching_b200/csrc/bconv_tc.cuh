@@ -116,7 +116,7 @@ __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
     __shared__ u32 tmem_base;
     __shared__ u32 half_s[TC_MAX_IN];
     unsigned char *Bs = tc_sm + TC_B_OFF;                         // [4 K chunks][N rows][16 B]
-    uint4 *trec = reinterpret_cast<uint4 *>(tc_sm + TC_REC_OFF);  // per target: (t, 2t, Shoup(2^16), row)
+    uint4 *trec = reinterpret_cast<uint4 *>(tc_sm + TC_REC_OFF);  // per target: (t, 2t, Shoup(2^16), row * N)
     const int tid = threadIdx.x, warp = tid >> 5;
     const int g = a.g_base + blockIdx.y;
     const int item = blockIdx.z / a.nchunk, chunk = blockIdx.z % a.nchunk;
@@ -159,7 +159,7 @@ __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
         const PrimeInfo pi = a.pinfo[prime_of(kk)];
         // floor(2^48 / t) = 2^16 floor(2^32 / t) + floor(2^16 [2^32]_t / t), the last term being
         // the Shoup companion of [2^32]_t shifted right by 16
-        trec[u] = make_uint4(pi.q, 2u * pi.q, (pi.onep << 16) + (pi.r64p >> 16), (u32)kk);
+        trec[u] = make_uint4(pi.q, 2u * pi.q, (pi.onep << 16) + (pi.r64p >> 16), (u32)kk * (u32)n);
     }
     for (int idx = tid; idx < 4 * N; idx += TC_THREADS) {        // B: (K chunk, column) -> 16 bytes
         const int kc = idx / N, col = idx - kc * N;
@@ -227,7 +227,7 @@ __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
                     const uint4 rec = trec[u];
                     const u32 s1 = r[4 * j] + (r[4 * j + 1] << 8);
                     const u32 s2 = r[4 * j + 2] + (r[4 * j + 3] << 8);
-                    ob[(size_t)rec.w * n + nc] = shoup_mul(s2, 65536u, rec.z, rec.x) + csub(s1, rec.y);
+                    ob[rec.w + (u32)nc] = shoup_mul(s2, 65536u, rec.z, rec.x) + csub(s1, rec.y);
                 }
             }
         }
