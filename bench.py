@@ -752,6 +752,57 @@ def run_workload(args, local_rank):
         ks_per_step, rot_per_step = 0, 0
         ops, blocks = R * rescale_ops(cfg, lvl), 0
         nbytes = R * (2 * na + 2 * lvl) * limb
+    elif key == "coeff-to-slot":
+        # CoeffToSlot of N=2^16 in 3 levels of 5 radix-2 stages: each level's 63 slot diagonals
+        # (shifts m s, |m| <= 31, s its smallest half-length) as 8 baby x 8 giant steps, then a
+        # rescale; plaintexts and keys are synthetic residues (the cost is data independent)
+        levels, n1 = 3, 8
+        ns = n // 2
+        halves = [1 << h for h in range(cfg.log_n - 2, -1, -1)]          # n/4 ... 1, applied in order
+        per = -(-len(halves) // levels)
+        steps = [min(halves[i:i + per]) for i in range(0, len(halves), per)]
+        plan, gk = [], {}
+        for li, st_ in enumerate(steps):
+            lv = lvl - li
+            # the level's shifts: signed sums of its stages' half-lengths, centred in [-n/2, n/2)
+            shifts = {0}
+            for h in halves[li * per:(li + 1) * per]:
+                shifts = {((x + d + ns // 2) % ns) - ns // 2 for x in shifts for d in (-h, 0, h)}
+            ms = sorted(x // st_ for x in shifts)
+            babies = [k * st_ for k in range(n1)]
+            giants = [g * n1 * st_ for g in range(ms[0] // n1, ms[-1] // n1 + 1)]
+            bg = [1 if b % ns == 0 else ks.galois_element(cfg.log_n, b) for b in babies]
+            gg = [1 if g_ % ns == 0 else ks.galois_element(cfg.log_n, g_) for g_ in giants]
+            for g_ in bg + gg:
+                if g_ != 1 and g_ not in gk:
+                    gk[g_] = ks.make_evk(res(mods * nd).view(nd, len(mods), n), cfg.chacha_seed, g_)
+            ext_l = lv + 1 + cfg.n_p
+            pt_l = res((q[:lv + 1] + p) * len(gg) * len(bg)).view(len(gg), len(bg), ext_l, n)
+            plan.append((lv, bg, gg, pt_l, ks.ckks_bsgs_workspace(ctx, lv, len(bg), len(gg), device=dev)))
+        cts = [res(q[:na] * 2).view(2, na, n) for _ in range(N_SETS)]
+        mids = [torch.empty((2, lv + 1, n), dtype=torch.uint32, device=dev) for lv, *_ in plan]
+        outs = [torch.empty((2, lv, n), dtype=torch.uint32, device=dev) for lv, *_ in plan]
+        ws_r = ctx.workspace(lvl, 1, device=dev)
+
+        def step(i):
+            cur = cts[i % N_SETS]
+            for (lv, bg, gg, pt_l, ws_l), mid, o in zip(plan, mids, outs):
+                ks.ckks_bsgs(ctx, cur, lv, bg, [gk.get(g_) for g_ in bg], gg, [gk.get(g_) for g_ in gg], pt_l,
+                             mid, ws_l, stream)
+                ks.ckks_rescale(ctx, mid, lv, o, ws_r, stream)
+                cur = o
+        ks_per_step = rot_per_step = sum(sum(1 for g_ in bg + gg if g_ != 1) for _, bg, gg, _, _ in plan)
+        ops = blocks = nbytes = 0
+        for lv, bg, gg, pt_l, _ in plan:
+            e_l, n_l = lv + 1 + cfg.n_p, lv + 1
+            nb_r, ng_r = sum(g_ != 1 for g_ in bg), sum(g_ != 1 for g_ in gg)
+            ops += (modup_ops(cfg, lv) + nb_r * ip_ops(cfg, lv) + len(gg) * len(bg) * 2 * e_l * n * MAC
+                    + len(gg) * 2 * e_l * n * RED + len(gg) * moddown_ops(cfg, lv)
+                    + ng_r * (keyswitch_ops(cfg, lv) + n_l * n * MADD) + len(gg) * 2 * n_l * n * MADD
+                    + rescale_ops(cfg, lv))
+            blocks += (nb_r + ng_r) * chacha_blocks(cfg, lv)
+            nbytes += (len(gg) * len(bg) * e_l + 2 * n_l + 2 * n_l + 2 * n_l + 2 * (n_l - 1)) * limb \
+                + (nb_r + ng_r) * key_limbs(cfg, lv) * limb
     else:                                          # bsgs, bsgs-n14
         n1, n2 = 16, 18
         baby = [1] + [ks.galois_element(cfg.log_n, k) for k in range(1, n1)]
@@ -807,6 +858,10 @@ def run_workload(args, local_rank):
             "ms_per_step": ms / args.steps, "steps": args.steps, "warmup": args.warmup}
     if key == "rescale":
         line["rescales_per_s"] = R / t_step
+    elif key == "coeff-to-slot":
+        line["ms_per_coeff_to_slot"] = t_step * 1e3
+        line["context"] = ("the EncryptedLLM summary (lpnh.cn page, Results) quotes 22-27 ms per whole "
+                           "bootstrap on an unnamed GPU; CoeffToSlot is one of its three parts")
     elif is_bsgs:
         line["transforms_per_s"] = 1 / t_step
         line["rotations_per_transform"] = rot_per_step
@@ -823,10 +878,13 @@ def run_workload(args, local_rank):
     print(json.dumps(line), flush=True)
 
 
-INFO_WORKLOADS = {"n14-hoisted8": "n14-hoisted8", "n16-bsgs32": "n16-bsgs32", "n16-stream64": "n16-stream64",
+INFO_WORKLOADS = {"coeff-to-slot": "n16-bsgs32",
+                  "n14-hoisted8": "n14-hoisted8", "n16-bsgs32": "n16-bsgs32", "n16-stream64": "n16-stream64",
                   "n16-stream64-rescale": "n16-stream64", "rescale": "n16-full", "bsgs": "n16-bsgs32",
                   "bsgs-n14": "n14-hoisted8"}
 INFO_DESCRIPTIONS = {
+    "coeff-to-slot": "N=2^16, 36+12 primes, dnum 4, from level 24; step = CoeffToSlot in 3 levels of 5 radix-2 "
+                     "stages, each an 8 baby x 8 giant step transform of 63 slot diagonals plus a rescale",
     "n14-hoisted8": "N=2^14, 12+4 primes, dnum 3, level 11; step = 8 units, each 8 hoisted rotations "
                     "(+-1, +-2, +-4, +-8) + tensor + relin",
     "n16-bsgs32": "N=2^16, 36+12 primes, dnum 4, level 24; step = 32 hoisted rotations of one ciphertext",
@@ -855,7 +913,7 @@ def info_cpu_baseline(key: str, max_seconds: float = 8.0):
     ct = W.uniform_residues(octx.q[:na] * 2, n, gen).reshape(2, na, n)
     b = W.uniform_residues(octx.mod * nd, n, gen).reshape(nd, len(octx.mod), n)
     seed = cfg.chacha_seed
-    if key == "bsgs":
+    if key in ("bsgs", "coeff-to-slot"):
         return None                 # the oracle's plaintext sums take minutes at N=2^16
     if key == "n14-hoisted8":
         gs = [octx.galois(r) for r in cfg.rot_steps]

@@ -32,7 +32,7 @@ constexpr int TC_M = 128;                 // coefficients per tile = tensor-memo
 constexpr int TC_K = 64;                  // K bytes (two MMAs of K = 32)
 constexpr int TC_MAX_IN = 15;             // 4 * 15 + 1 = 61 <= 64
 constexpr int TC_MAX_T = 32;              // targets per chunk: N = 4 T <= 128 columns
-constexpr int TC_THREADS = 128;
+constexpr int TC_THREADS = 256;           // 8 warps: two per tensor-memory lane quadrant
 constexpr int TC_TILES = 16;              // coefficient tiles per CTA
 constexpr int TC_STAGES = 3;              // A ring: the inputs of two tiles ahead are in flight
 constexpr int TC_COLS = 128;              // tensor-memory columns a CTA allocates
@@ -136,23 +136,30 @@ __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
     const u32 *yb = a.y + item * a.y_item + (size_t)(a.in_row0 + g * a.in_group_rows) * n;
     u32 *ob = a.out + item * a.out_item + ((size_t)g * a.map.out_group_rows + a.map.out_k_base) * n;
     auto a_stage = [&](int tile) { return tc_sm + (size_t)(tile % TC_STAGES) * TC_A_BYTES; };
-    // tile `tile`'s inputs: 4-byte copies straight into this thread's A row (word i of the row,
+    const int lane_row = tid & (TC_M - 1);                        // this thread's tile row (lane)
+    const bool loader = tid < TC_M;                               // threads 0..127 own the A rows
+    // tile `tile`'s inputs: 4-byte copies straight into the owner's A row (word i of the row,
     // i.e. K chunk i / 4, word i % 4), one commit group per tile (possibly empty)
     auto issue_loads = [&](int tile) {
-        if (tile < TC_TILES) {
-            const int nc = (blockIdx.x * TC_TILES + tile) * TC_M + tid;
-            unsigned char *row = a_stage(tile) + (size_t)tid * 16;
-            for (int i = 0; i < n_in; i++) tc_cp_async4(row + (i >> 2) * (TC_M * 16) + (i & 3) * 4, yb + (size_t)i * n + nc);
+        if (loader && tile < TC_TILES) {
+            const u32 *src = yb + (blockIdx.x * TC_TILES + tile) * TC_M + lane_row;
+            unsigned char *row = a_stage(tile) + (size_t)lane_row * 16;
+#pragma unroll
+            for (int i = 0; i < TC_MAX_IN; i++) {
+                if (i < n_in) tc_cp_async4(row + (i >> 2) * (TC_M * 16) + (i & 3) * 4, src);
+                src += n;
+            }
         }
         tc_cp_commit();
     };
     issue_loads(0);
     issue_loads(1);
     // words n_in + 1 .. 15 of every row stay zero (the copies never write them)
-    for (int st = 0; st < TC_STAGES; st++) {
-        u32 *row = reinterpret_cast<u32 *>(tc_sm + (size_t)st * TC_A_BYTES + (size_t)tid * 16);
-        for (int i = n_in + 1; i < 16; i++) row[(i >> 2) * (TC_M * 4) + (i & 3)] = 0u;
-    }
+    if (loader)
+        for (int st = 0; st < TC_STAGES; st++) {
+            u32 *row = reinterpret_cast<u32 *>(tc_sm + (size_t)st * TC_A_BYTES + (size_t)lane_row * 16);
+            for (int i = n_in + 1; i < 16; i++) row[(i >> 2) * (TC_M * 4) + (i & 3)] = 0u;
+        }
     for (int i = tid; i < n_in; i += TC_THREADS) half_s[i] = a.pinfo[p0 + i].half;
     for (int u = tid; u < Tc; u += TC_THREADS) {
         const int kk = target_pos(u);
@@ -181,20 +188,27 @@ __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
     __syncthreads();
     tc_fence_after();
     const u32 tmem = tmem_base;
-    const u32 taddr = tmem + ((u32)(warp * 32) << 16);            // this warp's 32 lanes
+    const u32 taddr = tmem + ((u32)((warp & 3) * 32) << 16);      // this warp's 32 lanes
+    const int half = warp >> 2;                                   // which column groups it reads
     const u32 idesc = tc_idesc(TC_M, N);
     const u32 b_base = tc_smem_u32(Bs);
     int failed_phase = -1;
     for (int tile = 0; tile < TC_TILES; tile++) {
-        const int nc = (blockIdx.x * TC_TILES + tile) * TC_M + tid;   // this thread's coefficient
+        const int nc = (blockIdx.x * TC_TILES + tile) * TC_M + lane_row;   // this thread's coefficient
         tc_cp_wait1();                                            // this tile's copies have landed
-        {   // the count v of negative representatives goes into word n_in of the row
-            u32 *row = reinterpret_cast<u32 *>(a_stage(tile) + (size_t)tid * 16);
+        if (loader) {   // the count v of negative representatives goes into word n_in of the row
+            uint4 *row4 = reinterpret_cast<uint4 *>(a_stage(tile) + (size_t)lane_row * 16);
+            u32 w[16];
+#pragma unroll
+            for (int kc = 0; kc < 4; kc++) {
+                const uint4 v4 = row4[kc * TC_M];
+                w[4 * kc] = v4.x; w[4 * kc + 1] = v4.y; w[4 * kc + 2] = v4.z; w[4 * kc + 3] = v4.w;
+            }
             u32 vcount = 0;
 #pragma unroll
             for (int i = 0; i < TC_MAX_IN; i++)
-                if (i < n_in) vcount += row[(i >> 2) * (TC_M * 4) + (i & 3)] > half_s[i] ? 1u : 0u;
-            row[(n_in >> 2) * (TC_M * 4) + (n_in & 3)] = vcount;
+                if (i < n_in) vcount += w[i] > half_s[i] ? 1u : 0u;
+            reinterpret_cast<u32 *>(row4)[(n_in >> 2) * (TC_M * 4) + (n_in & 3)] = vcount;
         }
         tc_fence_async_smem();                                    // A and B visible to the tensor cores
         tc_fence_before();
@@ -216,7 +230,7 @@ __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
             break;
         }
         tc_fence_after();
-        for (int c0 = 0; c0 < 4 * Tc; c0 += 16) {
+        for (int c0 = 16 * half; c0 < 4 * Tc; c0 += 32) {     // the two warps of a quadrant alternate
             u32 r[16];
             tc_ld16(taddr + (u32)c0, r);
             tc_wait_ld();
