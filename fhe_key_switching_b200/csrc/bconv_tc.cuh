@@ -31,7 +31,7 @@
 constexpr int TC_M = 128;                 // coefficients per tile = tensor-memory lanes
 constexpr int TC_K = 64;                  // K bytes (two MMAs of K = 32)
 constexpr int TC_MAX_IN = 15;             // 4 * 15 + 1 = 61 <= 64
-constexpr int TC_MAX_T = 32;              // targets per chunk: N = 4 T <= 128 columns
+constexpr int TC_MAX_T = 16;              // targets per chunk: N = 4 T <= 64 columns, two accumulators
 constexpr int TC_THREADS = 256;           // 8 warps: two per tensor-memory lane quadrant
 constexpr int TC_TILES = 16;              // coefficient tiles per CTA
 constexpr int TC_STAGES = 3;              // A ring: the inputs of two tiles ahead are in flight
@@ -112,7 +112,7 @@ static_assert(TC_REC_OFF + TC_MAX_T * 16 <= (int)TC_SMEM, "tensor-core conversio
 
 __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
     extern __shared__ __align__(1024) unsigned char tc_sm[];
-    __shared__ __align__(8) u64 bar;
+    __shared__ __align__(8) u64 bar[2];                           // one per tensor-memory accumulator
     __shared__ u32 tmem_base;
     __shared__ u32 half_s[TC_MAX_IN];
     unsigned char *Bs = tc_sm + TC_B_OFF;                         // [4 K chunks][N rows][16 B]
@@ -181,7 +181,8 @@ __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     if (tid == 0) {
-        mbar_init(&bar, 1);
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     tc_fence_before();
@@ -192,9 +193,34 @@ __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
     const int half = warp >> 2;                                   // which column groups it reads
     const u32 idesc = tc_idesc(TC_M, N);
     const u32 b_base = tc_smem_u32(Bs);
-    int failed_phase = -1;
+    int failed = 0, issued_upto = -1;
+    // accumulator b of tile k is k % 2 at column offset b N; the MMA of tile k runs while the
+    // epilogue of tile k - 1 reads the other accumulator
+    auto epilogue = [&](int tile) {
+        const int nc = (blockIdx.x * TC_TILES + tile) * TC_M + lane_row;
+        const u32 acc = taddr + (u32)((tile & 1) * N);
+        for (int c0 = 16 * half; c0 < 4 * Tc; c0 += 32) {         // the two warps of a quadrant alternate
+            u32 r[16];
+            tc_ld16(acc + (u32)c0, r);
+            tc_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                const int u = (c0 >> 2) + j;
+                if (u < Tc) {
+                    const uint4 rec = trec[u];
+                    const u32 s1 = r[4 * j] + (r[4 * j + 1] << 8);
+                    const u32 s2 = r[4 * j + 2] + (r[4 * j + 3] << 8);
+                    ob[rec.w + (u32)nc] = shoup_mul(s2, 65536u, rec.z, rec.x) + csub(s1, rec.y);
+                }
+            }
+        }
+    };
+    // waits for the MMA of tile `tile` (its accumulator's barrier, the tile's use of it as phase)
+    auto wait_mma = [&](int tile) {
+        const bool expired = !mbar_wait_bounded(&bar[tile & 1], (u32)((tile >> 1) & 1));
+        return __syncthreads_or(expired) != 0;
+    };
     for (int tile = 0; tile < TC_TILES; tile++) {
-        const int nc = (blockIdx.x * TC_TILES + tile) * TC_M + lane_row;   // this thread's coefficient
         tc_cp_wait1();                                            // this tile's copies have landed
         if (loader) {   // the count v of negative representatives goes into word n_in of the row
             uint4 *row4 = reinterpret_cast<uint4 *>(a_stage(tile) + (size_t)lane_row * 16);
@@ -211,49 +237,48 @@ __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
             reinterpret_cast<u32 *>(row4)[(n_in >> 2) * (TC_M * 4) + (n_in & 3)] = vcount;
         }
         tc_fence_async_smem();                                    // A and B visible to the tensor cores
-        tc_fence_before();
+        tc_fence_before();                                        // (and tile - 2's accumulator reads done)
         __syncthreads();
-        bool expired = false;
         if (tid == 0) {
             tc_fence_after();
             const u32 a_base = tc_smem_u32(a_stage(tile));
+            const u32 d = tmem + (u32)((tile & 1) * N);
 #pragma unroll
             for (int s = 0; s < 2; s++)
-                tc_mma(tmem, tc_smem_desc(a_base + (u32)(2 * s * TC_M * 16), TC_M * 16, 128),
+                tc_mma(d, tc_smem_desc(a_base + (u32)(2 * s * TC_M * 16), TC_M * 16, 128),
                        tc_smem_desc(b_base + (u32)(2 * s * N * 16), (u32)N * 16, 128), idesc, (u32)s);
-            tc_commit(&bar);
+            tc_commit(&bar[tile & 1]);
+        }
+        issued_upto = tile;
+        if (tile > 0) {
+            if (wait_mma(tile - 1)) { failed = 1; break; }
+            tc_fence_after();
         }
         issue_loads(tile + 2);                                    // into the stage of tile - 1 (its MMA is done)
-        if (tid == 0) expired = !mbar_wait_bounded(&bar, (u32)(tile & 1));
-        if (__syncthreads_or(expired)) {                          // leave together
-            failed_phase = tile & 1;
-            break;
+        if (tile > 0) {
+            epilogue(tile - 1);
+            tc_fence_before();
         }
-        tc_fence_after();
-        for (int c0 = 16 * half; c0 < 4 * Tc; c0 += 32) {     // the two warps of a quadrant alternate
-            u32 r[16];
-            tc_ld16(taddr + (u32)c0, r);
-            tc_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 4; j++) {
-                const int u = (c0 >> 2) + j;
-                if (u < Tc) {
-                    const uint4 rec = trec[u];
-                    const u32 s1 = r[4 * j] + (r[4 * j + 1] << 8);
-                    const u32 s2 = r[4 * j + 2] + (r[4 * j + 3] << 8);
-                    ob[rec.w + (u32)nc] = shoup_mul(s2, 65536u, rec.z, rec.x) + csub(s1, rec.y);
-                }
-            }
+    }
+    if (!failed) {
+        if (wait_mma(TC_TILES - 1)) {
+            failed = 1;
+        } else {
+            tc_fence_after();
+            epilogue(TC_TILES - 1);
+            tc_fence_before();
         }
-        tc_fence_before();                                        // reads done before the next MMA
     }
     tc_cp_wait0();                                                // no copy outlives the block
-    if (failed_phase >= 0) {
-        // record the failure and give the MMA in flight a second bounded wait before freeing its
-        // tensor memory
+    if (failed) {
+        // record the failure and give the MMAs in flight a second bounded wait (every commit made
+        // has completed once both barriers have passed their last phase) before freeing the
+        // tensor memory they write
         if (tid == 0) {
             atomicOr(a.err, CKKS_DEV_ERR_WAIT);
-            (void)mbar_wait_bounded(&bar, (u32)failed_phase);
+            // at most the last two tiles' commits can be pending, one per barrier
+            for (int t = issued_upto - 1; t <= issued_upto; t++)
+                if (t >= 0) (void)mbar_wait_bounded(&bar[t & 1], (u32)((t >> 1) & 1));
         }
     }
     __syncthreads();
