@@ -31,15 +31,15 @@
 constexpr int TC_M = 128;                 // coefficients per tile = tensor-memory lanes
 constexpr int TC_K = 64;                  // K bytes (two MMAs of K = 32)
 constexpr int TC_MAX_IN = 15;             // 4 * 15 + 1 = 61 <= 64
-constexpr int TC_MAX_T = 16;              // targets per chunk: N = 4 T <= 64 columns, two accumulators
-constexpr int TC_THREADS = 256;           // 8 warps: two per tensor-memory lane quadrant
+constexpr int TC_MAX_T = 32;              // targets per chunk: N = 4 T <= 128 columns per accumulator
+constexpr int TC_THREADS = 288;           // 4 producer warps, 4 epilogue warps, 1 MMA warp
 constexpr int TC_TILES = 16;              // coefficient tiles per CTA
 constexpr int TC_STAGES = 3;              // A ring: the inputs of two tiles ahead are in flight
-constexpr int TC_COLS = 128;              // tensor-memory columns a CTA allocates
+constexpr int TC_COLS = 256;              // tensor-memory columns a CTA allocates: two accumulators
 // Dynamic shared memory per CTA: the A ring (3 x 8 KB) + B (<= 8 KB) + target records, padded so
-// that at most 4 CTAs share an SM (4 x 128 columns = all 512 columns of tensor memory: no CTA
-// waits in alloc; 5 x 53 KB would exceed the SM's 228 KB).
-constexpr size_t TC_SMEM = 52 * 1024;
+// that at most 2 CTAs share an SM (2 x 256 columns = all 512 columns of tensor memory: no CTA
+// waits in alloc; 3 x 77 KB would exceed the SM's 228 KB).
+constexpr size_t TC_SMEM = 76 * 1024;
 constexpr int TC_A_BYTES = 4 * TC_M * 16;  // one A stage: [4 K chunks][128 rows][16 B]
 
 struct BconvTcArgs {
@@ -102,22 +102,37 @@ __device__ __forceinline__ void tc_cp_async4(void *dst, const void *src) {
 }
 __device__ __forceinline__ void tc_cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void tc_cp_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void tc_cp_wait2() { asm volatile("cp.async.wait_group 2;" ::: "memory"); }
 __device__ __forceinline__ void tc_cp_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 // Included by ks_kernels.cuh after the mbarrier helpers (mbar_init, mbar_wait_bounded,
 // CKKS_DEV_ERR_WAIT), which the kernel below uses.
+__device__ __forceinline__ void tc_arrive(u64 *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(tc_smem_u32(bar)) : "memory");
+}
 constexpr int TC_B_OFF = TC_STAGES * TC_A_BYTES;                          // B after the A ring
 constexpr int TC_REC_OFF = TC_B_OFF + 4 * (4 * TC_MAX_T) * 16;            // per-target records after B
 static_assert(TC_REC_OFF + TC_MAX_T * 16 <= (int)TC_SMEM, "tensor-core conversion: shared memory");
 
+// Roles: warps 0-3 produce the A tiles (thread t owns row t: 4-byte cp.async copies of its
+// coefficient's inputs, then the centred-lift count), warp 8 (one lane) issues the MMAs, warps
+// 4-7 read the accumulators back and store the outputs.  They meet on mbarriers only:
+//   a_full[s]   (128 producer arrivals)  stage s holds tile k's A;
+//   a_empty[s]  (tcgen05.commit)          the MMA of the stage's tile is done with it;
+//   acc_full[b] (tcgen05.commit)          accumulator b holds tile k's G;
+//   acc_empty[b](128 epilogue arrivals)   accumulator b has been read.
+// Every wait is bounded: on expiry the CTA's abort flag and the device error word are set and
+// every role leaves its loop; the MMA warp then waits (bounded) for its MMAs in flight before the
+// tensor memory is freed.
 __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
     extern __shared__ __align__(1024) unsigned char tc_sm[];
-    __shared__ __align__(8) u64 bar[2];                           // one per tensor-memory accumulator
+    __shared__ __align__(8) u64 a_full[TC_STAGES], a_empty[TC_STAGES], acc_full[2], acc_empty[2];
     __shared__ u32 tmem_base;
+    __shared__ volatile int abort_flag;
     __shared__ u32 half_s[TC_MAX_IN];
     unsigned char *Bs = tc_sm + TC_B_OFF;                         // [4 K chunks][N rows][16 B]
     uint4 *trec = reinterpret_cast<uint4 *>(tc_sm + TC_REC_OFF);  // per target: (t, 2t, Shoup(2^16), row * N)
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = a.g_base + blockIdx.y;
     const int item = blockIdx.z / a.nchunk, chunk = blockIdx.z % a.nchunk;
     const int n = 1 << a.log_n;
@@ -136,30 +151,7 @@ __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
     const u32 *yb = a.y + item * a.y_item + (size_t)(a.in_row0 + g * a.in_group_rows) * n;
     u32 *ob = a.out + item * a.out_item + ((size_t)g * a.map.out_group_rows + a.map.out_k_base) * n;
     auto a_stage = [&](int tile) { return tc_sm + (size_t)(tile % TC_STAGES) * TC_A_BYTES; };
-    const int lane_row = tid & (TC_M - 1);                        // this thread's tile row (lane)
-    const bool loader = tid < TC_M;                               // threads 0..127 own the A rows
-    // tile `tile`'s inputs: 4-byte copies straight into the owner's A row (word i of the row,
-    // i.e. K chunk i / 4, word i % 4), one commit group per tile (possibly empty)
-    auto issue_loads = [&](int tile) {
-        if (loader && tile < TC_TILES) {
-            const u32 *src = yb + (blockIdx.x * TC_TILES + tile) * TC_M + lane_row;
-            unsigned char *row = a_stage(tile) + (size_t)lane_row * 16;
-#pragma unroll
-            for (int i = 0; i < TC_MAX_IN; i++) {
-                if (i < n_in) tc_cp_async4(row + (i >> 2) * (TC_M * 16) + (i & 3) * 4, src);
-                src += n;
-            }
-        }
-        tc_cp_commit();
-    };
-    issue_loads(0);
-    issue_loads(1);
-    // words n_in + 1 .. 15 of every row stay zero (the copies never write them)
-    if (loader)
-        for (int st = 0; st < TC_STAGES; st++) {
-            u32 *row = reinterpret_cast<u32 *>(tc_sm + (size_t)st * TC_A_BYTES + (size_t)lane_row * 16);
-            for (int i = n_in + 1; i < 16; i++) row[(i >> 2) * (TC_M * 4) + (i & 3)] = 0u;
-        }
+    // ---- set-up (all threads): constants, B tile, zero padding of the A rows, barriers, memory
     for (int i = tid; i < n_in; i += TC_THREADS) half_s[i] = a.pinfo[p0 + i].half;
     for (int u = tid; u < Tc; u += TC_THREADS) {
         const int kk = target_pos(u);
@@ -175,55 +167,41 @@ __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
         if (u < Tc) v = a.tb[((size_t)cfg * a.n_primes + prime_of(target_pos(u))) * 16 + c * 4 + kc];
         reinterpret_cast<uint4 *>(Bs)[(size_t)kc * N + col] = v;
     }
-    if (warp == 0) {
+    if (tid < TC_M)          // words n_in + 1 .. 15 of every row stay zero (the copies never write them)
+        for (int st = 0; st < TC_STAGES; st++) {
+            u32 *row = reinterpret_cast<u32 *>(tc_sm + (size_t)st * TC_A_BYTES + (size_t)tid * 16);
+            for (int i = n_in + 1; i < 16; i++) row[(i >> 2) * (TC_M * 4) + (i & 3)] = 0u;
+        }
+    if (warp == 8) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                      ::"r"(tc_smem_u32(&tmem_base)), "r"(TC_COLS) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        if (lane == 0) {
+            for (int st = 0; st < TC_STAGES; st++) { mbar_init(&a_full[st], TC_M); mbar_init(&a_empty[st], 1); }
+            for (int b = 0; b < 2; b++) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], TC_M); }
+            abort_flag = 0;
+            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        }
     }
-    if (tid == 0) {
-        mbar_init(&bar[0], 1);
-        mbar_init(&bar[1], 1);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
+    tc_fence_async_smem();                                        // B visible to the tensor cores
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const u32 tmem = tmem_base;
-    const u32 taddr = tmem + ((u32)((warp & 3) * 32) << 16);      // this warp's 32 lanes
-    const int half = warp >> 2;                                   // which column groups it reads
-    const u32 idesc = tc_idesc(TC_M, N);
-    const u32 b_base = tc_smem_u32(Bs);
-    int failed = 0, issued_upto = -1;
-    // accumulator b of tile k is k % 2 at column offset b N; the MMA of tile k runs while the
-    // epilogue of tile k - 1 reads the other accumulator
-    auto epilogue = [&](int tile) {
-        const int nc = (blockIdx.x * TC_TILES + tile) * TC_M + lane_row;
-        const u32 acc = taddr + (u32)((tile & 1) * N);
-        for (int c0 = 16 * half; c0 < 4 * Tc; c0 += 32) {         // the two warps of a quadrant alternate
-            u32 r[16];
-            tc_ld16(acc + (u32)c0, r);
-            tc_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 4; j++) {
-                const int u = (c0 >> 2) + j;
-                if (u < Tc) {
-                    const uint4 rec = trec[u];
-                    const u32 s1 = r[4 * j] + (r[4 * j + 1] << 8);
-                    const u32 s2 = r[4 * j + 2] + (r[4 * j + 3] << 8);
-                    ob[rec.w + (u32)nc] = shoup_mul(s2, 65536u, rec.z, rec.x) + csub(s1, rec.y);
-                }
-            }
-        }
+    auto fail_wait = [&]() {
+        if (!abort_flag) atomicOr(a.err, CKKS_DEV_ERR_WAIT);
+        abort_flag = 1;
     };
-    // waits for the MMA of tile `tile` (its accumulator's barrier, the tile's use of it as phase)
-    auto wait_mma = [&](int tile) {
-        const bool expired = !mbar_wait_bounded(&bar[tile & 1], (u32)((tile >> 1) & 1));
-        return __syncthreads_or(expired) != 0;
+    auto wait_or_abort = [&](u64 *bar, u32 parity) {              // false: aborted
+        if (abort_flag) return false;
+        if (!mbar_wait_bounded(bar, parity)) { fail_wait(); return false; }
+        return true;
     };
-    for (int tile = 0; tile < TC_TILES; tile++) {
-        tc_cp_wait1();                                            // this tile's copies have landed
-        if (loader) {   // the count v of negative representatives goes into word n_in of the row
-            uint4 *row4 = reinterpret_cast<uint4 *>(a_stage(tile) + (size_t)lane_row * 16);
+    if (warp < 4) {
+        // ---- producers: row tid of every tile, two tiles of copies in flight
+        const int row_i = tid;
+        auto finish = [&](int k) {                                // tile k's copies have landed
+            uint4 *row4 = reinterpret_cast<uint4 *>(a_stage(k) + (size_t)row_i * 16);
             u32 w[16];
 #pragma unroll
             for (int kc = 0; kc < 4; kc++) {
@@ -235,54 +213,84 @@ __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
             for (int i = 0; i < TC_MAX_IN; i++)
                 if (i < n_in) vcount += w[i] > half_s[i] ? 1u : 0u;
             reinterpret_cast<u32 *>(row4)[(n_in >> 2) * (TC_M * 4) + (n_in & 3)] = vcount;
+            tc_fence_async_smem();                                // visible to the tensor cores
+            tc_arrive(&a_full[k % TC_STAGES]);
+        };
+        int k = 0;
+        for (; k < TC_TILES; k++) {
+            if (k >= TC_STAGES && !wait_or_abort(&a_empty[k % TC_STAGES], (u32)(((k / TC_STAGES) - 1) & 1))) break;
+            const u32 *src = yb + (blockIdx.x * TC_TILES + k) * TC_M + row_i;
+            unsigned char *row = a_stage(k) + (size_t)row_i * 16;
+#pragma unroll
+            for (int i = 0; i < TC_MAX_IN; i++) {
+                if (i < n_in) tc_cp_async4(row + (i >> 2) * (TC_M * 16) + (i & 3) * 4, src);
+                src += n;
+            }
+            tc_cp_commit();
+            if (k >= 2) {
+                tc_cp_wait2();
+                finish(k - 2);
+            }
         }
-        tc_fence_async_smem();                                    // A and B visible to the tensor cores
-        tc_fence_before();                                        // (and tile - 2's accumulator reads done)
-        __syncthreads();
-        if (tid == 0) {
+        tc_cp_wait0();
+        if (k == TC_TILES) {
+            if (TC_TILES >= 2) finish(TC_TILES - 2);
+            finish(TC_TILES - 1);
+        }
+    } else if (warp < 8) {
+        // ---- epilogue: lanes 32 (warp - 4) .. + 31 of each accumulator
+        const int q = warp - 4;
+        const int row_i = q * 32 + lane;
+        for (int k = 0; k < TC_TILES; k++) {
+            if (!wait_or_abort(&acc_full[k & 1], (u32)((k >> 1) & 1))) break;
             tc_fence_after();
-            const u32 a_base = tc_smem_u32(a_stage(tile));
-            const u32 d = tmem + (u32)((tile & 1) * N);
+            const int nc = (blockIdx.x * TC_TILES + k) * TC_M + row_i;
+            const u32 acc = tmem + ((u32)(q * 32) << 16) + (u32)((k & 1) * 128);
+            for (int c0 = 0; c0 < 4 * Tc; c0 += 16) {
+                u32 r[16];
+                tc_ld16(acc + (u32)c0, r);
+                tc_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 4; j++) {
+                    const int u = (c0 >> 2) + j;
+                    if (u < Tc) {
+                        const uint4 rec = trec[u];
+                        const u32 s1 = r[4 * j] + (r[4 * j + 1] << 8);
+                        const u32 s2 = r[4 * j + 2] + (r[4 * j + 3] << 8);
+                        ob[rec.w + (u32)nc] = shoup_mul(s2, 65536u, rec.z, rec.x) + csub(s1, rec.y);
+                    }
+                }
+            }
+            tc_fence_before();
+            tc_arrive(&acc_empty[k & 1]);
+        }
+    } else if (lane == 0) {
+        // ---- MMA issuer
+        const u32 idesc = tc_idesc(TC_M, N);
+        const u32 b_base = tc_smem_u32(Bs);
+        int issued = 0;
+        for (int k = 0; k < TC_TILES; k++) {
+            if (!wait_or_abort(&a_full[k % TC_STAGES], (u32)((k / TC_STAGES) & 1))) break;
+            if (k >= 2 && !wait_or_abort(&acc_empty[k & 1], (u32)(((k >> 1) - 1) & 1))) break;
+            tc_fence_after();
+            const u32 a_base = tc_smem_u32(a_stage(k));
+            const u32 d = tmem + (u32)((k & 1) * 128);
 #pragma unroll
             for (int s = 0; s < 2; s++)
                 tc_mma(d, tc_smem_desc(a_base + (u32)(2 * s * TC_M * 16), TC_M * 16, 128),
                        tc_smem_desc(b_base + (u32)(2 * s * N * 16), (u32)N * 16, 128), idesc, (u32)s);
-            tc_commit(&bar[tile & 1]);
+            tc_commit(&acc_full[k & 1]);
+            tc_commit(&a_empty[k % TC_STAGES]);
+            issued = k + 1;
         }
-        issued_upto = tile;
-        if (tile > 0) {
-            if (wait_mma(tile - 1)) { failed = 1; break; }
-            tc_fence_after();
-        }
-        issue_loads(tile + 2);                                    // into the stage of tile - 1 (its MMA is done)
-        if (tile > 0) {
-            epilogue(tile - 1);
-            tc_fence_before();
-        }
-    }
-    if (!failed) {
-        if (wait_mma(TC_TILES - 1)) {
-            failed = 1;
-        } else {
-            tc_fence_after();
-            epilogue(TC_TILES - 1);
-            tc_fence_before();
-        }
-    }
-    tc_cp_wait0();                                                // no copy outlives the block
-    if (failed) {
-        // record the failure and give the MMAs in flight a second bounded wait (every commit made
-        // has completed once both barriers have passed their last phase) before freeing the
-        // tensor memory they write
-        if (tid == 0) {
-            atomicOr(a.err, CKKS_DEV_ERR_WAIT);
-            // at most the last two tiles' commits can be pending, one per barrier
-            for (int t = issued_upto - 1; t <= issued_upto; t++)
-                if (t >= 0) (void)mbar_wait_bounded(&bar[t & 1], (u32)((t >> 1) & 1));
+        if (abort_flag) {
+            // the MMAs of the last two issued tiles may still run: wait for them (bounded)
+            for (int t = issued - 2; t < issued; t++)
+                if (t >= 0) (void)mbar_wait_bounded(&acc_full[t & 1], (u32)((t >> 1) & 1));
         }
     }
     __syncthreads();
-    if (warp == 0) {
+    if (warp == 8) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TC_COLS) : "memory");
     }
