@@ -34,9 +34,9 @@ constexpr int TC_MAX_IN = 15;             // 4 * 15 + 1 = 61 <= 64
 constexpr int TC_MAX_T = 32;              // targets per chunk: N = 4 T <= 128 columns per accumulator
 constexpr int TC_THREADS = 288;           // 4 producer warps, 4 epilogue warps, 1 MMA warp
 constexpr int TC_TILES = 16;              // coefficient tiles per CTA
-constexpr int TC_STAGES = 3;              // A ring: the inputs of two tiles ahead are in flight
+constexpr int TC_STAGES = 5;              // A ring: the inputs of four tiles ahead are in flight
 constexpr int TC_COLS = 256;              // tensor-memory columns a CTA allocates: two accumulators
-// Dynamic shared memory per CTA: the A ring (3 x 8 KB) + B (<= 8 KB) + target records, padded so
+// Dynamic shared memory per CTA: the A ring (5 x 8 KB) + B (<= 8 KB) + target records, padded so
 // that at most 2 CTAs share an SM (2 x 256 columns = all 512 columns of tensor memory: no CTA
 // waits in alloc; 3 x 77 KB would exceed the SM's 228 KB).
 constexpr size_t TC_SMEM = 76 * 1024;
@@ -103,6 +103,23 @@ __device__ __forceinline__ void tc_cp_async4(void *dst, const void *src) {
 __device__ __forceinline__ void tc_cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void tc_cp_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 __device__ __forceinline__ void tc_cp_wait2() { asm volatile("cp.async.wait_group 2;" ::: "memory"); }
+__device__ __forceinline__ void tc_cp_wait4() { asm volatile("cp.async.wait_group 4;" ::: "memory"); }
+
+// Bounded wait for `phase` of `bar` in which the waiting thread sleeps in try_wait (up to a
+// microsecond per try, the suspend-time hint) instead of spinning; false after 1 s of the
+// global timer or the try-count backstop.
+__device__ __forceinline__ bool tc_wait_bounded(u64 *bar, u32 phase) {
+    const u64 t0 = global_ns();
+    for (u32 i = 0; i < MBAR_WAIT_TRIES; i++) {
+        u32 ok;
+        asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+                     "selp.u32 %0, 1, 0, p;\n\t}"
+                     : "=r"(ok) : "r"(tc_smem_u32(bar)), "r"(phase), "r"(1000u) : "memory");
+        if (ok) return true;
+        if (global_ns() - t0 > MBAR_WAIT_NS) return false;
+    }
+    return false;
+}
 __device__ __forceinline__ void tc_cp_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 // Included by ks_kernels.cuh after the mbarrier helpers (mbar_init, mbar_wait_bounded,
@@ -113,6 +130,7 @@ __device__ __forceinline__ void tc_arrive(u64 *bar) {
 constexpr int TC_B_OFF = TC_STAGES * TC_A_BYTES;                          // B after the A ring
 constexpr int TC_REC_OFF = TC_B_OFF + 4 * (4 * TC_MAX_T) * 16;            // per-target records after B
 static_assert(TC_REC_OFF + TC_MAX_T * 16 <= (int)TC_SMEM, "tensor-core conversion: shared memory");
+static_assert(TC_STAGES == 5 && TC_TILES >= TC_STAGES, "the producer loop waits with cp.async.wait_group 4");
 
 // Roles: warps 0-3 produce the A tiles (thread t owns row t: 4-byte cp.async copies of its
 // coefficient's inputs, then the centred-lift count), warp 8 (one lane) issues the MMAs, warps
@@ -194,11 +212,11 @@ __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
     };
     auto wait_or_abort = [&](u64 *bar, u32 parity) {              // false: aborted
         if (abort_flag) return false;
-        if (!mbar_wait_bounded(bar, parity)) { fail_wait(); return false; }
+        if (!tc_wait_bounded(bar, parity)) { fail_wait(); return false; }
         return true;
     };
     if (warp < 4) {
-        // ---- producers: row tid of every tile, two tiles of copies in flight
+        // ---- producers: row tid of every tile, TC_STAGES - 1 tiles of copies in flight
         const int row_i = tid;
         auto finish = [&](int k) {                                // tile k's copies have landed
             uint4 *row4 = reinterpret_cast<uint4 *>(a_stage(k) + (size_t)row_i * 16);
@@ -227,16 +245,14 @@ __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
                 src += n;
             }
             tc_cp_commit();
-            if (k >= 2) {
-                tc_cp_wait2();
-                finish(k - 2);
+            if (k >= TC_STAGES - 1) {
+                tc_cp_wait4();                                    // tile k - 4 has landed
+                finish(k - (TC_STAGES - 1));
             }
         }
         tc_cp_wait0();
-        if (k == TC_TILES) {
-            if (TC_TILES >= 2) finish(TC_TILES - 2);
-            finish(TC_TILES - 1);
-        }
+        if (k == TC_TILES)
+            for (int t = TC_TILES - (TC_STAGES - 1); t < TC_TILES; t++) finish(t);
     } else if (warp < 8) {
         // ---- epilogue: lanes 32 (warp - 4) .. + 31 of each accumulator
         const int q = warp - 4;
@@ -286,7 +302,7 @@ __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
         if (abort_flag) {
             // the MMAs of the last two issued tiles may still run: wait for them (bounded)
             for (int t = issued - 2; t < issued; t++)
-                if (t >= 0) (void)mbar_wait_bounded(&acc_full[t & 1], (u32)((t >> 1) & 1));
+                if (t >= 0) (void)tc_wait_bounded(&acc_full[t & 1], (u32)((t >> 1) & 1));
         }
     }
     __syncthreads();
