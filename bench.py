@@ -1113,9 +1113,9 @@ def main():
     ap.add_argument("--graph", action="store_true",
                     help="time one CUDA graph replay per step instead of eager launches (pays at small "
                          "batches; at 2 streams x 4 units the other stream already hides launch gaps)")
-    ap.add_argument("--bconv", default="cuda", choices=sorted(BCONV_ENGINES),
-                    help="base-conversion engine: cuda (CUDA cores, default) or tensor (8-bit split on the "
-                         "tensor cores); the output bits are the same")
+    ap.add_argument("--bconv", default="tensor", choices=sorted(BCONV_ENGINES),
+                    help="base-conversion engine: tensor (8-bit split on the tensor cores, default) or cuda "
+                         "(CUDA cores); the output bits are the same")
     ap.add_argument("--int-peaks", action="store_true",
                     help="measure this GPU's integer throughput per instruction class (ckks_int_probe) and "
                          "print it as one JSON line")

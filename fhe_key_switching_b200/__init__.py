@@ -365,8 +365,8 @@ CKKS_BCONV_CUDA_CORES, CKKS_BCONV_TENSOR = 0, 1
 
 
 def ckks_set_bconv_mode(ctx, mode: int):
-    """Base-conversion engine of later calls on ctx: CKKS_BCONV_CUDA_CORES (default) or
-    CKKS_BCONV_TENSOR (8-bit contraction on the tensor cores); same output bits either way."""
+    """Base-conversion engine of later calls on ctx: CKKS_BCONV_TENSOR (default; 8-bit contraction
+    on the tensor cores) or CKKS_BCONV_CUDA_CORES; same output bits either way."""
     _check(_L.ckks_set_bconv_mode(ctx.handle, mode), "ckks_set_bconv_mode")
 
 

@@ -23,7 +23,7 @@ def _worker(rank, world, port, q):
     import torch.distributed as dist
     import bench
     r, w, lr = bench.rank_env()
-    dist.init_process_group("gloo", rank=r, world_size=w, timeout=timedelta(seconds=60))
+    dist.init_process_group("gloo", rank=r, world_size=w, timeout=timedelta(seconds=300))
     ms = 100.0 + 50.0 * rank                     # rank 1 is the slow one
     ms_max = bench.max_over_ranks(ms, w)
     value = bench.job_throughput(16, w, ms_max)
@@ -41,9 +41,9 @@ def test_replica_timing_two_gloo_ranks(world):
     for p in procs:
         p.start()
     for p in procs:
-        p.join(120)
+        p.join(600)             # a fresh process's first torch import can take a minute or more
         assert p.exitcode == 0
-    res = sorted(q.get(timeout=10) for _ in range(world))
+    res = sorted(q.get(timeout=60) for _ in range(world))
     for r, (rank, w, lr, ms_max, value) in enumerate(res):
         assert (rank, w, lr) == (r, world, r)
         assert ms_max == 150.0                               # max over ranks
