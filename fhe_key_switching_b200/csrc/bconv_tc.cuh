@@ -33,7 +33,7 @@ constexpr int TC_K = 64;                  // K bytes (two MMAs of K = 32)
 constexpr int TC_MAX_IN = 15;             // 4 * 15 + 1 = 61 <= 64
 constexpr int TC_MAX_T = 32;              // targets per chunk: N = 4 T <= 128 columns per accumulator
 constexpr int TC_THREADS = 288;           // 4 producer warps, 4 epilogue warps, 1 MMA warp
-constexpr int TC_TILES = 16;              // coefficient tiles per CTA
+constexpr int TC_TILES = 16;              // coefficient tiles per CTA, at most (BconvTcArgs::tiles)
 constexpr int TC_STAGES = 5;              // A ring: the inputs of four tiles ahead are in flight
 constexpr int TC_COLS = 256;              // tensor-memory columns a CTA allocates: two accumulators
 // Dynamic shared memory per CTA: the A ring (5 x 8 KB) + B (<= 8 KB) + target records, padded so
@@ -52,6 +52,7 @@ struct BconvTcArgs {
     int in_row0, in_group_rows, in_prime0, in_prime_step;
     int n_in_full, n_in_last, n_groups, cfg_per_group, g_base;
     int nchunk, tchunk;      // target chunks per item (blockIdx.z = item * nchunk + chunk)
+    int tiles;               // coefficient tiles of 128 per CTA (1 .. TC_TILES; fewer for small launches)
     size_t y_item, out_item;
     int *err;                // device error word: CKKS_DEV_ERR_WAIT when a wait expires
 };
@@ -130,7 +131,7 @@ __device__ __forceinline__ void tc_arrive(u64 *bar) {
 constexpr int TC_B_OFF = TC_STAGES * TC_A_BYTES;                          // B after the A ring
 constexpr int TC_REC_OFF = TC_B_OFF + 4 * (4 * TC_MAX_T) * 16;            // per-target records after B
 static_assert(TC_REC_OFF + TC_MAX_T * 16 <= (int)TC_SMEM, "tensor-core conversion: shared memory");
-static_assert(TC_STAGES == 5 && TC_TILES >= TC_STAGES, "the producer loop waits with cp.async.wait_group 4");
+static_assert(TC_STAGES == 5, "the producer loop waits with cp.async.wait_group 4");
 
 // Roles: warps 0-3 produce the A tiles (thread t owns row t: 4-byte cp.async copies of its
 // coefficient's inputs, then the centred-lift count), warp 8 (one lane) issues the MMAs, warps
@@ -151,6 +152,7 @@ __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
     unsigned char *Bs = tc_sm + TC_B_OFF;                         // [4 K chunks][N rows][16 B]
     uint4 *trec = reinterpret_cast<uint4 *>(tc_sm + TC_REC_OFF);  // per target: (t, 2t, Shoup(2^16), row * N)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tiles = a.tiles;
     const int g = a.g_base + blockIdx.y;
     const int item = blockIdx.z / a.nchunk, chunk = blockIdx.z % a.nchunk;
     const int n = 1 << a.log_n;
@@ -235,9 +237,9 @@ __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
             tc_arrive(&a_full[k % TC_STAGES]);
         };
         int k = 0;
-        for (; k < TC_TILES; k++) {
+        for (; k < tiles; k++) {
             if (k >= TC_STAGES && !wait_or_abort(&a_empty[k % TC_STAGES], (u32)(((k / TC_STAGES) - 1) & 1))) break;
-            const u32 *src = yb + (blockIdx.x * TC_TILES + k) * TC_M + row_i;
+            const u32 *src = yb + (blockIdx.x * tiles + k) * TC_M + row_i;
             unsigned char *row = a_stage(k) + (size_t)row_i * 16;
 #pragma unroll
             for (int i = 0; i < TC_MAX_IN; i++) {
@@ -251,16 +253,16 @@ __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
             }
         }
         tc_cp_wait0();
-        if (k == TC_TILES)
-            for (int t = TC_TILES - (TC_STAGES - 1); t < TC_TILES; t++) finish(t);
+        if (k == tiles)
+            for (int t = max(0, tiles - (TC_STAGES - 1)); t < tiles; t++) finish(t);
     } else if (warp < 8) {
         // ---- epilogue: lanes 32 (warp - 4) .. + 31 of each accumulator
         const int q = warp - 4;
         const int row_i = q * 32 + lane;
-        for (int k = 0; k < TC_TILES; k++) {
+        for (int k = 0; k < tiles; k++) {
             if (!wait_or_abort(&acc_full[k & 1], (u32)((k >> 1) & 1))) break;
             tc_fence_after();
-            const int nc = (blockIdx.x * TC_TILES + k) * TC_M + row_i;
+            const int nc = (blockIdx.x * tiles + k) * TC_M + row_i;
             const u32 acc = tmem + ((u32)(q * 32) << 16) + (u32)((k & 1) * 128);
             for (int c0 = 0; c0 < 4 * Tc; c0 += 16) {
                 u32 r[16];
@@ -285,7 +287,7 @@ __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
         const u32 idesc = tc_idesc(TC_M, N);
         const u32 b_base = tc_smem_u32(Bs);
         int issued = 0;
-        for (int k = 0; k < TC_TILES; k++) {
+        for (int k = 0; k < tiles; k++) {
             if (!wait_or_abort(&a_full[k % TC_STAGES], (u32)((k / TC_STAGES) & 1))) break;
             if (k >= 2 && !wait_or_abort(&acc_empty[k & 1], (u32)(((k >> 1) - 1) & 1))) break;
             tc_fence_after();
