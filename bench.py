@@ -970,11 +970,14 @@ def info_cpu_baseline(key: str, max_seconds: float = 8.0):
 
 
 BCONV_ENGINES = {"cuda": "CUDA cores (32x32->64-bit multiply-adds)",
-                 "tensor": "tensor cores (8-bit split, tcgen05.mma kind::i8)"}
+                 "tensor": "tensor cores (8-bit split, tcgen05.mma kind::i8)",
+                 "auto": "automatic: tensor cores (8-bit split, tcgen05.mma kind::i8) for launches of at least "
+                         "4 tiles per block, CUDA cores below"}
 
 
 def set_bconv(ks, ctx, args):
-    ks.ckks_set_bconv_mode(ctx, ks.CKKS_BCONV_TENSOR if args.bconv == "tensor" else ks.CKKS_BCONV_CUDA_CORES)
+    ks.ckks_set_bconv_mode(ctx, {"tensor": ks.CKKS_BCONV_TENSOR, "cuda": ks.CKKS_BCONV_CUDA_CORES,
+                                 "auto": ks.CKKS_BCONV_AUTO}[args.bconv])
 
 
 def run_int_peaks(local_rank):
@@ -1113,9 +1116,9 @@ def main():
     ap.add_argument("--graph", action="store_true",
                     help="time one CUDA graph replay per step instead of eager launches (pays at small "
                          "batches; at 2 streams x 4 units the other stream already hides launch gaps)")
-    ap.add_argument("--bconv", default="tensor", choices=sorted(BCONV_ENGINES),
-                    help="base-conversion engine: tensor (8-bit split on the tensor cores, default) or cuda "
-                         "(CUDA cores); the output bits are the same")
+    ap.add_argument("--bconv", default="auto", choices=sorted(BCONV_ENGINES),
+                    help="base-conversion engine: auto (default: tensor cores for large launches), tensor "
+                         "(8-bit split on the tensor cores) or cuda (CUDA cores); the output bits are the same")
     ap.add_argument("--int-peaks", action="store_true",
                     help="measure this GPU's integer throughput per instruction class (ckks_int_probe) and "
                          "print it as one JSON line")

@@ -34,6 +34,7 @@ constexpr int TC_MAX_IN = 15;             // 4 * 15 + 1 = 61 <= 64
 constexpr int TC_MAX_T = 32;              // targets per chunk: N = 4 T <= 128 columns per accumulator
 constexpr int TC_THREADS = 288;           // 4 producer warps, 4 epilogue warps, 1 MMA warp
 constexpr int TC_TILES = 16;              // coefficient tiles per CTA, at most (BconvTcArgs::tiles)
+constexpr int TC_MIN_TILES = 4;           // smaller launches use the CUDA-core kernel
 constexpr int TC_STAGES = 5;              // A ring: the inputs of four tiles ahead are in flight
 constexpr int TC_COLS = 256;              // tensor-memory columns a CTA allocates: two accumulators
 // Dynamic shared memory per CTA: the A ring (5 x 8 KB) + B (<= 8 KB) + target records, padded so

@@ -449,7 +449,6 @@ struct IpRowArgs {
     u32 hoist_g[KS_MAXB], cdig_g[KS_MAXB];
     // groups (blockIdx.z): items grp_item[grp_first[g] .. grp_first[g] + grp_count[g] - 1]
     int grp_first[KS_MAXB], grp_count[KS_MAXB], grp_item[KS_MAXB];
-    int *err;                     // device error word (k_ip_row_ws's bounded waits)
 };
 
 __global__ void __launch_bounds__(ROW_THREADS)
@@ -844,6 +843,3 @@ k_sum_parts(SumArgs a) {
 
 // ---------------------------------------------------------------- base conversion on the tensor cores
 #include "bconv_tc.cuh"
-
-// ---------------------------------------------------------------- inner product, warp-specialized
-#include "ip_row_ws.cuh"

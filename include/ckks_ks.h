@@ -238,14 +238,16 @@ int ckks_modraise(ckks_ctx *ctx, const uint32_t *ct, int level, uint32_t *out, v
 
 /* Base-conversion engine (the results are the same residues either way; the bits of every
  * entry point's output are identical):
- *  CKKS_BCONV_TENSOR (default): the conversion as an exact 8-bit contraction on the tensor cores
+ *  CKKS_BCONV_TENSOR: the conversion as an exact 8-bit contraction on the tensor cores
  *    (tcgen05.mma kind::i8, sm_100a): inputs split into bytes along K with the byte shifts folded
  *    into the constants, 4 byte columns per target summed with shifts 0, 8, 16, 24 in the
  *    epilogue.  Groups of more than 15 primes use the CUDA cores;
- *  CKKS_BCONV_CUDA_CORES: 32 x 32 -> 64-bit multiply-adds on the CUDA cores.
+ *  CKKS_BCONV_CUDA_CORES: 32 x 32 -> 64-bit multiply-adds on the CUDA cores;
+ *  CKKS_BCONV_AUTO (default): the tensor cores for launches large enough to give each block of
+ *    the tensor-core kernel at least 4 tiles of 128 coefficients, the CUDA cores otherwise.
  * The mode applies to later calls on the context; it is not synchronised with calls in flight
  * from other threads.  CKKS_ERR_ARG for an unknown mode. */
-enum { CKKS_BCONV_CUDA_CORES = 0, CKKS_BCONV_TENSOR = 1 };
+enum { CKKS_BCONV_CUDA_CORES = 0, CKKS_BCONV_TENSOR = 1, CKKS_BCONV_AUTO = 2 };
 int ckks_set_bconv_mode(ckks_ctx *ctx, int mode);
 
 /* The key's regenerated uniform half for one (digit, global limb): out [N] (device),

@@ -79,9 +79,10 @@ def test_tc_rotate_relin_and_modes_agree(ks_lib, oracle_mod, key):
     ks.ckks_relin(ctx, d, lvl, evk_0, out, ws)
     want_rel = octx.relin(octx.tensor(x, y, lvl), lvl, cfg.alpha, b0, cfg.chacha_seed, 0)
     assert np.array_equal(_host(out), want_rel)
-    ks.ckks_set_bconv_mode(ctx, ks.CKKS_BCONV_CUDA_CORES)
-    ks.ckks_rotate(ctx, _dev(x), lvl, g, evk_g, out, ws)
-    assert np.array_equal(_host(out), want_rot)
+    for mode in (ks.CKKS_BCONV_CUDA_CORES, ks.CKKS_BCONV_AUTO):
+        ks.ckks_set_bconv_mode(ctx, mode)
+        ks.ckks_rotate(ctx, _dev(x), lvl, g, evk_g, out, ws)
+        assert np.array_equal(_host(out), want_rot), mode
 
 
 def test_tc_batch_and_hoisted(ks_lib, oracle_mod):
