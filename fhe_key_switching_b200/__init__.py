@@ -72,6 +72,12 @@ _SIGS = {
     "ckks_prof_begin": (_ci, [_vp, ctypes.c_char_p, _ci]),
     "ckks_prof_end": (_ci, [_vp, ctypes.POINTER(_ci), ctypes.POINTER(ctypes.c_double)]),
     "ckks_set_bconv_mode": (_ci, [_vp, _ci]),
+    "ckks_mul_const": (_ci, [_vp, _vp, _ci, _ci, ctypes.c_longlong, _vp, _vp]),
+    "ckks_add_const": (_ci, [_vp, _vp, _ci, ctypes.c_longlong, _vp, _vp]),
+    "ckks_add": (_ci, [_vp, _vp, _vp, _ci, _ci, _vp, _vp]),
+    "ckks_evalmod_workspace_bytes": (_sz, [_vp, _ci]),
+    "ckks_evalmod": (_ci, [_vp, _vp, _ci, ctypes.c_double, _ci, _ci, ctypes.POINTER(ckks_evk), _vp,
+                           ctypes.POINTER(_ci), ctypes.POINTER(ctypes.c_double), _vp, _sz, _vp]),
     "ckks_modraise": (_ci, [_vp, _vp, _ci, _vp, _vp, _sz, _vp]),
     "ckks_encode": (_ci, [_vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double), ctypes.c_double,
                           _ci, _ci, _vp, _vp, _sz, _vp]),
@@ -353,6 +359,36 @@ def ckks_encode(ctx, slots, scale: float, level: int, out, ws, with_special: boo
     im = (ctypes.c_double * n)(*[complex(v).imag for v in slots])
     _check(_L.ckks_encode(ctx.handle, re, im, float(scale), level, 1 if with_special else 0, _ptr(out), _ptr(ws),
                           ws.numel() * ws.element_size(), _stream(stream)), "ckks_encode")
+
+
+def ckks_mul_const(ctx, ct, n_comp: int, level: int, v: int, out, stream=None):
+    _check(_L.ckks_mul_const(ctx.handle, _ptr(ct), n_comp, level, v, _ptr(out), _stream(stream)), "ckks_mul_const")
+
+
+def ckks_add_const(ctx, ct, level: int, v: int, out, stream=None):
+    _check(_L.ckks_add_const(ctx.handle, _ptr(ct), level, v, _ptr(out), _stream(stream)), "ckks_add_const")
+
+
+def ckks_add(ctx, x, y, n_comp: int, level: int, out, stream=None):
+    _check(_L.ckks_add(ctx.handle, _ptr(x), _ptr(y), n_comp, level, _ptr(out), _stream(stream)), "ckks_add")
+
+
+def ckks_evalmod_workspace(ctx, level: int, device=None):
+    import torch
+    nb = int(_L.ckks_evalmod_workspace_bytes(ctx.handle, level))
+    if nb == 0:
+        raise ValueError("ckks_evalmod_workspace_bytes: level out of range")
+    return torch.empty(nb, dtype=torch.uint8, device=device or torch.device("cuda", torch.cuda.current_device()))
+
+
+def ckks_evalmod(ctx, ct, level: int, scale: float, r: int, d: int, relin_evk: ckks_evk, out, ws, stream=None):
+    """EvalMod: out's slots ~ sin(2 pi x) / (2 pi) for ct's real slots x; returns (out_level, out_scale)."""
+    lv = _ci()
+    sc = ctypes.c_double()
+    _check(_L.ckks_evalmod(ctx.handle, _ptr(ct), level, float(scale), r, d, ctypes.byref(relin_evk), _ptr(out),
+                           ctypes.byref(lv), ctypes.byref(sc), _ptr(ws), ws.numel() * ws.element_size(),
+                           _stream(stream)), "ckks_evalmod")
+    return lv.value, sc.value
 
 
 def ckks_modraise(ctx, ct, level: int, out, ws, stream=None):

@@ -236,6 +236,42 @@ int ckks_encode(ckks_ctx *ctx, const double *re, const double *im, double scale,
 int ckks_modraise(ckks_ctx *ctx, const uint32_t *ct, int level, uint32_t *out, void *ws, size_t ws_bytes,
                   ckks_stream_t stream);
 
+/* Ciphertext arithmetic for polynomial evaluation (EvalMod).  All in the evaluation domain over
+ * q_0..q_level, canonical; out may equal the input (elementwise).
+ *  ckks_mul_const: every component of ct [n_comp][l+1][N] times the integer v (reduced mod q_i;
+ *    the plaintext scale is unchanged, the slots are multiplied by v);
+ *  ckks_add_const: ct [2][l+1][N] plus the constant polynomial v on component 0 (the slots gain
+ *    v / scale);
+ *  ckks_add: x + y, both [n_comp][l+1][N].
+ * n_comp in 1..3; errors as for the other calls. */
+int ckks_mul_const(ckks_ctx *ctx, const uint32_t *ct, int n_comp, int level, long long v, uint32_t *out,
+                   ckks_stream_t stream);
+int ckks_add_const(ckks_ctx *ctx, const uint32_t *ct, int level, long long v, uint32_t *out, ckks_stream_t stream);
+int ckks_add(ckks_ctx *ctx, const uint32_t *x, const uint32_t *y, int n_comp, int level, uint32_t *out,
+             ckks_stream_t stream);
+
+/* EvalMod, the modular reduction of CKKS bootstrapping (Cheon, Han, Kim, Kim, Song, Eurocrypt
+ * 2018; the pages give no construction): for a ciphertext whose slots hold real x with
+ * |x| small, out's slots approximate sin(2 pi x) / (2 pi), which equals x - round(x) near the
+ * integers.  Fixed sequence (every constant an integer by std::llround, half away from zero, of
+ * an IEEE double product; the nominal scale S tracked in double):
+ *   theta = (2 pi / 2^r)(x - 1/4): ct * llround(c1 q_l), rescale, + llround(-(c1/4) S);
+ *   u = theta^2 (tensor, relinearisation, rescale; S_u = S^2 / q_l);
+ *   cos(theta) = sum_{k<=d} (-1)^k u^k / (2k)! by Horner: p = u * llround(a_d q_l), rescale,
+ *     + llround(a_(d-1) S_u), then d - 1 times p = p * u (u dropped to p's level), + llround(a_k S_p);
+ *   r double angles: p = 2 p^2 - 1 (square, relinearisation, rescale, * 2, + llround(-S_p));
+ *   out = p * llround(q_l / (2 pi)), rescale.
+ * It consumes d + r + 3 levels: *out_level = level - d - r - 3, *out_scale = the tracked scale of
+ * out.  ct: [2][level+1][N]; out: room for 2 (level+1) N words, of which the first
+ * 2 (*out_level+1) N hold the result as [2][*out_level+1][N]; relin_key: the key for s^2
+ * (key_id 0); ws: ckks_evalmod_workspace_bytes(ctx, level)
+ * bytes.  r in 0..16, d in 1..16.  Errors: CKKS_ERR_ARG (null, ranges, scale, overlap),
+ * CKKS_ERR_UNSUPPORTED (level below d + r + 3 or above the chain), CKKS_ERR_ALIGN,
+ * CKKS_ERR_WORKSPACE. */
+size_t ckks_evalmod_workspace_bytes(const ckks_ctx *ctx, int level);
+int ckks_evalmod(ckks_ctx *ctx, const uint32_t *ct, int level, double scale, int r, int d, const ckks_evk *relin_key,
+                 uint32_t *out, int *out_level, double *out_scale, void *ws, size_t ws_bytes, ckks_stream_t stream);
+
 /* Base-conversion engine (the results are the same residues either way; the bits of every
  * entry point's output are identical):
  *  CKKS_BCONV_TENSOR: the conversion as an exact 8-bit contraction on the tensor cores

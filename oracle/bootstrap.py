@@ -26,6 +26,8 @@ signed sums of the stages' half-lengths.
 """
 from __future__ import annotations
 
+import math
+
 import numpy as np
 
 
@@ -234,3 +236,83 @@ def linear_level(ctx, ct, level: int, alpha: int, babies, giants, pt_enc, keys: 
     gk = [None if g == 1 else (keys[g], g) for g in gg]
     out = ctx.bsgs(ct, level, alpha, bg, bk, gg, gk, pt_enc, seed)
     return ctx.rescale(out, level)
+
+
+# ----------------------------------------------------------------------------- EvalMod
+# The modular reduction of bootstrapping: slots x (real, near the integers) -> x - round(x),
+# approximated by sin(2 pi x) / (2 pi) = cos(2 pi (x - 1/4)) / (2 pi), the cosine evaluated as an
+# even Taylor polynomial of theta = 2 pi (x - 1/4) / 2^r followed by r double angles
+# cos(2t) = 2 cos(t)^2 - 1 (the scaled-sine approach of Cheon, Han, Kim, Kim, Song, Eurocrypt
+# 2018, with the double-angle step of Han and Ki, CT-RSA 2020).  Every constant is an integer:
+# the IEEE double product rounded half away from zero (C's llround), so that the library's
+# evaluation of the same sequence is comparable bit for bit.
+
+def llround(x: float) -> int:
+    """Round half away from zero, exactly as C's llround for doubles below 2^52 in magnitude."""
+    f = math.floor(x)
+    d = x - f                       # exact
+    if d > 0.5:
+        return int(f) + 1
+    if d < 0.5:
+        return int(f)
+    return int(f) + 1 if x > 0 else int(f)
+
+
+def mul_const(ctx, ct: np.ndarray, level: int, v: int) -> np.ndarray:
+    """Every component times the integer v, limb by limb modulo q_i."""
+    q = np.array(ctx.q[: level + 1], dtype=np.uint64)[:, None]
+    w = np.array([v % int(qi) for qi in ctx.q[: level + 1]], dtype=np.uint64)[:, None]
+    return ((np.asarray(ct, dtype=np.uint64) * w) % q).astype(np.uint32)
+
+
+def add_const(ctx, ct: np.ndarray, level: int, v: int) -> np.ndarray:
+    """The constant polynomial v (every evaluation slot) added to component 0."""
+    q = np.array(ctx.q[: level + 1], dtype=np.uint64)[:, None]
+    w = np.array([v % int(qi) for qi in ctx.q[: level + 1]], dtype=np.uint64)[:, None]
+    out = np.array(ct, dtype=np.uint32, copy=True)
+    out[0] = ((out[0].astype(np.uint64) + w) % q).astype(np.uint32)
+    return out
+
+
+def evalmod(ctx, ct: np.ndarray, level: int, scale: float, r: int, d: int, alpha: int,
+            relin_b: np.ndarray, seed: bytes):
+    """Returns (ciphertext [2][level_out+1][N], level_out, scale_out); consumes d + r + 3 levels."""
+    a = []
+    fact = 1.0
+    for k in range(d + 1):
+        a.append((-1.0 if k & 1 else 1.0) / fact)
+        fact *= float(2 * k + 1) * float(2 * k + 2)
+    c1 = 2.0 * math.pi / float(1 << r)
+    q = lambda lv: float(ctx.q[lv])
+
+    def mult(x, y, lv):
+        return ctx.rescale(ctx.relin(ctx.tensor(x, y, lv), lv, alpha, relin_b, seed, 0), lv)
+
+    lv, S = level, scale
+    t = ctx.rescale(mul_const(ctx, ct, lv, llround(c1 * q(lv))), lv)
+    lv -= 1
+    t = add_const(ctx, t, lv, llround(-(c1 / 4.0) * S))
+    u = mult(t, t, lv)
+    Su = S * S / q(lv)
+    lv -= 1
+    lu = lv
+    p = ctx.rescale(mul_const(ctx, u, lv, llround(a[d] * q(lv))), lv)
+    lv -= 1
+    Sp = Su
+    p = add_const(ctx, p, lv, llround(a[d - 1] * Sp))
+    for k in range(d - 2, -1, -1):
+        ua = np.ascontiguousarray(u[:, : lv + 1])
+        p = mult(p, ua, lv)
+        Sp = Sp * Su / q(lv)
+        lv -= 1
+        p = add_const(ctx, p, lv, llround(a[k] * Sp))
+    for _ in range(r):
+        p = mult(p, p, lv)
+        Sp = Sp * Sp / q(lv)
+        lv -= 1
+        p = mul_const(ctx, p, lv, 2)
+        p = add_const(ctx, p, lv, llround(-1.0 * Sp))
+    out = ctx.rescale(mul_const(ctx, p, lv, llround(1.0 / (2.0 * math.pi) * q(lv))), lv)
+    lv -= 1
+    assert lu >= lv
+    return out, lv, Sp

@@ -94,3 +94,67 @@ def _dft_levels(ks_lib, key, levels, n1, direction):
     ref = bt.coeff_to_slot(z, log_n, levels) if inverse else bt.slot_to_coeff(z, log_n, levels)
     err = np.max(np.abs(got - ref))
     assert err < (2.0 ** -8 if inverse else 2.0 ** -9 * np.max(np.abs(ref))), err
+
+
+def test_constant_ops_parity(ks_lib, oracle_mod):
+    """ckks_mul_const, ckks_add_const and ckks_add against the oracle's restatement, bit for bit,
+    with negative constants and constants above the primes."""
+    from oracle import bootstrap as bt
+    ks = ks_lib
+    cfg = W.CONFIGS["n14-hoisted8"]
+    q, p = ks.ckks_gen_primes(cfg.log_n, cfg.n_q, cfg.n_p)
+    octx = oracle_mod.Ctx(cfg.log_n, cfg.n_q, cfg.n_p)
+    ctx = ks.Context(cfg.log_n, q, p, cfg.dnum)
+    lvl, n = cfg.level, cfg.n
+    gen = W.rng(cfg.seed, W.TAG_SYNTH, 9300)
+    x = W.uniform_residues(q[: lvl + 1] * 2, n, gen).reshape(2, lvl + 1, n)
+    y = W.uniform_residues(q[: lvl + 1] * 2, n, gen).reshape(2, lvl + 1, n)
+    out = torch.empty((2, lvl + 1, n), dtype=torch.uint32, device="cuda")
+    for v in (-3, 2, 5 * (1 << 40) + 7, -(1 << 45) - 1):
+        ks.ckks_mul_const(ctx, _dev(x), 2, lvl, v, out)
+        assert np.array_equal(_host(out), bt.mul_const(octx, x, lvl, v)), v
+        ks.ckks_add_const(ctx, _dev(x), lvl, v, out)
+        assert np.array_equal(_host(out), bt.add_const(octx, x, lvl, v)), v
+    ks.ckks_add(ctx, _dev(x), _dev(y), 2, lvl, out)
+    mods = np.array(q[: lvl + 1], dtype=np.uint64)[:, None]
+    assert np.array_equal(_host(out), ((x.astype(np.uint64) + y) % mods).astype(np.uint32))
+
+
+def _evalmod_case(ks, oracle_mod, key, level, r, d, check_decode):
+    from oracle import bootstrap as bt
+    from oracle.scenario import Scenario
+    cfg = W.CONFIGS[key]
+    sc = Scenario(cfg)
+    octx = sc.ctx
+    q, p = ks.ckks_gen_primes(cfg.log_n, cfg.n_q, cfg.n_p)
+    ctx = ks.Context(cfg.log_n, q, p, cfg.dnum)
+    S = float(octx.q[level])
+    x = np.random.default_rng(5).uniform(-2, 2, cfg.n // 2)
+    m = oracle_mod.encode(x.astype(complex), cfg.n, S)
+    e = W.gaussian_error(cfg.n, cfg.sigma, W.rng(cfg.seed, W.TAG_ENC_ERR, 77))[0]
+    a = W.uniform_residues(octx.q[: level + 1], cfg.n, W.rng(cfg.seed, W.TAG_ENC_A, 77))
+    ct = octx.encrypt(sc.s, m, e, a, level)
+    b0 = sc.key(0)
+    want, lv, so = bt.evalmod(octx, ct, level, S, r, d, cfg.alpha, b0, cfg.chacha_seed)
+    evk = ks.make_evk(_dev(b0), cfg.chacha_seed, 0)
+    out = torch.empty((2, level + 1, cfg.n), dtype=torch.uint32, device="cuda")
+    g_lv, g_so = ks.ckks_evalmod(ctx, _dev(ct), level, S, r, d, evk, out, ks.ckks_evalmod_workspace(ctx, level))
+    assert (g_lv, g_so) == (lv, so)
+    got = _host(out).reshape(-1)[: 2 * (lv + 1) * cfg.n].reshape(2, lv + 1, cfg.n)
+    assert np.array_equal(got, want)
+    if check_decode:
+        err = np.abs(sc.decrypt_slots(got, lv, so).real - np.sin(2 * np.pi * x) / (2 * np.pi))
+        assert err.max() < 2.0 ** -9
+
+
+def test_evalmod_parity_n14(ks_lib, oracle_mod):
+    """EvalMod (degree 8 in theta, two double angles) at N=2^14 from level 11, bit for bit (this
+    chain's key-switching noise is too large for the decoded values to mean much)."""
+    _evalmod_case(ks_lib, oracle_mod, "n14-hoisted8", 11, 2, 4, False)
+
+
+@pytest.mark.slow
+def test_evalmod_parity_n16(ks_lib, oracle_mod):
+    """EvalMod (degree 12, three double angles) at N=2^16, dnum 4, from level 35: bit for bit with
+    the oracle, and decoding to sin(2 pi x) / (2 pi) within 2^-9."""
+    _evalmod_case(ks_lib, oracle_mod, "n16-stream64", 35, 3, 6, True)

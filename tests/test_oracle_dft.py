@@ -142,3 +142,55 @@ def test_homomorphic_levels_decode(direction):
         assert err < 2.0 ** -8, err
     else:
         assert err < 2.0 ** -9 * np.max(np.abs(want)), (err, np.max(np.abs(want)))
+
+
+def test_llround_is_half_away_from_zero():
+    for x, want in [(2.5, 3), (-2.5, -3), (0.49999999999999994, 0), (-0.5, -1), (1e15 + 0.5, int(1e15) + 1),
+                    (3.2, 3), (-3.7, -4), (0.0, 0)]:
+        assert bt.llround(x) == want, x
+
+
+@pytest.mark.slow
+def test_evalmod_decodes_to_scaled_sine():
+    """EvalMod (cosine Taylor polynomial of degree 12 in theta = 2 pi (x - 1/4) / 8, three double
+    angles) on an encryption of real slots x in [-2, 2] at N=2^16, dnum 4, level 35, scale q_35,
+    decodes to sin(2 pi x) / (2 pi): the polynomial itself is within 4.3e-8 of it; the measured
+    error (CKKS noise of the input amplified up to 64 times by the double angles) has median
+    1.9e-6 and maximum 1.1e-3 (2^-9.85) over the 32768 slots.  Pinned: median below 2^-17 and
+    maximum below 2^-9; a wrong coefficient, sign or step gives errors of order 0.1."""
+    import workloads as W
+    from oracle.scenario import Scenario
+    cfg = W.CONFIGS["n16-stream64"]
+    sc = Scenario(cfg)
+    ctx = sc.ctx
+    L = 35
+    S = float(ctx.q[L])
+    x = np.random.default_rng(5).uniform(-2, 2, cfg.n // 2)
+    m = oracle.encode(x.astype(complex), cfg.n, S)
+    e = W.gaussian_error(cfg.n, cfg.sigma, W.rng(cfg.seed, W.TAG_ENC_ERR, 77))[0]
+    a = W.uniform_residues(ctx.q[: L + 1], cfg.n, W.rng(cfg.seed, W.TAG_ENC_A, 77))
+    ct = ctx.encrypt(sc.s, m, e, a, L)
+    out, lv, so = bt.evalmod(ctx, ct, L, S, 3, 6, cfg.alpha, sc.key(0), cfg.chacha_seed)
+    assert lv == L - (6 + 3 + 3)
+    err = np.abs(sc.decrypt_slots(out, lv, so).real - np.sin(2 * np.pi * x) / (2 * np.pi))
+    assert np.median(err) < 2.0 ** -17 and err.max() < 2.0 ** -9, (np.median(err), err.max())
+
+
+def test_constant_ops_by_definition():
+    """mul_const and add_const against the slot values they must produce (decoded), and the
+    residue arithmetic against Python integers."""
+    import workloads as W
+    from oracle.scenario import Scenario
+    cfg = W.CONFIGS["n12-dnum4"]
+    sc = Scenario(cfg)
+    ctx = sc.ctx
+    z, ct = sc.ciphertext(0)
+    lvl = cfg.level
+    m3 = bt.mul_const(ctx, ct, lvl, -3)
+    for i in range(lvl + 1):
+        qi = ctx.q[i]
+        assert int(m3[1, i, 5]) == (int(ct[1, i, 5]) * -3) % qi
+    assert np.max(np.abs(sc.decrypt_slots(m3) - (-3) * z)) < 1e-3
+    c = bt.add_const(ctx, ct, lvl, bt.llround(0.75 * sc.scale))
+    assert np.array_equal(c[1], ct[1])
+    assert np.max(np.abs(sc.decrypt_slots(c) - (z + 0.75))) < 1e-3
