@@ -752,6 +752,73 @@ def run_workload(args, local_rank):
         ks_per_step, rot_per_step = 0, 0
         ops, blocks = R * rescale_ops(cfg, lvl), 0
         nbytes = R * (2 * na + 2 * lvl) * limb
+    elif key == "bootstrap-steps":
+        # the bootstrapping steps this library has, in sequence, at N=2^16 (dnum 4, levels 35 -> 17):
+        # ModRaise to level 35, CoeffToSlot (3 levels), one conjugation, EvalMod twice (the real and
+        # the imaginary halves: degree 12, 3 double angles, 12 levels each), SlotToCoeff (3 levels);
+        # synthetic plaintexts and keys (the cost is data independent)
+        levels, n1, L = 3, 8, cfg.n_q - 1
+        ns = n // 2
+        halves_fwd = [1 << h for h in range(cfg.log_n - 2, -1, -1)]
+        per = -(-len(halves_fwd) // levels)
+
+        def dft_plan(top, inverse):
+            hs_all = halves_fwd if inverse else halves_fwd[::-1]
+            plan_ = []
+            for li in range(levels):
+                hs = hs_all[li * per:(li + 1) * per]
+                st_ = min(hs)
+                shifts = {0}
+                for h in hs:
+                    shifts = {((x_ + dd + ns // 2) % ns) - ns // 2 for x_ in shifts for dd in (-h, 0, h)}
+                ms_ = sorted(x_ // st_ for x_ in shifts)
+                bg_ = [1 if k == 0 else ks.galois_element(cfg.log_n, k * st_) for k in range(n1)]
+                gg_ = [1 if g_ == 0 else ks.galois_element(cfg.log_n, g_ * n1 * st_)
+                       for g_ in range(ms_[0] // n1, ms_[-1] // n1 + 1)]
+                lv_ = top - li
+                pt_ = res((q[:lv_ + 1] + p) * len(gg_) * len(bg_)).view(len(gg_), len(bg_), lv_ + 1 + cfg.n_p, n)
+                plan_.append((lv_, bg_, gg_, pt_, ks.ckks_bsgs_workspace(ctx, lv_, len(bg_), len(gg_), device=dev)))
+            return plan_
+        c2s, s2c = dft_plan(L, True), dft_plan(L - 3 - 12, False)
+        gk = {}
+        for _, bg_, gg_, _, _ in c2s + s2c:
+            for g_ in bg_ + gg_:
+                if g_ != 1 and g_ not in gk:
+                    gk[g_] = ks.make_evk(res(mods * nd).view(nd, len(mods), n), cfg.chacha_seed, g_)
+        gconj = ks.conjugation_element(cfg.log_n)
+        k_conj = ks.make_evk(res(mods * nd).view(nd, len(mods), n), cfg.chacha_seed, gconj)
+        k_rel = ks.make_evk(res(mods * nd).view(nd, len(mods), n), cfg.chacha_seed, 0)
+        cts0 = [res(q[:1] * 2).view(2, 1, n) for _ in range(N_SETS)]
+        big = torch.empty((2, L + 1, n), dtype=torch.uint32, device=dev)
+        bufs = [torch.empty((2, L + 1, n), dtype=torch.uint32, device=dev) for _ in range(4)]
+        ws_mr = torch.empty(2 * n, dtype=torch.uint32, device=dev)
+        ws_ks = ctx.workspace(L, 1, device=dev)
+        ws_em = ks.ckks_evalmod_workspace(ctx, L - 3, device=dev)
+
+        def run_levels(plan_, src):
+            cur = src
+            for i_, (lv_, bg_, gg_, pt_, ws_l) in enumerate(plan_):
+                ks.ckks_bsgs(ctx, cur, lv_, bg_, [gk.get(g_) for g_ in bg_], gg_, [gk.get(g_) for g_ in gg_],
+                             pt_, bufs[0].view(-1)[: 2 * (lv_ + 1) * n].view(2, lv_ + 1, n), ws_l, stream)
+                dst = bufs[1 + (i_ & 1)].view(-1)[: 2 * lv_ * n].view(2, lv_, n)
+                ks.ckks_rescale(ctx, bufs[0].view(-1)[: 2 * (lv_ + 1) * n].view(2, lv_ + 1, n), lv_, dst, ws_ks,
+                                stream)
+                cur = dst
+            return cur
+
+        def step(i):
+            ks.ckks_modraise(ctx, cts0[i % N_SETS], L, big, ws_mr, stream)
+            z = run_levels(c2s, big)
+            lz = L - 3
+            zc = bufs[3].view(-1)[: 2 * (lz + 1) * n].view(2, lz + 1, n)
+            ks.ckks_rotate(ctx, z, lz, gconj, k_conj, zc, ws_ks, stream)
+            e1 = bufs[0].view(-1)[: 2 * (lz + 1) * n].view(2, lz + 1, n)
+            ks.ckks_evalmod(ctx, z, lz, float(q[lz]), 3, 6, k_rel, e1, ws_em, stream)
+            ks.ckks_evalmod(ctx, zc, lz, float(q[lz]), 3, 6, k_rel, big, ws_em, stream)
+            run_levels(s2c, big.view(-1)[: 2 * (lz - 12 + 1) * n].view(2, lz - 12 + 1, n))
+        ks_per_step = rot_per_step = (sum(sum(1 for g_ in bg_ + gg_ if g_ != 1) for _, bg_, gg_, _, _ in c2s + s2c)
+                                      + 1)
+        ops = blocks = nbytes = 0        # reported as a time only: its op model is not tabulated
     elif key == "coeff-to-slot":
         # CoeffToSlot of N=2^16 in 3 levels of 5 radix-2 stages: each level's 63 slot diagonals
         # (shifts m s, |m| <= 31, s its smallest half-length) as 8 baby x 8 giant steps, then a
@@ -858,6 +925,11 @@ def run_workload(args, local_rank):
             "ms_per_step": ms / args.steps, "steps": args.steps, "warmup": args.warmup}
     if key == "rescale":
         line["rescales_per_s"] = R / t_step
+    elif key == "bootstrap-steps":
+        line["ms_per_bootstrap_steps"] = t_step * 1e3
+        line["context"] = ("the EncryptedLLM summary (lpnh.cn page, Results) quotes 22-27 ms per whole bootstrap "
+                           "on an unnamed GPU; these are the steps this library has, not a complete bootstrap "
+                           "(the real/imaginary split and recombination are not timed)")
     elif key == "coeff-to-slot":
         line["ms_per_coeff_to_slot"] = t_step * 1e3
         line["context"] = ("the EncryptedLLM summary (lpnh.cn page, Results) quotes 22-27 ms per whole "
@@ -869,7 +941,8 @@ def run_workload(args, local_rank):
         line["key_switches_per_s"] = ks_per_step / t_step
         line["rotations_per_s"] = rot_per_step / t_step
         line["key_switches_per_step"] = ks_per_step
-    line["path_roofline"] = dict(path_roofline(ops, blocks, nbytes, t_step, peaks), per="one step")
+    if ops:
+        line["path_roofline"] = dict(path_roofline(ops, blocks, nbytes, t_step, peaks), per="one step")
     line.update(extra)
     line["int_peaks"] = int_peaks_summary(peaks)
     line["clocks"] = clk
@@ -878,11 +951,14 @@ def run_workload(args, local_rank):
     print(json.dumps(line), flush=True)
 
 
-INFO_WORKLOADS = {"coeff-to-slot": "n16-bsgs32",
+INFO_WORKLOADS = {"coeff-to-slot": "n16-bsgs32", "bootstrap-steps": "n16-stream64",
                   "n14-hoisted8": "n14-hoisted8", "n16-bsgs32": "n16-bsgs32", "n16-stream64": "n16-stream64",
                   "n16-stream64-rescale": "n16-stream64", "rescale": "n16-full", "bsgs": "n16-bsgs32",
                   "bsgs-n14": "n14-hoisted8"}
 INFO_DESCRIPTIONS = {
+    "bootstrap-steps": "N=2^16, 36+12 primes, dnum 4; step = ModRaise to level 35, CoeffToSlot (3 levels), "
+                       "a conjugation, EvalMod twice (12 levels each, degree 12, 3 double angles), "
+                       "SlotToCoeff (3 levels)",
     "coeff-to-slot": "N=2^16, 36+12 primes, dnum 4, from level 24; step = CoeffToSlot in 3 levels of 5 radix-2 "
                      "stages, each an 8 baby x 8 giant step transform of 63 slot diagonals plus a rescale",
     "n14-hoisted8": "N=2^14, 12+4 primes, dnum 3, level 11; step = 8 units, each 8 hoisted rotations "
@@ -913,7 +989,7 @@ def info_cpu_baseline(key: str, max_seconds: float = 8.0):
     ct = W.uniform_residues(octx.q[:na] * 2, n, gen).reshape(2, na, n)
     b = W.uniform_residues(octx.mod * nd, n, gen).reshape(nd, len(octx.mod), n)
     seed = cfg.chacha_seed
-    if key in ("bsgs", "coeff-to-slot"):
+    if key in ("bsgs", "coeff-to-slot", "bootstrap-steps"):
         return None                 # the oracle's plaintext sums take minutes at N=2^16
     if key == "n14-hoisted8":
         gs = [octx.galois(r) for r in cfg.rot_steps]
