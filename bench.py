@@ -593,7 +593,7 @@ def roofline(cfg, launches, total_ms, clk, batch, single_step_ms, launches_ov, t
 # them the figure is reported as null until a new capture replaces it.
 IP_ROW_TRAFFIC = {"sources_sha16": "cab75b06f246685b", "bytes_per_unit": (473.90e6 + 471.65e6) / 2 / 4,
                   "capture": "profiles/k_ip_row_n16_full.md (dram__bytes read + write of two 4-unit launches)"}
-KERNEL_HEADERS = ("modarith.cuh", "chacha.cuh", "ntt.cuh", "ks_kernels.cuh")
+KERNEL_HEADERS = ("debug_bounds.cuh", "modarith.cuh", "chacha.cuh", "ntt.cuh", "ks_kernels.cuh")
 
 
 def kernel_sources_sha16() -> str:

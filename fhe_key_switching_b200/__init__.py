@@ -6,6 +6,10 @@ memory and streams.  The functions keep the C names; buffers are CUDA tensors of
 uint32 or int32 (reinterpreted), contiguous, laid out as the header states.
 
 There is no CPU fallback: if the compiled library is missing, importing this package raises.
+
+``FHE_KS_B200_BUILD=debug`` in the environment loads the debug-bounds build of the same sources
+(``libckks_ks_debug.so``, from ``python fhe_key_switching_b200/build.py --debug``), whose kernels
+check every access span against the call's buffers (see ckks_debug_bounds_report).
 """
 from __future__ import annotations
 
@@ -13,17 +17,20 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "_build", "libckks_ks.so")
+BUILD = os.environ.get("FHE_KS_B200_BUILD", "release")
+if BUILD not in ("release", "debug"):
+    raise ImportError(f"FHE_KS_B200_BUILD={BUILD!r}: expected 'release' or 'debug'")
+LIB_PATH = os.path.join(_HERE, "_build", "libckks_ks_debug.so" if BUILD == "debug" else "libckks_ks.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"CUDA library {LIB_PATH} is not built; run `python fhe_key_switching_b200/build.py` "
-        "(nvcc, sm_100a) or `python __graft_entry__.py` first")
+        f"CUDA library {LIB_PATH} is not built; run `python fhe_key_switching_b200/build.py"
+        f"{' --debug' if BUILD == 'debug' else ''}` (nvcc, sm_100a) or `python __graft_entry__.py` first")
 
 _L = ctypes.CDLL(LIB_PATH)
 
 CKKS_OK, CKKS_ERR_ARG, CKKS_ERR_UNSUPPORTED, CKKS_ERR_ALIGN = 0, -1, -2, -3
-CKKS_ERR_WORKSPACE, CKKS_ERR_CUDA, CKKS_ERR_TIMEOUT = -4, -5, -6
+CKKS_ERR_WORKSPACE, CKKS_ERR_CUDA, CKKS_ERR_TIMEOUT, CKKS_ERR_BOUNDS = -4, -5, -6, -7
 
 _u32p = ctypes.POINTER(ctypes.c_uint32)
 _vp = ctypes.c_void_p
@@ -83,6 +90,11 @@ _SIGS = {
                           _ci, _ci, _vp, _vp, _sz, _vp]),
     "ckks_int_probe": (_ci, [_ci, _ci, _ci, _vp, _vp, ctypes.POINTER(ctypes.c_float),
                              ctypes.POINTER(ctypes.c_double)]),
+    "ckks_debug_bounds_enabled": (_ci, []),
+    "ckks_debug_bounds_report": (_ci, [ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(_ci),
+                                       ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_uint64), _ci]),
+    "ckks_debug_bounds_site_name": (ctypes.c_char_p, [_ci]),
+    "ckks_selftest_bounds": (_ci, [_vp, _vp]),
     "ckks_last_error": (ctypes.c_char_p, []),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -335,6 +347,27 @@ def ckks_sync_status(ctx, stream=None, timeout_ms: int = 10000) -> int:
 
 def ckks_selftest_wait_expiry(ctx, stream=None):
     _check(_L.ckks_selftest_wait_expiry(ctx.handle, _stream(stream)), "ckks_selftest_wait_expiry")
+
+
+def ckks_debug_bounds_enabled() -> bool:
+    return bool(_L.ckks_debug_bounds_enabled())
+
+
+def ckks_debug_bounds_report(clear: bool = True):
+    """(failed checks, first site's name, its address, its size in bytes) since the last clear."""
+    count, site, addr, nbytes = ctypes.c_uint64(), _ci(), ctypes.c_uint64(), ctypes.c_uint64()
+    _check(_L.ckks_debug_bounds_report(ctypes.byref(count), ctypes.byref(site), ctypes.byref(addr),
+                                       ctypes.byref(nbytes), int(clear)), "ckks_debug_bounds_report")
+    name = _L.ckks_debug_bounds_site_name(site.value).decode()
+    return int(count.value), name, int(addr.value), int(nbytes.value)
+
+
+def ckks_debug_bounds_site_name(site: int) -> str:
+    return _L.ckks_debug_bounds_site_name(site).decode()
+
+
+def ckks_selftest_bounds(ctx, stream=None):
+    _check(_L.ckks_selftest_bounds(ctx.handle, _stream(stream)), "ckks_selftest_bounds")
 
 
 def ckks_prof_begin(ctx, kernel: str, max_launches: int):

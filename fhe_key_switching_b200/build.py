@@ -1,4 +1,6 @@
-"""Build the CUDA library (sm_100a) in-tree: fhe_key_switching_b200/_build/libckks_ks.so."""
+"""Build the CUDA library (sm_100a) in-tree: fhe_key_switching_b200/_build/libckks_ks.so, and with
+``--debug`` the debug-bounds build of the same sources (-DCKKS_DEBUG_BOUNDS: index checks in every
+kernel, see include/ckks_ks.h) as fhe_key_switching_b200/_build/libckks_ks_debug.so."""
 from __future__ import annotations
 
 import glob
@@ -10,6 +12,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 OUT_DIR = os.path.join(HERE, "_build")
 LIB = os.path.join(OUT_DIR, "libckks_ks.so")
+LIB_DEBUG = os.path.join(OUT_DIR, "libckks_ks_debug.so")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 
 NVCC_FLAGS = [
@@ -24,26 +27,28 @@ def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(INCLUDE, "*.h"))
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
+def build(force: bool = False, verbose_ptxas: bool = False, debug: bool = False) -> str:
     os.makedirs(OUT_DIR, exist_ok=True)
-    if not force and not _stale():
-        return LIB
+    lib = LIB_DEBUG if debug else LIB
+    if not force and not _stale(lib):
+        return lib
     nvcc = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
-    cmd = [nvcc, *NVCC_FLAGS, "-I", INCLUDE, "-o", LIB + ".tmp", *sources()]
+    cmd = [nvcc, *NVCC_FLAGS, *(["-DCKKS_DEBUG_BOUNDS"] if debug else []), "-I", INCLUDE, "-o", lib + ".tmp",
+           *sources()]
     if verbose_ptxas:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.run(cmd, check=True)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(lib + ".tmp", lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose_ptxas="-v" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose_ptxas="-v" in sys.argv, debug="--debug" in sys.argv))

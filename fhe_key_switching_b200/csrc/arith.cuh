@@ -15,6 +15,9 @@ __global__ void k_mul_const(const u32 *in, u32 *out, ConstRns cw, const PrimeInf
     const int c4 = blockIdx.x * blockDim.x + threadIdx.x;
     if (4 * c4 >= n) return;
     const int r = blockIdx.y, i = r % (level + 1);
+    if (!CKKS_SPAN(pinfo + i, 1, CKKS_DBG_CONST) || !CKKS_SPAN(in + (size_t)r * n + 4 * c4, 4, CKKS_DBG_CONST) ||
+        !CKKS_SPAN(out + (size_t)r * n + 4 * c4, 4, CKKS_DBG_CONST))
+        return;
     const u32 q = pinfo[i].q;
     const tw_t w = cw.w[i];
     const uint4 v = reinterpret_cast<const uint4 *>(in + (size_t)r * n)[c4];
@@ -28,6 +31,9 @@ __global__ void k_add_const(const u32 *in, u32 *out, ConstRns cw, const PrimeInf
     const int c4 = blockIdx.x * blockDim.x + threadIdx.x;
     if (4 * c4 >= n) return;
     const int r = blockIdx.y, i = r % (level + 1);
+    if (!CKKS_SPAN(pinfo + i, 1, CKKS_DBG_CONST) || !CKKS_SPAN(in + (size_t)r * n + 4 * c4, 4, CKKS_DBG_CONST) ||
+        !CKKS_SPAN(out + (size_t)r * n + 4 * c4, 4, CKKS_DBG_CONST))
+        return;
     const u32 q = pinfo[i].q;
     const u32 c = r <= level ? cw.w[i].x : 0u;        // the constant polynomial: every slot, component 0
     const uint4 v = reinterpret_cast<const uint4 *>(in + (size_t)r * n)[c4];
@@ -40,6 +46,10 @@ __global__ void k_add(const u32 *x, const u32 *y, u32 *out, const PrimeInfo *pin
     const int c4 = blockIdx.x * blockDim.x + threadIdx.x;
     if (4 * c4 >= n) return;
     const int r = blockIdx.y, i = r % (level + 1);
+    if (!CKKS_SPAN(pinfo + i, 1, CKKS_DBG_CONST) || !CKKS_SPAN(x + (size_t)r * n + 4 * c4, 4, CKKS_DBG_CONST) ||
+        !CKKS_SPAN(y + (size_t)r * n + 4 * c4, 4, CKKS_DBG_CONST) ||
+        !CKKS_SPAN(out + (size_t)r * n + 4 * c4, 4, CKKS_DBG_CONST))
+        return;
     const u32 q = pinfo[i].q;
     const uint4 a = reinterpret_cast<const uint4 *>(x + (size_t)r * n)[c4];
     const uint4 b = reinterpret_cast<const uint4 *>(y + (size_t)r * n)[c4];

@@ -172,6 +172,11 @@ __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
     const u32 *yb = a.y + item * a.y_item + (size_t)(a.in_row0 + g * a.in_group_rows) * n;
     u32 *ob = a.out + item * a.out_item + ((size_t)g * a.map.out_group_rows + a.map.out_k_base) * n;
     auto a_stage = [&](int tile) { return tc_sm + (size_t)(tile % TC_STAGES) * TC_A_BYTES; };
+    if (!CKKS_SPAN(a.pinfo + p0, n_in, CKKS_DBG_TC_TABLES) ||
+        !CKKS_SPAN(a.pinfo + a.map.lo_base, a.map.split, CKKS_DBG_TC_TABLES) ||
+        (T > a.map.split && !CKKS_SPAN(a.pinfo + a.map.hi_base, T - a.map.split, CKKS_DBG_TC_TABLES)))
+        return;                                                   // (the same for the whole block)
+    CKKS_POISON_DYNAMIC(tc_sm);
     // ---- set-up (all threads): constants, B tile, zero padding of the A rows, barriers, memory
     for (int i = tid; i < n_in; i += TC_THREADS) half_s[i] = a.pinfo[p0 + i].half;
     for (int u = tid; u < Tc; u += TC_THREADS) {
@@ -185,7 +190,10 @@ __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
         const int kc = idx / N, col = idx - kc * N;
         const int u = col >> 2, c = col & 3;
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (u < Tc) v = a.tb[((size_t)cfg * a.n_primes + prime_of(target_pos(u))) * 16 + c * 4 + kc];
+        if (u < Tc) {
+            const uint4 *e = a.tb + ((size_t)cfg * a.n_primes + prime_of(target_pos(u))) * 16 + c * 4 + kc;
+            if (CKKS_SPAN(e, 1, CKKS_DBG_TC_TABLES)) v = *e;
+        }
         reinterpret_cast<uint4 *>(Bs)[(size_t)kc * N + col] = v;
     }
     if (tid < TC_M)          // words n_in + 1 .. 15 of every row stay zero (the copies never write them)
@@ -210,7 +218,7 @@ __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
     tc_fence_after();
     const u32 tmem = tmem_base;
     auto fail_wait = [&]() {
-        if (!abort_flag) atomicOr(a.err, CKKS_DEV_ERR_WAIT);
+        if (!abort_flag && CKKS_SPAN(a.err, 1, CKKS_DBG_ERR_WORD)) atomicOr(a.err, CKKS_DEV_ERR_WAIT);
         abort_flag = 1;
     };
     auto wait_or_abort = [&](u64 *bar, u32 parity) {              // false: aborted
@@ -242,9 +250,10 @@ __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
             if (k >= TC_STAGES && !wait_or_abort(&a_empty[k % TC_STAGES], (u32)(((k / TC_STAGES) - 1) & 1))) break;
             const u32 *src = yb + (blockIdx.x * tiles + k) * TC_M + row_i;
             unsigned char *row = a_stage(k) + (size_t)row_i * 16;
+            const bool ok_in = CKKS_SPAN2(src, src + (size_t)(n_in - 1) * n, CKKS_DBG_TC_IN);
 #pragma unroll
             for (int i = 0; i < TC_MAX_IN; i++) {
-                if (i < n_in) tc_cp_async4(row + (i >> 2) * (TC_M * 16) + (i & 3) * 4, src);
+                if (i < n_in && ok_in) tc_cp_async4(row + (i >> 2) * (TC_M * 16) + (i & 3) * 4, src);
                 src += n;
             }
             tc_cp_commit();
@@ -276,7 +285,8 @@ __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
                         const uint4 rec = trec[u];
                         const u32 s1 = r[4 * j] + (r[4 * j + 1] << 8);
                         const u32 s2 = r[4 * j + 2] + (r[4 * j + 3] << 8);
-                        ob[rec.w + (u32)nc] = shoup_mul(s2, 65536u, rec.z, rec.x) + csub(s1, rec.y);
+                        if (CKKS_SPAN(ob + rec.w + (u32)nc, 1, CKKS_DBG_TC_OUT))
+                            ob[rec.w + (u32)nc] = shoup_mul(s2, 65536u, rec.z, rec.x) + csub(s1, rec.y);
                     }
                 }
             }

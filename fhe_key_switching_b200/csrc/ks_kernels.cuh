@@ -9,6 +9,7 @@ __global__ void k_chacha_expand(ChachaKey key, u32 key_id, u32 digit, u32 limb,
                                 const PrimeInfo *pinfo, u32 *out, int n) {
     const int b = blockIdx.x * blockDim.x + threadIdx.x;
     if (b >= n / 8) return;
+    if (!CKKS_SPAN(pinfo + limb, 1, CKKS_DBG_NTT_TABLES) || !CKKS_SPAN(out + 8 * b, 8, CKKS_DBG_CHACHA_OUT)) return;
     const PrimeInfo pi = pinfo[limb];
     u32 a[8];
     chacha_coeffs<true>(key, key_id, digit, limb, (u32)b, pi, a);
@@ -66,6 +67,12 @@ k_bconv(BconvArgs a) {
     const int T = a.map.per_group;
     const int row0 = a.in_row0 + g * a.in_group_rows;
     const int p0 = a.in_prime0 + g * a.in_prime_step;
+    if (!CKKS_SPAN(bm, (size_t)n_in * a.n_primes, CKKS_DBG_BCONV_TABLES) ||
+        !CKKS_SPAN(nd, a.n_primes, CKKS_DBG_BCONV_TABLES) || !CKKS_SPAN(a.pinfo + p0, n_in, CKKS_DBG_BCONV_TABLES) ||
+        !CKKS_SPAN(a.pinfo + a.map.lo_base, a.map.split, CKKS_DBG_BCONV_TABLES) ||
+        (T > a.map.split && !CKKS_SPAN(a.pinfo + a.map.hi_base, T - a.map.split, CKKS_DBG_BCONV_TABLES)))
+        return;                                               // (the same for the whole block)
+    CKKS_POISON_DYNAMIC(smb);
     u32 *half = smb + (n_in + 1) * T;
     for (int idx = threadIdx.x; idx < (n_in + 1) * T; idx += blockDim.x) {
         const int i = idx / T, kk = idx - i * T;
@@ -78,10 +85,12 @@ k_bconv(BconvArgs a) {
     if (2 * c2 >= n) return;
     u32 y0[MAXIN], y1[MAXIN];
     u32 v0 = 0, v1 = 0;
+    const bool ok_in = CKKS_SPAN2(yb + (size_t)row0 * n + 2 * c2, yb + (size_t)(row0 + n_in - 1) * n + 2 * c2 + 1,
+                                  CKKS_DBG_BCONV_IN);
 #pragma unroll
     for (int i = 0; i < MAXIN; i++) {
         if (i < n_in) {
-            const uint2 t = reinterpret_cast<const uint2 *>(yb + (size_t)(row0 + i) * n)[c2];
+            const uint2 t = ok_in ? reinterpret_cast<const uint2 *>(yb + (size_t)(row0 + i) * n)[c2] : make_uint2(0u, 0u);
             const u32 h = half[i];
             y0[i] = t.x; y1[i] = t.y;
             v0 += t.x > h ? 1u : 0u;
@@ -91,6 +100,10 @@ k_bconv(BconvArgs a) {
     const int lo = a.map.skip_alpha > 0 ? g * a.map.skip_alpha : 0;
     const int hi = a.map.skip_alpha > 0 ? min(lo + a.map.skip_alpha, a.map.split) : 0;
     const int k_end = min(T, (chunk + 1) * a.tchunk);
+    const bool ok_out = chunk * a.tchunk >= k_end ||
+                        CKKS_SPAN2(ob + ((size_t)g * a.map.out_group_rows + a.map.out_k_base + chunk * a.tchunk) * n + 2 * c2,
+                                   ob + ((size_t)g * a.map.out_group_rows + a.map.out_k_base + k_end - 1) * n + 2 * c2 + 1,
+                                   CKKS_DBG_BCONV_OUT);
     for (int kk = chunk * a.tchunk; kk < k_end; kk++) {
         if (kk >= lo && kk < hi) continue;
         const int t = kk < a.map.split ? a.map.lo_base + kk : a.map.hi_base + (kk - a.map.split);
@@ -111,7 +124,7 @@ k_bconv(BconvArgs a) {
         }
         const uint2 r = make_uint2(reduce64(s0, pi.q, pi.r64, pi.r64p, pi.onep),
                                    reduce64(s1, pi.q, pi.r64, pi.r64p, pi.onep));
-        reinterpret_cast<uint2 *>(ob + ((size_t)g * a.map.out_group_rows + a.map.out_k_base + kk) * n)[c2] = r;
+        if (ok_out) reinterpret_cast<uint2 *>(ob + ((size_t)g * a.map.out_group_rows + a.map.out_k_base + kk) * n)[c2] = r;
     }
 }
 
@@ -144,6 +157,12 @@ k_bconv_n(BconvArgs a) {
     const int T4 = (T + 3) & ~3;
     const int row0 = a.in_row0 + g * a.in_group_rows;
     const int p0 = a.in_prime0 + g * a.in_prime_step;
+    if (!CKKS_SPAN(bm, (size_t)NIN * a.n_primes, CKKS_DBG_BCONV_TABLES) ||
+        !CKKS_SPAN(nd, a.n_primes, CKKS_DBG_BCONV_TABLES) || !CKKS_SPAN(a.pinfo + p0, NIN, CKKS_DBG_BCONV_TABLES) ||
+        !CKKS_SPAN(a.pinfo + a.map.lo_base, a.map.split, CKKS_DBG_BCONV_TABLES) ||
+        (T > a.map.split && !CKKS_SPAN(a.pinfo + a.map.hi_base, T - a.map.split, CKKS_DBG_BCONV_TABLES)))
+        return;                                               // (the same for the whole block)
+    CKKS_POISON_DYNAMIC(smc);
     for (int idx = threadIdx.x; idx < (NIN + 1) * T4; idx += blockDim.x) {
         const int i = idx / T4, kk = idx - i * T4;
         u32 val = 0;
@@ -168,10 +187,12 @@ k_bconv_n(BconvArgs a) {
     if (CPT * cv >= n) return;
     u32 y[CPT][NIN + 1];
     u32 v[CPT] = {0, 0, 0, 0};
+    const bool ok_in = CKKS_SPAN2(yb + (size_t)row0 * n + CPT * cv, yb + (size_t)(row0 + NIN - 1) * n + CPT * cv + CPT - 1,
+                                  CKKS_DBG_BCONV_IN);
 #pragma unroll
     for (int i = 0; i < NIN; i++) {
         const u32 h = a.pinfo[p0 + i].half;
-        const uint4 w = reinterpret_cast<const uint4 *>(yb + (size_t)(row0 + i) * n)[cv];
+        const uint4 w = ok_in ? reinterpret_cast<const uint4 *>(yb + (size_t)(row0 + i) * n)[cv] : make_uint4(0u, 0u, 0u, 0u);
         const u32 t[CPT] = {w.x, w.y, w.z, w.w};
 #pragma unroll
         for (int c = 0; c < CPT; c++) { y[c][i] = t[c]; v[c] += t[c] > h ? 1u : 0u; }
@@ -182,6 +203,11 @@ k_bconv_n(BconvArgs a) {
     const int hi = a.map.skip_alpha > 0 ? min(lo + a.map.skip_alpha, a.map.split) : 0;
     const int k_beg = chunk * a.tchunk;
     const int k_end = min(T, k_beg + a.tchunk);
+    const bool ok_out = k_beg >= k_end ||
+                        CKKS_SPAN2(ob + ((size_t)g * a.map.out_group_rows + a.map.out_k_base + k_beg) * n + CPT * cv,
+                                   ob + ((size_t)g * a.map.out_group_rows + a.map.out_k_base + k_end - 1) * n + CPT * cv +
+                                       CPT - 1,
+                                   CKKS_DBG_BCONV_OUT);
     for (int k4 = k_beg; k4 < k_end; k4 += 4) {
         u64 s[CPT][4];
 #pragma unroll
@@ -206,7 +232,7 @@ k_bconv_n(BconvArgs a) {
 #pragma unroll
             for (int c = 0; c < CPT; c++) r[c] = reduce64_lazy(s[c][m], pq.x, pq.y, pq.z, pq.w);
             u32 *dst = ob + ((size_t)g * a.map.out_group_rows + a.map.out_k_base + kk) * n;
-            reinterpret_cast<uint4 *>(dst)[cv] = make_uint4(r[0], r[1], r[2], r[3]);
+            if (ok_out) reinterpret_cast<uint4 *>(dst)[cv] = make_uint4(r[0], r[1], r[2], r[3]);
         }
     }
 }
@@ -240,6 +266,7 @@ k_inner_product(IpArgs a) {
     const int u = blockIdx.y;
     const int na = a.level + 1;
     const int t = u < na ? u : a.n_q + (u - na);
+    if (!CKKS_SPAN(a.pinfo + t, 1, CKKS_DBG_IP_TABLES)) return;
     const PrimeInfo pi = a.pinfo[t];
     u64 s0[8], s1[8];
 #pragma unroll
@@ -250,21 +277,25 @@ k_inner_product(IpArgs a) {
         const u32 g = in_digit ? (a.hoist_g ? a.hoist_g : a.cdig_g) : a.hoist_g;
         u32 d[8];
         if (g) {
+            const bool ok = CKKS_SPAN(src, n, CKKS_DBG_IP_IN);             // automorph_src < n
 #pragma unroll
-            for (int m = 0; m < 8; m++) d[m] = src[automorph_src((u32)(8 * blk + m), g, a.log_n)];
+            for (int m = 0; m < 8; m++) d[m] = ok ? src[automorph_src((u32)(8 * blk + m), g, a.log_n)] : 0u;
         } else {
             const uint4 *s4 = reinterpret_cast<const uint4 *>(src + 8 * blk);
-            const uint4 p = s4[0], q4 = s4[1];
+            const bool ok = CKKS_SPAN(s4, 2, CKKS_DBG_IP_IN);
+            const uint4 p = ok ? s4[0] : make_uint4(0u, 0u, 0u, 0u), q4 = ok ? s4[1] : make_uint4(0u, 0u, 0u, 0u);
             d[0] = p.x; d[1] = p.y; d[2] = p.z; d[3] = p.w;
             d[4] = q4.x; d[5] = q4.y; d[6] = q4.z; d[7] = q4.w;
         }
         const uint4 *b4 = reinterpret_cast<const uint4 *>(a.b + ((size_t)j * a.n_primes + t) * n + 8 * blk);
-        const uint4 bp = b4[0], bq = b4[1];
+        const bool ok_b = CKKS_SPAN(b4, 2, CKKS_DBG_IP_KEY);
+        const uint4 bp = ok_b ? b4[0] : make_uint4(0u, 0u, 0u, 0u), bq = ok_b ? b4[1] : make_uint4(0u, 0u, 0u, 0u);
         const u32 bb[8] = {bp.x, bp.y, bp.z, bp.w, bq.x, bq.y, bq.z, bq.w};
         u32 av[8];
         if (a.a_stored) {
             const uint4 *a4 = reinterpret_cast<const uint4 *>(a.a_stored + ((size_t)j * a.n_primes + t) * n + 8 * blk);
-            const uint4 ap = a4[0], aq = a4[1];
+            const bool ok_a = CKKS_SPAN(a4, 2, CKKS_DBG_IP_KEY);
+            const uint4 ap = ok_a ? a4[0] : make_uint4(0u, 0u, 0u, 0u), aq = ok_a ? a4[1] : make_uint4(0u, 0u, 0u, 0u);
             av[0] = ap.x; av[1] = ap.y; av[2] = ap.z; av[3] = ap.w;
             av[4] = aq.x; av[5] = aq.y; av[6] = aq.z; av[7] = aq.w;
         } else {
@@ -291,6 +322,7 @@ k_inner_product(IpArgs a) {
     }
     uint4 *o0 = reinterpret_cast<uint4 *>(a.acc + (size_t)u * n + 8 * blk);
     uint4 *o1 = reinterpret_cast<uint4 *>(a.acc + ((size_t)a.ext + u) * n + 8 * blk);
+    if (!CKKS_SPAN(o0, 2, CKKS_DBG_IP_OUT) || !CKKS_SPAN(o1, 2, CKKS_DBG_IP_OUT)) return;
     o0[0] = make_uint4(r0[0], r0[1], r0[2], r0[3]);
     o0[1] = make_uint4(r0[4], r0[5], r0[6], r0[7]);
     o1[0] = make_uint4(r1[0], r1[1], r1[2], r1[3]);
@@ -310,6 +342,10 @@ __global__ void k_tensor(const u32 *x, const u32 *y, u32 *d, const PrimeInfo *pi
     x += blockIdx.z * 2 * pl;
     y += blockIdx.z * 2 * pl;
     d += blockIdx.z * 3 * pl;
+    if (!CKKS_SPAN(pinfo + i, 1, CKKS_DBG_TENSOR) || !CKKS_SPAN2(x + off + 4 * c4, x + pl + off + 4 * c4 + 3, CKKS_DBG_TENSOR) ||
+        !CKKS_SPAN2(y + off + 4 * c4, y + pl + off + 4 * c4 + 3, CKKS_DBG_TENSOR) ||
+        !CKKS_SPAN2(d + off + 4 * c4, d + 2 * pl + off + 4 * c4 + 3, CKKS_DBG_TENSOR))
+        return;
     const uint4 x0 = reinterpret_cast<const uint4 *>(x + off)[c4];
     const uint4 x1 = reinterpret_cast<const uint4 *>(x + pl + off)[c4];
     const uint4 y0 = reinterpret_cast<const uint4 *>(y + off)[c4];
@@ -334,6 +370,7 @@ __global__ void k_automorph(const u32 *in, u32 *out, int log_n, u32 g) {
     const int k = blockIdx.x * blockDim.x + threadIdx.x;
     if (k >= n) return;
     const size_t off = (size_t)blockIdx.y * n;
+    if (!CKKS_SPAN(in + off, n, CKKS_DBG_AUTOMORPH) || !CKKS_SPAN(out + off + k, 1, CKKS_DBG_AUTOMORPH)) return;
     out[off + k] = in[off + automorph_src((u32)k, g, log_n)];
 }
 
@@ -346,6 +383,9 @@ __global__ void k_encode_rns(const long long *m, u32 *out, const PrimeInfo *pinf
     int prime, kk;
     size_t in_row, out_row;
     if (!map_job(map, blockIdx.y, prime, in_row, out_row, kk)) return;
+    if (!CKKS_SPAN(pinfo + prime, 1, CKKS_DBG_ENCODE) || !CKKS_SPAN(m + k, 1, CKKS_DBG_ENCODE) ||
+        !CKKS_SPAN(out + out_row * n + k, 1, CKKS_DBG_ENCODE))
+        return;
     const long long q = pinfo[prime].q;
     long long r = m[k] % q;
     if (r < 0) r += q;
@@ -359,6 +399,9 @@ __global__ void k_copy_digit_limbs(const u32 *c, u32 *dt, int log_n, int level, 
     if (c4 >= n / 4) return;
     const int u = blockIdx.y;            // 0..level
     const int j = u / alpha;
+    if (!CKKS_SPAN(c + (size_t)u * n + 4 * c4, 4, CKKS_DBG_COPY_DIGIT) ||
+        !CKKS_SPAN(dt + ((size_t)j * ext + u) * n + 4 * c4, 4, CKKS_DBG_COPY_DIGIT))
+        return;
     reinterpret_cast<uint4 *>(dt + ((size_t)j * ext + u) * n)[c4] =
         reinterpret_cast<const uint4 *>(c + (size_t)u * n)[c4];
 }
@@ -381,6 +424,27 @@ __device__ __forceinline__ void store16_vec(u32 *p, const u32 (&x)[16]) {
     uint4 *p4 = reinterpret_cast<uint4 *>(p);
 #pragma unroll
     for (int v = 0; v < 4; v++) p4[v] = make_uint4(x[4 * v], x[4 * v + 1], x[4 * v + 2], x[4 * v + 3]);
+}
+
+// the same behind the debug-bounds check of the 16 words (zeros / nothing when it fails)
+__device__ __forceinline__ void load16_chk(const u32 *p, u32 (&x)[16], int site) {
+    if (CKKS_SPAN(p, 16, site)) {
+        load16_vec(p, x);
+    } else {
+#pragma unroll
+        for (int v = 0; v < 16; v++) x[v] = 0u;
+    }
+}
+
+__device__ __forceinline__ void store16_chk(u32 *p, const u32 (&x)[16], int site) {
+    if (CKKS_SPAN(p, 16, site)) store16_vec(p, x);
+}
+
+// x[v] = row[lo + 16 v], the round-0 input of a row pass, behind the check of its span
+__device__ __forceinline__ void load_row16_chk(const u32 *row, int lo, u32 (&x)[16], int site) {
+    const bool ok = CKKS_SPAN2(row + lo, row + lo + 16 * 15, site);
+#pragma unroll
+    for (int v = 0; v < 16; v++) x[v] = ok ? row[lo + 16 * v] : 0u;
 }
 
 // Forward row pass of one row held as round-0 input x[v] = row element lo + 16 v; returns the
@@ -460,6 +524,10 @@ k_ip_row(IpRowArgs a) {
     const int u = blockIdx.y;
     const int g0 = a.grp_first[blockIdx.z], gcnt = a.grp_count[blockIdx.z];
     const int t = u < na ? u : a.n_q + (u - na);
+    if (!CKKS_SPAN(a.pinfo + t, 1, CKKS_DBG_IPROW_TABLES) || !CKKS_SPAN(a.twf + (size_t)t * n, n, CKKS_DBG_IPROW_TABLES))
+        return;                                               // (the same for the whole block)
+    CKKS_POISON(sm, sizeof(sm));
+    CKKS_POISON_DYNAMIC(sa);
     const PrimeInfo pi = a.pinfo[t];
     const u32 q = pi.q, two_q = 2 * q;
     const int r = threadIdx.x >> 4, lo = threadIdx.x & 15;
@@ -502,15 +570,15 @@ k_ip_row(IpRowArgs a) {
                 const u32 *src = cdb + (size_t)u * n;
                 const u32 g = hoist_g ? hoist_g : cdig_g;
                 if (g) {
+                    const bool ok = CKKS_SPAN(src, n, CKKS_DBG_IPROW_CDIG);       // automorph_src < n
 #pragma unroll
-                    for (int v = 0; v < 16; v++) x[v] = src[automorph_src((u32)(k0 + v), g, a.log_n)];
+                    for (int v = 0; v < 16; v++) x[v] = ok ? src[automorph_src((u32)(k0 + v), g, a.log_n)] : 0u;
                 } else {
-                    load16_vec(src + k0, x);
+                    load16_chk(src + k0, x, CKKS_DBG_IPROW_CDIG);
                 }
             } else {
                 const u32 *src = xb + ((size_t)j * a.ext + u) * n + (size_t)src_row * 256;
-#pragma unroll
-                for (int v = 0; v < 16; v++) x[v] = src[lo + 16 * v];
+                load_row16_chk(src, lo, x, CKKS_DBG_IPROW_X);
                 row_fwd_regs(x, twf, R1 + (u32)src_row, lo, srow, q);
                 if (hoist_g) {        // permute inside the row: slot k takes source slot src(k)
 #pragma unroll
@@ -525,13 +593,13 @@ k_ip_row(IpRowArgs a) {
                 }
             }
             u32 bv[16], av[16];
-            load16_vec(bkey + ((size_t)j * a.n_primes + t) * n + k0, bv);
+            load16_chk(bkey + ((size_t)j * a.n_primes + t) * n + k0, bv, CKKS_DBG_IPROW_KEY);
             if (gcnt > 1) {
                 const u32 *src = sa + (size_t)j * 16 * ROW_THREADS + threadIdx.x;
 #pragma unroll
                 for (int v = 0; v < 16; v++) av[v] = src[v * ROW_THREADS];
             } else if (astore) {
-                load16_vec(astore + ((size_t)j * a.n_primes + t) * n + k0, av);
+                load16_chk(astore + ((size_t)j * a.n_primes + t) * n + k0, av, CKKS_DBG_IPROW_KEY);
             } else {
                 u32 h[8];
                 chacha_coeffs<false>(a.key[item], a.key_id[item], (u32)j, (u32)t, (u32)(k0 >> 3), pi, h);
@@ -553,8 +621,8 @@ k_ip_row(IpRowArgs a) {
             acc0[v] = csub(shoup_mul(acc0[v], pi.r64, pi.r64p, q), q);
             acc1[v] = csub(shoup_mul(acc1[v], pi.r64, pi.r64p, q), q);
         }
-        store16_vec(accb + (size_t)u * n + (size_t)row * 256 + 16 * lo, acc0);
-        store16_vec(accb + ((size_t)a.ext + u) * n + (size_t)row * 256 + 16 * lo, acc1);
+        store16_chk(accb + (size_t)u * n + (size_t)row * 256 + 16 * lo, acc0, CKKS_DBG_IPROW_OUT);
+        store16_chk(accb + ((size_t)a.ext + u) * n + (size_t)row * 256 + 16 * lo, acc1, CKKS_DBG_IPROW_OUT);
     }
 }
 
@@ -583,6 +651,10 @@ k_row_combine(RowCombineArgs a) {
     const int i = blockIdx.y, comp = blockIdx.z % a.n_comp, item = blockIdx.z / a.n_comp;
     const u32 add_g = a.add_g[item];
     const int na = a.level + 1;
+    if (!CKKS_SPAN(a.pinfo + i, 1, CKKS_DBG_COMBINE_TABLES) || !CKKS_SPAN(a.pinv + i, 1, CKKS_DBG_COMBINE_TABLES) ||
+        !CKKS_SPAN(a.twf + (size_t)i * n, n, CKKS_DBG_COMBINE_TABLES))
+        return;                                               // (the same for the whole block)
+    CKKS_POISON(sm, sizeof(sm));
     const PrimeInfo pi = a.pinfo[i];
     const u32 q = pi.q;
     const int r = threadIdx.x >> 4, lo = threadIdx.x & 15;
@@ -591,11 +663,10 @@ k_row_combine(RowCombineArgs a) {
     u32 *srow = sm + r * 272;
     u32 x[16];
     const u32 *src = a.conv + item * a.conv_item + ((size_t)comp * na + i) * n + (size_t)row * 256;
-#pragma unroll
-    for (int v = 0; v < 16; v++) x[v] = src[lo + 16 * v];
+    load_row16_chk(src, lo, x, CKKS_DBG_COMBINE_IN);
     row_fwd_regs(x, a.twf + (size_t)i * n, (u32)(n >> 8) + (u32)row, lo, srow, q);
     u32 ac[16];
-    load16_vec(a.acc + item * a.acc_item + ((size_t)comp * a.acc_comp_rows + i) * n + k0, ac);
+    load16_chk(a.acc + item * a.acc_item + ((size_t)comp * a.acc_comp_rows + i) * n + k0, ac, CKKS_DBG_COMBINE_IN);
     const tw_t w = a.pinv[i];
 #pragma unroll
     for (int v = 0; v < 16; v++) x[v] = csub(shoup_mul(ac[v] + q - x[v], w.x, w.y, q), q);
@@ -603,15 +674,16 @@ k_row_combine(RowCombineArgs a) {
         const u32 *ad = a.add + item * a.add_item + ((size_t)comp * na + i) * n;
         u32 y[16];
         if (add_g) {
+            const bool ok = CKKS_SPAN(ad, n, CKKS_DBG_COMBINE_ADD);          // automorph_src < n
 #pragma unroll
-            for (int v = 0; v < 16; v++) y[v] = ad[automorph_src((u32)(k0 + v), add_g, a.log_n)];
+            for (int v = 0; v < 16; v++) y[v] = ok ? ad[automorph_src((u32)(k0 + v), add_g, a.log_n)] : 0u;
         } else {
-            load16_vec(ad + k0, y);
+            load16_chk(ad + k0, y, CKKS_DBG_COMBINE_ADD);
         }
 #pragma unroll
         for (int v = 0; v < 16; v++) x[v] = csub(x[v] + y[v], q);
     }
-    store16_vec(a.out + item * a.out_item + ((size_t)comp * na + i) * n + k0, x);
+    store16_chk(a.out + item * a.out_item + ((size_t)comp * na + i) * n + k0, x, CKKS_DBG_COMBINE_OUT);
 }
 
 // ---------------------------------------------------------------- baby-step giant-step transform
@@ -701,7 +773,7 @@ __global__ void k_wait_expiry_probe(int *err) {
     }
     __syncthreads();
     const bool expired = !mbar_wait_bounded(&bar, 0u);
-    if (threadIdx.x == 0 && expired) atomicOr(err, CKKS_DEV_ERR_WAIT);
+    if (threadIdx.x == 0 && expired && CKKS_SPAN(err, 1, CKKS_DBG_ERR_WORD)) atomicOr(err, CKKS_DEV_ERR_WAIT);
 }
 
 // The plaintexts stream through shared memory: a block covers 512 coefficients (2 per thread)
@@ -722,6 +794,9 @@ k_bsgs_combine(BsgsArgs a) {
     const int u = blockIdx.y;
     const int na = a.level + 1;
     const int t = u < na ? u : a.n_q + (u - na);
+    if (!CKKS_SPAN(a.pinfo + t, 1, CKKS_DBG_BSGS_TABLES) || (u < na && !CKKS_SPAN(a.pmod + u, 1, CKKS_DBG_BSGS_TABLES)))
+        return;                                               // (the same for the whole block)
+    CKKS_POISON_DYNAMIC(sp);
     const PrimeInfo pi = a.pinfo[t];
     const u32 q = pi.q;
     const tw_t pm = u < na ? a.pmod[u] : make_uint2(0u, 0u);
@@ -737,11 +812,27 @@ k_bsgs_combine(BsgsArgs a) {
     // thread 0: giant step j's plaintext chunks into stage j % BSGS_STAGES
     auto issue = [&](int j) {
         const int st = j % BSGS_STAGES;
-        mbar_expect_tx(&full[st], stage_bytes);
         const u32 *src = pbase + (size_t)j * a.n_baby * plane;
+#ifdef CKKS_DEBUG_BOUNDS
+        // a chunk outside the registered regions is not copied, and the stage expects its bytes less
+        u32 okm = 0, bytes = 0;
+        (void)stage_bytes;
+        for (int kk = 0; kk < a.kc; kk++)
+            if (CKKS_SPAN(src + (size_t)kk * plane, BSGS_CHUNK, CKKS_DBG_BSGS_PT)) {
+                okm |= 1u << kk;
+                bytes += BSGS_CHUNK * sizeof(u32);
+            }
+        mbar_expect_tx(&full[st], bytes);
+        for (int kk = 0; kk < a.kc; kk++)
+            if ((okm >> kk) & 1u)
+                bulk_load(sp + ((size_t)st * BSGS_KC + kk) * BSGS_CHUNK, src + (size_t)kk * plane,
+                          BSGS_CHUNK * sizeof(u32), &full[st]);
+#else
+        mbar_expect_tx(&full[st], stage_bytes);
         for (int kk = 0; kk < a.kc; kk++)
             bulk_load(sp + ((size_t)st * BSGS_KC + kk) * BSGS_CHUNK, src + (size_t)kk * plane,
                       BSGS_CHUNK * sizeof(u32), &full[st]);
+#endif
     };
     if (tid == 0)
         for (int j = 0; j < BSGS_STAGES && j < a.n_giant; j++) issue(j);
@@ -754,7 +845,8 @@ k_bsgs_combine(BsgsArgs a) {
             const int k = a.k0 + kk;
             const int z = a.item_of[k];
             if (z < 0) {
-                if (u < na) {
+                if (u < na && CKKS_SPAN2(a.ct + (size_t)u * n + 2 * c2, a.ct + ((size_t)na + u) * n + 2 * c2 + 1,
+                                         CKKS_DBG_BSGS_IN)) {
                     const uint2 v0 = reinterpret_cast<const uint2 *>(a.ct + (size_t)u * n)[c2];
                     const uint2 v1 = reinterpret_cast<const uint2 *>(a.ct + ((size_t)na + u) * n)[c2];
                     x0[kk][0] = csub(shoup_mul(v0.x, pm.x, pm.y, q), q);
@@ -764,10 +856,11 @@ k_bsgs_combine(BsgsArgs a) {
                 }
             } else {
                 const u32 *ac = a.acc + (size_t)z * a.acc_item;
-                const uint2 v0 = reinterpret_cast<const uint2 *>(ac + r0)[c2];
-                const uint2 v1 = reinterpret_cast<const uint2 *>(ac + r1)[c2];
+                const bool ok = CKKS_SPAN2(ac + r0 + 2 * c2, ac + r1 + 2 * c2 + 1, CKKS_DBG_BSGS_IN);
+                const uint2 v0 = ok ? reinterpret_cast<const uint2 *>(ac + r0)[c2] : make_uint2(0u, 0u);
+                const uint2 v1 = ok ? reinterpret_cast<const uint2 *>(ac + r1)[c2] : make_uint2(0u, 0u);
                 u32 e0 = v0.x, e1 = v0.y;
-                if (u < na) {
+                if (u < na && CKKS_SPAN(a.ct + (size_t)u * n, n, CKKS_DBG_BSGS_IN)) {     // automorph_src < n
                     const u32 *c0 = a.ct + (size_t)u * n;
                     const u32 g = a.galois[k];
                     e0 = csub(e0 + csub(shoup_mul(c0[automorph_src((u32)(2 * c2), g, a.log_n)], pm.x, pm.y, q), q), q);
@@ -784,16 +877,17 @@ k_bsgs_combine(BsgsArgs a) {
         if (__syncthreads_or(expired)) {
             // leave together: record the failure, let this block's copies in flight land
             if (tid == 0) {
-                atomicOr(a.err, CKKS_DEV_ERR_WAIT);
+                if (CKKS_SPAN(a.err, 1, CKKS_DBG_ERR_WORD)) atomicOr(a.err, CKKS_DEV_ERR_WAIT);
                 for (int jj = j; jj < j + BSGS_STAGES && jj < a.n_giant; jj++)
                     (void)mbar_wait_bounded(&full[jj % BSGS_STAGES], (u32)(jj / BSGS_STAGES) & 1u);
             }
             return;
         }
         u32 *vj = a.v + (size_t)j * a.v_item;
+        const bool ok_v = CKKS_SPAN2(vj + r0 + 2 * c2, vj + r1 + 2 * c2 + 1, CKKS_DBG_BSGS_V);
         // a canonical carry plus 16 products of two values below q < 2^30 stays below 2^64
         u64 s00 = 0, s01 = 0, s10 = 0, s11 = 0;              // [component][coefficient]
-        if (a.k0) {
+        if (a.k0 && ok_v) {
             const uint2 w0 = reinterpret_cast<const uint2 *>(vj + r0)[c2];
             const uint2 w1 = reinterpret_cast<const uint2 *>(vj + r1)[c2];
             s00 = w0.x; s01 = w0.y; s10 = w1.x; s11 = w1.y;
@@ -807,10 +901,12 @@ k_bsgs_combine(BsgsArgs a) {
                 s10 += (u64)p.x * x1[kk][0]; s11 += (u64)p.y * x1[kk][1];
             }
         }
-        reinterpret_cast<uint2 *>(vj + r0)[c2] =
-            make_uint2(reduce64(s00, q, pi.r64, pi.r64p, pi.onep), reduce64(s01, q, pi.r64, pi.r64p, pi.onep));
-        reinterpret_cast<uint2 *>(vj + r1)[c2] =
-            make_uint2(reduce64(s10, q, pi.r64, pi.r64p, pi.onep), reduce64(s11, q, pi.r64, pi.r64p, pi.onep));
+        if (ok_v) {
+            reinterpret_cast<uint2 *>(vj + r0)[c2] =
+                make_uint2(reduce64(s00, q, pi.r64, pi.r64p, pi.onep), reduce64(s01, q, pi.r64, pi.r64p, pi.onep));
+            reinterpret_cast<uint2 *>(vj + r1)[c2] =
+                make_uint2(reduce64(s10, q, pi.r64, pi.r64p, pi.onep), reduce64(s11, q, pi.r64, pi.r64p, pi.onep));
+        }
         __syncthreads();                                     // stage st fully read
         if (tid == 0 && j + BSGS_STAGES < a.n_giant) issue(j + BSGS_STAGES);
     }
@@ -832,9 +928,13 @@ k_sum_parts(SumArgs a) {
     const int c4 = blockIdx.x * blockDim.x + threadIdx.x;
     if (4 * c4 >= n) return;
     const int r = blockIdx.y;
+    if (!CKKS_SPAN(a.pinfo + r % (a.level + 1), 1, CKKS_DBG_SUM) ||
+        !CKKS_SPAN(a.out + (size_t)r * n + 4 * c4, 4, CKKS_DBG_SUM))
+        return;
     const u32 q = a.pinfo[r % (a.level + 1)].q;
     uint4 s = make_uint4(0u, 0u, 0u, 0u);
     for (int i = 0; i < a.n_src; i++) {
+        if (!CKKS_SPAN(a.src[i] + (size_t)r * n + 4 * c4, 4, CKKS_DBG_SUM)) continue;
         const uint4 v = reinterpret_cast<const uint4 *>(a.src[i] + (size_t)r * n)[c4];
         s.x = csub(s.x + v.x, q); s.y = csub(s.y + v.y, q); s.z = csub(s.z + v.z, q); s.w = csub(s.w + v.w, q);
     }

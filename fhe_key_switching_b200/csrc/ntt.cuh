@@ -18,6 +18,7 @@
 // The inverse passes undo the forward stages in reverse order with Gentleman-Sande
 // butterflies and the psi^-brv(idx) table.
 #pragma once
+#include "debug_bounds.cuh"
 #include "modarith.cuh"
 
 // Twiddle record: (w, Shoup companion of w).
@@ -168,6 +169,11 @@ k_ntt_col(NttArgs a) {
     size_t in_row, out_row;
     if (!map_job(a.map, blockIdx.y, prime, in_row, out_row, k)) return;
     const int n = 1 << a.log_n;
+    if (!CKKS_SPAN(a.pinfo + prime, 1, CKKS_DBG_NTT_TABLES) ||
+        !CKKS_SPAN(a.tw + (size_t)prime * n, n, CKKS_DBG_NTT_TABLES) ||
+        (!FWD && a.scale && !CKKS_SPAN(a.scale + k, 1, CKKS_DBG_NTT_TABLES)))
+        return;                                               // (the same for the whole block)
+    CKKS_POISON(sm, sizeof(sm));
     const PrimeInfo pi = a.pinfo[prime];
     const u32 q = pi.q, two_q = 2 * q;
     const tw_t *tw = a.tw + (size_t)prime * n;
@@ -180,8 +186,10 @@ k_ntt_col(NttArgs a) {
     u32 *dst = a.out + blockIdx.z * a.out_item + out_row * n;
     u32 x[16];
     if (FWD) {
+        const bool ok_in = CKKS_SPAN2(src + (size_t)lo * 256 + col, src + (size_t)(lo + C::LOS * 15) * 256 + col,
+                                      CKKS_DBG_NTT_IN);
 #pragma unroll
-        for (int u = 0; u < 16; u++) x[u] = src[(size_t)(lo + C::LOS * u) * 256 + col];
+        for (int u = 0; u < 16; u++) x[u] = ok_in ? src[(size_t)(lo + C::LOS * u) * 256 + col] : 0u;
         if (a.lift_q) {
             // y - lift_q + 2q lies in (2q - lift_q/2, 2q), inside the butterflies' [0, 4q) input
 #pragma unroll
@@ -194,11 +202,15 @@ k_ntt_col(NttArgs a) {
 #pragma unroll
         for (int u = 0; u < 16; u++) x[u] = sm[(16 * lo + u) * C::CPB + ccol];
         fwd_low<R1LOG>(x, tw, 1u, (u32)lo, q, two_q);
+        if (CKKS_SPAN2(dst + (size_t)(16 * lo) * 256 + col, dst + (size_t)(16 * lo + 15) * 256 + col, CKKS_DBG_NTT_OUT)) {
 #pragma unroll
-        for (int u = 0; u < 16; u++) dst[(size_t)(16 * lo + u) * 256 + col] = x[u];
+            for (int u = 0; u < 16; u++) dst[(size_t)(16 * lo + u) * 256 + col] = x[u];
+        }
     } else {
+        const bool ok_in = CKKS_SPAN2(src + (size_t)(16 * lo) * 256 + col, src + (size_t)(16 * lo + 15) * 256 + col,
+                                      CKKS_DBG_NTT_IN);
 #pragma unroll
-        for (int u = 0; u < 16; u++) x[u] = src[(size_t)(16 * lo + u) * 256 + col];
+        for (int u = 0; u < 16; u++) x[u] = ok_in ? src[(size_t)(16 * lo + u) * 256 + col] : 0u;
         inv_low<R1LOG>(x, tw, 1u, (u32)lo, q, two_q);
 #pragma unroll
         for (int u = 0; u < 16; u++) sm[(16 * lo + u) * C::CPB + ccol] = x[u];
@@ -208,9 +220,11 @@ k_ntt_col(NttArgs a) {
         inv_top4(x, tw, 1u, q, two_q);
         u32 w = pi.n_inv, wp = pi.n_invp;
         if (a.scale) { const tw_t s = a.scale[k]; w = s.x; wp = s.y; }
+        if (CKKS_SPAN2(dst + (size_t)lo * 256 + col, dst + (size_t)(lo + C::LOS * 15) * 256 + col, CKKS_DBG_NTT_OUT)) {
 #pragma unroll
-        for (int u = 0; u < 16; u++)
-            dst[(size_t)(lo + C::LOS * u) * 256 + col] = csub(shoup_mul(x[u], w, wp, q), q);
+            for (int u = 0; u < 16; u++)
+                dst[(size_t)(lo + C::LOS * u) * 256 + col] = csub(shoup_mul(x[u], w, wp, q), q);
+        }
     }
 }
 
@@ -230,6 +244,9 @@ k_ntt_row(NttArgs a) {
     size_t in_row, out_row;
     if (!map_job(a.map, blockIdx.y, prime, in_row, out_row, k)) return;
     const int n = 1 << a.log_n;
+    if (!CKKS_SPAN(a.pinfo + prime, 1, CKKS_DBG_NTT_TABLES) || !CKKS_SPAN(a.tw + (size_t)prime * n, n, CKKS_DBG_NTT_TABLES))
+        return;                                               // (the same for the whole block)
+    CKKS_POISON(sm, sizeof(sm));
     const PrimeInfo pi = a.pinfo[prime];
     const u32 q = pi.q, two_q = 2 * q;
     const tw_t *tw = a.tw + (size_t)prime * n;
@@ -243,8 +260,9 @@ k_ntt_row(NttArgs a) {
     u32 x[16];
     if (FWD) {
         const u32 *s = src + (size_t)row * 256;
+        const bool ok_in = CKKS_SPAN2(s + lo, s + lo + 16 * 15, CKKS_DBG_NTT_IN);
 #pragma unroll
-        for (int u = 0; u < 16; u++) x[u] = s[lo + 16 * u];
+        for (int u = 0; u < 16; u++) x[u] = ok_in ? s[lo + 16 * u] : 0u;
         fwd_top4(x, tw, base, q, two_q);
 #pragma unroll
         for (int u = 0; u < 16; u++) srow[lo + 17 * u] = x[u];
@@ -252,6 +270,7 @@ k_ntt_row(NttArgs a) {
 #pragma unroll
         for (int u = 0; u < 16; u++) x[u] = srow[17 * lo + u];
         fwd_low<8>(x, tw, base, (u32)lo, q, two_q);
+        const bool ok_out = CKKS_SPAN(dst + 16 * lo, 16, CKKS_DBG_NTT_OUT);
 #pragma unroll
         for (int v = 0; v < 4; v++) {
             uint4 o;
@@ -259,18 +278,20 @@ k_ntt_row(NttArgs a) {
             o.y = csub(csub(x[4 * v + 1], two_q), q);
             o.z = csub(csub(x[4 * v + 2], two_q), q);
             o.w = csub(csub(x[4 * v + 3], two_q), q);
-            reinterpret_cast<uint4 *>(dst + 16 * lo)[v] = o;
+            if (ok_out) reinterpret_cast<uint4 *>(dst + 16 * lo)[v] = o;
         }
     } else {
         if (galois) {
+            const bool ok_in = CKKS_SPAN(src, n, CKKS_DBG_NTT_IN);          // automorph_src < n
 #pragma unroll
             for (int u = 0; u < 16; u++)
-                x[u] = src[automorph_src((u32)(row * 256 + 16 * lo + u), galois, a.log_n)];
+                x[u] = ok_in ? src[automorph_src((u32)(row * 256 + 16 * lo + u), galois, a.log_n)] : 0u;
         } else {
             const uint4 *s4 = reinterpret_cast<const uint4 *>(src + (size_t)row * 256 + 16 * lo);
+            const bool ok_in = CKKS_SPAN(s4, 4, CKKS_DBG_NTT_IN);
 #pragma unroll
             for (int v = 0; v < 4; v++) {
-                const uint4 t = s4[v];
+                const uint4 t = ok_in ? s4[v] : make_uint4(0u, 0u, 0u, 0u);
                 x[4 * v] = t.x; x[4 * v + 1] = t.y; x[4 * v + 2] = t.z; x[4 * v + 3] = t.w;
             }
         }
@@ -281,7 +302,9 @@ k_ntt_row(NttArgs a) {
 #pragma unroll
         for (int u = 0; u < 16; u++) x[u] = srow[lo + 17 * u];
         inv_top4(x, tw, base, q, two_q);
+        if (CKKS_SPAN2(dst + lo, dst + lo + 16 * 15, CKKS_DBG_NTT_OUT)) {
 #pragma unroll
-        for (int u = 0; u < 16; u++) dst[lo + 16 * u] = x[u];
+            for (int u = 0; u < 16; u++) dst[lo + 16 * u] = x[u];
+        }
     }
 }

@@ -56,7 +56,8 @@ enum {
     CKKS_ERR_ALIGN = -3,        /* a device pointer is not 16-byte aligned */
     CKKS_ERR_WORKSPACE = -4,    /* workspace smaller than ckks_workspace_bytes() */
     CKKS_ERR_CUDA = -5,         /* a CUDA call or kernel launch failed */
-    CKKS_ERR_TIMEOUT = -6       /* ckks_sync_status: stream still busy at the deadline */
+    CKKS_ERR_TIMEOUT = -6,      /* ckks_sync_status: stream still busy at the deadline */
+    CKKS_ERR_BOUNDS = -7        /* ckks_sync_status, debug-bounds build only: an index check failed */
 };
 
 typedef struct ckks_ctx ckks_ctx; /* opaque; owns read-only device tables only */
@@ -325,7 +326,8 @@ size_t ckks_workspace_bytes(const ckks_ctx *ctx, int level, int n);
  * context's device error word: kernels whose waits are bounded (the shared-memory pipeline of
  * ckks_bsgs) record an expired wait there and return early, and ckks_sync_status reports it as
  * CKKS_ERR_TIMEOUT; the results of the calls since the previous check are then invalid, and the
- * context stays usable. */
+ * context stays usable.  In the debug-bounds build it last reads (and clears) the index-check
+ * record and returns CKKS_ERR_BOUNDS when a check failed since the previous clear. */
 int ckks_sync_status(ckks_ctx *ctx, ckks_stream_t stream, int timeout_ms);
 
 /* Self-test of the failure path of bounded device waits (no counterpart in the pages):
@@ -334,6 +336,33 @@ int ckks_sync_status(ckks_ctx *ctx, ckks_stream_t stream, int timeout_ms);
  * ckks_sync_status on `stream` returns CKKS_ERR_TIMEOUT and clears it, and the context stays
  * usable.  Nothing faults or hangs. */
 int ckks_selftest_wait_expiry(ckks_ctx *ctx, ckks_stream_t stream);
+
+/* Debug-bounds build (a checking aid; the pages have no counterpart).  The same sources compiled
+ * with -DCKKS_DEBUG_BOUNDS (`python fhe_key_switching_b200/build.py --debug` writes
+ * libckks_ks_debug.so beside the release library) give every kernel index checks: before each
+ * group of global-memory accesses it checks that the group's span lies inside one region of the
+ * running call -- the caller's buffers, sized from the call's arguments as this header states
+ * (a workspace by the ws_bytes passed), the keys ([D][n_q+n_p][N] words per half), and the
+ * context's device tables.  A failed check is counted in a device record that keeps the first
+ * failure's site, address and size, and the accesses of that group are skipped (loads read 0), so
+ * a wrong index is reported and no memory outside the call's buffers is touched.  Shared memory is
+ * filled with a poison word at the start of each kernel that stages data in it, so that a read of
+ * a word never written gives a wrong result.  The region table is global per device: use the
+ * debug build with one stream at a time.  The release build has no checks and the same
+ * results; the integer-throughput probe is not instrumented.
+ *   ckks_debug_bounds_enabled: 1 in the debug-bounds build, 0 otherwise.
+ *   ckks_debug_bounds_report: waits for the current device, then stores the number of failed
+ *     checks since the last clear and the first failure's site (see ckks_debug_bounds_site_name),
+ *     address and size (each pointer but count may be NULL); clear != 0 empties the record.
+ *     CKKS_ERR_UNSUPPORTED in the release build.
+ *   ckks_debug_bounds_site_name: the name of a check site ("unknown" outside the list).
+ *   ckks_selftest_bounds: enqueues on `stream` one check of the 4 bytes after the context's
+ *     device error word (a region of its own), which fails and is recorded at site "selftest";
+ *     nothing is read or written.  CKKS_ERR_UNSUPPORTED in the release build. */
+int ckks_debug_bounds_enabled(void);
+int ckks_debug_bounds_report(uint64_t *count, int *site, uint64_t *addr, uint64_t *bytes, int clear);
+const char *ckks_debug_bounds_site_name(int site);
+int ckks_selftest_bounds(ckks_ctx *ctx, ckks_stream_t stream);
 
 /* Kernel timing.  Between ckks_prof_begin and ckks_prof_end, every launch of the kernel named
  * `kernel` ("ip_row", "bconv", "ntt_col_fwd", "ntt_col_inv", "ntt_row_fwd", "ntt_row_inv",

@@ -24,6 +24,26 @@ def test_header_symbols_exported(ks_lib):
     assert set(names) == set(ks_lib.EXPORTED)
 
 
+def test_debug_build_exports_the_same_symbols(ks_lib):
+    """The debug-bounds build exports the header's entry points too and says which build it is;
+    neither question needs a GPU."""
+    from conftest import build_library
+    lib = ctypes.CDLL(build_library(debug=True))
+    for name in _declared():
+        assert hasattr(lib, name), name
+    rel = ctypes.CDLL(os.path.join(os.path.dirname(ks_lib.LIB_PATH), "libckks_ks.so"))
+    assert lib.ckks_debug_bounds_enabled() == 1 and rel.ckks_debug_bounds_enabled() == 0
+    for l in (lib, rel):
+        l.ckks_debug_bounds_site_name.restype = ctypes.c_char_p
+        assert l.ckks_debug_bounds_site_name(1) == b"selftest"
+        assert l.ckks_debug_bounds_site_name(10 ** 6) == b"unknown"
+    count = ctypes.c_uint64()
+    rel.ckks_debug_bounds_report.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int]
+    assert rel.ckks_debug_bounds_report(ctypes.byref(count), None, None, None, 1) == ks_lib.CKKS_ERR_UNSUPPORTED
+    lib.ckks_debug_bounds_report.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int]
+    assert lib.ckks_debug_bounds_report(None, None, None, None, 1) == ks_lib.CKKS_ERR_ARG
+
+
 @pytest.mark.parametrize("log_n,n_q,n_p", [(12, 4, 1), (14, 12, 4), (16, 36, 12), (13, 3, 2), (15, 5, 5)])
 def test_gen_primes_matches_oracle(ks_lib, oracle_mod, log_n, n_q, n_p):
     q, p = ks_lib.ckks_gen_primes(log_n, n_q, n_p)
