@@ -591,7 +591,7 @@ def roofline(cfg, launches, total_ms, clk, batch, single_step_ms, launches_ov, t
 # DRAM bytes (read + write) per unit of a k_ip_row launch from an ncu capture, valid only for the
 # kernel sources it was taken on (sha-256 prefix of the device-code headers): after any change to
 # them the figure is reported as null until a new capture replaces it.
-IP_ROW_TRAFFIC = {"sources_sha16": "cab75b06f246685b", "bytes_per_unit": (473.90e6 + 471.65e6) / 2 / 4,
+IP_ROW_TRAFFIC = {"sources_sha16": "4c48c3054b3353e0", "bytes_per_unit": (477.75e6 + 472.51e6) / 2 / 4,
                   "capture": "profiles/k_ip_row_n16_full.md (dram__bytes read + write of two 4-unit launches)"}
 KERNEL_HEADERS = ("debug_bounds.cuh", "modarith.cuh", "chacha.cuh", "ntt.cuh", "ks_kernels.cuh")
 
@@ -1048,12 +1048,14 @@ def info_cpu_baseline(key: str, max_seconds: float = 8.0):
 BCONV_ENGINES = {"cuda": "CUDA cores (32x32->64-bit multiply-adds)",
                  "tensor": "tensor cores (8-bit split, tcgen05.mma kind::i8)",
                  "auto": "automatic: tensor cores (8-bit split, tcgen05.mma kind::i8) for launches of at least "
-                         "4 tiles per block, CUDA cores below"}
+                         "4 tiles per block, CUDA cores below",
+                 "fused": "tensor cores (8-bit split, tcgen05.mma kind::i8) fused with the first forward NTT "
+                          "pass of the converted limbs"}
 
 
 def set_bconv(ks, ctx, args):
     ks.ckks_set_bconv_mode(ctx, {"tensor": ks.CKKS_BCONV_TENSOR, "cuda": ks.CKKS_BCONV_CUDA_CORES,
-                                 "auto": ks.CKKS_BCONV_AUTO}[args.bconv])
+                                 "auto": ks.CKKS_BCONV_AUTO, "fused": ks.CKKS_BCONV_FUSED}[args.bconv])
 
 
 def run_int_peaks(local_rank):
@@ -1194,7 +1196,8 @@ def main():
                          "batches; at 2 streams x 4 units the other stream already hides launch gaps)")
     ap.add_argument("--bconv", default="auto", choices=sorted(BCONV_ENGINES),
                     help="base-conversion engine: auto (default: tensor cores for large launches), tensor "
-                         "(8-bit split on the tensor cores) or cuda (CUDA cores); the output bits are the same")
+                         "(8-bit split on the tensor cores), fused (that, fused with the first forward NTT "
+                         "pass) or cuda (CUDA cores); the output bits are the same")
     ap.add_argument("--int-peaks", action="store_true",
                     help="measure this GPU's integer throughput per instruction class (ckks_int_probe) and "
                          "print it as one JSON line")
