@@ -1048,14 +1048,12 @@ def info_cpu_baseline(key: str, max_seconds: float = 8.0):
 BCONV_ENGINES = {"cuda": "CUDA cores (32x32->64-bit multiply-adds)",
                  "tensor": "tensor cores (8-bit split, tcgen05.mma kind::i8)",
                  "auto": "automatic: tensor cores (8-bit split, tcgen05.mma kind::i8) for launches of at least "
-                         "4 tiles per block, CUDA cores below",
-                 "fused": "tensor cores (8-bit split, tcgen05.mma kind::i8) fused with the first forward NTT "
-                          "pass of the converted limbs"}
+                         "4 tiles per block, CUDA cores below"}
 
 
 def set_bconv(ks, ctx, args):
     ks.ckks_set_bconv_mode(ctx, {"tensor": ks.CKKS_BCONV_TENSOR, "cuda": ks.CKKS_BCONV_CUDA_CORES,
-                                 "auto": ks.CKKS_BCONV_AUTO, "fused": ks.CKKS_BCONV_FUSED}[args.bconv])
+                                 "auto": ks.CKKS_BCONV_AUTO}[args.bconv])
 
 
 def run_int_peaks(local_rank):
@@ -1196,8 +1194,7 @@ def main():
                          "batches; at 2 streams x 4 units the other stream already hides launch gaps)")
     ap.add_argument("--bconv", default="auto", choices=sorted(BCONV_ENGINES),
                     help="base-conversion engine: auto (default: tensor cores for large launches), tensor "
-                         "(8-bit split on the tensor cores), fused (that, fused with the first forward NTT "
-                         "pass) or cuda (CUDA cores); the output bits are the same")
+                         "(8-bit split on the tensor cores) or cuda (CUDA cores); the output bits are the same")
     ap.add_argument("--int-peaks", action="store_true",
                     help="measure this GPU's integer throughput per instruction class (ckks_int_probe) and "
                          "print it as one JSON line")

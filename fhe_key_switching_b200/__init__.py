@@ -430,13 +430,12 @@ def ckks_modraise(ctx, ct, level: int, out, ws, stream=None):
                             _stream(stream)), "ckks_modraise")
 
 
-CKKS_BCONV_CUDA_CORES, CKKS_BCONV_TENSOR, CKKS_BCONV_AUTO, CKKS_BCONV_FUSED = 0, 1, 2, 3
+CKKS_BCONV_CUDA_CORES, CKKS_BCONV_TENSOR, CKKS_BCONV_AUTO = 0, 1, 2
 
 
 def ckks_set_bconv_mode(ctx, mode: int):
     """Base-conversion engine of later calls on ctx: CKKS_BCONV_AUTO (default: the tensor cores for
-    large launches), CKKS_BCONV_TENSOR (8-bit contraction on the tensor cores),
-    CKKS_BCONV_FUSED (that contraction fused with the first forward NTT pass) or
+    large launches), CKKS_BCONV_TENSOR (8-bit contraction on the tensor cores) or
     CKKS_BCONV_CUDA_CORES; same output bits either way."""
     _check(_L.ckks_set_bconv_mode(ctx.handle, mode), "ckks_set_bconv_mode")
 

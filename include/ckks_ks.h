@@ -281,14 +281,10 @@ int ckks_evalmod(ckks_ctx *ctx, const uint32_t *ct, int level, double scale, int
  *    epilogue.  Groups of more than 15 primes use the CUDA cores;
  *  CKKS_BCONV_CUDA_CORES: 32 x 32 -> 64-bit multiply-adds on the CUDA cores;
  *  CKKS_BCONV_AUTO (default): the tensor cores for launches large enough to give each block of
- *    the tensor-core kernel at least 4 tiles of 128 coefficients, the CUDA cores otherwise;
- *  CKKS_BCONV_FUSED: the tensor-core conversion fused with the first forward NTT pass of the
- *    converted limbs (ModUp and ModDown): one kernel converts a block of 8 NTT columns for up to
- *    8 targets into shared memory and runs their column passes there, so the converted limbs
- *    never go to HBM and back.  Groups of more than 15 primes use the CUDA cores.
+ *    the tensor-core kernel at least 4 tiles of 128 coefficients, the CUDA cores otherwise.
  * The mode applies to later calls on the context; it is not synchronised with calls in flight
  * from other threads.  CKKS_ERR_ARG for an unknown mode. */
-enum { CKKS_BCONV_CUDA_CORES = 0, CKKS_BCONV_TENSOR = 1, CKKS_BCONV_AUTO = 2, CKKS_BCONV_FUSED = 3 };
+enum { CKKS_BCONV_CUDA_CORES = 0, CKKS_BCONV_TENSOR = 1, CKKS_BCONV_AUTO = 2 };
 int ckks_set_bconv_mode(ckks_ctx *ctx, int mode);
 
 /* The key's regenerated uniform half for one (digit, global limb): out [N] (device),

@@ -1,9 +1,7 @@
-"""Base conversion on the tensor cores against the oracle, bit for bit: the conversion alone
-(CKKS_BCONV_TENSOR) and fused with the first forward NTT pass (CKKS_BCONV_FUSED), each test in
-both modes.
+"""Base conversion on the tensor cores (CKKS_BCONV_TENSOR) against the oracle, bit for bit.
 
-The tensor-core engines compute the same residues as the CUDA-core one through an exact 8-bit
-contraction, so every entry point must give the oracle's bits in every mode.  Covered: ModUp and
+The tensor-core engine computes the same residues as the CUDA-core one through an exact 8-bit
+contraction, so every entry point must give the oracle's bits in either mode.  Covered: ModUp and
 ModDown alone (full and partial last digits, groups of 1 to 12 primes), the key switch, rotation
 and relinearisation, a batch of items with several target chunks, hoisted rotations, the
 centred-lift thresholds, and groups wider than 15 primes (which fall back to the CUDA cores)."""
@@ -26,27 +24,22 @@ def _host(t):
     return t.cpu().numpy()
 
 
-@pytest.fixture(params=["tensor", "fused"])
-def mode(request):
-    return request.param
-
-
-def _ctx(ks, oracle_mod, log_n, n_q, n_p, dnum, mode):
+def _ctx(ks, oracle_mod, log_n, n_q, n_p, dnum):
     q, p = ks.ckks_gen_primes(log_n, n_q, n_p)
     octx = oracle_mod.Ctx(log_n, n_q, n_p)
     assert octx.q == q and octx.p == p
     ctx = ks.Context(log_n, q, p, dnum)
-    ks.ckks_set_bconv_mode(ctx, ks.CKKS_BCONV_FUSED if mode == "fused" else ks.CKKS_BCONV_TENSOR)
+    ks.ckks_set_bconv_mode(ctx, ks.CKKS_BCONV_TENSOR)
     return q, p, octx, ctx
 
 
 @pytest.mark.parametrize("key,level", [("n12-dnum2", 3), ("n12-dnum4", 2), ("n14-hoisted8", 11),
                                        ("n14-hoisted8", 6), ("n16-full", 35), ("n16-stream64", 20),
                                        ("n16-full", 0)])
-def test_tc_modup_moddown(ks_lib, oracle_mod, key, level, mode):
+def test_tc_modup_moddown(ks_lib, oracle_mod, key, level):
     ks = ks_lib
     cfg = W.CONFIGS[key]
-    q, p, octx, ctx = _ctx(ks, oracle_mod, cfg.log_n, cfg.n_q, cfg.n_p, cfg.dnum, mode)
+    q, p, octx, ctx = _ctx(ks, oracle_mod, cfg.log_n, cfg.n_q, cfg.n_p, cfg.dnum)
     n, na = cfg.n, level + 1
     gen = W.rng(cfg.seed, W.TAG_SYNTH, 8100 + level)
     c = W.uniform_residues(q[:na], n, gen)
@@ -62,11 +55,11 @@ def test_tc_modup_moddown(ks_lib, oracle_mod, key, level, mode):
 
 
 @pytest.mark.parametrize("log_n,level", [(13, 5), (13, 2), (15, 5), (15, 4)])
-def test_tc_modup_moddown_every_ring(ks_lib, oracle_mod, log_n, level, mode):
-    """N = 2^13 and 2^15 (the column passes of 32 and 128 rows), 6 + 2 primes, dnum 3, full and
-    partial last digits: ModUp and ModDown equal the oracle."""
+def test_tc_modup_moddown_every_ring(ks_lib, oracle_mod, log_n, level):
+    """N = 2^13 and 2^15, 6 + 2 primes, dnum 3, full and partial last digits: ModUp and ModDown
+    equal the oracle."""
     ks = ks_lib
-    q, p, octx, ctx = _ctx(ks, oracle_mod, log_n, 6, 2, 3, mode)
+    q, p, octx, ctx = _ctx(ks, oracle_mod, log_n, 6, 2, 3)
     n, na, alpha = 1 << log_n, level + 1, 2
     gen = W.rng(3, W.TAG_SYNTH, 8400 + 16 * log_n + level)
     c = W.uniform_residues(q[:na], n, gen)
@@ -81,13 +74,13 @@ def test_tc_modup_moddown_every_ring(ks_lib, oracle_mod, log_n, level, mode):
 
 
 @pytest.mark.parametrize("key", ["n12-dnum2", "n14-hoisted8", "n16-full"])
-def test_tc_rotate_relin_and_modes_agree(ks_lib, oracle_mod, key, mode):
+def test_tc_rotate_relin_and_modes_agree(ks_lib, oracle_mod, key):
     """Rotation and relinearisation with oracle-built keys; every other mode gives the same bits."""
     from oracle.scenario import Scenario
     ks = ks_lib
     cfg = W.CONFIGS[key]
     sc = Scenario(cfg)
-    q, p, octx, ctx = _ctx(ks, oracle_mod, cfg.log_n, cfg.n_q, cfg.n_p, cfg.dnum, mode)
+    q, p, octx, ctx = _ctx(ks, oracle_mod, cfg.log_n, cfg.n_q, cfg.n_p, cfg.dnum)
     lvl = cfg.level
     _, x = sc.ciphertext(0)
     _, y = sc.ciphertext(1)
@@ -105,18 +98,18 @@ def test_tc_rotate_relin_and_modes_agree(ks_lib, oracle_mod, key, mode):
     ks.ckks_relin(ctx, d, lvl, evk_0, out, ws)
     want_rel = octx.relin(octx.tensor(x, y, lvl), lvl, cfg.alpha, b0, cfg.chacha_seed, 0)
     assert np.array_equal(_host(out), want_rel)
-    for other in (ks.CKKS_BCONV_CUDA_CORES, ks.CKKS_BCONV_AUTO, ks.CKKS_BCONV_TENSOR, ks.CKKS_BCONV_FUSED):
+    for other in (ks.CKKS_BCONV_CUDA_CORES, ks.CKKS_BCONV_AUTO):
         ks.ckks_set_bconv_mode(ctx, other)
         ks.ckks_rotate(ctx, _dev(x), lvl, g, evk_g, out, ws)
         assert np.array_equal(_host(out), want_rot), other
 
 
-def test_tc_batch_and_hoisted(ks_lib, oracle_mod, mode):
+def test_tc_batch_and_hoisted(ks_lib, oracle_mod):
     """A 5-item key-switch batch (several items per launch and two target chunks per group) and
     4 hoisted rotations at N=2^14; every item equals the oracle."""
     ks = ks_lib
     cfg = W.CONFIGS["n14-hoisted8"]
-    q, p, octx, ctx = _ctx(ks, oracle_mod, cfg.log_n, cfg.n_q, cfg.n_p, cfg.dnum, mode)
+    q, p, octx, ctx = _ctx(ks, oracle_mod, cfg.log_n, cfg.n_q, cfg.n_p, cfg.dnum)
     lvl, n = cfg.level, cfg.n
     na, items = lvl + 1, 5
     gen = W.rng(cfg.seed, W.TAG_SYNTH, 8200)
@@ -139,11 +132,11 @@ def test_tc_batch_and_hoisted(ks_lib, oracle_mod, mode):
     assert np.array_equal(_host(rot), want)
 
 
-def test_tc_wide_groups_fall_back(ks_lib, oracle_mod, mode):
+def test_tc_wide_groups_fall_back(ks_lib, oracle_mod):
     """dnum 1 at N=2^12 (a digit of 36 primes, 24 special primes): both conversions are wider
     than the tensor-core tile and run on the CUDA cores; the output is the oracle's."""
     ks = ks_lib
-    q, p, octx, ctx = _ctx(ks, oracle_mod, 12, 36, 24, 1, mode)
+    q, p, octx, ctx = _ctx(ks, oracle_mod, 12, 36, 24, 1)
     n, lvl = 1 << 12, 35
     gen = W.rng(1, W.TAG_SYNTH, 8300)
     c = W.uniform_residues(q, n, gen)

@@ -51,13 +51,12 @@ def _setup(ks, oracle_mod, key, mode):
     octx = oracle_mod.Ctx(cfg.log_n, cfg.n_q, cfg.n_p)
     assert octx.q == q and octx.p == p
     ctx = ks.Context(cfg.log_n, q, p, cfg.dnum)
-    ks.ckks_set_bconv_mode(ctx, {"tensor": ks.CKKS_BCONV_TENSOR, "fused": ks.CKKS_BCONV_FUSED,
-                                 "cuda_cores": ks.CKKS_BCONV_CUDA_CORES}[mode])
+    ks.ckks_set_bconv_mode(ctx, ks.CKKS_BCONV_TENSOR if mode == "tensor" else ks.CKKS_BCONV_CUDA_CORES)
     return cfg, octx, ctx
 
 
 CASES = [("n12-dnum2", 3), ("n14-hoisted8", 11), ("n14-hoisted8", 6), ("n16-full", 35)]
-MODES = ["cuda_cores", "tensor", "fused"]   # the base-conversion engine (same bits in every mode)
+MODES = ["cuda_cores", "tensor"]       # the base-conversion engine (same bits either way)
 
 
 @pytest.mark.gpu
