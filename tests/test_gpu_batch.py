@@ -178,6 +178,47 @@ def test_bench_launch_configuration(ks_lib, oracle_mod):
         assert np.array_equal(out[i].cpu().numpy(), want), i
 
 
+def test_two_streams_share_a_context(ks_lib):
+    """The benchmark's concurrency: one context, two streams with a workspace each, each stream
+    running tensor -> relin -> rotate on its own 2 units of n16-full while the other runs.  Both
+    results equal the same calls made one after the other on the default stream."""
+    import hashlib
+    ks = ks_lib
+    cfg, q, p, ctx = _setup(ks, "n16-full")
+    lvl, N = cfg.level, cfg.n
+    na, B, S = lvl + 1, 4, 2
+    gen = W.rng(cfg.seed, W.TAG_SYNTH, 779)
+    nd = -(-cfg.n_q // cfg.alpha)
+    g = ks.galois_element(cfg.log_n, 1)
+    seeds = [hashlib.sha256(cfg.chacha_seed + bytes([1, i])).digest() for i in range(B)]
+    k_rel = [ks.make_evk(_res((q + p) * nd, N, gen).view(nd, len(q) + len(p), N), seeds[i], 0) for i in range(B)]
+    k_rot = [ks.make_evk(_res((q + p) * nd, N, gen).view(nd, len(q) + len(p), N), seeds[i], g) for i in range(B)]
+    x = _res(q[:na] * 2 * B, N, gen).view(B, 2, na, N)
+    y = _res(q[:na] * 2 * B, N, gen).view(B, 2, na, N)
+
+    def run(streams):
+        d = torch.empty((B, 3, na, N), dtype=torch.uint32, device="cuda")
+        r = torch.empty((B, 2, na, N), dtype=torch.uint32, device="cuda")
+        out = torch.empty((B, 2, na, N), dtype=torch.uint32, device="cuda")
+        per = B // len(streams)
+        wss = [ctx.workspace(lvl, per) for _ in streams]
+        torch.cuda.synchronize()
+        for si, st in enumerate(streams):
+            z = slice(si * per, (si + 1) * per)
+            with torch.cuda.stream(st):
+                ks.ckks_tensor_batch(ctx, per, x[z], y[z], lvl, d[z], st)
+                ks.ckks_relin_batch(ctx, d[z], lvl, k_rel[z], r[z], wss[si], st)
+                ks.ckks_rotate_batch(ctx, r[z], lvl, [g] * per, k_rot[z], out[z], wss[si], st)
+        torch.cuda.synchronize()
+        for st in streams:
+            assert ks.ckks_sync_status(ctx, st, 10000) == ks.CKKS_OK
+        return out
+
+    want = run([torch.cuda.default_stream()])
+    got = run([torch.cuda.Stream() for _ in range(S)])
+    assert torch.equal(got, want)
+
+
 @pytest.mark.slow
 def test_n16_stream64_shared_keystream_batches(ks_lib, oracle_mod):
     """The n16-stream64 line's launch configuration (N=2^16, level 20, dnum 4, so beta = 3):
