@@ -1,6 +1,7 @@
 """Seeded sweep of small parameter sets on the GPU against the oracle, bit for bit.
 
-Chains at N=2^12 (6 + 2 primes) and N=2^13 (5 + 3 primes); every dnum from 1 to L+1, so digit
+Chains at N=2^12 (6 + 2 primes), N=2^13 (5 + 3 primes) and N=2^15 (4 + 2 primes; the column
+passes of 128 rows, which the N = 2^14 and 2^16 configurations do not reach); every dnum from 1 to L+1, so digit
 widths from the whole chain down to one prime; for each, two levels drawn from a seeded
 generator, one of them chosen so that the last digit is partial whenever the digit width allows
 it.  At each point: a key switch, two hoisted rotations (steps 1 and -3) and a rescale (level >= 1),
@@ -13,7 +14,7 @@ import workloads as W
 
 torch = pytest.importorskip("torch")
 
-CHAINS = [(12, 6, 2), (13, 5, 3)]
+CHAINS = [(12, 6, 2), (13, 5, 3), (15, 4, 2)]
 
 
 def _grid():
