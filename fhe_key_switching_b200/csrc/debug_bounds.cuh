@@ -116,6 +116,24 @@ __device__ __forceinline__ unsigned ckks_dbg_dynamic_smem_bytes() {
 #define CKKS_POISON(p, bytes) ckks_dbg_poison((p), (bytes))
 #define CKKS_POISON_DYNAMIC(p) ckks_dbg_poison((p), ckks_dbg_dynamic_smem_bytes())
 
+// The host's region slots reach the device through this kernel, launched on the registering
+// call's stream before its first launch: it writes that call's slots only and raises the table
+// length with atomicMax, so that calls on other streams never see their own slots shrink away.
+constexpr int CKKS_DBG_PUBLISH_MAX = 64;
+struct CkksDbgPublish {
+    int n;
+    int slot[CKKS_DBG_PUBLISH_MAX];
+    CkksDbgRegion r[CKKS_DBG_PUBLISH_MAX];
+};
+__global__ void k_dbg_publish(CkksDbgPublish p) {
+    const int i = threadIdx.x;
+    if (i < p.n && p.slot[i] >= 0 && p.slot[i] < CKKS_DBG_MAX_REGIONS) {
+        g_dbg_regions[p.slot[i]] = p.r[i];
+        __threadfence();
+        atomicMax(&g_dbg_n_regions, p.slot[i] + 1);
+    }
+}
+
 // Self-test of the record: checks the 4 bytes after a word the host registered as a region of its
 // own (a cudaMalloc'd word: no other allocation starts before the next 256-byte boundary), so the
 // check fails; nothing is read or written.

@@ -347,9 +347,10 @@ int ckks_selftest_wait_expiry(ckks_ctx *ctx, ckks_stream_t stream);
  * failure's site, address and size, and the accesses of that group are skipped (loads read 0), so
  * a wrong index is reported and no memory outside the call's buffers is touched.  Shared memory is
  * filled with a poison word at the start of each kernel that stages data in it, so that a read of
- * a word never written gives a wrong result.  The region table is global per device: use the
- * debug build with one stream at a time.  The release build has no checks and the same
- * results; the integer-throughput probe is not instrumented.
+ * a word never written gives a wrong result.  Calls may run on several streams at once: each
+ * call's regions stay in the table until its stream has run the call's last launch.  The
+ * release build has no checks and the same results; the integer-throughput probe is not
+ * instrumented.
  *   ckks_debug_bounds_enabled: 1 in the debug-bounds build, 0 otherwise.
  *   ckks_debug_bounds_report: waits for the current device, then stores the number of failed
  *     checks since the last clear and the first failure's site (see ckks_debug_bounds_site_name),
