@@ -75,6 +75,7 @@ _SIGS = {
     "ckks_workspace_bytes": (_sz, [_vp, _ci, _ci]),
     "ckks_sync_status": (_ci, [_vp, _vp, _ci]),
     "ckks_selftest_wait_expiry": (_ci, [_vp, _vp]),
+    "ckks_selftest_launch_error": (_ci, [_vp, _vp]),
     "ckks_keyswitch_noalloc": (_ci, [_vp, _vp, _ci, ctypes.POINTER(ckks_evk), _vp, _vp]),
     "ckks_prof_begin": (_ci, [_vp, ctypes.c_char_p, _ci]),
     "ckks_prof_end": (_ci, [_vp, ctypes.POINTER(_ci), ctypes.POINTER(ctypes.c_double)]),
@@ -347,6 +348,15 @@ def ckks_sync_status(ctx, stream=None, timeout_ms: int = 10000) -> int:
 
 def ckks_selftest_wait_expiry(ctx, stream=None):
     _check(_L.ckks_selftest_wait_expiry(ctx.handle, _stream(stream)), "ckks_selftest_wait_expiry")
+
+
+def ckks_selftest_launch_error(ctx, stream=None) -> int:
+    """The status of a launch the CUDA runtime rejects (CKKS_ERR_CUDA); see ckks_last_error()."""
+    return int(_L.ckks_selftest_launch_error(ctx.handle, _stream(stream)))
+
+
+def ckks_last_error() -> str:
+    return _L.ckks_last_error().decode(errors="replace")
 
 
 def ckks_debug_bounds_enabled() -> bool:

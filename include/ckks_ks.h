@@ -337,6 +337,13 @@ int ckks_sync_status(ckks_ctx *ctx, ckks_stream_t stream, int timeout_ms);
  * usable.  Nothing faults or hangs. */
 int ckks_selftest_wait_expiry(ckks_ctx *ctx, ckks_stream_t stream);
 
+/* Self-test of the CUDA-error path (no counterpart in the pages): launches a kernel with an
+ * invalid configuration (2048 threads per block), which the CUDA runtime rejects on the host
+ * before anything reaches the GPU, and returns what every entry point returns after a failed
+ * launch: CKKS_ERR_CUDA, with the runtime's message in ckks_last_error().  The error is not
+ * sticky: the context and the stream stay usable. */
+int ckks_selftest_launch_error(ckks_ctx *ctx, ckks_stream_t stream);
+
 /* Debug-bounds build (a checking aid; the pages have no counterpart).  The same sources compiled
  * with -DCKKS_DEBUG_BOUNDS (`python fhe_key_switching_b200/build.py --debug` writes
  * libckks_ks_debug.so beside the release library) give every kernel index checks: before each
