@@ -515,6 +515,10 @@ struct IpRowArgs {
     int grp_first[KS_MAXB], grp_count[KS_MAXB], grp_item[KS_MAXB];
 };
 
+// XDONE: x already holds every non-digit limb in the evaluation domain (a hoisted batch whose
+// shared ModUp ran its forward row pass once); those rows are then read like the digit limbs,
+// through kappa_{hoist_g}, instead of being transformed again for every item.
+template <bool XDONE>
 __global__ void __launch_bounds__(ROW_THREADS)
 k_ip_row(IpRowArgs a) {
     __shared__ u32 sm[16 * 272];
@@ -566,9 +570,9 @@ k_ip_row(IpRowArgs a) {
         for (int j = 0; j < a.beta; j++) {
             const bool in_digit = u < na && u >= j * a.alpha && u < min(j * a.alpha + a.alpha, na);
             u32 x[16];
-            if (in_digit) {
-                const u32 *src = cdb + (size_t)u * n;
-                const u32 g = hoist_g ? hoist_g : cdig_g;
+            if (in_digit || XDONE) {
+                const u32 *src = in_digit ? cdb + (size_t)u * n : xb + ((size_t)j * a.ext + u) * n;
+                const u32 g = in_digit ? (hoist_g ? hoist_g : cdig_g) : hoist_g;
                 if (g) {
                     const bool ok = CKKS_SPAN(src, n, CKKS_DBG_IPROW_CDIG);       // automorph_src < n
 #pragma unroll
