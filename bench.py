@@ -591,7 +591,7 @@ def roofline(cfg, launches, total_ms, clk, batch, single_step_ms, launches_ov, t
 # DRAM bytes (read + write) per unit of a k_ip_row launch from an ncu capture, valid only for the
 # kernel sources it was taken on (sha-256 prefix of the device-code headers): after any change to
 # them the figure is reported as null until a new capture replaces it.
-IP_ROW_TRAFFIC = {"sources_sha16": "f7525bba23c6f0ee", "bytes_per_unit": (473.82e6 + 471.26e6) / 2 / 4,
+IP_ROW_TRAFFIC = {"sources_sha16": "f6416638b40c5a0a", "bytes_per_unit": (473.86e6 + 471.79e6) / 2 / 4,
                   "capture": "profiles/k_ip_row_n16_full.md (dram__bytes read + write of two 4-unit launches)"}
 KERNEL_HEADERS = ("debug_bounds.cuh", "modarith.cuh", "chacha.cuh", "ntt.cuh", "ks_kernels.cuh")
 
