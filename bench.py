@@ -754,9 +754,9 @@ def run_workload(args, local_rank):
         nbytes = R * (2 * na + 2 * lvl) * limb
     elif key == "bootstrap-steps":
         # the bootstrapping steps this library has, in sequence, at N=2^16 (dnum 4, levels 35 -> 17):
-        # ModRaise to level 35, CoeffToSlot (3 levels), one conjugation, EvalMod twice (the real and
-        # the imaginary halves: degree 12, 3 double angles, 12 levels each), SlotToCoeff (3 levels);
-        # synthetic plaintexts and keys (the cost is data independent)
+        # ModRaise to level 35, CoeffToSlot (3 levels), one conjugation, EvalMod on the real and the
+        # imaginary halves as one batch of two (degree 12, 3 double angles, 12 levels), SlotToCoeff
+        # (3 levels); synthetic plaintexts and keys (the cost is data independent)
         levels, n1, L = 3, 8, cfg.n_q - 1
         ns = n // 2
         halves_fwd = [1 << h for h in range(cfg.log_n - 2, -1, -1)]
@@ -793,14 +793,17 @@ def run_workload(args, local_rank):
         bufs = [torch.empty((2, L + 1, n), dtype=torch.uint32, device=dev) for _ in range(4)]
         ws_mr = torch.empty(2 * n, dtype=torch.uint32, device=dev)
         ws_ks = ctx.workspace(L, 1, device=dev)
-        ws_em = ks.ckks_evalmod_workspace(ctx, L - 3, device=dev)
+        ws_em = ks.ckks_evalmod_batch_workspace(ctx, L - 3, 2, device=dev)
+        pair = torch.empty((2, 2, L + 1, n), dtype=torch.uint32, device=dev)    # z and its conjugate
+        em_out = torch.empty((2, 2, L + 1, n), dtype=torch.uint32, device=dev)
 
-        def run_levels(plan_, src):
+        def run_levels(plan_, src, final=None):
             cur = src
             for i_, (lv_, bg_, gg_, pt_, ws_l) in enumerate(plan_):
                 ks.ckks_bsgs(ctx, cur, lv_, bg_, [gk.get(g_) for g_ in bg_], gg_, [gk.get(g_) for g_ in gg_],
                              pt_, bufs[0].view(-1)[: 2 * (lv_ + 1) * n].view(2, lv_ + 1, n), ws_l, stream)
-                dst = bufs[1 + (i_ & 1)].view(-1)[: 2 * lv_ * n].view(2, lv_, n)
+                last = i_ == len(plan_) - 1 and final is not None
+                dst = final if last else bufs[1 + (i_ & 1)].view(-1)[: 2 * lv_ * n].view(2, lv_, n)
                 ks.ckks_rescale(ctx, bufs[0].view(-1)[: 2 * (lv_ + 1) * n].view(2, lv_ + 1, n), lv_, dst, ws_ks,
                                 stream)
                 cur = dst
@@ -808,14 +811,13 @@ def run_workload(args, local_rank):
 
         def step(i):
             ks.ckks_modraise(ctx, cts0[i % N_SETS], L, big, ws_mr, stream)
-            z = run_levels(c2s, big)
             lz = L - 3
-            zc = bufs[3].view(-1)[: 2 * (lz + 1) * n].view(2, lz + 1, n)
-            ks.ckks_rotate(ctx, z, lz, gconj, k_conj, zc, ws_ks, stream)
-            e1 = bufs[0].view(-1)[: 2 * (lz + 1) * n].view(2, lz + 1, n)
-            ks.ckks_evalmod(ctx, z, lz, float(q[lz]), 3, 6, k_rel, e1, ws_em, stream)
-            ks.ckks_evalmod(ctx, zc, lz, float(q[lz]), 3, 6, k_rel, big, ws_em, stream)
-            run_levels(s2c, big.view(-1)[: 2 * (lz - 12 + 1) * n].view(2, lz - 12 + 1, n))
+            zz = pair.view(-1)[: 4 * (lz + 1) * n].view(2, 2, lz + 1, n)
+            run_levels(c2s, big, final=zz[0])
+            ks.ckks_rotate(ctx, zz[0], lz, gconj, k_conj, zz[1], ws_ks, stream)
+            lv_em, _ = ks.ckks_evalmod_batch(ctx, zz, lz, float(q[lz]), 3, 6, k_rel, em_out, ws_em, stream)
+            em = em_out.view(-1)[: 4 * (lv_em + 1) * n].view(2, 2, lv_em + 1, n)
+            run_levels(s2c, em[1])
         ks_per_step = rot_per_step = (sum(sum(1 for g_ in bg_ + gg_ if g_ != 1) for _, bg_, gg_, _, _ in c2s + s2c)
                                       + 1)
         ops = blocks = nbytes = 0        # reported as a time only: its op model is not tabulated

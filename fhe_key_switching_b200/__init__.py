@@ -84,6 +84,9 @@ _SIGS = {
     "ckks_add_const": (_ci, [_vp, _vp, _ci, ctypes.c_longlong, _vp, _vp]),
     "ckks_add": (_ci, [_vp, _vp, _vp, _ci, _ci, _vp, _vp]),
     "ckks_evalmod_workspace_bytes": (_sz, [_vp, _ci]),
+    "ckks_evalmod_batch_workspace_bytes": (_sz, [_vp, _ci, _ci]),
+    "ckks_evalmod_batch": (_ci, [_vp, _ci, _vp, _ci, ctypes.c_double, _ci, _ci, ctypes.POINTER(ckks_evk), _vp,
+                                 ctypes.POINTER(_ci), ctypes.POINTER(ctypes.c_double), _vp, _sz, _vp]),
     "ckks_evalmod": (_ci, [_vp, _vp, _ci, ctypes.c_double, _ci, _ci, ctypes.POINTER(ckks_evk), _vp,
                            ctypes.POINTER(_ci), ctypes.POINTER(ctypes.c_double), _vp, _sz, _vp]),
     "ckks_modraise": (_ci, [_vp, _vp, _ci, _vp, _vp, _sz, _vp]),
@@ -431,6 +434,25 @@ def ckks_evalmod(ctx, ct, level: int, scale: float, r: int, d: int, relin_evk: c
     _check(_L.ckks_evalmod(ctx.handle, _ptr(ct), level, float(scale), r, d, ctypes.byref(relin_evk), _ptr(out),
                            ctypes.byref(lv), ctypes.byref(sc), _ptr(ws), ws.numel() * ws.element_size(),
                            _stream(stream)), "ckks_evalmod")
+    return lv.value, sc.value
+
+
+def ckks_evalmod_batch_workspace(ctx, level: int, n: int, device=None):
+    import torch
+    nb = int(_L.ckks_evalmod_batch_workspace_bytes(ctx.handle, level, n))
+    if nb == 0:
+        raise ValueError("ckks_evalmod_batch_workspace_bytes: level or batch out of range")
+    return torch.empty(nb, dtype=torch.uint8, device=device or torch.device("cuda", torch.cuda.current_device()))
+
+
+def ckks_evalmod_batch(ctx, ct, level: int, scale: float, r: int, d: int, relin_evk: ckks_evk, out, ws,
+                       stream=None):
+    """EvalMod on the n ciphertexts of ct [n][2][level+1][N]; returns (out_level, out_scale)."""
+    lv = _ci()
+    sc = ctypes.c_double()
+    _check(_L.ckks_evalmod_batch(ctx.handle, int(ct.shape[0]), _ptr(ct), level, float(scale), r, d,
+                                 ctypes.byref(relin_evk), _ptr(out), ctypes.byref(lv), ctypes.byref(sc), _ptr(ws),
+                                 ws.numel() * ws.element_size(), _stream(stream)), "ckks_evalmod_batch")
     return lv.value, sc.value
 
 

@@ -4,8 +4,9 @@
 #include "ntt.cuh"
 
 // Ciphertext-constant arithmetic over [n_comp][l+1] rows (row r has the prime of limb r mod (l+1)):
-//   k_mul_const: out = in * [c]_q (every component); k_add_const: out = in + [c]_q on component 0,
-//   component 1 copied; k_add: out = x + y.  cw: per limb (w, Shoup companion) of [c]_q_i.
+//   k_mul_const: out = in * [c]_q (every component); k_add_const: out = in + [c]_q on component 0
+//   of every ciphertext ([n][2][l+1] rows: the even components), the odd components copied;
+//   k_add: out = x + y.  cw: per limb (w, Shoup companion) of [c]_q_i.
 struct ConstRns {
     tw_t w[64];
 };
@@ -35,7 +36,7 @@ __global__ void k_add_const(const u32 *in, u32 *out, ConstRns cw, const PrimeInf
         !CKKS_SPAN(out + (size_t)r * n + 4 * c4, 4, CKKS_DBG_CONST))
         return;
     const u32 q = pinfo[i].q;
-    const u32 c = r <= level ? cw.w[i].x : 0u;        // the constant polynomial: every slot, component 0
+    const u32 c = ((r / (level + 1)) & 1) == 0 ? cw.w[i].x : 0u;   // component 0 of each ciphertext
     const uint4 v = reinterpret_cast<const uint4 *>(in + (size_t)r * n)[c4];
     reinterpret_cast<uint4 *>(out + (size_t)r * n)[c4] =
         make_uint4(csub(v.x + c, q), csub(v.y + c, q), csub(v.z + c, q), csub(v.w + c, q));

@@ -273,6 +273,19 @@ size_t ckks_evalmod_workspace_bytes(const ckks_ctx *ctx, int level);
 int ckks_evalmod(ckks_ctx *ctx, const uint32_t *ct, int level, double scale, int r, int d, const ckks_evk *relin_key,
                  uint32_t *out, int *out_level, double *out_scale, void *ws, size_t ws_bytes, ckks_stream_t stream);
 
+/* The same EvalMod on n ciphertexts at one level and scale (1 <= n <= 64; bootstrapping applies it
+ * to the real and the imaginary halves): ct [n][2][level+1][N]; out: room for n 2 (level+1) N
+ * words, of which the first n 2 (*out_level+1) N hold the results as [n][2][*out_level+1][N];
+ * ws: ckks_evalmod_batch_workspace_bytes(ctx, level, n) bytes (0 for n or level out of range).
+ * Every step runs once for the whole batch (the batched tensor, relinearisation and rescale
+ * calls; the items' relinearisations share the one key's regenerated a half).  Each item's
+ * result equals ckks_evalmod on that item alone, bit for bit.  Errors as ckks_evalmod, and
+ * CKKS_ERR_ARG for n out of range. */
+size_t ckks_evalmod_batch_workspace_bytes(const ckks_ctx *ctx, int level, int n);
+int ckks_evalmod_batch(ckks_ctx *ctx, int n, const uint32_t *ct, int level, double scale, int r, int d,
+                       const ckks_evk *relin_key, uint32_t *out, int *out_level, double *out_scale, void *ws,
+                       size_t ws_bytes, ckks_stream_t stream);
+
 /* Base-conversion engine (the results are the same residues either way; the bits of every
  * entry point's output are identical):
  *  CKKS_BCONV_TENSOR: the conversion as an exact 8-bit contraction on the tensor cores

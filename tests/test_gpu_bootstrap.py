@@ -153,6 +153,31 @@ def test_evalmod_parity_n14(ks_lib, oracle_mod):
     _evalmod_case(ks_lib, oracle_mod, "n14-hoisted8", 11, 2, 4, False)
 
 
+def test_evalmod_batch_equals_single_calls(ks_lib, oracle_mod):
+    """ckks_evalmod_batch on 3 ciphertexts at N=2^14 (level 11, degree 8, two double angles): each
+    item equals ckks_evalmod on it alone, bit for bit (and that call equals the oracle, above)."""
+    ks = ks_lib
+    cfg = W.CONFIGS["n14-hoisted8"]
+    q, p = ks.ckks_gen_primes(cfg.log_n, cfg.n_q, cfg.n_p)
+    ctx = ks.Context(cfg.log_n, q, p, cfg.dnum)
+    lvl, n, nb = 11, cfg.n, 3
+    gen = W.rng(cfg.seed, W.TAG_SYNTH, 9400)
+    ct = W.uniform_residues(q[: lvl + 1] * 2 * nb, n, gen).reshape(nb, 2, lvl + 1, n)
+    nd = -(-cfg.n_q // cfg.alpha)
+    b0 = W.uniform_residues((q + p) * nd, n, gen).reshape(nd, len(q) + len(p), n)
+    evk = ks.make_evk(_dev(b0), cfg.chacha_seed, 0)
+    S = float(q[lvl])
+    out = torch.empty((nb, 2, lvl + 1, n), dtype=torch.uint32, device="cuda")
+    lv, so = ks.ckks_evalmod_batch(ctx, _dev(ct), lvl, S, 2, 4, evk, out, ks.ckks_evalmod_batch_workspace(ctx, lvl, nb))
+    got = _host(out).reshape(-1)[: nb * 2 * (lv + 1) * n].reshape(nb, 2, lv + 1, n)
+    one = torch.empty((2, lvl + 1, n), dtype=torch.uint32, device="cuda")
+    ws1 = ks.ckks_evalmod_workspace(ctx, lvl)
+    for i in range(nb):
+        assert ks.ckks_evalmod(ctx, _dev(ct[i]), lvl, S, 2, 4, evk, one, ws1) == (lv, so)
+        assert np.array_equal(_host(one).reshape(-1)[: 2 * (lv + 1) * n].reshape(2, lv + 1, n), got[i]), i
+    assert ks.ckks_sync_status(ctx, None, 10000) == ks.CKKS_OK
+
+
 @pytest.mark.slow
 def test_evalmod_parity_n16(ks_lib, oracle_mod):
     """EvalMod (degree 12, three double angles) at N=2^16, dnum 4, from level 35: bit for bit with
