@@ -462,7 +462,7 @@ def unit_model(cfg, level: int) -> dict:
 
 
 def ip_row_ops(cfg) -> float:
-    """Algorithmic int32 operations of one key switch's share of a k_ip_row launch, with the unit costs
+    """Algorithmic int32 operations of one key switch's share of a k_ip_row8 launch, with the unit costs
     of the op model: ChaCha12 block 608 (8 coefficients), 64-bit word reduction 8, NTT butterfly
     8, variable modular product 6, modular addition 2.  Units: beta*ext (digit, limb) pairs of N
     coefficients; the row pass (8 of log N stages) runs on the pairs outside their digit."""
@@ -570,7 +570,7 @@ def roofline(cfg, launches, total_ms, clk, batch, single_step_ms, launches_ov, t
     achieved = ops / avg_s / 1e12
     peak = ops / t_floor / 1e12
     traffic = ip_row_traffic_per_unit()
-    out = {"kernel": "k_ip_row (ModUp last NTT pass + ChaCha12 + key inner product)",
+    out = {"kernel": "k_ip_row8 (ModUp last NTT pass + ChaCha12 + key inner product)",
            "bound": "alu", "achieved": achieved, "peak": peak, "unit": "Tops (int32)",
            "frac": achieved / peak,
            "traffic": None if traffic is None else traffic * batch,
@@ -588,11 +588,11 @@ def roofline(cfg, launches, total_ms, clk, batch, single_step_ms, launches_ov, t
     return out
 
 
-# DRAM bytes (read + write) per unit of a k_ip_row launch from an ncu capture, valid only for the
+# DRAM bytes (read + write) per unit of a k_ip_row8 launch from an ncu capture, valid only for the
 # kernel sources it was taken on (sha-256 prefix of the device-code headers): after any change to
 # them the figure is reported as null until a new capture replaces it.
-IP_ROW_TRAFFIC = {"sources_sha16": "f6416638b40c5a0a", "bytes_per_unit": (473.86e6 + 471.79e6) / 2 / 4,
-                  "capture": "profiles/k_ip_row_n16_full.md (dram__bytes read + write of two 4-unit launches)"}
+IP_ROW_TRAFFIC = {"sources_sha16": "fa9b0e41cf836996", "bytes_per_unit": (479.04e6 + 476.39e6) / 2 / 4,
+                  "capture": "profiles/k_ip_row8_n16_full.md (dram__bytes read + write of two 4-unit launches)"}
 KERNEL_HEADERS = ("debug_bounds.cuh", "modarith.cuh", "chacha.cuh", "ntt.cuh", "ks_kernels.cuh")
 
 

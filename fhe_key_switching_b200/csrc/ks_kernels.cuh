@@ -479,11 +479,10 @@ __device__ __forceinline__ void row_inv_regs(u32 (&x)[16], const tw_t *tw, u32 b
     inv_top4(x, tw, base, q, two_q);
 }
 
-// Key inner product fused with the last forward NTT pass of ModUp.  Block (16 rows, u, group):
-// for every active digit j, the extended digit dt_j[u] is completed in registers (forward row
-// pass of the column-pass output x[j][u], or the input polynomial itself for u inside digit
-// j), the key's a half for (digit j, limb t) is regenerated by ChaCha12 for the same 16
-// slots, and
+// Key inner product, with the last forward NTT pass of ModUp fused in (k_ip_row8 below): for every
+// active digit j, the extended digit dt_j[u] is completed in registers (forward row pass of the
+// column-pass output x[j][u], or the input polynomial itself for u inside digit j), the key's a
+// half for (digit j, limb t) is regenerated by ChaCha12 for the same slots, and
 //   acc0 += dt_j[u] * b_j[t],  acc1 += dt_j[u] * a_j[t]   (Montgomery products, mod t).
 // Rotations: hoist_g != 0 reads every dt_j[u] through kappa_{hoist_g} (hoisted rotation:
 // the source row is transformed, then permuted inside the row); cdig_g != 0 reads only the
@@ -515,31 +514,27 @@ struct IpRowArgs {
     int grp_first[KS_MAXB], grp_count[KS_MAXB], grp_item[KS_MAXB];
 };
 
-// XDONE: x already holds every non-digit limb in the evaluation domain (a hoisted batch whose
-// shared ModUp ran its forward row pass once); those rows are then read like the digit limbs,
-// through kappa_{hoist_g}, instead of being transformed again for every item.
-template <bool XDONE>
+// The inner product of a hoisted batch whose shared ModUp is already complete in the evaluation
+// domain (run_modup_rows transformed every non-digit limb of x once): every dt_j[u] is read through
+// kappa_{hoist_g} -- x for the non-digit limbs, the input polynomial for the digit limbs -- so no
+// item repeats the row pass.  16 rows x 16 threads per block, 16 consecutive slots per thread
+// (at 128 registers this layout runs hoisted batches faster than k_ip_row8's); groups as above,
+// the shared a half as [digit][16][ROW_THREADS].
 __global__ void __launch_bounds__(ROW_THREADS)
-k_ip_row(IpRowArgs a) {
-    __shared__ u32 sm[16 * 272];
+k_ip_hoisted(IpRowArgs a) {
     extern __shared__ u32 sa[];                      // shared a half: [digit][16][ROW_THREADS]
     const int n = 1 << a.log_n;
     const int na = a.level + 1;
     const int u = blockIdx.y;
     const int g0 = a.grp_first[blockIdx.z], gcnt = a.grp_count[blockIdx.z];
     const int t = u < na ? u : a.n_q + (u - na);
-    if (!CKKS_SPAN(a.pinfo + t, 1, CKKS_DBG_IPROW_TABLES) || !CKKS_SPAN(a.twf + (size_t)t * n, n, CKKS_DBG_IPROW_TABLES))
-        return;                                               // (the same for the whole block)
-    CKKS_POISON(sm, sizeof(sm));
+    if (!CKKS_SPAN(a.pinfo + t, 1, CKKS_DBG_IPROW_TABLES)) return;   // (the same for the whole block)
     CKKS_POISON_DYNAMIC(sa);
     const PrimeInfo pi = a.pinfo[t];
     const u32 q = pi.q, two_q = 2 * q;
     const int r = threadIdx.x >> 4, lo = threadIdx.x & 15;
     const int row = blockIdx.x * 16 + r;
-    const u32 R1 = (u32)(n >> 8);
-    u32 *srow = sm + r * 272;
     const int k0 = row * 256 + 16 * lo;              // first evaluation slot of this thread
-    const tw_t *twf = a.twf + (size_t)t * n;
     if (gcnt > 1) {                                  // the group's shared a half, once per digit
         const int item = a.grp_item[g0];
         for (int j = 0; j < a.beta; j++) {
@@ -562,46 +557,27 @@ k_ip_row(IpRowArgs a) {
         const u32 *bkey = a.b[item];
         const u32 *astore = a.a_stored[item];
         const u32 hoist_g = a.hoist_g[item], cdig_g = a.cdig_g[item];
-        // hoisted rotation: source row of this row under kappa_g
-        const int src_row = hoist_g ? (int)(automorph_src((u32)(row * 256), hoist_g, a.log_n) >> 8) : row;
         u32 acc0[16], acc1[16];
 #pragma unroll
         for (int v = 0; v < 16; v++) acc0[v] = acc1[v] = 0;
         for (int j = 0; j < a.beta; j++) {
             const bool in_digit = u < na && u >= j * a.alpha && u < min(j * a.alpha + a.alpha, na);
+            const u32 *src = in_digit ? cdb + (size_t)u * n : xb + ((size_t)j * a.ext + u) * n;
+            const u32 g = in_digit ? (hoist_g ? hoist_g : cdig_g) : hoist_g;
             u32 x[16];
-            if (in_digit || XDONE) {
-                const u32 *src = in_digit ? cdb + (size_t)u * n : xb + ((size_t)j * a.ext + u) * n;
-                const u32 g = in_digit ? (hoist_g ? hoist_g : cdig_g) : hoist_g;
-                if (g) {
-                    const bool ok = CKKS_SPAN(src, n, CKKS_DBG_IPROW_CDIG);       // automorph_src < n
+            if (g) {
+                const bool ok = CKKS_SPAN(src, n, CKKS_DBG_IPROW_CDIG);       // automorph_src < n
 #pragma unroll
-                    for (int v = 0; v < 16; v++) x[v] = ok ? src[automorph_src((u32)(k0 + v), g, a.log_n)] : 0u;
-                } else {
-                    load16_chk(src + k0, x, CKKS_DBG_IPROW_CDIG);
-                }
+                for (int v = 0; v < 16; v++) x[v] = ok ? src[automorph_src((u32)(k0 + v), g, a.log_n)] : 0u;
             } else {
-                const u32 *src = xb + ((size_t)j * a.ext + u) * n + (size_t)src_row * 256;
-                load_row16_chk(src, lo, x, CKKS_DBG_IPROW_X);
-                row_fwd_regs(x, twf, R1 + (u32)src_row, lo, srow, q);
-                if (hoist_g) {        // permute inside the row: slot k takes source slot src(k)
-#pragma unroll
-                    for (int v = 0; v < 16; v++) srow[17 * lo + v] = x[v];
-                    __syncwarp();
-#pragma unroll
-                    for (int v = 0; v < 16; v++) {
-                        const u32 m = automorph_src((u32)(k0 + v), hoist_g, a.log_n) & 255u;
-                        x[v] = srow[m + (m >> 4)];
-                    }
-                    __syncwarp();
-                }
+                load16_chk(src + k0, x, CKKS_DBG_IPROW_CDIG);
             }
             u32 bv[16], av[16];
             load16_chk(bkey + ((size_t)j * a.n_primes + t) * n + k0, bv, CKKS_DBG_IPROW_KEY);
             if (gcnt > 1) {
-                const u32 *src = sa + (size_t)j * 16 * ROW_THREADS + threadIdx.x;
+                const u32 *s2 = sa + (size_t)j * 16 * ROW_THREADS + threadIdx.x;
 #pragma unroll
-                for (int v = 0; v < 16; v++) av[v] = src[v * ROW_THREADS];
+                for (int v = 0; v < 16; v++) av[v] = s2[v * ROW_THREADS];
             } else if (astore) {
                 load16_chk(astore + ((size_t)j * a.n_primes + t) * n + k0, av, CKKS_DBG_IPROW_KEY);
             } else {
@@ -625,8 +601,200 @@ k_ip_row(IpRowArgs a) {
             acc0[v] = csub(shoup_mul(acc0[v], pi.r64, pi.r64p, q), q);
             acc1[v] = csub(shoup_mul(acc1[v], pi.r64, pi.r64p, q), q);
         }
-        store16_chk(accb + (size_t)u * n + (size_t)row * 256 + 16 * lo, acc0, CKKS_DBG_IPROW_OUT);
-        store16_chk(accb + ((size_t)a.ext + u) * n + (size_t)row * 256 + 16 * lo, acc1, CKKS_DBG_IPROW_OUT);
+        store16_chk(accb + (size_t)u * n + k0, acc0, CKKS_DBG_IPROW_OUT);
+        store16_chk(accb + ((size_t)a.ext + u) * n + k0, acc1, CKKS_DBG_IPROW_OUT);
+    }
+}
+
+// ---- the inner product with one row per warp: 32 threads x 8 values per 256-point row
+// (k_ip_row8).  The forward row pass runs in three register rounds:
+//   A: m = lo + 32 u (u = 0..7), local stages 0..2;
+//   B: m = 32 (lo >> 2) + 4 u + (lo & 3), stages 3..5;
+//   C: m = 8 lo + u, stages 6..7,
+// local stage s pairing (m, m + 2^(7-s)) with twiddle (base << s) + (m >> (8 - s)), as the
+// 16-value rounds of fwd_top4 / fwd_low<8>.  The exchanges go through the row's 288 words of
+// shared memory at m + 4 (m >> 5) (A -> B) and m + (m >> 3) (B -> C), both free of bank conflicts.
+__device__ __forceinline__ int row8_x1(int m) { return m + 4 * (m >> 5); }
+__device__ __forceinline__ int row8_x2(int m) { return m + (m >> 3); }
+
+// x[u] = element lo + 32 u of the row (round A's input) -> canonical evaluation values of the
+// elements 8 lo + u
+__device__ __forceinline__ void row8_fwd(u32 (&x)[8], const tw_t *__restrict__ tw, u32 base, int lo, u32 *srow,
+                                         u32 q) {
+    const u32 two_q = 2 * q;
+#pragma unroll
+    for (int s = 0; s < 3; s++) {
+        const int d = 4 >> s;
+#pragma unroll
+        for (int g = 0; g < (1 << s); g++) {
+            const tw_t w = __ldg(tw + (base << s) + g);
+#pragma unroll
+            for (int i = 0; i < d; i++) ct_bfly(x[2 * d * g + i], x[2 * d * g + i + d], w.x, w.y, q, two_q);
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; u++) srow[row8_x1(lo + 32 * u)] = x[u];
+    __syncwarp();
+    const int a = lo >> 2, b = lo & 3;
+#pragma unroll
+    for (int u = 0; u < 8; u++) x[u] = srow[row8_x1(32 * a + 4 * u + b)];
+    __syncwarp();
+#pragma unroll
+    for (int s = 3; s < 6; s++) {
+        const int d = 4 >> (s - 3);
+#pragma unroll
+        for (int g = 0; g < (1 << (s - 3)); g++) {
+            const tw_t w = __ldg(tw + (base << s) + ((u32)a << (s - 3)) + g);
+#pragma unroll
+            for (int i = 0; i < d; i++) ct_bfly(x[2 * d * g + i], x[2 * d * g + i + d], w.x, w.y, q, two_q);
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; u++) srow[row8_x2(32 * a + 4 * u + b)] = x[u];
+    __syncwarp();
+#pragma unroll
+    for (int u = 0; u < 8; u++) x[u] = srow[row8_x2(8 * lo + u)];
+    __syncwarp();
+#pragma unroll
+    for (int s = 6; s < 8; s++) {
+        const int d = 1 << (7 - s);
+#pragma unroll
+        for (int g = 0; g < 8 / (2 * d); g++) {
+            const tw_t w = __ldg(tw + (base << s) + ((u32)lo << (s - 5)) + g);
+#pragma unroll
+            for (int i = 0; i < d; i++) ct_bfly(x[2 * d * g + i], x[2 * d * g + i + d], w.x, w.y, q, two_q);
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; u++) x[u] = csub(csub(x[u], two_q), q);
+}
+
+__device__ __forceinline__ void load8_chk(const u32 *p, u32 (&x)[8], int site) {
+    if (CKKS_SPAN(p, 8, site)) {
+        const uint4 *p4 = reinterpret_cast<const uint4 *>(p);
+        const uint4 t0 = p4[0], t1 = p4[1];
+        x[0] = t0.x; x[1] = t0.y; x[2] = t0.z; x[3] = t0.w; x[4] = t1.x; x[5] = t1.y; x[6] = t1.z; x[7] = t1.w;
+    } else {
+#pragma unroll
+        for (int v = 0; v < 8; v++) x[v] = 0u;
+    }
+}
+
+__device__ __forceinline__ void store8_chk(u32 *p, const u32 (&x)[8], int site) {
+    if (CKKS_SPAN(p, 8, site)) {
+        uint4 *p4 = reinterpret_cast<uint4 *>(p);
+        p4[0] = make_uint4(x[0], x[1], x[2], x[3]);
+        p4[1] = make_uint4(x[4], x[5], x[6], x[7]);
+    }
+}
+
+constexpr int IP8_ROWS = ROW_THREADS / 32;       // rows per block: one per warp
+
+// The inner product with the row pass fused in (every launch but a hoisted batch's over finished
+// rows): one 256-slot row per warp, a thread holding the 8 consecutive slots
+// k0 = 256 row + 8 lo .. + 7, so one ChaCha12 block per digit; 80 registers, 3 blocks of 8 warps
+// per SM.  Shared a half of a group: [digit][8][ROW_THREADS].
+__global__ void __launch_bounds__(ROW_THREADS, 3)
+k_ip_row8(IpRowArgs a) {
+    __shared__ u32 sm[IP8_ROWS * 288];
+    extern __shared__ u32 sa[];
+    const int n = 1 << a.log_n;
+    const int na = a.level + 1;
+    const int u = blockIdx.y;
+    const int g0 = a.grp_first[blockIdx.z], gcnt = a.grp_count[blockIdx.z];
+    const int t = u < na ? u : a.n_q + (u - na);
+    if (!CKKS_SPAN(a.pinfo + t, 1, CKKS_DBG_IPROW_TABLES) || !CKKS_SPAN(a.twf + (size_t)t * n, n, CKKS_DBG_IPROW_TABLES))
+        return;                                               // (the same for the whole block)
+    CKKS_POISON(sm, sizeof(sm));
+    CKKS_POISON_DYNAMIC(sa);
+    const PrimeInfo pi = a.pinfo[t];
+    const u32 q = pi.q, two_q = 2 * q;
+    const int r = threadIdx.x >> 5, lo = threadIdx.x & 31;
+    const int row = blockIdx.x * IP8_ROWS + r;
+    const u32 R1 = (u32)(n >> 8);
+    u32 *srow = sm + r * 288;
+    const int k0 = row * 256 + 8 * lo;               // first evaluation slot of this thread
+    const u32 blk = (u32)(k0 >> 3);                  // its ChaCha12 block
+    const tw_t *twf = a.twf + (size_t)t * n;
+    if (gcnt > 1) {                                  // the group's shared a half, once per digit
+        const int item = a.grp_item[g0];
+        for (int j = 0; j < a.beta; j++) {
+            u32 h[8];
+            u32 *dst = sa + (size_t)j * 8 * ROW_THREADS + threadIdx.x;
+            chacha_coeffs<false>(a.key[item], a.key_id[item], (u32)j, (u32)t, blk, pi, h);
+#pragma unroll
+            for (int v = 0; v < 8; v++) dst[v * ROW_THREADS] = h[v];
+        }
+        __syncthreads();
+    }
+    for (int it = 0; it < gcnt; it++) {
+        const int item = a.grp_item[g0 + it];
+        const u32 *xb = a.x + item * a.x_item;
+        const u32 *cdb = a.cdig + item * a.cdig_item;
+        u32 *accb = a.acc + item * a.acc_item;
+        const u32 *bkey = a.b[item];
+        const u32 *astore = a.a_stored[item];
+        const u32 hoist_g = a.hoist_g[item], cdig_g = a.cdig_g[item];
+        const int src_row = hoist_g ? (int)(automorph_src((u32)(row * 256), hoist_g, a.log_n) >> 8) : row;
+        u32 acc0[8], acc1[8];
+#pragma unroll
+        for (int v = 0; v < 8; v++) acc0[v] = acc1[v] = 0;
+        for (int j = 0; j < a.beta; j++) {
+            const bool in_digit = u < na && u >= j * a.alpha && u < min(j * a.alpha + a.alpha, na);
+            u32 x[8];
+            if (in_digit) {
+                const u32 *src = cdb + (size_t)u * n;
+                const u32 g = hoist_g ? hoist_g : cdig_g;
+                if (g) {
+                    const bool ok = CKKS_SPAN(src, n, CKKS_DBG_IPROW_CDIG);       // automorph_src < n
+#pragma unroll
+                    for (int v = 0; v < 8; v++) x[v] = ok ? src[automorph_src((u32)(k0 + v), g, a.log_n)] : 0u;
+                } else {
+                    load8_chk(src + k0, x, CKKS_DBG_IPROW_CDIG);
+                }
+            } else {
+                const u32 *src = xb + ((size_t)j * a.ext + u) * n + (size_t)src_row * 256;
+                const bool ok = CKKS_SPAN2(src + lo, src + lo + 32 * 7, CKKS_DBG_IPROW_X);
+#pragma unroll
+                for (int v = 0; v < 8; v++) x[v] = ok ? src[lo + 32 * v] : 0u;
+                row8_fwd(x, twf, R1 + (u32)src_row, lo, srow, q);
+                if (hoist_g) {        // permute inside the row: slot k takes source slot src(k)
+#pragma unroll
+                    for (int v = 0; v < 8; v++) srow[row8_x2(8 * lo + v)] = x[v];
+                    __syncwarp();
+#pragma unroll
+                    for (int v = 0; v < 8; v++) {
+                        const int m = (int)(automorph_src((u32)(k0 + v), hoist_g, a.log_n) & 255u);
+                        x[v] = srow[row8_x2(m)];
+                    }
+                    __syncwarp();
+                }
+            }
+            u32 bv[8], av[8];
+            load8_chk(bkey + ((size_t)j * a.n_primes + t) * n + k0, bv, CKKS_DBG_IPROW_KEY);
+            if (gcnt > 1) {
+                const u32 *src = sa + (size_t)j * 8 * ROW_THREADS + threadIdx.x;
+#pragma unroll
+                for (int v = 0; v < 8; v++) av[v] = src[v * ROW_THREADS];
+            } else if (astore) {
+                load8_chk(astore + ((size_t)j * a.n_primes + t) * n + k0, av, CKKS_DBG_IPROW_KEY);
+            } else {
+                chacha_coeffs<false>(a.key[item], a.key_id[item], (u32)j, (u32)t, blk, pi, av);
+            }
+#pragma unroll
+            for (int v = 0; v < 8; v++) {
+                acc0[v] = csub(acc0[v] + mont_mul(x[v], bv[v], q, pi.qinv), two_q);
+                acc1[v] = csub(acc1[v] + mont_mul(x[v], av[v], q, pi.qinv), two_q);
+            }
+        }
+        // undo the Montgomery factor 2^-32
+#pragma unroll
+        for (int v = 0; v < 8; v++) {
+            acc0[v] = csub(shoup_mul(acc0[v], pi.r64, pi.r64p, q), q);
+            acc1[v] = csub(shoup_mul(acc1[v], pi.r64, pi.r64p, q), q);
+        }
+        store8_chk(accb + (size_t)u * n + k0, acc0, CKKS_DBG_IPROW_OUT);
+        store8_chk(accb + ((size_t)a.ext + u) * n + k0, acc1, CKKS_DBG_IPROW_OUT);
     }
 }
 
