@@ -514,27 +514,36 @@ struct IpRowArgs {
     int grp_first[KS_MAXB], grp_count[KS_MAXB], grp_item[KS_MAXB];
 };
 
-// The inner product of a hoisted batch whose shared ModUp is already complete in the evaluation
-// domain (run_modup_rows transformed every non-digit limb of x once): every dt_j[u] is read through
-// kappa_{hoist_g} -- x for the non-digit limbs, the input polynomial for the digit limbs -- so no
-// item repeats the row pass.  16 rows x 16 threads per block, 16 consecutive slots per thread
-// (at 128 registers this layout runs hoisted batches faster than k_ip_row8's); groups as above,
-// the shared a half as [digit][16][ROW_THREADS].
+// The 16-slot inner product (16 rows x 16 threads per block, 16 consecutive slots and two
+// ChaCha12 blocks per thread, 128 registers).  XDONE = true is what runs now: a hoisted batch whose
+// shared ModUp already holds every non-digit limb in the evaluation domain (run_modup_rows
+// transformed them once); those rows are read like the digit limbs, through kappa_{hoist_g},
+// instead of being transformed again for every item.  XDONE = false, the same layout with the row
+// pass fused in, was the benchmark's kernel until k_ip_row8 replaced it and is no longer launched;
+// it stays in this template because the XDONE = true kernel compiled without it measured 1.5-3%
+// slower on the hoisted lines (same box).
+template <bool XDONE>
 __global__ void __launch_bounds__(ROW_THREADS)
-k_ip_hoisted(IpRowArgs a) {
+k_ip_row(IpRowArgs a) {
+    __shared__ u32 sm[16 * 272];
     extern __shared__ u32 sa[];                      // shared a half: [digit][16][ROW_THREADS]
     const int n = 1 << a.log_n;
     const int na = a.level + 1;
     const int u = blockIdx.y;
     const int g0 = a.grp_first[blockIdx.z], gcnt = a.grp_count[blockIdx.z];
     const int t = u < na ? u : a.n_q + (u - na);
-    if (!CKKS_SPAN(a.pinfo + t, 1, CKKS_DBG_IPROW_TABLES)) return;   // (the same for the whole block)
+    if (!CKKS_SPAN(a.pinfo + t, 1, CKKS_DBG_IPROW_TABLES) || !CKKS_SPAN(a.twf + (size_t)t * n, n, CKKS_DBG_IPROW_TABLES))
+        return;                                               // (the same for the whole block)
+    CKKS_POISON(sm, sizeof(sm));
     CKKS_POISON_DYNAMIC(sa);
     const PrimeInfo pi = a.pinfo[t];
     const u32 q = pi.q, two_q = 2 * q;
     const int r = threadIdx.x >> 4, lo = threadIdx.x & 15;
     const int row = blockIdx.x * 16 + r;
+    const u32 R1 = (u32)(n >> 8);
+    u32 *srow = sm + r * 272;
     const int k0 = row * 256 + 16 * lo;              // first evaluation slot of this thread
+    const tw_t *twf = a.twf + (size_t)t * n;
     if (gcnt > 1) {                                  // the group's shared a half, once per digit
         const int item = a.grp_item[g0];
         for (int j = 0; j < a.beta; j++) {
@@ -557,27 +566,46 @@ k_ip_hoisted(IpRowArgs a) {
         const u32 *bkey = a.b[item];
         const u32 *astore = a.a_stored[item];
         const u32 hoist_g = a.hoist_g[item], cdig_g = a.cdig_g[item];
+        // hoisted rotation: source row of this row under kappa_g
+        const int src_row = hoist_g ? (int)(automorph_src((u32)(row * 256), hoist_g, a.log_n) >> 8) : row;
         u32 acc0[16], acc1[16];
 #pragma unroll
         for (int v = 0; v < 16; v++) acc0[v] = acc1[v] = 0;
         for (int j = 0; j < a.beta; j++) {
             const bool in_digit = u < na && u >= j * a.alpha && u < min(j * a.alpha + a.alpha, na);
-            const u32 *src = in_digit ? cdb + (size_t)u * n : xb + ((size_t)j * a.ext + u) * n;
-            const u32 g = in_digit ? (hoist_g ? hoist_g : cdig_g) : hoist_g;
             u32 x[16];
-            if (g) {
-                const bool ok = CKKS_SPAN(src, n, CKKS_DBG_IPROW_CDIG);       // automorph_src < n
+            if (in_digit || XDONE) {
+                const u32 *src = in_digit ? cdb + (size_t)u * n : xb + ((size_t)j * a.ext + u) * n;
+                const u32 g = in_digit ? (hoist_g ? hoist_g : cdig_g) : hoist_g;
+                if (g) {
+                    const bool ok = CKKS_SPAN(src, n, CKKS_DBG_IPROW_CDIG);       // automorph_src < n
 #pragma unroll
-                for (int v = 0; v < 16; v++) x[v] = ok ? src[automorph_src((u32)(k0 + v), g, a.log_n)] : 0u;
+                    for (int v = 0; v < 16; v++) x[v] = ok ? src[automorph_src((u32)(k0 + v), g, a.log_n)] : 0u;
+                } else {
+                    load16_chk(src + k0, x, CKKS_DBG_IPROW_CDIG);
+                }
             } else {
-                load16_chk(src + k0, x, CKKS_DBG_IPROW_CDIG);
+                const u32 *src = xb + ((size_t)j * a.ext + u) * n + (size_t)src_row * 256;
+                load_row16_chk(src, lo, x, CKKS_DBG_IPROW_X);
+                row_fwd_regs(x, twf, R1 + (u32)src_row, lo, srow, q);
+                if (hoist_g) {        // permute inside the row: slot k takes source slot src(k)
+#pragma unroll
+                    for (int v = 0; v < 16; v++) srow[17 * lo + v] = x[v];
+                    __syncwarp();
+#pragma unroll
+                    for (int v = 0; v < 16; v++) {
+                        const u32 m = automorph_src((u32)(k0 + v), hoist_g, a.log_n) & 255u;
+                        x[v] = srow[m + (m >> 4)];
+                    }
+                    __syncwarp();
+                }
             }
             u32 bv[16], av[16];
             load16_chk(bkey + ((size_t)j * a.n_primes + t) * n + k0, bv, CKKS_DBG_IPROW_KEY);
             if (gcnt > 1) {
-                const u32 *s2 = sa + (size_t)j * 16 * ROW_THREADS + threadIdx.x;
+                const u32 *src = sa + (size_t)j * 16 * ROW_THREADS + threadIdx.x;
 #pragma unroll
-                for (int v = 0; v < 16; v++) av[v] = s2[v * ROW_THREADS];
+                for (int v = 0; v < 16; v++) av[v] = src[v * ROW_THREADS];
             } else if (astore) {
                 load16_chk(astore + ((size_t)j * a.n_primes + t) * n + k0, av, CKKS_DBG_IPROW_KEY);
             } else {
@@ -601,8 +629,8 @@ k_ip_hoisted(IpRowArgs a) {
             acc0[v] = csub(shoup_mul(acc0[v], pi.r64, pi.r64p, q), q);
             acc1[v] = csub(shoup_mul(acc1[v], pi.r64, pi.r64p, q), q);
         }
-        store16_chk(accb + (size_t)u * n + k0, acc0, CKKS_DBG_IPROW_OUT);
-        store16_chk(accb + ((size_t)a.ext + u) * n + k0, acc1, CKKS_DBG_IPROW_OUT);
+        store16_chk(accb + (size_t)u * n + (size_t)row * 256 + 16 * lo, acc0, CKKS_DBG_IPROW_OUT);
+        store16_chk(accb + ((size_t)a.ext + u) * n + (size_t)row * 256 + 16 * lo, acc1, CKKS_DBG_IPROW_OUT);
     }
 }
 
