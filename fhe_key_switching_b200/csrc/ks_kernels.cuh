@@ -407,9 +407,9 @@ __global__ void k_copy_digit_limbs(const u32 *c, u32 *dt, int log_n, int level, 
 }
 
 // ---------------------------------------------------------------- fused row kernels
-// Both kernels use the row-pass geometry of k_ntt_row (16 rows x 16 threads per block); at
-// the end of a forward row pass thread (r, lo) holds the 16 consecutive evaluation slots
-// k = 256*row + 16*lo + v, v = 0..15.
+// The 16-slot layout (k_ip_row): 16 rows x 16 threads per block; at the end of a forward row
+// pass (row_fwd_regs) thread (r, lo) holds the 16 consecutive evaluation slots
+// k = 256*row + 16*lo + v, v = 0..15.  The other row kernels hold one row per warp (ntt.cuh).
 
 __device__ __forceinline__ void load16_vec(const u32 *p, u32 (&x)[16]) {
     const uint4 *p4 = reinterpret_cast<const uint4 *>(p);
@@ -635,68 +635,7 @@ k_ip_row(IpRowArgs a) {
 }
 
 // ---- the inner product with one row per warp: 32 threads x 8 values per 256-point row
-// (k_ip_row8).  The forward row pass runs in three register rounds:
-//   A: m = lo + 32 u (u = 0..7), local stages 0..2;
-//   B: m = 32 (lo >> 2) + 4 u + (lo & 3), stages 3..5;
-//   C: m = 8 lo + u, stages 6..7,
-// local stage s pairing (m, m + 2^(7-s)) with twiddle (base << s) + (m >> (8 - s)), as the
-// 16-value rounds of fwd_top4 / fwd_low<8>.  The exchanges go through the row's 288 words of
-// shared memory at m + 4 (m >> 5) (A -> B) and m + (m >> 3) (B -> C), both free of bank conflicts.
-__device__ __forceinline__ int row8_x1(int m) { return m + 4 * (m >> 5); }
-__device__ __forceinline__ int row8_x2(int m) { return m + (m >> 3); }
-
-// x[u] = element lo + 32 u of the row (round A's input) -> canonical evaluation values of the
-// elements 8 lo + u
-__device__ __forceinline__ void row8_fwd(u32 (&x)[8], const tw_t *__restrict__ tw, u32 base, int lo, u32 *srow,
-                                         u32 q) {
-    const u32 two_q = 2 * q;
-#pragma unroll
-    for (int s = 0; s < 3; s++) {
-        const int d = 4 >> s;
-#pragma unroll
-        for (int g = 0; g < (1 << s); g++) {
-            const tw_t w = __ldg(tw + (base << s) + g);
-#pragma unroll
-            for (int i = 0; i < d; i++) ct_bfly(x[2 * d * g + i], x[2 * d * g + i + d], w.x, w.y, q, two_q);
-        }
-    }
-#pragma unroll
-    for (int u = 0; u < 8; u++) srow[row8_x1(lo + 32 * u)] = x[u];
-    __syncwarp();
-    const int a = lo >> 2, b = lo & 3;
-#pragma unroll
-    for (int u = 0; u < 8; u++) x[u] = srow[row8_x1(32 * a + 4 * u + b)];
-    __syncwarp();
-#pragma unroll
-    for (int s = 3; s < 6; s++) {
-        const int d = 4 >> (s - 3);
-#pragma unroll
-        for (int g = 0; g < (1 << (s - 3)); g++) {
-            const tw_t w = __ldg(tw + (base << s) + ((u32)a << (s - 3)) + g);
-#pragma unroll
-            for (int i = 0; i < d; i++) ct_bfly(x[2 * d * g + i], x[2 * d * g + i + d], w.x, w.y, q, two_q);
-        }
-    }
-#pragma unroll
-    for (int u = 0; u < 8; u++) srow[row8_x2(32 * a + 4 * u + b)] = x[u];
-    __syncwarp();
-#pragma unroll
-    for (int u = 0; u < 8; u++) x[u] = srow[row8_x2(8 * lo + u)];
-    __syncwarp();
-#pragma unroll
-    for (int s = 6; s < 8; s++) {
-        const int d = 1 << (7 - s);
-#pragma unroll
-        for (int g = 0; g < 8 / (2 * d); g++) {
-            const tw_t w = __ldg(tw + (base << s) + ((u32)lo << (s - 5)) + g);
-#pragma unroll
-            for (int i = 0; i < d; i++) ct_bfly(x[2 * d * g + i], x[2 * d * g + i + d], w.x, w.y, q, two_q);
-        }
-    }
-#pragma unroll
-    for (int u = 0; u < 8; u++) x[u] = csub(csub(x[u], two_q), q);
-}
-
+// (k_ip_row8), its forward row pass in registers (row8_fwd, ntt.cuh).
 __device__ __forceinline__ void load8_chk(const u32 *p, u32 (&x)[8], int site) {
     if (CKKS_SPAN(p, 8, site)) {
         const uint4 *p4 = reinterpret_cast<const uint4 *>(p);
@@ -716,7 +655,6 @@ __device__ __forceinline__ void store8_chk(u32 *p, const u32 (&x)[8], int site) 
     }
 }
 
-constexpr int IP8_ROWS = ROW_THREADS / 32;       // rows per block: one per warp
 
 // The inner product with the row pass fused in (every launch but a hoisted batch's over finished
 // rows): one 256-slot row per warp, a thread holding the 8 consecutive slots
@@ -724,7 +662,7 @@ constexpr int IP8_ROWS = ROW_THREADS / 32;       // rows per block: one per warp
 // per SM.  Shared a half of a group: [digit][8][ROW_THREADS].
 __global__ void __launch_bounds__(ROW_THREADS, 3)
 k_ip_row8(IpRowArgs a) {
-    __shared__ u32 sm[IP8_ROWS * 288];
+    __shared__ u32 sm[ROW_ROWS * ROW_SMEM];
     extern __shared__ u32 sa[];
     const int n = 1 << a.log_n;
     const int na = a.level + 1;
@@ -738,9 +676,9 @@ k_ip_row8(IpRowArgs a) {
     const PrimeInfo pi = a.pinfo[t];
     const u32 q = pi.q, two_q = 2 * q;
     const int r = threadIdx.x >> 5, lo = threadIdx.x & 31;
-    const int row = blockIdx.x * IP8_ROWS + r;
+    const int row = blockIdx.x * ROW_ROWS + r;
     const u32 R1 = (u32)(n >> 8);
-    u32 *srow = sm + r * 288;
+    u32 *srow = sm + r * ROW_SMEM;
     const int k0 = row * 256 + 8 * lo;               // first evaluation slot of this thread
     const u32 blk = (u32)(k0 >> 3);                  // its ChaCha12 block
     const tw_t *twf = a.twf + (size_t)t * n;
@@ -844,9 +782,11 @@ struct RowCombineArgs {
     u32 add_g[KS_MAXB];
 };
 
+// One 256-slot row per warp and 8 slots per thread (the layout of k_ip_row8): 32 registers, 8 blocks
+// per SM, so the latency of the three input streams is hidden by occupancy.
 __global__ void __launch_bounds__(ROW_THREADS)
 k_row_combine(RowCombineArgs a) {
-    __shared__ u32 sm[16 * 272];
+    __shared__ u32 sm[ROW_ROWS * ROW_SMEM];
     const int n = 1 << a.log_n;
     const int i = blockIdx.y, comp = blockIdx.z % a.n_comp, item = blockIdx.z / a.n_comp;
     const u32 add_g = a.add_g[item];
@@ -857,33 +797,35 @@ k_row_combine(RowCombineArgs a) {
     CKKS_POISON(sm, sizeof(sm));
     const PrimeInfo pi = a.pinfo[i];
     const u32 q = pi.q;
-    const int r = threadIdx.x >> 4, lo = threadIdx.x & 15;
-    const int row = blockIdx.x * 16 + r;
-    const int k0 = row * 256 + 16 * lo;
-    u32 *srow = sm + r * 272;
-    u32 x[16];
+    const int r = threadIdx.x >> 5, lo = threadIdx.x & 31;
+    const int row = blockIdx.x * ROW_ROWS + r;
+    const int k0 = row * 256 + 8 * lo;
+    u32 *srow = sm + r * ROW_SMEM;
+    u32 x[8];
     const u32 *src = a.conv + item * a.conv_item + ((size_t)comp * na + i) * n + (size_t)row * 256;
-    load_row16_chk(src, lo, x, CKKS_DBG_COMBINE_IN);
-    row_fwd_regs(x, a.twf + (size_t)i * n, (u32)(n >> 8) + (u32)row, lo, srow, q);
-    u32 ac[16];
-    load16_chk(a.acc + item * a.acc_item + ((size_t)comp * a.acc_comp_rows + i) * n + k0, ac, CKKS_DBG_COMBINE_IN);
+    const bool ok = CKKS_SPAN2(src + lo, src + lo + 32 * 7, CKKS_DBG_COMBINE_IN);
+#pragma unroll
+    for (int v = 0; v < 8; v++) x[v] = ok ? src[lo + 32 * v] : 0u;
+    row8_fwd(x, a.twf + (size_t)i * n, (u32)(n >> 8) + (u32)row, lo, srow, q);
+    u32 ac[8];
+    load8_chk(a.acc + item * a.acc_item + ((size_t)comp * a.acc_comp_rows + i) * n + k0, ac, CKKS_DBG_COMBINE_IN);
     const tw_t w = a.pinv[i];
 #pragma unroll
-    for (int v = 0; v < 16; v++) x[v] = csub(shoup_mul(ac[v] + q - x[v], w.x, w.y, q), q);
+    for (int v = 0; v < 8; v++) x[v] = csub(shoup_mul(ac[v] + q - x[v], w.x, w.y, q), q);
     if (comp < a.add_comps) {
         const u32 *ad = a.add + item * a.add_item + ((size_t)comp * na + i) * n;
-        u32 y[16];
+        u32 y[8];
         if (add_g) {
-            const bool ok = CKKS_SPAN(ad, n, CKKS_DBG_COMBINE_ADD);          // automorph_src < n
+            const bool okg = CKKS_SPAN(ad, n, CKKS_DBG_COMBINE_ADD);          // automorph_src < n
 #pragma unroll
-            for (int v = 0; v < 16; v++) y[v] = ok ? ad[automorph_src((u32)(k0 + v), add_g, a.log_n)] : 0u;
+            for (int v = 0; v < 8; v++) y[v] = okg ? ad[automorph_src((u32)(k0 + v), add_g, a.log_n)] : 0u;
         } else {
-            load16_chk(ad + k0, y, CKKS_DBG_COMBINE_ADD);
+            load8_chk(ad + k0, y, CKKS_DBG_COMBINE_ADD);
         }
 #pragma unroll
-        for (int v = 0; v < 16; v++) x[v] = csub(x[v] + y[v], q);
+        for (int v = 0; v < 8; v++) x[v] = csub(x[v] + y[v], q);
     }
-    store16_chk(a.out + item * a.out_item + ((size_t)comp * na + i) * n + k0, x, CKKS_DBG_COMBINE_OUT);
+    store8_chk(a.out + item * a.out_item + ((size_t)comp * na + i) * n + k0, x, CKKS_DBG_COMBINE_OUT);
 }
 
 // ---------------------------------------------------------------- baby-step giant-step transform

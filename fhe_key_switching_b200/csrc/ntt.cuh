@@ -229,17 +229,130 @@ k_ntt_col(NttArgs a) {
 }
 
 // ---------------------------------------------------------------- row pass (stages r1..log_n-1)
-// Block: 16 rows x 16 threads.  The register exchange stays inside a warp (2 rows per warp).
-// Shared layout per row: element m at m + (m >> 4) (row stride 272), conflict-free for both
-// the lo + 16u and the 16 lo + u patterns.
+// One 256-point row per warp: 32 threads x 8 values.  A row pass runs in three register rounds,
+//   A: m = lo + 32 u (u = 0..7), local stages 0..2;
+//   B: m = 32 (lo >> 2) + 4 u + (lo & 3), stages 3..5;
+//   C: m = 8 lo + u, stages 6..7,
+// local stage s pairing (m, m + 2^(7-s)) with twiddle (base << s) + (m >> (8 - s)) of the
+// bit-reversed table (base = N/256 + row); the inverse runs the rounds backwards (C, B, A).  The
+// exchanges go through the row's 288 words of shared memory at m + 4 (m >> 5) (A <-> B) and
+// m + (m >> 3) (B <-> C), both free of bank conflicts for the two patterns that use them.
 constexpr int ROW_THREADS = 256;
+constexpr int ROW_ROWS = ROW_THREADS / 32;       // rows per block: one per warp
+constexpr int ROW_SMEM = 288;                    // shared words per row
+
+__device__ __forceinline__ int row8_x1(int m) { return m + 4 * (m >> 5); }
+__device__ __forceinline__ int row8_x2(int m) { return m + (m >> 3); }
+
+// Forward: x[u] = element lo + 32 u of the row (round A's input) -> canonical evaluation values of
+// the elements 8 lo + u.
+__device__ __forceinline__ void row8_fwd(u32 (&x)[8], const tw_t *__restrict__ tw, u32 base, int lo, u32 *srow,
+                                         u32 q) {
+    const u32 two_q = 2 * q;
+#pragma unroll
+    for (int s = 0; s < 3; s++) {
+        const int d = 4 >> s;
+#pragma unroll
+        for (int g = 0; g < (1 << s); g++) {
+            const tw_t w = __ldg(tw + (base << s) + g);
+#pragma unroll
+            for (int i = 0; i < d; i++) ct_bfly(x[2 * d * g + i], x[2 * d * g + i + d], w.x, w.y, q, two_q);
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; u++) srow[row8_x1(lo + 32 * u)] = x[u];
+    __syncwarp();
+    const int a = lo >> 2, b = lo & 3;
+#pragma unroll
+    for (int u = 0; u < 8; u++) x[u] = srow[row8_x1(32 * a + 4 * u + b)];
+    __syncwarp();
+#pragma unroll
+    for (int s = 3; s < 6; s++) {
+        const int d = 4 >> (s - 3);
+#pragma unroll
+        for (int g = 0; g < (1 << (s - 3)); g++) {
+            const tw_t w = __ldg(tw + (base << s) + ((u32)a << (s - 3)) + g);
+#pragma unroll
+            for (int i = 0; i < d; i++) ct_bfly(x[2 * d * g + i], x[2 * d * g + i + d], w.x, w.y, q, two_q);
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; u++) srow[row8_x2(32 * a + 4 * u + b)] = x[u];
+    __syncwarp();
+#pragma unroll
+    for (int u = 0; u < 8; u++) x[u] = srow[row8_x2(8 * lo + u)];
+    __syncwarp();
+#pragma unroll
+    for (int s = 6; s < 8; s++) {
+        const int d = 1 << (7 - s);
+#pragma unroll
+        for (int g = 0; g < 8 / (2 * d); g++) {
+            const tw_t w = __ldg(tw + (base << s) + ((u32)lo << (s - 5)) + g);
+#pragma unroll
+            for (int i = 0; i < d; i++) ct_bfly(x[2 * d * g + i], x[2 * d * g + i + d], w.x, w.y, q, two_q);
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; u++) x[u] = csub(csub(x[u], two_q), q);
+}
+
+
+// Inverse: x[u] = element 8 lo + u of the row (round C's layout), inputs in [0, 2q) -> elements
+// lo + 32 u after the inverse stages 7..0, lazy in [0, 2q).
+__device__ __forceinline__ void row8_inv(u32 (&x)[8], const tw_t *__restrict__ tw, u32 base, int lo, u32 *srow,
+                                         u32 q) {
+    const u32 two_q = 2 * q;
+#pragma unroll
+    for (int s = 7; s >= 6; s--) {
+        const int d = 1 << (7 - s);
+#pragma unroll
+        for (int g = 0; g < 8 / (2 * d); g++) {
+            const tw_t w = __ldg(tw + (base << s) + ((u32)lo << (s - 5)) + g);
+#pragma unroll
+            for (int i = 0; i < d; i++) gs_bfly(x[2 * d * g + i], x[2 * d * g + i + d], w.x, w.y, q, two_q);
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; u++) srow[row8_x2(8 * lo + u)] = x[u];
+    __syncwarp();
+    const int a = lo >> 2, b = lo & 3;
+#pragma unroll
+    for (int u = 0; u < 8; u++) x[u] = srow[row8_x2(32 * a + 4 * u + b)];
+    __syncwarp();
+#pragma unroll
+    for (int s = 5; s >= 3; s--) {
+        const int d = 4 >> (s - 3);
+#pragma unroll
+        for (int g = 0; g < (1 << (s - 3)); g++) {
+            const tw_t w = __ldg(tw + (base << s) + ((u32)a << (s - 3)) + g);
+#pragma unroll
+            for (int i = 0; i < d; i++) gs_bfly(x[2 * d * g + i], x[2 * d * g + i + d], w.x, w.y, q, two_q);
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; u++) srow[row8_x1(32 * a + 4 * u + b)] = x[u];
+    __syncwarp();
+#pragma unroll
+    for (int u = 0; u < 8; u++) x[u] = srow[row8_x1(lo + 32 * u)];
+    __syncwarp();
+#pragma unroll
+    for (int s = 2; s >= 0; s--) {
+        const int d = 4 >> s;
+#pragma unroll
+        for (int g = 0; g < (1 << s); g++) {
+            const tw_t w = __ldg(tw + (base << s) + g);
+#pragma unroll
+            for (int i = 0; i < d; i++) gs_bfly(x[2 * d * g + i], x[2 * d * g + i + d], w.x, w.y, q, two_q);
+        }
+    }
+}
 
 // FWD: forward stages, canonical output.  !FWD: inverse stages (input gathered through
 // kappa_g when galois != 0), output lazy in [0, 2q).
 template <bool FWD>
 __global__ void __launch_bounds__(ROW_THREADS)
 k_ntt_row(NttArgs a) {
-    __shared__ u32 sm[16 * 272];
+    __shared__ u32 sm[ROW_ROWS * ROW_SMEM];
     int prime, k;
     size_t in_row, out_row;
     if (!map_job(a.map, blockIdx.y, prime, in_row, out_row, k)) return;
@@ -247,64 +360,44 @@ k_ntt_row(NttArgs a) {
     if (!CKKS_SPAN(a.pinfo + prime, 1, CKKS_DBG_NTT_TABLES) || !CKKS_SPAN(a.tw + (size_t)prime * n, n, CKKS_DBG_NTT_TABLES))
         return;                                               // (the same for the whole block)
     CKKS_POISON(sm, sizeof(sm));
-    const PrimeInfo pi = a.pinfo[prime];
-    const u32 q = pi.q, two_q = 2 * q;
+    const u32 q = a.pinfo[prime].q;
     const tw_t *tw = a.tw + (size_t)prime * n;
-    const int r = threadIdx.x >> 4, lo = threadIdx.x & 15;
-    const int row = blockIdx.x * 16 + r;
+    const int r = threadIdx.x >> 5, lo = threadIdx.x & 31;
+    const int row = blockIdx.x * ROW_ROWS + r;
     const u32 base = (u32)(n >> 8) + (u32)row;
     const u32 *src = a.in + blockIdx.z * a.in_item + in_row * n;
     u32 *dst = a.out + blockIdx.z * a.out_item + out_row * n + (size_t)row * 256;
     const u32 galois = a.galois[blockIdx.z];
-    u32 *srow = sm + r * 272;
-    u32 x[16];
+    u32 *srow = sm + r * ROW_SMEM;
+    u32 x[8];
     if (FWD) {
         const u32 *s = src + (size_t)row * 256;
-        const bool ok_in = CKKS_SPAN2(s + lo, s + lo + 16 * 15, CKKS_DBG_NTT_IN);
+        const bool ok_in = CKKS_SPAN2(s + lo, s + lo + 32 * 7, CKKS_DBG_NTT_IN);
 #pragma unroll
-        for (int u = 0; u < 16; u++) x[u] = ok_in ? s[lo + 16 * u] : 0u;
-        fwd_top4(x, tw, base, q, two_q);
-#pragma unroll
-        for (int u = 0; u < 16; u++) srow[lo + 17 * u] = x[u];
-        __syncwarp();
-#pragma unroll
-        for (int u = 0; u < 16; u++) x[u] = srow[17 * lo + u];
-        fwd_low<8>(x, tw, base, (u32)lo, q, two_q);
-        const bool ok_out = CKKS_SPAN(dst + 16 * lo, 16, CKKS_DBG_NTT_OUT);
-#pragma unroll
-        for (int v = 0; v < 4; v++) {
-            uint4 o;
-            o.x = csub(csub(x[4 * v + 0], two_q), q);
-            o.y = csub(csub(x[4 * v + 1], two_q), q);
-            o.z = csub(csub(x[4 * v + 2], two_q), q);
-            o.w = csub(csub(x[4 * v + 3], two_q), q);
-            if (ok_out) reinterpret_cast<uint4 *>(dst + 16 * lo)[v] = o;
+        for (int u = 0; u < 8; u++) x[u] = ok_in ? s[lo + 32 * u] : 0u;
+        row8_fwd(x, tw, base, lo, srow, q);
+        if (CKKS_SPAN(dst + 8 * lo, 8, CKKS_DBG_NTT_OUT)) {
+            uint4 *d4 = reinterpret_cast<uint4 *>(dst + 8 * lo);
+            d4[0] = make_uint4(x[0], x[1], x[2], x[3]);
+            d4[1] = make_uint4(x[4], x[5], x[6], x[7]);
         }
     } else {
         if (galois) {
             const bool ok_in = CKKS_SPAN(src, n, CKKS_DBG_NTT_IN);          // automorph_src < n
 #pragma unroll
-            for (int u = 0; u < 16; u++)
-                x[u] = ok_in ? src[automorph_src((u32)(row * 256 + 16 * lo + u), galois, a.log_n)] : 0u;
+            for (int u = 0; u < 8; u++)
+                x[u] = ok_in ? src[automorph_src((u32)(row * 256 + 8 * lo + u), galois, a.log_n)] : 0u;
         } else {
-            const uint4 *s4 = reinterpret_cast<const uint4 *>(src + (size_t)row * 256 + 16 * lo);
-            const bool ok_in = CKKS_SPAN(s4, 4, CKKS_DBG_NTT_IN);
-#pragma unroll
-            for (int v = 0; v < 4; v++) {
-                const uint4 t = ok_in ? s4[v] : make_uint4(0u, 0u, 0u, 0u);
-                x[4 * v] = t.x; x[4 * v + 1] = t.y; x[4 * v + 2] = t.z; x[4 * v + 3] = t.w;
-            }
+            const uint4 *s4 = reinterpret_cast<const uint4 *>(src + (size_t)row * 256 + 8 * lo);
+            const bool ok_in = CKKS_SPAN(s4, 2, CKKS_DBG_NTT_IN);
+            const uint4 t0 = ok_in ? s4[0] : make_uint4(0u, 0u, 0u, 0u);
+            const uint4 t1 = ok_in ? s4[1] : make_uint4(0u, 0u, 0u, 0u);
+            x[0] = t0.x; x[1] = t0.y; x[2] = t0.z; x[3] = t0.w; x[4] = t1.x; x[5] = t1.y; x[6] = t1.z; x[7] = t1.w;
         }
-        inv_low<8>(x, tw, base, (u32)lo, q, two_q);
+        row8_inv(x, tw, base, lo, srow, q);
+        if (CKKS_SPAN2(dst + lo, dst + lo + 32 * 7, CKKS_DBG_NTT_OUT)) {
 #pragma unroll
-        for (int u = 0; u < 16; u++) srow[17 * lo + u] = x[u];
-        __syncwarp();
-#pragma unroll
-        for (int u = 0; u < 16; u++) x[u] = srow[lo + 17 * u];
-        inv_top4(x, tw, base, q, two_q);
-        if (CKKS_SPAN2(dst + lo, dst + lo + 16 * 15, CKKS_DBG_NTT_OUT)) {
-#pragma unroll
-            for (int u = 0; u < 16; u++) dst[lo + 16 * u] = x[u];
+            for (int u = 0; u < 8; u++) dst[lo + 32 * u] = x[u];
         }
     }
 }
