@@ -591,7 +591,7 @@ def roofline(cfg, launches, total_ms, clk, batch, single_step_ms, launches_ov, t
 # DRAM bytes (read + write) per unit of a k_ip_row8 launch from an ncu capture, valid only for the
 # kernel sources it was taken on (sha-256 prefix of the device-code headers): after any change to
 # them the figure is reported as null until a new capture replaces it.
-IP_ROW_TRAFFIC = {"sources_sha16": "90ac1c3524a44979", "bytes_per_unit": (478.41e6 + 476.34e6) / 2 / 4,
+IP_ROW_TRAFFIC = {"sources_sha16": "93f7aa389dfb0d6d", "bytes_per_unit": (478.58e6 + 476.20e6) / 2 / 4,
                   "capture": "profiles/k_ip_row8_n16_full.md (dram__bytes read + write of two 4-unit launches)"}
 KERNEL_HEADERS = ("debug_bounds.cuh", "modarith.cuh", "chacha.cuh", "ntt.cuh", "ks_kernels.cuh")
 
