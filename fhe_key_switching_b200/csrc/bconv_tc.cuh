@@ -17,11 +17,14 @@
 // the forward NTT that always follows accepts.
 //
 // Tile: M = 128 coefficients (one per tensor-memory lane), K = 64 bytes (n_in <= 15), N = 4 x
-// (targets of the chunk), at most 128 columns.  A CTA of 128 threads (4 warps) stages the
-// chunk's B once, then loops over coefficient tiles: every thread transposes its coefficient's
-// n_in inputs into one A row in shared memory, thread 0 issues the two K = 32 MMAs and commits
-// them to an mbarrier, and every thread reads its row's accumulators back (tcgen05.ld), combines
-// them and stores its targets' outputs (one coalesced 128-byte row segment per warp and target).
+// (targets of the chunk), at most 256 columns, so that one chunk covers every target of a ModUp
+// digit or of ModDown at the supported sizes and each input is gathered once.  A CTA stages the
+// chunk's B once, then loops over coefficient tiles with warp-specialized roles (producers
+// transpose each coefficient's n_in inputs into one A row in shared memory, one lane issues the
+// two K = 32 MMAs, epilogue warps read the accumulators back with tcgen05.ld, combine them and
+// store one coalesced 128-byte row segment per warp and target; see k_bconv_tc).  Accumulators:
+// two of 128 columns when N <= 128, so that the MMAs of a tile overlap the read-back of the
+// previous one, else one of N columns.
 // Both operands are K-major without swizzle: core matrices of 8 rows x 16 bytes, stored
 // [16-byte K chunk][row][16 bytes], so the leading-dimension offset (next K chunk) is
 // rows x 16 bytes and the stride-dimension offset (next 8 rows) is 128 bytes.
@@ -31,13 +34,13 @@
 constexpr int TC_M = 128;                 // coefficients per tile = tensor-memory lanes
 constexpr int TC_K = 64;                  // K bytes (two MMAs of K = 32)
 constexpr int TC_MAX_IN = 15;             // 4 * 15 + 1 = 61 <= 64
-constexpr int TC_MAX_T = 32;              // targets per chunk: N = 4 T <= 128 columns per accumulator
+constexpr int TC_MAX_T = 64;              // targets per chunk: N = 4 T <= 256 columns (one MMA)
 constexpr int TC_THREADS = 288;           // 4 producer warps, 4 epilogue warps, 1 MMA warp
 constexpr int TC_TILES = 16;              // coefficient tiles per CTA, at most (BconvTcArgs::tiles)
 constexpr int TC_MIN_TILES = 4;           // smaller launches use the CUDA-core kernel
 constexpr int TC_STAGES = 5;              // A ring: the inputs of four tiles ahead are in flight
-constexpr int TC_COLS = 256;              // tensor-memory columns a CTA allocates: two accumulators
-// Dynamic shared memory per CTA: the A ring (5 x 8 KB) + B (<= 8 KB) + target records, padded so
+constexpr int TC_COLS = 256;              // tensor-memory columns a CTA allocates: the accumulator(s)
+// Dynamic shared memory per CTA: the A ring (5 x 8 KB) + B (<= 16 KB) + target records, padded so
 // that at most 2 CTAs share an SM (2 x 256 columns = all 512 columns of tensor memory: no CTA
 // waits in alloc; 3 x 77 KB would exceed the SM's 228 KB).
 constexpr size_t TC_SMEM = 76 * 1024;
@@ -166,6 +169,11 @@ __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
     const int Tc = min(a.tchunk, T - (hi - lo) - u0);             // targets of this chunk
     if (Tc <= 0) return;                                          // (uniform: before any barrier)
     const int N = (4 * Tc + 15) & ~15;
+    // two accumulators of 128 columns when N fits one, else a single one of N <= 256 columns
+    // (the MMA of tile k + 1 then waits until tile k's accumulator has been read)
+    const int nacc = N <= 128 ? 2 : 1;
+    auto acc_slot = [&](int k) { return nacc == 2 ? (k & 1) : 0; };
+    auto acc_phase = [&](int k) { return (u32)((nacc == 2 ? (k >> 1) : k) & 1); };
     auto target_pos = [&](int u) { const int idx = u0 + u; return idx < lo ? idx : idx + (hi - lo); };
     auto prime_of = [&](int kk) { return kk < a.map.split ? a.map.lo_base + kk : a.map.hi_base + (kk - a.map.split); };
     const int p0 = a.in_prime0 + g * a.in_prime_step;
@@ -270,10 +278,10 @@ __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
         const int q = warp - 4;
         const int row_i = q * 32 + lane;
         for (int k = 0; k < tiles; k++) {
-            if (!wait_or_abort(&acc_full[k & 1], (u32)((k >> 1) & 1))) break;
+            if (!wait_or_abort(&acc_full[acc_slot(k)], acc_phase(k))) break;
             tc_fence_after();
             const int nc = (blockIdx.x * tiles + k) * TC_M + row_i;
-            const u32 acc = tmem + ((u32)(q * 32) << 16) + (u32)((k & 1) * 128);
+            const u32 acc = tmem + ((u32)(q * 32) << 16) + (u32)(acc_slot(k) * 128);
             for (int c0 = 0; c0 < 4 * Tc; c0 += 16) {
                 u32 r[16];
                 tc_ld16(acc + (u32)c0, r);
@@ -291,7 +299,7 @@ __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
                 }
             }
             tc_fence_before();
-            tc_arrive(&acc_empty[k & 1]);
+            tc_arrive(&acc_empty[acc_slot(k)]);
         }
     } else if (lane == 0) {
         // ---- MMA issuer
@@ -300,22 +308,22 @@ __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
         int issued = 0;
         for (int k = 0; k < tiles; k++) {
             if (!wait_or_abort(&a_full[k % TC_STAGES], (u32)((k / TC_STAGES) & 1))) break;
-            if (k >= 2 && !wait_or_abort(&acc_empty[k & 1], (u32)(((k >> 1) - 1) & 1))) break;
+            if (k >= nacc && !wait_or_abort(&acc_empty[acc_slot(k)], acc_phase(k - nacc))) break;
             tc_fence_after();
             const u32 a_base = tc_smem_u32(a_stage(k));
-            const u32 d = tmem + (u32)((k & 1) * 128);
+            const u32 d = tmem + (u32)(acc_slot(k) * 128);
 #pragma unroll
             for (int s = 0; s < 2; s++)
                 tc_mma(d, tc_smem_desc(a_base + (u32)(2 * s * TC_M * 16), TC_M * 16, 128),
                        tc_smem_desc(b_base + (u32)(2 * s * N * 16), (u32)N * 16, 128), idesc, (u32)s);
-            tc_commit(&acc_full[k & 1]);
+            tc_commit(&acc_full[acc_slot(k)]);
             tc_commit(&a_empty[k % TC_STAGES]);
             issued = k + 1;
         }
         if (abort_flag) {
-            // the MMAs of the last two issued tiles may still run: wait for them (bounded)
-            for (int t = issued - 2; t < issued; t++)
-                if (t >= 0) (void)tc_wait_bounded(&acc_full[t & 1], (u32)((t >> 1) & 1));
+            // the MMAs of the last nacc issued tiles may still run: wait for them (bounded)
+            for (int t = issued - nacc; t < issued; t++)
+                if (t >= 0) (void)tc_wait_bounded(&acc_full[acc_slot(t)], acc_phase(t));
         }
     }
     __syncthreads();
