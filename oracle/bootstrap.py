@@ -316,3 +316,106 @@ def evalmod(ctx, ct: np.ndarray, level: int, scale: float, r: int, d: int, alpha
     lv -= 1
     assert lu >= lv
     return out, lv, Sp
+
+
+# ----------------------------------------------------------------------------- the whole bootstrap
+# ModRaise, CoeffToSlot, the split into real and imaginary halves, EvalMod on each half, their
+# recombination and SlotToCoeff (Cheon, Han, Kim, Kim, Song, Eurocrypt 2018, Sec. 4, with the
+# linear maps of Chen, Chillotti, Song, Eurocrypt 2019).  After CoeffToSlot the slots hold
+# t_k / q_0 = M_k / q_0 + i M_(k+n) / q_0 (bit-reversed order) for the raised plaintext
+# M = m + q_0 I.  The real half (z + conj z) / 2 and the imaginary half (z - conj z) / (2 i) are
+# formed with one conjugation; the 1/2 is folded into the last CoeffToSlot level's diagonals and the
+# division by i is a product with the monomial X^(N/2), which multiplies every slot by i.
+
+def mul_monomial_half(ctx, ct: np.ndarray, level: int) -> np.ndarray:
+    """X^(N/2) times every component of ct [n_comp][level+1][N] (evaluation domain).  Done in the
+    coefficient domain as the plain negacyclic product: coefficient a_k moves to k + N/2, and the
+    upper half wraps round to the bottom with a minus sign (X^N = -1).  Each slot root
+    w_j = zeta^(5^j) has w_j^(N/2) = exp(i pi 5^j / 2) = i (5^j = 1 mod 4), so the slots are
+    multiplied by i."""
+    ct = np.ascontiguousarray(ct, dtype=np.uint32)
+    h = ctx.n // 2
+    q = np.array(ctx.q[: level + 1], dtype=np.int64)[:, None]
+    out = np.empty_like(ct)
+    for comp in range(ct.shape[0]):
+        coef = ctx.ntt_inv(ct[comp], 0).astype(np.int64)
+        sh = np.empty_like(coef)
+        sh[:, h:] = coef[:, :h]
+        sh[:, :h] = (q - coef[:, h:]) % q
+        out[comp] = ctx.ntt_fwd(sh.astype(np.uint32), 0)
+    return out
+
+
+def _add(ctx, x, y, level):
+    q = np.array(ctx.q[: level + 1], dtype=np.uint64)[:, None]
+    return ((np.asarray(x, dtype=np.uint64) + np.asarray(y, dtype=np.uint64)) % q).astype(np.uint32)
+
+
+def _sub(ctx, x, y, level):
+    q = np.array(ctx.q[: level + 1], dtype=np.uint64)[:, None]
+    return ((np.asarray(x, dtype=np.uint64) + q - np.asarray(y, dtype=np.uint64)) % q).astype(np.uint32)
+
+
+def bootstrap_plans(log_n: int, levels: int, n1: int):
+    """The complex baby-step giant-step plans of CoeffToSlot and SlotToCoeff, `levels` levels each:
+    lists of (baby shifts, giant shifts, pt[giant][baby][n_slots]).  The last CoeffToSlot level
+    carries the factor 1/2 of the split into real and imaginary halves."""
+    ns = 1 << (log_n - 1)
+    c2s = []
+    for i, lens in enumerate(split_levels(log_n, levels, True)):
+        diags = level_diagonals(log_n, lens, True)
+        if i == levels - 1:
+            diags = {r: 0.5 * v for r, v in diags.items()}
+        c2s.append(bsgs_plan(diags, ns, n1))
+    s2c = [bsgs_plan(level_diagonals(log_n, lens, False), ns, n1) for lens in split_levels(log_n, levels, False)]
+    return c2s, s2c
+
+
+def bootstrap_levels(top: int, n_c2s: int, n_s2c: int, r: int, d: int):
+    """Levels at which the CoeffToSlot and SlotToCoeff transforms run, and the output level."""
+    c2s = [top - i for i in range(n_c2s)]
+    lz = top - n_c2s - (d + r + 3)
+    s2c = [lz - i for i in range(n_s2c)]
+    return c2s, s2c, lz - n_s2c
+
+
+def bootstrap(ctx, ct0: np.ndarray, top: int, alpha: int, c2s, s2c, keys: dict, conj_b, relin_b,
+              seed: bytes, r: int, d: int):
+    """Bootstraps ct0 ([2][1][N] or [2][N] at level 0).  c2s, s2c: per level (baby shifts, giant
+    shifts, plaintexts encoded at scale q_level over the extended basis, uint32
+    [giant][baby][ext][N]), at the levels of bootstrap_levels.  keys: Galois element -> b half of
+    the rotation key; conj_b: the key of g = 2N - 1; relin_b: the key of s^2 (key_id 0).
+    Returns (ciphertext [2][level_out+1][N], level_out, ratio): the output decodes at scale
+    ratio * Delta to the input's slots, Delta being the input's scale (its plaintext m becomes
+    sin(2 pi m / q_0) q_0 / (2 pi) ~ m, times ratio)."""
+    g_conj = 2 * ctx.n - 1
+    lv = top
+    ct = modraise(ctx, ct0, top)
+    for babies, giants, enc in c2s:
+        ct = linear_level(ctx, ct, lv, alpha, babies, giants, enc, keys, seed)
+        lv -= 1
+    cj = ctx.rotate(ct, lv, alpha, g_conj, conj_b, seed, g_conj)
+    re = _add(ctx, ct, cj, lv)
+    im = mul_monomial_half(ctx, _sub(ctx, cj, ct, lv), lv)
+    s_in = float(ctx.q[0])
+    re, lo, sp = evalmod(ctx, re, lv, s_in, r, d, alpha, relin_b, seed)
+    im, lo2, sp2 = evalmod(ctx, im, lv, s_in, r, d, alpha, relin_b, seed)
+    assert (lo, sp) == (lo2, sp2)
+    lv = lo
+    ct = _add(ctx, re, mul_monomial_half(ctx, im, lv), lv)
+    for babies, giants, enc in s2c:
+        ct = linear_level(ctx, ct, lv, alpha, babies, giants, enc, keys, seed)
+        lv -= 1
+    return ct, lv, sp / s_in
+
+
+def encoded_plans(ctx, plans, lvls):
+    """Encodes each complex plan at its level (scale q_level, extended basis).  Returns the list of
+    (baby shifts, giant shifts, encoded plaintexts) and the sorted Galois elements the plans rotate
+    by (1 excluded)."""
+    out, gal = [], set()
+    for (babies, giants, pt), lv in zip(plans, lvls):
+        gal.update(galois_of_shift(ctx, s) for s in babies + giants)
+        out.append((babies, giants, encode_plan(ctx, pt, lv, float(ctx.q[lv]))))
+    gal.discard(1)
+    return out, sorted(gal)

@@ -22,6 +22,11 @@ Workloads (named by ring size and shape):
 * ``n16-stream64`` -- the N=2^16 chain at level 20 with dnum=4: 64 independent ct x ct tensor
   products, each relinearised and then rotated by 2^(i mod 15); slots Gaussian sigma=1
   clipped to [-4, 4].
+* ``n12-boot``     -- a test chain for the whole bootstrap: N=2^12, 24 + 6 primes, dnum=4, a
+  level-0 ciphertext at scale 2^29 raised to level 23.  Its secret has Hamming weight 2, which is
+  insecure and chosen on purpose: the raised plaintext m + q_0 I then has |I| <= 1, inside the
+  range on which the 12-level EvalMod (degree 12, three double angles) is accurate, so that the
+  output can be decoded and compared with the input.
 """
 from __future__ import annotations
 
@@ -78,6 +83,7 @@ CONFIGS = {
                          hoisted=True, relin=False, seed=1004),
     "n16-stream64": Config("n16-stream64", 16, 36, 12, 4, 20, 192, 3.2, 28, "gauss_clip4",
                            rot_steps=_stream_steps(), n_pairs=64, seed=1005),
+    "n12-boot": Config("n12-boot", 12, 24, 6, 4, 23, 2, 3.2, 29, "uniform", relin=False, seed=1006),
 }
 
 
