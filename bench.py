@@ -752,11 +752,11 @@ def run_workload(args, local_rank):
         ks_per_step, rot_per_step = 0, 0
         ops, blocks = R * rescale_ops(cfg, lvl), 0
         nbytes = R * (2 * na + 2 * lvl) * limb
-    elif key == "bootstrap-steps":
-        # the bootstrapping steps this library has, in sequence, at N=2^16 (dnum 4, levels 35 -> 17):
-        # ModRaise to level 35, CoeffToSlot (3 levels), one conjugation, EvalMod on the real and the
-        # imaginary halves as one batch of two (degree 12, 3 double angles, 12 levels), SlotToCoeff
-        # (3 levels); synthetic plaintexts and keys (the cost is data independent)
+    elif key == "bootstrap":
+        # one whole bootstrap per step (ckks_bootstrap) at N=2^16, dnum 4, levels 0 -> 35 -> 17: ModRaise
+        # to level 35, CoeffToSlot (3 levels), the real/imaginary split (one conjugation), EvalMod on both
+        # halves as one batch of two (degree 12, 3 double angles, 12 levels), the recombination,
+        # SlotToCoeff (3 levels); synthetic plaintexts and keys (the cost is data independent)
         levels, n1, L = 3, 8, cfg.n_q - 1
         ns = n // 2
         halves_fwd = [1 << h for h in range(cfg.log_n - 2, -1, -1)]
@@ -777,7 +777,7 @@ def run_workload(args, local_rank):
                        for g_ in range(ms_[0] // n1, ms_[-1] // n1 + 1)]
                 lv_ = top - li
                 pt_ = res((q[:lv_ + 1] + p) * len(gg_) * len(bg_)).view(len(gg_), len(bg_), lv_ + 1 + cfg.n_p, n)
-                plan_.append((lv_, bg_, gg_, pt_, ks.ckks_bsgs_workspace(ctx, lv_, len(bg_), len(gg_), device=dev)))
+                plan_.append((lv_, bg_, gg_, pt_, None))
             return plan_
         c2s, s2c = dft_plan(L, True), dft_plan(L - 3 - 12, False)
         gk = {}
@@ -789,37 +789,19 @@ def run_workload(args, local_rank):
         k_conj = ks.make_evk(res(mods * nd).view(nd, len(mods), n), cfg.chacha_seed, gconj)
         k_rel = ks.make_evk(res(mods * nd).view(nd, len(mods), n), cfg.chacha_seed, 0)
         cts0 = [res(q[:1] * 2).view(2, 1, n) for _ in range(N_SETS)]
-        big = torch.empty((2, L + 1, n), dtype=torch.uint32, device=dev)
-        bufs = [torch.empty((2, L + 1, n), dtype=torch.uint32, device=dev) for _ in range(4)]
-        ws_mr = torch.empty(2 * n, dtype=torch.uint32, device=dev)
-        ws_ks = ctx.workspace(L, 1, device=dev)
-        ws_em = ks.ckks_evalmod_batch_workspace(ctx, L - 3, 2, device=dev)
-        pair = torch.empty((2, 2, L + 1, n), dtype=torch.uint32, device=dev)    # z and its conjugate
-        em_out = torch.empty((2, 2, L + 1, n), dtype=torch.uint32, device=dev)
 
-        def run_levels(plan_, src, final=None):
-            cur = src
-            for i_, (lv_, bg_, gg_, pt_, ws_l) in enumerate(plan_):
-                ks.ckks_bsgs(ctx, cur, lv_, bg_, [gk.get(g_) for g_ in bg_], gg_, [gk.get(g_) for g_ in gg_],
-                             pt_, bufs[0].view(-1)[: 2 * (lv_ + 1) * n].view(2, lv_ + 1, n), ws_l, stream)
-                last = i_ == len(plan_) - 1 and final is not None
-                dst = final if last else bufs[1 + (i_ & 1)].view(-1)[: 2 * lv_ * n].view(2, lv_, n)
-                ks.ckks_rescale(ctx, bufs[0].view(-1)[: 2 * (lv_ + 1) * n].view(2, lv_ + 1, n), lv_, dst, ws_ks,
-                                stream)
-                cur = dst
-            return cur
+        def plan_levels(plan_):
+            return [(bg_, [gk.get(g_) for g_ in bg_], gg_, [gk.get(g_) for g_ in gg_], pt_)
+                    for _, bg_, gg_, pt_, _ in plan_]
+        bplan = ks.BootstrapPlan(L, plan_levels(c2s), plan_levels(s2c), k_conj, k_rel, 3, 6)
+        ws_bt = ks.ckks_bootstrap_workspace(ctx, bplan, device=dev)
+        out = torch.empty((2, bplan.out_level + 1, n), dtype=torch.uint32, device=dev)
 
         def step(i):
-            ks.ckks_modraise(ctx, cts0[i % N_SETS], L, big, ws_mr, stream)
-            lz = L - 3
-            zz = pair.view(-1)[: 4 * (lz + 1) * n].view(2, 2, lz + 1, n)
-            run_levels(c2s, big, final=zz[0])
-            ks.ckks_rotate(ctx, zz[0], lz, gconj, k_conj, zz[1], ws_ks, stream)
-            lv_em, _ = ks.ckks_evalmod_batch(ctx, zz, lz, float(q[lz]), 3, 6, k_rel, em_out, ws_em, stream)
-            em = em_out.view(-1)[: 4 * (lv_em + 1) * n].view(2, 2, lv_em + 1, n)
-            run_levels(s2c, em[1])
-        ks_per_step = rot_per_step = (sum(sum(1 for g_ in bg_ + gg_ if g_ != 1) for _, bg_, gg_, _, _ in c2s + s2c)
-                                      + 1)
+            ks.ckks_bootstrap(ctx, cts0[i % N_SETS], bplan, out, ws_bt, stream)
+        # the transforms' rotations and the conjugation, plus EvalMod's d + r relinearisations per half
+        rot_per_step = sum(sum(1 for g_ in bg_ + gg_ if g_ != 1) for _, bg_, gg_, _, _ in c2s + s2c) + 1
+        ks_per_step = rot_per_step + 2 * (6 + 3)
         ops = blocks = nbytes = 0        # reported as a time only: its op model is not tabulated
     elif key == "coeff-to-slot":
         # CoeffToSlot of N=2^16 in 3 levels of 5 radix-2 stages: each level's 63 slot diagonals
@@ -927,11 +909,10 @@ def run_workload(args, local_rank):
             "ms_per_step": ms / args.steps, "steps": args.steps, "warmup": args.warmup}
     if key == "rescale":
         line["rescales_per_s"] = R / t_step
-    elif key == "bootstrap-steps":
-        line["ms_per_bootstrap_steps"] = t_step * 1e3
-        line["context"] = ("the EncryptedLLM summary (lpnh.cn page, Results) quotes 22-27 ms per whole bootstrap "
-                           "on an unnamed GPU; these are the steps this library has, not a complete bootstrap "
-                           "(the real/imaginary split and recombination are not timed)")
+    elif key == "bootstrap":
+        line["ms_per_bootstrap"] = t_step * 1e3
+        line["context"] = ("the EncryptedLLM summary (lpnh.cn page, Results) quotes 22-27 ms per bootstrap on an "
+                           "unnamed GPU with its own parameters; context only, not a target")
     elif key == "coeff-to-slot":
         line["ms_per_coeff_to_slot"] = t_step * 1e3
         line["context"] = ("the EncryptedLLM summary (lpnh.cn page, Results) quotes 22-27 ms per whole "
@@ -953,14 +934,14 @@ def run_workload(args, local_rank):
     print(json.dumps(line), flush=True)
 
 
-INFO_WORKLOADS = {"coeff-to-slot": "n16-bsgs32", "bootstrap-steps": "n16-stream64",
+INFO_WORKLOADS = {"coeff-to-slot": "n16-bsgs32", "bootstrap": "n16-stream64",
                   "n14-hoisted8": "n14-hoisted8", "n16-bsgs32": "n16-bsgs32", "n16-stream64": "n16-stream64",
                   "n16-stream64-rescale": "n16-stream64", "rescale": "n16-full", "bsgs": "n16-bsgs32",
                   "bsgs-n14": "n14-hoisted8"}
 INFO_DESCRIPTIONS = {
-    "bootstrap-steps": "N=2^16, 36+12 primes, dnum 4; step = ModRaise to level 35, CoeffToSlot (3 levels), "
-                       "a conjugation, EvalMod twice (12 levels each, degree 12, 3 double angles), "
-                       "SlotToCoeff (3 levels)",
+    "bootstrap": "N=2^16, 36+12 primes, dnum 4; step = one ckks_bootstrap from level 0: ModRaise to level 35, "
+                 "CoeffToSlot (3 levels), the real/imaginary split (a conjugation), EvalMod on both halves (12 "
+                 "levels, degree 12, 3 double angles), the recombination, SlotToCoeff (3 levels), output at level 17",
     "coeff-to-slot": "N=2^16, 36+12 primes, dnum 4, from level 24; step = CoeffToSlot in 3 levels of 5 radix-2 "
                      "stages, each an 8 baby x 8 giant step transform of 63 slot diagonals plus a rescale",
     "n14-hoisted8": "N=2^14, 12+4 primes, dnum 3, level 11; step = 8 units, each 8 hoisted rotations "
@@ -991,7 +972,7 @@ def info_cpu_baseline(key: str, max_seconds: float = 8.0):
     ct = W.uniform_residues(octx.q[:na] * 2, n, gen).reshape(2, na, n)
     b = W.uniform_residues(octx.mod * nd, n, gen).reshape(nd, len(octx.mod), n)
     seed = cfg.chacha_seed
-    if key in ("bsgs", "coeff-to-slot", "bootstrap-steps"):
+    if key in ("bsgs", "coeff-to-slot", "bootstrap"):
         return None                 # the oracle's plaintext sums take minutes at N=2^16
     if key == "n14-hoisted8":
         gs = [octx.galois(r) for r in cfg.rot_steps]
@@ -1187,7 +1168,8 @@ def main():
                     help="independent units per step (default 8 for n16-full, 64 for the N=2^12 lines)")
     ap.add_argument("--workload", default=CONFIG_KEY,
                     help="n16-full (benchmark line), or n12-dnum2 / n12-dnum4 / n14-hoisted8 / n16-bsgs32 / "
-                         "n16-stream64 / n16-stream64-rescale / rescale / bsgs / bsgs-n14 (informational lines)")
+                         "n16-stream64 / n16-stream64-rescale / rescale / bsgs / bsgs-n14 / coeff-to-slot / bootstrap "
+                         "(informational lines)")
     ap.add_argument("--streams", type=int, default=None,
                     help="CUDA streams the batch is split over, each running batch/streams units "
                          "(default 2 for an even batch, else 1)")

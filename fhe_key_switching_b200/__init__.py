@@ -46,6 +46,17 @@ class ckks_evk(ctypes.Structure):
     _fields_ = [("b", _vp), ("a", _vp), ("seed", ctypes.c_uint8 * 32), ("key_id", _cu)]
 
 
+class ckks_bsgs_level(ctypes.Structure):
+    _fields_ = [("n_baby", _ci), ("baby_galois", _u32p), ("baby_keys", ctypes.POINTER(ckks_evk)),
+                ("n_giant", _ci), ("giant_galois", _u32p), ("giant_keys", ctypes.POINTER(ckks_evk)), ("pt", _vp)]
+
+
+class ckks_bootstrap_plan(ctypes.Structure):
+    _fields_ = [("top_level", _ci), ("n_c2s", _ci), ("c2s", ctypes.POINTER(ckks_bsgs_level)), ("n_s2c", _ci),
+                ("s2c", ctypes.POINTER(ckks_bsgs_level)), ("conj_key", ctypes.POINTER(ckks_evk)),
+                ("relin_key", ctypes.POINTER(ckks_evk)), ("r", _ci), ("d", _ci)]
+
+
 _SIGS = {
     "ckks_gen_primes": (_ci, [_cu, _cu, _cu, _u32p, _u32p]),
     "ckks_ctx_create": (_ci, [ctypes.POINTER(ckks_params), ctypes.POINTER(_vp)]),
@@ -90,6 +101,10 @@ _SIGS = {
     "ckks_evalmod": (_ci, [_vp, _vp, _ci, ctypes.c_double, _ci, _ci, ctypes.POINTER(ckks_evk), _vp,
                            ctypes.POINTER(_ci), ctypes.POINTER(ctypes.c_double), _vp, _sz, _vp]),
     "ckks_modraise": (_ci, [_vp, _vp, _ci, _vp, _vp, _sz, _vp]),
+    "ckks_mul_i": (_ci, [_vp, _vp, _ci, _ci, _vp, _vp]),
+    "ckks_bootstrap_workspace_bytes": (_sz, [_vp, ctypes.POINTER(ckks_bootstrap_plan)]),
+    "ckks_bootstrap": (_ci, [_vp, _vp, ctypes.POINTER(ckks_bootstrap_plan), _vp, ctypes.POINTER(_ci),
+                             ctypes.POINTER(ctypes.c_double), _vp, _sz, _vp]),
     "ckks_encode": (_ci, [_vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double), ctypes.c_double,
                           _ci, _ci, _vp, _vp, _sz, _vp]),
     "ckks_int_probe": (_ci, [_ci, _ci, _ci, _vp, _vp, ctypes.POINTER(ctypes.c_float),
@@ -495,3 +510,52 @@ def conjugation_element(log_n: int) -> int:
     """Galois element of complex conjugation of the slots: 2N - 1 (X -> X^-1); its key has
     key_id 2N - 1 and it runs through ckks_rotate like any rotation."""
     return (2 << log_n) - 1
+
+
+def ckks_mul_i(ctx, ct, n_comp: int, level: int, out, stream=None):
+    """out = X^(N/2) ct: every slot times i."""
+    _check(_L.ckks_mul_i(ctx.handle, _ptr(ct), n_comp, level, _ptr(out), _stream(stream)), "ckks_mul_i")
+
+
+class BootstrapPlan:
+    """Holds a ckks_bootstrap_plan and the host arrays and tensors it points to.
+    c2s, s2c: per level (baby Galois elements, baby evks, giant Galois elements, giant evks, pt tensor),
+    None standing for the key of element 1; conj_evk, relin_evk: ckks_evk."""
+
+    def __init__(self, top_level: int, c2s, s2c, conj_evk, relin_evk, r: int, d: int):
+        empty = ckks_evk()
+        self._keep = []
+
+        def levels(lst):
+            arr = (ckks_bsgs_level * len(lst))()
+            for i, (bg, bk, gg, gk, pt) in enumerate(lst):
+                bga = (ctypes.c_uint32 * len(bg))(*bg)
+                gga = (ctypes.c_uint32 * len(gg))(*gg)
+                bka = (ckks_evk * len(bk))(*[e if e is not None else empty for e in bk])
+                gka = (ckks_evk * len(gk))(*[e if e is not None else empty for e in gk])
+                self._keep += [bga, gga, bka, gka, pt]
+                arr[i] = ckks_bsgs_level(len(bg), bga, bka, len(gg), gga, gka, _ptr(pt))
+            self._keep.append(arr)
+            return arr
+
+        self._conj, self._relin = conj_evk, relin_evk
+        self.plan = ckks_bootstrap_plan(top_level, len(c2s), levels(c2s), len(s2c), levels(s2c),
+                                        ctypes.pointer(self._conj), ctypes.pointer(self._relin), r, d)
+        self.out_level = top_level - len(c2s) - (d + r + 3) - len(s2c)
+
+
+def ckks_bootstrap_workspace(ctx, plan: BootstrapPlan, device=None):
+    import torch
+    nbytes = _L.ckks_bootstrap_workspace_bytes(ctx.handle, ctypes.byref(plan.plan))
+    if nbytes == 0:
+        raise CkksError(CKKS_ERR_ARG, "ckks_bootstrap_workspace_bytes")
+    return torch.empty((nbytes + 3) // 4, dtype=torch.uint32, device=device or "cuda")
+
+
+def ckks_bootstrap(ctx, ct, plan: BootstrapPlan, out, ws, stream=None):
+    """Bootstraps ct [2][1][N] into out [2][plan.out_level+1][N]; returns (out_level, ratio)."""
+    lv, ratio = _ci(), ctypes.c_double()
+    _check(_L.ckks_bootstrap(ctx.handle, _ptr(ct), ctypes.byref(plan.plan), _ptr(out), ctypes.byref(lv),
+                             ctypes.byref(ratio), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "ckks_bootstrap")
+    return lv.value, ratio.value

@@ -286,6 +286,63 @@ int ckks_evalmod_batch(ckks_ctx *ctx, int n, const uint32_t *ct, int level, doub
                        const ckks_evk *relin_key, uint32_t *out, int *out_level, double *out_scale, void *ws,
                        size_t ws_bytes, ckks_stream_t stream);
 
+/* Product with the monomial X^(N/2): every slot is multiplied by i, since each slot root
+ * zeta^(5^j) raised to N/2 is i (5^j = 1 mod 4).  Bootstrapping uses it to take the imaginary half of
+ * CoeffToSlot's output and to put it back (Cheon, Han, Kim, Kim, Song, Eurocrypt 2018; the pages give
+ * no construction).  In the evaluation domain it is a multiplication by w = psi^(N/2) on the first
+ * N/2 entries of every limb and by -w on the rest.  ct, out: [n_comp][level+1][N] (out may equal
+ * ct), n_comp in 1..3; errors as for ckks_add, and CKKS_ERR_ALIGN. */
+int ckks_mul_i(ckks_ctx *ctx, const uint32_t *ct, int n_comp, int level, uint32_t *out, ckks_stream_t stream);
+
+/* One level of a slot DFT for ckks_bootstrap: the arguments of one ckks_bsgs call (host arrays of
+ * n_baby and n_giant entries; pt on the device, [n_giant][n_baby][l+1+k][N] at the level the
+ * transform runs at, encoded at scale q_l so that the rescale after it keeps the scale). */
+typedef struct {
+    int n_baby;
+    const uint32_t *baby_galois;
+    const ckks_evk *baby_keys;
+    int n_giant;
+    const uint32_t *giant_galois;
+    const ckks_evk *giant_keys;
+    const uint32_t *pt;
+} ckks_bsgs_level;
+
+/* What ckks_bootstrap runs: ModRaise to top_level; n_c2s CoeffToSlot levels at top_level,
+ * top_level - 1, ...; EvalMod of degree 2 d with r double angles (d + r + 3 levels); n_s2c
+ * SlotToCoeff levels.  conj_key switches kappa_(2N-1)(s) -> s, relin_key s^2 -> s (key_id 0).  The
+ * CoeffToSlot diagonals carry the factor 1/2 of the split into real and imaginary halves. */
+typedef struct {
+    int top_level;
+    int n_c2s;
+    const ckks_bsgs_level *c2s;
+    int n_s2c;
+    const ckks_bsgs_level *s2c;
+    const ckks_evk *conj_key;
+    const ckks_evk *relin_key;
+    int r, d;
+} ckks_bootstrap_plan;
+
+/* CKKS bootstrapping (Cheon, Han, Kim, Kim, Song, Eurocrypt 2018; the linear maps as levels of the
+ * slot DFT, Chen, Chillotti, Song, Eurocrypt 2019; the pages name bootstrapping and its cost but give
+ * no construction): a ciphertext at level 0, ct [2][1][N], is raised to top_level (its plaintext
+ * becomes m + q_0 I); CoeffToSlot (each level one ckks_bsgs and one ckks_rescale) leaves the slots
+ * holding the raised coefficients over q_0, in bit-reversed order, at scale q_0; one conjugation
+ * splits them into the real half z + conj(z) and the imaginary half X^(N/2) (conj(z) - z); EvalMod
+ * (ckks_evalmod_batch on both halves) replaces each value x by sin(2 pi x) / (2 pi), which removes
+ * I; the halves are recombined as real + X^(N/2) imag; SlotToCoeff moves the values back into the
+ * coefficients.  The output decrypts to m (the input's message), scaled by *out_ratio: it decodes
+ * at the input's scale times *out_ratio.  It is exact where m is small against q_0, up to the
+ * approximation of EvalMod and the noise of the steps.
+ *   out: [2][*out_level+1][N] with *out_level = top_level - n_c2s - (d + r + 3) - n_s2c;
+ *   ws: ckks_bootstrap_workspace_bytes(ctx, plan) bytes (0 for a plan out of range).
+ * Errors: CKKS_ERR_ARG (null pointers, level counts outside 1..16, r outside 0..16, d outside 1..16,
+ * overlaps between the input, the output, the workspace and the plaintexts, and every error of the
+ * ckks_bsgs calls), CKKS_ERR_UNSUPPORTED (top_level above the chain or below the levels consumed),
+ * CKKS_ERR_ALIGN, CKKS_ERR_WORKSPACE. */
+size_t ckks_bootstrap_workspace_bytes(ckks_ctx *ctx, const ckks_bootstrap_plan *plan);
+int ckks_bootstrap(ckks_ctx *ctx, const uint32_t *ct, const ckks_bootstrap_plan *plan, uint32_t *out, int *out_level,
+                   double *out_ratio, void *ws, size_t ws_bytes, ckks_stream_t stream);
+
 /* Base-conversion engine (the results are the same residues either way; the bits of every
  * entry point's output are identical):
  *  CKKS_BCONV_TENSOR: the conversion as an exact 8-bit contraction on the tensor cores

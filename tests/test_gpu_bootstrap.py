@@ -183,3 +183,68 @@ def test_evalmod_parity_n16(ks_lib, oracle_mod):
     """EvalMod (degree 12, three double angles) at N=2^16, dnum 4, from level 35: bit for bit with
     the oracle, and decoding to sin(2 pi x) / (2 pi) within 2^-9."""
     _evalmod_case(ks_lib, oracle_mod, "n16-stream64", 35, 3, 6, True)
+
+
+def test_mul_i_parity(ks_lib, oracle_mod):
+    """ckks_mul_i (X^(N/2) in the evaluation domain: w or -w per half) against the oracle's
+    coefficient-domain negacyclic shift, bit for bit, on 3 components at level 7 of n12-boot."""
+    from oracle import bootstrap as bt
+    ks = ks_lib
+    cfg = W.CONFIGS["n12-boot"]
+    q, p = ks.ckks_gen_primes(cfg.log_n, cfg.n_q, cfg.n_p)
+    octx = oracle_mod.Ctx(cfg.log_n, cfg.n_q, cfg.n_p)
+    ctx = ks.Context(cfg.log_n, q, p, cfg.dnum)
+    lvl = 7
+    x = W.uniform_residues(q[: lvl + 1] * 3, cfg.n, W.rng(cfg.seed, W.TAG_SYNTH, 9500)).reshape(3, lvl + 1, cfg.n)
+    out = torch.empty((3, lvl + 1, cfg.n), dtype=torch.uint32, device="cuda")
+    ks.ckks_mul_i(ctx, _dev(x), 3, lvl, out)
+    assert np.array_equal(_host(out), bt.mul_monomial_half(octx, x, lvl))
+
+
+def test_bootstrap_parity_n12(ks_lib, oracle_mod):
+    """ckks_bootstrap on the n12-boot chain (level 0 -> 23 -> 5: CoeffToSlot and SlotToCoeff in 3
+    levels of 8 baby steps, EvalMod of degree 12 with three double angles) equals the oracle's
+    bootstrap bit for bit, twice in a row on one workspace; the output decodes to the input slots
+    (the oracle's own pin, tests/test_oracle_bootstrap.py)."""
+    from oracle import bootstrap as bt
+    from oracle.scenario import Scenario
+    ks = ks_lib
+    cfg = W.CONFIGS["n12-boot"]
+    sc = Scenario(cfg)
+    octx = sc.ctx
+    q, p = ks.ckks_gen_primes(cfg.log_n, cfg.n_q, cfg.n_p)
+    ctx = ks.Context(cfg.log_n, q, p, cfg.dnum)
+    r, d, levels, n1 = 3, 6, 3, 8
+    c2s_p, s2c_p = bt.bootstrap_plans(cfg.log_n, levels, n1)
+    lc, ls, lout = bt.bootstrap_levels(cfg.level, levels, levels, r, d)
+    c2s, g1 = bt.encoded_plans(octx, c2s_p, lc)
+    s2c, g2 = bt.encoded_plans(octx, s2c_p, ls)
+    keys = {g: sc.key(g) for g in sorted(set(g1) | set(g2))}
+    evks = {g: ks.make_evk(_dev(b), cfg.chacha_seed, g) for g, b in keys.items()}
+    g_conj = 2 * cfg.n - 1
+    conj_b, relin_b = sc.key(g_conj), sc.key(0)
+
+    def gpu_levels(plans):
+        out = []
+        for babies, giants, enc in plans:
+            bg = [bt.galois_of_shift(octx, s) for s in babies]
+            gg = [bt.galois_of_shift(octx, s) for s in giants]
+            out.append((bg, [evks.get(g) for g in bg], gg, [evks.get(g) for g in gg], _dev(enc)))
+        return out
+
+    plan = ks.BootstrapPlan(cfg.level, gpu_levels(c2s), gpu_levels(s2c),
+                            ks.make_evk(_dev(conj_b), cfg.chacha_seed, g_conj),
+                            ks.make_evk(_dev(relin_b), cfg.chacha_seed, 0), r, d)
+    assert plan.out_level == lout
+    ws = ks.ckks_bootstrap_workspace(ctx, plan)
+    out = torch.empty((2, lout + 1, cfg.n), dtype=torch.uint32, device="cuda")
+    for index in (0, 1):
+        z, ct = sc.ciphertext(index, level=0)
+        want, lv, ratio = bt.bootstrap(octx, ct, cfg.level, cfg.alpha, c2s, s2c, keys, conj_b, relin_b,
+                                       cfg.chacha_seed, r, d)
+        g_lv, g_ratio = ks.ckks_bootstrap(ctx, _dev(ct.reshape(2, 1, cfg.n)), plan, out, ws)
+        assert ks.ckks_sync_status(ctx, None, 10000) == ks.CKKS_OK
+        assert (g_lv, g_ratio) == (lv, ratio)
+        got = _host(out)
+        assert np.array_equal(got, want), index
+        assert np.max(np.abs(sc.decrypt_slots(got, lv, sc.scale * ratio) - z)) < 2.0 ** -6
