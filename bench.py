@@ -453,6 +453,60 @@ def key_limbs(cfg, level: int) -> int:
     return len(digit_sizes(cfg, level)) * (level + 1 + cfg.n_p)
 
 
+def bsgs_level_model(cfg, lv: int, bg, gg):
+    """One level of a slot DFT at level lv: the baby-step giant-step transform (one ModUp, the hoisted
+    baby inner products, the plaintext sums in PQ, one ModDown per giant step, the giant rotations,
+    the sum of the partials) and its rescale.  bg, gg: the Galois elements (1 = no rotation).
+    Returns (op-model int32 operations, ChaCha12 blocks, compulsory bytes: input, plaintexts, the
+    keys' b halves, output)."""
+    n, limb = cfg.n, cfg.n * 4
+    e_l, n_l = lv + 1 + cfg.n_p, lv + 1
+    nb_r, ng_r = sum(g_ != 1 for g_ in bg), sum(g_ != 1 for g_ in gg)
+    ops = (modup_ops(cfg, lv) + nb_r * ip_ops(cfg, lv) + len(gg) * len(bg) * 2 * e_l * n * MAC
+           + len(gg) * 2 * e_l * n * RED + len(gg) * moddown_ops(cfg, lv)
+           + ng_r * (keyswitch_ops(cfg, lv) + n_l * n * MADD) + len(gg) * 2 * n_l * n * MADD
+           + rescale_ops(cfg, lv))
+    blocks = (nb_r + ng_r) * chacha_blocks(cfg, lv)
+    nbytes = ((len(gg) * len(bg) * e_l + 2 * n_l + 2 * n_l + 2 * n_l + 2 * (n_l - 1)) * limb
+              + (nb_r + ng_r) * key_limbs(cfg, lv) * limb)
+    return ops, blocks, nbytes
+
+
+def evalmod_model(cfg, level: int, r: int, d: int, items: int):
+    """EvalMod (degree 2d Taylor polynomial by Horner in theta^2, r double angles) on `items`
+    ciphertexts that share the relinearisation key: (ops, ChaCha12 blocks, compulsory bytes: the
+    key's b half once per product; inputs and outputs are counted by the caller).  The key's
+    keystream is counted once per product, as the batched call regenerates it once."""
+    n = cfg.n
+    ops = blocks = nbytes = 0
+    l = level
+
+    def mult(l):
+        # the items' relinearisations regenerate the key's a half once (they share one keystream)
+        shared = (items - 1) * chacha_blocks(cfg, l) * CHACHA_BLOCK
+        return (items * (tensor_ops(cfg, l) + keyswitch_ops(cfg, l) + 2 * (l + 1) * n * MADD + rescale_ops(cfg, l))
+                - shared, chacha_blocks(cfg, l), key_limbs(cfg, l) * n * 4)
+
+    def cmul_rescale(l):
+        return items * (2 * (l + 1) * n * CMUL + rescale_ops(cfg, l))
+
+    def addc(l):
+        return items * (l + 1) * n * MADD
+    ops += cmul_rescale(l) + addc(l - 1)                  # theta
+    l -= 1
+    for k in range(d + r):                                # theta^2, d - 1 Horner steps, r double angles
+        if k == 1:                                        # the leading coefficient times u, rescale, + a_(d-1)
+            ops += cmul_rescale(l) + addc(l - 1)
+            l -= 1
+        o, b, kb = mult(l)
+        ops, blocks, nbytes = ops + o, blocks + b, nbytes + kb
+        l -= 1
+        if k > 0:                                         # + a_k, or (times 2) - 1 after a double angle
+            ops += addc(l) + (items * 2 * (l + 1) * n * CMUL if k >= d else 0)
+    ops += cmul_rescale(l)                                # times 1 / (2 pi)
+    return ops, blocks, nbytes
+
+
 def unit_model(cfg, level: int) -> dict:
     """One unit of the benchmark step (tensor, relinearisation, rotation): op-model int32 operations,
     ChaCha12 blocks and compulsory HBM bytes."""
@@ -802,7 +856,23 @@ def run_workload(args, local_rank):
         # the transforms' rotations and the conjugation, plus EvalMod's d + r relinearisations per half
         rot_per_step = sum(sum(1 for g_ in bg_ + gg_ if g_ != 1) for _, bg_, gg_, _, _ in c2s + s2c) + 1
         ks_per_step = rot_per_step + 2 * (6 + 3)
-        ops = blocks = nbytes = 0        # reported as a time only: its op model is not tabulated
+        # op model: ModRaise (inverse NTT of limb 0, lift and NTT into 36 limbs, both components),
+        # the six DFT levels, the conjugation, the split and the recombination, EvalMod on both
+        # halves; compulsory bytes: the input, plaintexts and keys (the levels' and EvalMod's), output
+        lz, lo = L - levels, L - levels - 12
+        ntt1 = limb_ntt_ops(cfg.log_n)
+        ops = 2 * (ntt1 + (L + 1) * (n * RED + ntt1))
+        blocks = 0
+        nbytes = 2 * limb + 2 * (bplan.out_level + 1) * limb + key_limbs(cfg, lz) * limb
+        for lv_, bg_, gg_, _, _ in c2s + s2c:
+            o_, b_, _ = bsgs_level_model(cfg, lv_, bg_, gg_)
+            ops, blocks = ops + o_, blocks + b_
+            nbytes += (len(gg_) * len(bg_) * (lv_ + 1 + cfg.n_p)
+                       + sum(g_ != 1 for g_ in bg_ + gg_) * key_limbs(cfg, lv_)) * limb
+        ops += keyswitch_ops(cfg, lz) + (lz + 1) * n * MADD + 2 * (lz + 1) * n * (2 * MADD + CMUL)
+        blocks += chacha_blocks(cfg, lz)
+        o_, b_, n_ = evalmod_model(cfg, lz, 3, 6, 2)
+        ops, blocks, nbytes = ops + o_ + 2 * (lo + 1) * n * (MADD + CMUL), blocks + b_, nbytes + n_
     elif key == "coeff-to-slot":
         # CoeffToSlot of N=2^16 in 3 levels of 5 radix-2 stages: each level's 63 slot diagonals
         # (shifts m s, |m| <= 31, s its smallest half-length) as 8 baby x 8 giant steps, then a
@@ -845,15 +915,8 @@ def run_workload(args, local_rank):
         ks_per_step = rot_per_step = sum(sum(1 for g_ in bg + gg if g_ != 1) for _, bg, gg, _, _ in plan)
         ops = blocks = nbytes = 0
         for lv, bg, gg, pt_l, _ in plan:
-            e_l, n_l = lv + 1 + cfg.n_p, lv + 1
-            nb_r, ng_r = sum(g_ != 1 for g_ in bg), sum(g_ != 1 for g_ in gg)
-            ops += (modup_ops(cfg, lv) + nb_r * ip_ops(cfg, lv) + len(gg) * len(bg) * 2 * e_l * n * MAC
-                    + len(gg) * 2 * e_l * n * RED + len(gg) * moddown_ops(cfg, lv)
-                    + ng_r * (keyswitch_ops(cfg, lv) + n_l * n * MADD) + len(gg) * 2 * n_l * n * MADD
-                    + rescale_ops(cfg, lv))
-            blocks += (nb_r + ng_r) * chacha_blocks(cfg, lv)
-            nbytes += (len(gg) * len(bg) * e_l + 2 * n_l + 2 * n_l + 2 * n_l + 2 * (n_l - 1)) * limb \
-                + (nb_r + ng_r) * key_limbs(cfg, lv) * limb
+            o_, b_, n_ = bsgs_level_model(cfg, lv, bg, gg)
+            ops, blocks, nbytes = ops + o_, blocks + b_, nbytes + n_
     else:                                          # bsgs, bsgs-n14
         n1, n2 = 16, 18
         baby = [1] + [ks.galois_element(cfg.log_n, k) for k in range(1, n1)]

@@ -97,3 +97,20 @@ def test_compulsory_bytes_per_unit():
     # at least the two input ciphertexts, the two keys' b halves and the output
     na, ext, beta = cfg.level + 1, cfg.level + 1 + cfg.n_p, -(-(cfg.level + 1) // cfg.alpha)
     assert b >= (4 * na + 2 * beta * ext + 2 * na) * limb
+
+
+def test_evalmod_model_counts_the_products_and_the_shared_keystream():
+    """EvalMod of degree 2d with r double angles makes d + r ciphertext products (each a tensor, a
+    relinearisation and a rescale); items that share the key regenerate its keystream once."""
+    cfg = W.CONFIGS["n16-stream64"]
+    lvl, r, d = 32, 3, 6
+    o1, b1, k1 = bench.evalmod_model(cfg, lvl, r, d, 1)
+    o2, b2, k2 = bench.evalmod_model(cfg, lvl, r, d, 2)
+    levels = range(lvl - 1, lvl - 1 - (d + r + 1), -1)
+    prod_levels = [lvl - 1] + list(range(lvl - 3, lvl - 3 - (d - 1 + r), -1))
+    assert len(prod_levels) == d + r and min(levels) >= 0
+    assert b1 == b2 == sum(bench.chacha_blocks(cfg, l) for l in prod_levels)
+    assert k1 == k2 == sum(bench.key_limbs(cfg, l) for l in prod_levels) * cfg.n * 4
+    chacha = b1 * bench.CHACHA_BLOCK
+    assert o2 == 2 * o1 - chacha
+    assert o1 > sum(bench.keyswitch_ops(cfg, l) for l in prod_levels)
