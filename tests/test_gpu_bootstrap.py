@@ -248,3 +248,45 @@ def test_bootstrap_parity_n12(ks_lib, oracle_mod):
         got = _host(out)
         assert np.array_equal(got, want), index
         assert np.max(np.abs(sc.decrypt_slots(got, lv, sc.scale * ratio) - z)) < 2.0 ** -6
+
+
+def test_bootstrap_rejects_bad_plans(ks_lib):
+    """ckks_bootstrap's argument checks: a plan that consumes more levels than the top level has
+    (CKKS_ERR_UNSUPPORTED), level counts outside 1..16 and an output overlapping the input
+    (CKKS_ERR_ARG), a short workspace (CKKS_ERR_WORKSPACE); nothing runs on the GPU for any of them."""
+    ks = ks_lib
+    cfg = W.CONFIGS["n12-boot"]
+    q, p = ks.ckks_gen_primes(cfg.log_n, cfg.n_q, cfg.n_p)
+    ctx = ks.Context(cfg.log_n, q, p, cfg.dnum)
+    n, nd = cfg.n, -(-cfg.n_q // cfg.alpha)
+    gen = W.rng(cfg.seed, W.TAG_SYNTH, 9600)
+    mods = q + p
+    evk = ks.make_evk(_dev(W.uniform_residues(mods * nd, n, gen).reshape(nd, len(mods), n)), cfg.chacha_seed, 0)
+    conj = ks.make_evk(_dev(W.uniform_residues(mods * nd, n, gen).reshape(nd, len(mods), n)), cfg.chacha_seed,
+                       2 * n - 1)
+
+    def level(lv):
+        pt = _dev(W.uniform_residues(q[: lv + 1] + p, n, gen)).reshape(1, 1, lv + 1 + cfg.n_p, n)
+        return ([1], [None], [1], [None], pt)
+
+    ct = _dev(W.uniform_residues([q[0]] * 2, n, gen)).reshape(2, 1, n)
+
+    def call(plan, out=None, ws_bytes=None):
+        lv, ratio = ks._ci(), ks.ctypes.c_double()
+        need = ks._L.ckks_bootstrap_workspace_bytes(ctx.handle, ks.ctypes.byref(plan.plan))
+        ws = torch.empty(max(need, 1 << 20) // 4 + 64, dtype=torch.uint32, device="cuda")
+        o = out if out is not None else torch.empty((2, 24, n), dtype=torch.uint32, device="cuda")
+        nb = ws.numel() * 4 if ws_bytes is None else ws_bytes
+        return need, ks._L.ckks_bootstrap(ctx.handle, ks._ptr(ct), ks.ctypes.byref(plan.plan), ks._ptr(o),
+                                          ks.ctypes.byref(lv), ks.ctypes.byref(ratio), ks._ptr(ws), nb, None)
+
+    # 1 + (1 + 0 + 3) + 1 = 6 levels from top level 5
+    need, rc = call(ks.BootstrapPlan(5, [level(5)], [level(0)], conj, evk, 0, 1))
+    assert need == 0 and rc == ks.CKKS_ERR_UNSUPPORTED
+    ok = ks.BootstrapPlan(23, [level(23)], [level(18)], conj, evk, 0, 1)
+    need, rc = call(ok, ws_bytes=1024)
+    assert need > 0 and rc == ks.CKKS_ERR_WORKSPACE
+    empty = ks.BootstrapPlan(23, [], [level(18)], conj, evk, 0, 1)
+    assert call(empty)[1] == ks.CKKS_ERR_ARG
+    assert call(ok, out=ct.view(-1)[: 2 * n].view(2, 1, n))[1] == ks.CKKS_ERR_ARG
+    assert ks.ckks_sync_status(ctx, None, 10000) == ks.CKKS_OK
