@@ -19,10 +19,11 @@
 // Tile: M = 128 coefficients (one per tensor-memory lane), K = 64 bytes (n_in <= 15), N = 4 x
 // (targets of the chunk), at most 256 columns, so that one chunk covers every target of a ModUp
 // digit or of ModDown at the supported sizes and each input is gathered once.  A CTA stages the
-// chunk's B once, then loops over coefficient tiles with warp-specialized roles (producers
-// transpose each coefficient's n_in inputs into one A row in shared memory, one lane issues the
-// two K = 32 MMAs, epilogue warps read the accumulators back with tcgen05.ld, combine them and
-// store one coalesced 128-byte row segment per warp and target; see k_bconv_tc).  Accumulators:
+// chunk's B once, then loops over coefficient tiles with warp-specialized roles (one producer
+// thread brings each tile's n_in input rows of 512 bytes into a staging ring with bulk copies,
+// producer warps transpose each coefficient's n_in inputs into one A row in shared memory, one
+// lane issues the two K = 32 MMAs, epilogue warps read the accumulators back with tcgen05.ld,
+// combine them and store one coalesced 128-byte row segment per warp and target; see k_bconv_tc).  Accumulators:
 // two of 128 columns when N <= 128, so that the MMAs of a tile overlap the read-back of the
 // previous one, else one of N columns.
 // Both operands are K-major without swizzle: core matrices of 8 rows x 16 bytes, stored
@@ -40,11 +41,12 @@ constexpr int TC_TILES = 16;              // coefficient tiles per CTA, at most 
 constexpr int TC_MIN_TILES = 4;           // smaller launches use the CUDA-core kernel
 constexpr int TC_STAGES = 5;              // A ring: the inputs of four tiles ahead are in flight
 constexpr int TC_COLS = 256;              // tensor-memory columns a CTA allocates: the accumulator(s)
-// Dynamic shared memory per CTA: the A ring (5 x 8 KB) + B (<= 16 KB) + target records, padded so
-// that at most 2 CTAs share an SM (2 x 256 columns = all 512 columns of tensor memory: no CTA
-// waits in alloc; 3 x 77 KB would exceed the SM's 228 KB).
-constexpr size_t TC_SMEM = 76 * 1024;
+// Dynamic shared memory per CTA: the A ring (5 x 8 KB) + B (<= 16 KB) + target records + the input
+// staging ring (5 x 7.5 KB), at most 2 CTAs per SM (2 x 256 columns = all 512 columns of tensor
+// memory: no CTA waits in alloc; 3 x 96 KB would exceed the SM's 228 KB).
+constexpr size_t TC_SMEM = 96 * 1024;
 constexpr int TC_A_BYTES = 4 * TC_M * 16;  // one A stage: [4 K chunks][128 rows][16 B]
+constexpr int TC_RAW_BYTES = TC_MAX_IN * TC_M * 4;   // one staging stage: [input row][128 words]
 
 struct BconvTcArgs {
     const u32 *y;            // input rows
@@ -101,15 +103,6 @@ __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence:
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-// 4-byte asynchronous copy global -> shared (completed by cp.async.wait_group)
-__device__ __forceinline__ void tc_cp_async4(void *dst, const void *src) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(tc_smem_u32(dst)), "l"(src) : "memory");
-}
-__device__ __forceinline__ void tc_cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void tc_cp_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
-__device__ __forceinline__ void tc_cp_wait2() { asm volatile("cp.async.wait_group 2;" ::: "memory"); }
-__device__ __forceinline__ void tc_cp_wait4() { asm volatile("cp.async.wait_group 4;" ::: "memory"); }
-
 // Bounded wait for `phase` of `bar` in which the waiting thread sleeps in try_wait (up to a
 // microsecond per try, the suspend-time hint) instead of spinning; false after 1 s of the
 // global timer or the try-count backstop.
@@ -125,31 +118,36 @@ __device__ __forceinline__ bool tc_wait_bounded(u64 *bar, u32 phase) {
     }
     return false;
 }
-__device__ __forceinline__ void tc_cp_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
-// Included by ks_kernels.cuh after the mbarrier helpers (mbar_init, mbar_wait_bounded,
-// CKKS_DEV_ERR_WAIT), which the kernel below uses.
+// Included by ks_kernels.cuh after the mbarrier and bulk-copy helpers (mbar_init, mbar_expect_tx,
+// bulk_load, CKKS_DEV_ERR_WAIT), which the kernel below uses.
 __device__ __forceinline__ void tc_arrive(u64 *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(tc_smem_u32(bar)) : "memory");
 }
 constexpr int TC_B_OFF = TC_STAGES * TC_A_BYTES;                          // B after the A ring
 constexpr int TC_REC_OFF = TC_B_OFF + 4 * (4 * TC_MAX_T) * 16;            // per-target records after B
-static_assert(TC_REC_OFF + TC_MAX_T * 16 <= (int)TC_SMEM, "tensor-core conversion: shared memory");
-static_assert(TC_STAGES == 5, "the producer loop waits with cp.async.wait_group 4");
+constexpr int TC_RAW_OFF = TC_REC_OFF + TC_MAX_T * 16;                    // input staging ring after them
+static_assert(TC_RAW_OFF % 128 == 0 && TC_RAW_BYTES % 16 == 0, "tensor-core conversion: staging alignment");
+static_assert(TC_RAW_OFF + TC_STAGES * TC_RAW_BYTES <= (int)TC_SMEM, "tensor-core conversion: shared memory");
 
-// Roles: warps 0-3 produce the A tiles (thread t owns row t: 4-byte cp.async copies of its
-// coefficient's inputs, then the centred-lift count), warp 8 (one lane) issues the MMAs, warps
-// 4-7 read the accumulators back and store the outputs.  They meet on mbarriers only:
+// Roles: warps 0-3 produce the A tiles (thread 0 also issues the bulk copies of every tile's input
+// rows into the staging ring, TC_STAGES tiles ahead; thread t then transposes coefficient t's
+// inputs into row t of the A tile and appends the centred-lift count), warp 8 (one lane) issues
+// the MMAs, warps 4-7 read the accumulators back and store the outputs.  They meet on mbarriers
+// only:
+//   raw_full[s] (thread 0's expect_tx + the copies' bytes)  staging stage s holds tile k's inputs;
+//   raw_empty[s](128 producer arrivals)   every producer has read staging stage s;
 //   a_full[s]   (128 producer arrivals)  stage s holds tile k's A;
 //   a_empty[s]  (tcgen05.commit)          the MMA of the stage's tile is done with it;
 //   acc_full[b] (tcgen05.commit)          accumulator b holds tile k's G;
 //   acc_empty[b](128 epilogue arrivals)   accumulator b has been read.
 // Every wait is bounded: on expiry the CTA's abort flag and the device error word are set and
-// every role leaves its loop; the MMA warp then waits (bounded) for its MMAs in flight before the
-// tensor memory is freed.
+// every role leaves its loop; thread 0 then waits (bounded) for the copies it issued and the MMA
+// warp for its MMAs in flight, before the CTA ends and the tensor memory is freed.
 __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
     extern __shared__ __align__(1024) unsigned char tc_sm[];
     __shared__ __align__(8) u64 a_full[TC_STAGES], a_empty[TC_STAGES], acc_full[2], acc_empty[2];
+    __shared__ __align__(8) u64 raw_full[TC_STAGES], raw_empty[TC_STAGES];
     __shared__ u32 tmem_base;
     __shared__ volatile int abort_flag;
     __shared__ u32 half_s[TC_MAX_IN];
@@ -204,17 +202,15 @@ __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
         }
         reinterpret_cast<uint4 *>(Bs)[(size_t)kc * N + col] = v;
     }
-    if (tid < TC_M)          // words n_in + 1 .. 15 of every row stay zero (the copies never write them)
-        for (int st = 0; st < TC_STAGES; st++) {
-            u32 *row = reinterpret_cast<u32 *>(tc_sm + (size_t)st * TC_A_BYTES + (size_t)tid * 16);
-            for (int i = n_in + 1; i < 16; i++) row[(i >> 2) * (TC_M * 4) + (i & 3)] = 0u;
-        }
     if (warp == 8) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                      ::"r"(tc_smem_u32(&tmem_base)), "r"(TC_COLS) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
         if (lane == 0) {
-            for (int st = 0; st < TC_STAGES; st++) { mbar_init(&a_full[st], TC_M); mbar_init(&a_empty[st], 1); }
+            for (int st = 0; st < TC_STAGES; st++) {
+                mbar_init(&a_full[st], TC_M); mbar_init(&a_empty[st], 1);
+                mbar_init(&raw_full[st], 1); mbar_init(&raw_empty[st], TC_M);
+            }
             for (int b = 0; b < 2; b++) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], TC_M); }
             abort_flag = 0;
             asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -235,44 +231,63 @@ __global__ void __launch_bounds__(TC_THREADS) k_bconv_tc(BconvTcArgs a) {
         return true;
     };
     if (warp < 4) {
-        // ---- producers: row tid of every tile, TC_STAGES - 1 tiles of copies in flight
+        // ---- producers: row tid of every tile; thread 0 keeps TC_STAGES tiles of copies in flight
         const int row_i = tid;
-        auto finish = [&](int k) {                                // tile k's copies have landed
-            uint4 *row4 = reinterpret_cast<uint4 *>(a_stage(k) + (size_t)row_i * 16);
-            u32 w[16];
-#pragma unroll
-            for (int kc = 0; kc < 4; kc++) {
-                const uint4 v4 = row4[kc * TC_M];
-                w[4 * kc] = v4.x; w[4 * kc + 1] = v4.y; w[4 * kc + 2] = v4.z; w[4 * kc + 3] = v4.w;
-            }
-            u32 vcount = 0;
-#pragma unroll
-            for (int i = 0; i < TC_MAX_IN; i++)
-                if (i < n_in) vcount += w[i] > half_s[i] ? 1u : 0u;
-            reinterpret_cast<u32 *>(row4)[(n_in >> 2) * (TC_M * 4) + (n_in & 3)] = vcount;
-            tc_fence_async_smem();                                // visible to the tensor cores
-            tc_arrive(&a_full[k % TC_STAGES]);
+        auto raw_stage = [&](int t) { return tc_sm + TC_RAW_OFF + (size_t)(t % TC_STAGES) * TC_RAW_BYTES; };
+        auto issue = [&](int t) {                                 // thread 0: tile t's input rows
+            u64 *bar = &raw_full[t % TC_STAGES];
+            unsigned char *dst = raw_stage(t);
+            const u32 *src = yb + (size_t)(blockIdx.x * tiles + t) * TC_M;
+#ifdef CKKS_DEBUG_BOUNDS
+            // a row outside the registered regions is not copied, and the stage expects its bytes less
+            u32 okm = 0, bytes = 0;
+            for (int i = 0; i < n_in; i++)
+                if (CKKS_SPAN(src + (size_t)i * n, TC_M, CKKS_DBG_TC_IN)) { okm |= 1u << i; bytes += TC_M * 4; }
+            mbar_expect_tx(bar, bytes);
+            for (int i = 0; i < n_in; i++)
+                if ((okm >> i) & 1u) bulk_load(dst + (size_t)i * TC_M * 4, src + (size_t)i * n, TC_M * 4, bar);
+#else
+            mbar_expect_tx(bar, (u32)(n_in * TC_M * 4));
+            for (int i = 0; i < n_in; i++) bulk_load(dst + (size_t)i * TC_M * 4, src + (size_t)i * n, TC_M * 4, bar);
+#endif
         };
+        int issued = 0;
+        if (tid == 0)
+            for (; issued < TC_STAGES && issued < tiles; issued++) issue(issued);
         int k = 0;
         for (; k < tiles; k++) {
-            if (k >= TC_STAGES && !wait_or_abort(&a_empty[k % TC_STAGES], (u32)(((k / TC_STAGES) - 1) & 1))) break;
-            const u32 *src = yb + (blockIdx.x * tiles + k) * TC_M + row_i;
-            unsigned char *row = a_stage(k) + (size_t)row_i * 16;
-            const bool ok_in = CKKS_SPAN2(src, src + (size_t)(n_in - 1) * n, CKKS_DBG_TC_IN);
+            const int st = k % TC_STAGES;
+            const u32 ph = (u32)((k / TC_STAGES) & 1);
+            if (k >= TC_STAGES && !wait_or_abort(&a_empty[st], ph ^ 1u)) break;
+            if (!wait_or_abort(&raw_full[st], ph)) break;
+            const u32 *raw = reinterpret_cast<const u32 *>(raw_stage(k));
+            u32 w[16];
+            u32 vcount = 0;
 #pragma unroll
-            for (int i = 0; i < TC_MAX_IN; i++) {
-                if (i < n_in && ok_in) tc_cp_async4(row + (i >> 2) * (TC_M * 16) + (i & 3) * 4, src);
-                src += n;
+            for (int i = 0; i < 16; i++) {
+                w[i] = 0u;
+                if (i < n_in) {
+                    w[i] = raw[i * TC_M + row_i];
+                    vcount += w[i] > half_s[i] ? 1u : 0u;
+                }
             }
-            tc_cp_commit();
-            if (k >= TC_STAGES - 1) {
-                tc_cp_wait4();                                    // tile k - 4 has landed
-                finish(k - (TC_STAGES - 1));
+#pragma unroll
+            for (int i = 0; i < 16; i++)
+                if (i == n_in) w[i] = vcount;
+            uint4 *row4 = reinterpret_cast<uint4 *>(a_stage(k) + (size_t)row_i * 16);
+#pragma unroll
+            for (int kc = 0; kc < 4; kc++) row4[kc * TC_M] = make_uint4(w[4 * kc], w[4 * kc + 1], w[4 * kc + 2], w[4 * kc + 3]);
+            tc_fence_async_smem();                                // visible to the tensor cores
+            tc_arrive(&a_full[st]);
+            tc_arrive(&raw_empty[st]);
+            if (tid == 0 && issued < tiles) {                     // refill this staging stage
+                if (!wait_or_abort(&raw_empty[st], ph)) break;
+                tc_fence_async_smem();                            // the reads above before the copies' writes
+                issue(issued++);
             }
         }
-        tc_cp_wait0();
-        if (k == tiles)
-            for (int t = max(0, tiles - (TC_STAGES - 1)); t < tiles; t++) finish(t);
+        if (tid == 0 && abort_flag)                               // copies still in flight: wait (bounded)
+            for (int t = k; t < issued; t++) (void)tc_wait_bounded(&raw_full[t % TC_STAGES], (u32)((t / TC_STAGES) & 1));
     } else if (warp < 8) {
         // ---- epilogue: lanes 32 (warp - 4) .. + 31 of each accumulator
         const int q = warp - 4;
