@@ -873,6 +873,7 @@ def run_workload(args, local_rank):
         blocks += chacha_blocks(cfg, lz)
         o_, b_, n_ = evalmod_model(cfg, lz, 3, 6, 2)
         ops, blocks, nbytes = ops + o_ + 2 * (lo + 1) * n * (MADD + CMUL), blocks + b_, nbytes + n_
+        extra["_boot_level"] = (c2s[0][0], c2s[0][1], c2s[0][2])
     elif key == "coeff-to-slot":
         # CoeffToSlot of N=2^16 in 3 levels of 5 radix-2 stages: each level's 63 slot diagonals
         # (shifts m s, |m| <= 31, s its smallest half-length) as 8 baby x 8 giant steps, then a
@@ -989,11 +990,12 @@ def run_workload(args, local_rank):
         line["key_switches_per_step"] = ks_per_step
     if ops:
         line["path_roofline"] = dict(path_roofline(ops, blocks, nbytes, t_step, peaks), per="one step")
+    boot_level = extra.pop("_boot_level", None)
     line.update(extra)
     line["int_peaks"] = int_peaks_summary(peaks)
     line["clocks"] = clk
     if not args.no_cpu_baseline:
-        line["cpu_baseline"] = info_cpu_baseline(key)
+        line["cpu_baseline"] = info_cpu_baseline(key, ops_step=ops, boot_level=boot_level)
     print(json.dumps(line), flush=True)
 
 
@@ -1020,9 +1022,11 @@ INFO_DESCRIPTIONS = {
 }
 
 
-def info_cpu_baseline(key: str, max_seconds: float = 8.0):
+def info_cpu_baseline(key: str, max_seconds: float = 8.0, ops_step: float = 0.0, boot_level=None):
     """The oracle on a bounded sample of an informational line's step (synthetic residues; the cost
-    is data independent), in the line's own unit."""
+    is data independent), in the line's own unit.  For the whole bootstrap the sample is its first
+    CoeffToSlot level (boot_level: its level and Galois elements) and one EvalMod half, and the
+    step's time is estimated from the sample by the op model (ops_step: the step's count)."""
     import numpy as np
     import oracle
 
@@ -1035,7 +1039,29 @@ def info_cpu_baseline(key: str, max_seconds: float = 8.0):
     ct = W.uniform_residues(octx.q[:na] * 2, n, gen).reshape(2, na, n)
     b = W.uniform_residues(octx.mod * nd, n, gen).reshape(nd, len(octx.mod), n)
     seed = cfg.chacha_seed
-    if key in ("bsgs", "coeff-to-slot", "bootstrap"):
+    if key == "bootstrap":
+        from oracle import bootstrap as obt
+        lz = cfg.n_q - 1 - 3                            # EvalMod's input level in the bootstrap
+        ctz = W.uniform_residues(octx.q[:lz + 1] * 2, n, gen).reshape(2, lz + 1, n)
+        lv, bg, gg = boot_level
+        ct_l = W.uniform_residues(octx.q[:lv + 1] * 2, n, gen).reshape(2, lv + 1, n)
+        ext_l = lv + 1 + cfg.n_p
+        pt = W.uniform_residues((octx.q[:lv + 1] + octx.p) * len(gg) * len(bg), n, gen).reshape(
+            len(gg), len(bg), ext_l, n)
+        bk = [None if g_ == 1 else (b, g_) for g_ in bg]
+        gk = [None if g_ == 1 else (b, g_) for g_ in gg]
+        t0 = time.perf_counter()
+        octx.rescale(octx.bsgs(ct_l, lv, cfg.alpha, bg, bk, gg, gk, pt, seed), lv)
+        obt.evalmod(octx, ctz, lz, float(octx.q[0]), 3, 6, cfg.alpha, b, seed)
+        dt = time.perf_counter() - t0
+        ratio = ops_step / (evalmod_model(cfg, lz, 3, 6, 1)[0] + bsgs_level_model(cfg, lv, bg, gg)[0])
+        return {"value": dt * ratio * 1e3, "unit": "ms per bootstrap (estimate)", "cores": _omp_threads(),
+                "kind": "oracle",
+                "sample": f"the first CoeffToSlot level (level {lv}, {len(bg)} baby x {len(gg)} giant steps, "
+                          f"rescale) and one EvalMod half (9 products, level {lz} -> {lz - 12}) on synthetic "
+                          f"residues, {dt:.2f} s, scaled by the op model's ratio of the whole bootstrap to them "
+                          f"({ratio:.2f}); plain C oracle with OpenMP over limbs"}
+    if key in ("bsgs", "coeff-to-slot"):
         return None                 # the oracle's plaintext sums take minutes at N=2^16
     if key == "n14-hoisted8":
         gs = [octx.galois(r) for r in cfg.rot_steps]

@@ -206,10 +206,23 @@ def test_bootstrap_parity_n12(ks_lib, oracle_mod):
     levels of 8 baby steps, EvalMod of degree 12 with three double angles) equals the oracle's
     bootstrap bit for bit, twice in a row on one workspace; the output decodes to the input slots
     (the oracle's own pin, tests/test_oracle_bootstrap.py)."""
+    _bootstrap_case(ks_lib, "n12-boot", (0, 1))
+
+
+@pytest.mark.slow
+def test_bootstrap_parity_n16(ks_lib, oracle_mod):
+    """The benchmark's bootstrap shape at full size: N=2^16, 36+12 primes, dnum 4, level 0 -> 35 ->
+    17 (CoeffToSlot and SlotToCoeff in 3 levels of 8 baby x 8 giant steps, EvalMod of degree 12 with
+    three double angles), bit for bit with the oracle, and decoding to the input slots (measured
+    2^-8.7 at most with the oracle; the oracle takes minutes here)."""
+    _bootstrap_case(ks_lib, "n16-boot", (0,))
+
+
+def _bootstrap_case(ks_lib, key, indices):
     from oracle import bootstrap as bt
     from oracle.scenario import Scenario
     ks = ks_lib
-    cfg = W.CONFIGS["n12-boot"]
+    cfg = W.CONFIGS[key]
     sc = Scenario(cfg)
     octx = sc.ctx
     q, p = ks.ckks_gen_primes(cfg.log_n, cfg.n_q, cfg.n_p)
@@ -238,7 +251,7 @@ def test_bootstrap_parity_n12(ks_lib, oracle_mod):
     assert plan.out_level == lout
     ws = ks.ckks_bootstrap_workspace(ctx, plan)
     out = torch.empty((2, lout + 1, cfg.n), dtype=torch.uint32, device="cuda")
-    for index in (0, 1):
+    for index in indices:
         z, ct = sc.ciphertext(index, level=0)
         want, lv, ratio = bt.bootstrap(octx, ct, cfg.level, cfg.alpha, c2s, s2c, keys, conj_b, relin_b,
                                        cfg.chacha_seed, r, d)

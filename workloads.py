@@ -27,6 +27,8 @@ Workloads (named by ring size and shape):
   insecure and chosen on purpose: the raised plaintext m + q_0 I then has |I| <= 1, inside the
   range on which the 12-level EvalMod (degree 12, three double angles) is accurate, so that the
   output can be decoded and compared with the input.
+* ``n16-boot``     -- the same on the N=2^16 chain of n16-full with dnum=4 (the benchmark's bootstrap
+  shape): level 0 -> 35 -> 17, secret of Hamming weight 2.
 """
 from __future__ import annotations
 
@@ -84,6 +86,7 @@ CONFIGS = {
     "n16-stream64": Config("n16-stream64", 16, 36, 12, 4, 20, 192, 3.2, 28, "gauss_clip4",
                            rot_steps=_stream_steps(), n_pairs=64, seed=1005),
     "n12-boot": Config("n12-boot", 12, 24, 6, 4, 23, 2, 3.2, 29, "uniform", relin=False, seed=1006),
+    "n16-boot": Config("n16-boot", 16, 36, 12, 4, 35, 2, 3.2, 29, "uniform", relin=False, seed=1007),
 }
 
 
