@@ -789,9 +789,13 @@ def run_workload(args, local_rank):
             ks.ckks_rotate_batch(ctx, r2, lr, gs, ev, out, ws, stream)
         ks_per_step, rot_per_step = 2 * P_, P_
         nr = lr + 1
-        ops = P_ * (tensor_ops(cfg, lvl) + ksw + 2 * na * n * MADD + keyswitch_ops(cfg, lr) + nr * n * MADD
-                    + (rescale_ops(cfg, lvl) if rs else 0))
-        blocks = P_ * (chacha_blocks(cfg, lvl) + chacha_blocks(cfg, lr))
+        # the keystreams counted once per distinct key and step (one relinearisation key, 15 rotation
+        # keys), like the key bytes below: the items that share a key need its a half only once
+        n_rk = len(set(gs))
+        ops = (P_ * (tensor_ops(cfg, lvl) + ksw + 2 * na * n * MADD + keyswitch_ops(cfg, lr) + nr * n * MADD
+                     + (rescale_ops(cfg, lvl) if rs else 0))
+               - ((P_ - 1) * chacha_blocks(cfg, lvl) + (P_ - n_rk) * chacha_blocks(cfg, lr)) * CHACHA_BLOCK)
+        blocks = chacha_blocks(cfg, lvl) + n_rk * chacha_blocks(cfg, lr)
         # per call, each key once (one relinearisation key, 15 rotation keys)
         nbytes = (P_ * (7 * na + 3 * na + 2 * na + (2 * na + 2 * nr if rs else 0) + 2 * nr + 2 * nr) * limb
                   + kl + len(steps_g) * key_limbs(cfg, lr) * limb)
