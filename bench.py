@@ -747,9 +747,12 @@ def run_workload(args, local_rank):
             ks.ckks_tensor_batch(ctx, U, x, y, lvl, d, stream)
             ks.ckks_relin_batch(ctx, d, lvl, [k_rel] * U, rl, ws_b, stream)
         ks_per_step, rot_per_step = U * (R + 1), U * R
-        ops = U * (modup_ops(cfg, lvl) + R * (ip_ops(cfg, lvl) + moddown_ops(cfg, lvl) + na * n * MADD)
-                   + tensor_ops(cfg, lvl) + ksw + 2 * na * n * MADD)
-        blocks = U * (R + 1) * chacha_blocks(cfg, lvl)
+        # the units share the 8 rotation keys and the relinearisation key: their keystreams are
+        # counted once per step, like their key bytes
+        ops = (U * (modup_ops(cfg, lvl) + R * (ip_ops(cfg, lvl) + moddown_ops(cfg, lvl) + na * n * MADD)
+                    + tensor_ops(cfg, lvl) + ksw + 2 * na * n * MADD)
+               - (U - 1) * (R + 1) * chacha_blocks(cfg, lvl) * CHACHA_BLOCK)
+        blocks = (R + 1) * chacha_blocks(cfg, lvl)
         nbytes = U * (2 * na * limb + R * 2 * na * limb + 7 * na * limb + 5 * na * limb) + (R + 1) * kl
     elif key == "n16-bsgs32":
         cts = [res(q[:na] * 2).view(2, na, n) for _ in range(N_SETS)]
