@@ -737,13 +737,14 @@ def run_workload(args, local_rank):
         rot = torch.empty((U, R, 2, na, n), dtype=torch.uint32, device=dev)
         d = torch.empty((U, 3, na, n), dtype=torch.uint32, device=dev)
         rl = torch.empty((U, 2, na, n), dtype=torch.uint32, device=dev)
-        ws_h = [ctx.workspace(lvl, R, device=dev) for _ in range(U)]
+        ws_h = ctx.workspace(lvl, U * R, device=dev)
         ws_b = ctx.workspace(lvl, U, device=dev)
 
         def step(i):
             x, y = cts[i % N_SETS], ys[i % N_SETS]
-            for u in range(U):
-                ks.ckks_rotate_hoisted(ctx, x[u], lvl, gs, ev, rot[u], ws_h[u], stream)
+            # the 8 units' hoisted rotations in one call: one ModUp per unit, one inner-product
+            # launch over the 64 pairs, whose items with the same key share its keystream
+            ks.ckks_rotate_hoisted_batch(ctx, x, lvl, gs, ev, rot, ws_h, stream)
             ks.ckks_tensor_batch(ctx, U, x, y, lvl, d, stream)
             ks.ckks_relin_batch(ctx, d, lvl, [k_rel] * U, rl, ws_b, stream)
         ks_per_step, rot_per_step = U * (R + 1), U * R

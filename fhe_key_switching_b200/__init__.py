@@ -71,6 +71,8 @@ _SIGS = {
     "ckks_rotate": (_ci, [_vp, _vp, _ci, _cu, ctypes.POINTER(ckks_evk), _vp, _vp, _sz, _vp]),
     "ckks_rotate_hoisted": (_ci, [_vp, _vp, _ci, _ci, _u32p, ctypes.POINTER(ckks_evk), _vp, _vp,
                                   _sz, _vp]),
+    "ckks_rotate_hoisted_batch": (_ci, [_vp, _ci, _vp, _ci, _ci, _u32p, ctypes.POINTER(ckks_evk), _vp, _vp,
+                                        _sz, _vp]),
     "ckks_relin": (_ci, [_vp, _vp, _ci, ctypes.POINTER(ckks_evk), _vp, _vp, _sz, _vp]),
     "ckks_keyswitch_batch": (_ci, [_vp, _ci, _vp, _ci, ctypes.POINTER(ckks_evk), _vp, _vp, _sz, _vp]),
     "ckks_rotate_batch": (_ci, [_vp, _ci, _vp, _ci, _u32p, ctypes.POINTER(ckks_evk), _vp, _vp, _sz, _vp]),
@@ -559,3 +561,13 @@ def ckks_bootstrap(ctx, ct, plan: BootstrapPlan, out, ws, stream=None):
                              ctypes.byref(ratio), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "ckks_bootstrap")
     return lv.value, ratio.value
+
+
+def ckks_rotate_hoisted_batch(ctx, ct, level: int, galois, evks, out, ws, stream=None):
+    """ct [n_ct][2][l+1][N] -> out [n_ct][n_rot][2][l+1][N]: every ciphertext rotated by every
+    Galois element, one ModUp per ciphertext."""
+    n_rot = len(galois)
+    ga = (ctypes.c_uint32 * n_rot)(*galois)
+    _check(_L.ckks_rotate_hoisted_batch(ctx.handle, ct.shape[0], _ptr(ct), level, n_rot, ga, _evk_array(evks),
+                                        _ptr(out), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "ckks_rotate_hoisted_batch")

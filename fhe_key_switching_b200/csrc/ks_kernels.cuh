@@ -501,6 +501,8 @@ struct IpRowArgs {
     const u32 *cdig;         // [l+1][N] input polynomial, evaluation domain
     u32 *acc;                // [2][ext][N]
     size_t x_item, cdig_item, acc_item;        // item strides (words; 0 = shared)
+    int item_div;            // item z reads x and cdig of source z / item_div (hoisted batches of
+                             // several ciphertexts: item_div rotations per ciphertext; 0 reads as 1)
     const tw_t *twf, *twi;
     const PrimeInfo *pinfo;
     int log_n, level, n_q, n_primes, alpha, beta, ext;
@@ -560,8 +562,9 @@ k_ip_row(IpRowArgs a) {
     }
     for (int it = 0; it < gcnt; it++) {
         const int item = a.grp_item[g0 + it];
-        const u32 *xb = a.x + item * a.x_item;
-        const u32 *cdb = a.cdig + item * a.cdig_item;
+        const int src_item = item / max(1, a.item_div);
+        const u32 *xb = a.x + src_item * a.x_item;
+        const u32 *cdb = a.cdig + src_item * a.cdig_item;
         u32 *accb = a.acc + item * a.acc_item;
         const u32 *bkey = a.b[item];
         const u32 *astore = a.a_stored[item];
@@ -695,8 +698,9 @@ k_ip_row8(IpRowArgs a) {
     }
     for (int it = 0; it < gcnt; it++) {
         const int item = a.grp_item[g0 + it];
-        const u32 *xb = a.x + item * a.x_item;
-        const u32 *cdb = a.cdig + item * a.cdig_item;
+        const int src_item = item / max(1, a.item_div);
+        const u32 *xb = a.x + src_item * a.x_item;
+        const u32 *cdb = a.cdig + src_item * a.cdig_item;
         u32 *accb = a.acc + item * a.acc_item;
         const u32 *bkey = a.b[item];
         const u32 *astore = a.a_stored[item];
@@ -775,6 +779,7 @@ struct RowCombineArgs {
     const u32 *add;
     u32 *out;                // [n_comp][l+1][N]
     size_t conv_item, acc_item, add_item, out_item;   // item strides (words; 0 = shared)
+    int add_div;             // item z adds the polynomial of source z / add_div (0 reads as 1)
     const tw_t *twf;
     const PrimeInfo *pinfo;
     const tw_t *pinv;
@@ -813,7 +818,7 @@ k_row_combine(RowCombineArgs a) {
 #pragma unroll
     for (int v = 0; v < 8; v++) x[v] = csub(shoup_mul(ac[v] + q - x[v], w.x, w.y, q), q);
     if (comp < a.add_comps) {
-        const u32 *ad = a.add + item * a.add_item + ((size_t)comp * na + i) * n;
+        const u32 *ad = a.add + (item / max(1, a.add_div)) * a.add_item + ((size_t)comp * na + i) * n;
         u32 y[8];
         if (add_g) {
             const bool okg = CKKS_SPAN(ad, n, CKKS_DBG_COMBINE_ADD);          // automorph_src < n

@@ -141,6 +141,20 @@ int ckks_rotate_hoisted(ckks_ctx *ctx, const uint32_t *ct, int level, int n_rot,
                         const uint32_t *galois, const ckks_evk *keys, uint32_t *out, void *ws,
                         size_t ws_bytes, ckks_stream_t stream);
 
+/* Hoisted rotations of several ciphertexts by the same n_rot rotations: ct [n_ct][2][l+1][N],
+ * out [n_ct][n_rot][2][l+1][N]; output (u, r) equals ckks_rotate_hoisted of ciphertext u, rotation
+ * r, bit for bit (and so ckks_rotate).  One ModUp per ciphertext, then one inner product and
+ * ModDown launch over up to 64 (ciphertext, rotation) pairs, in which the pairs that use the same
+ * key regenerate its a half once per group of up to 8 (the a half is regenerated inside the kernel
+ * that uses the key: ai4snews write-up of Perseus, Interpretation, 2nd paragraph; hoisting several
+ * rotations over one ModUp is Halevi and Shoup's).  1 <= n_rot <= 64; the workspace is
+ * ckks_workspace_bytes(ctx, level, min(n_ct, 64 / n_rot) * n_rot).  Errors as for
+ * ckks_rotate_hoisted, and CKKS_ERR_ARG for n_ct < 0, n_rot outside 0..64 and overlaps between
+ * the input, the output and the workspace; n_ct = 0 or n_rot = 0 does nothing. */
+int ckks_rotate_hoisted_batch(ckks_ctx *ctx, int n_ct, const uint32_t *ct, int level, int n_rot,
+                              const uint32_t *galois, const ckks_evk *keys, uint32_t *out, void *ws,
+                              size_t ws_bytes, ckks_stream_t stream);
+
 /* Relinearisation: d [3][l+1][N] (decrypting under 1, s, s^2) -> out [2][l+1][N] =
  * (d0, d1) + keyswitch(d2) with the key for s^2. */
 int ckks_relin(ckks_ctx *ctx, const uint32_t *d, int level, const ckks_evk *evk, uint32_t *out,

@@ -257,3 +257,53 @@ def test_n16_stream64_shared_keystream_batches(ks_lib, oracle_mod):
         r = cfg.rot_steps[i]
         want = octx.rotate(got_r[i], lvl, cfg.alpha, gal[r], b_rot[r], cfg.chacha_seed, gal[r])
         assert np.array_equal(got_o[i], want), ("rotate", i)
+
+
+@pytest.mark.parametrize("key,n_ct,steps", [("n14-hoisted8", 8, (1, -1, 2, -2, 4, -4, 8, -8)),
+                                            ("n12-dnum4", 9, (1, -1, 2, -2, 4, -4, 8, -8)),
+                                            ("n14-hoisted8", 3, (5,))])
+def test_hoisted_batch_equals_per_ciphertext(ks_lib, key, n_ct, steps):
+    """ckks_rotate_hoisted_batch: output (u, r) equals ckks_rotate_hoisted of ciphertext u alone
+    (pinned to the oracle in test_gpu_parity), bit for bit; 9 x 8 pairs span two launches of 64 and
+    8, and one rotation per ciphertext takes the fused row pass."""
+    ks = ks_lib
+    cfg, q, p, ctx = _setup(ks, key)
+    lvl, N = cfg.level, cfg.n
+    na = lvl + 1
+    gen = W.rng(cfg.seed, W.TAG_SYNTH, 9700 + n_ct)
+    nd = -(-cfg.n_q // cfg.alpha)
+    gs = [ks.galois_element(cfg.log_n, r) for r in steps]
+    evks = [ks.make_evk(_res((q + p) * nd, N, gen).view(nd, len(q) + len(p), N), cfg.chacha_seed, g) for g in gs]
+    R = len(gs)
+    x = _res(q[:na] * 2 * n_ct, N, gen).view(n_ct, 2, na, N)
+    out = torch.empty((n_ct, R, 2, na, N), dtype=torch.uint32, device="cuda")
+    ws = ctx.workspace(lvl, min(n_ct, 64 // R) * R)
+    ks.ckks_rotate_hoisted_batch(ctx, x, lvl, gs, evks, out, ws)
+    one = torch.empty((R, 2, na, N), dtype=torch.uint32, device="cuda")
+    ws_1 = ctx.workspace(lvl, R)
+    for u in range(n_ct):
+        ks.ckks_rotate_hoisted(ctx, x[u], lvl, gs, evks, one, ws_1)
+        assert torch.equal(one, out[u]), u
+    assert ks.ckks_sync_status(ctx, None, 10000) == ks.CKKS_OK
+
+
+def test_hoisted_batch_sampled_oracle(ks_lib, oracle_mod):
+    """ckks_rotate_hoisted_batch at n14-hoisted8 with the oracle's keys: ciphertexts 0 and 5 of 8,
+    all 8 rotations, equal the oracle's hoisted rotations bit for bit."""
+    from oracle.scenario import Scenario
+    ks = ks_lib
+    cfg, q, p, ctx = _setup(ks, "n14-hoisted8")
+    sc = Scenario(cfg)
+    lvl, N = cfg.level, cfg.n
+    gs = [sc.galois(r) for r in cfg.rot_steps]
+    keys = [sc.key(g) for g in gs]
+    evks = [ks.make_evk(torch.from_numpy(k).cuda(), cfg.chacha_seed, g) for k, g in zip(keys, gs)]
+    cts = [sc.ciphertext(u)[1] for u in range(8)]
+    x = torch.from_numpy(np.stack(cts)).cuda()
+    out = torch.empty((8, len(gs), 2, lvl + 1, N), dtype=torch.uint32, device="cuda")
+    ks.ckks_rotate_hoisted_batch(ctx, x, lvl, gs, evks, out, ctx.workspace(lvl, 8 * len(gs)))
+    torch.cuda.synchronize()
+    got = out.cpu().numpy()
+    for u in (0, 5):
+        want = sc.ctx.rotate_hoisted(cts[u], lvl, cfg.alpha, gs, keys, [cfg.chacha_seed] * len(gs), gs)
+        assert np.array_equal(got[u], want), u
