@@ -63,3 +63,23 @@ def test_bootstrap_decodes_to_input(boot_case):
     assert lv == lout and out.shape == (2, lv + 1, cfg.n)
     got = sc.decrypt_slots(out, lv, sc.scale * ratio)
     assert np.max(np.abs(got - z)) < 2.0 ** -6
+
+
+def test_bootstrap_plans_are_the_dft_maps():
+    """The plans bootstrap_plans builds, applied in the clear level by level (baby-step giant-step
+    form), are half the CoeffToSlot map (the 1/2 of the real/imaginary split) and the SlotToCoeff
+    map of the oracle's stage factorisation, at N=2^7 with 2 and 3 levels."""
+    from oracle import bootstrap as bt
+    rng = np.random.default_rng(11)
+    for log_n, levels, n1 in ((7, 2, 4), (7, 3, 2)):
+        ns = 1 << (log_n - 1)
+        z = rng.normal(size=ns) + 1j * rng.normal(size=ns)
+        c2s, s2c = bt.bootstrap_plans(log_n, levels, n1)
+        x = z
+        for babies, giants, pt in c2s:
+            x = bt.apply_bsgs(x, babies, giants, pt)
+        assert np.allclose(x, 0.5 * bt.coeff_to_slot(z, log_n, levels), atol=1e-12)
+        y = z
+        for babies, giants, pt in s2c:
+            y = bt.apply_bsgs(y, babies, giants, pt)
+        assert np.allclose(y, bt.slot_to_coeff(z, log_n, levels), atol=1e-9)
