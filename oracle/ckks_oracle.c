@@ -107,8 +107,8 @@ typedef struct {
     int log_n, n, n_q, n_p;
     u32 *mod;          /* [n_q + n_p] */
     u32 *psi;          /* [n_q + n_p] */
-    u32 *psi_rev;      /* [n_q + n_p][N]: psi^brv(i) */
-    u32 *psi_inv_rev;  /* [n_q + n_p][N]: psi^-brv(i) */
+    u32 *psi_pow;      /* [n_q + n_p][N]: psi^i */
+    u32 *psi_inv_pow;  /* [n_q + n_p][N]: psi^-i */
 } or_ctx;
 
 or_ctx *or_ctx_create(int log_n, int n_q, int n_p, const u32 *q, const u32 *p) {
@@ -117,8 +117,8 @@ or_ctx *or_ctx_create(int log_n, int n_q, int n_p, const u32 *q, const u32 *p) {
     c->log_n = log_n; c->n = n; c->n_q = n_q; c->n_p = n_p;
     c->mod = (u32 *)malloc(sizeof(u32) * nt);
     c->psi = (u32 *)malloc(sizeof(u32) * nt);
-    c->psi_rev = (u32 *)malloc(sizeof(u32) * (size_t)nt * n);
-    c->psi_inv_rev = (u32 *)malloc(sizeof(u32) * (size_t)nt * n);
+    c->psi_pow = (u32 *)malloc(sizeof(u32) * (size_t)nt * n);
+    c->psi_inv_pow = (u32 *)malloc(sizeof(u32) * (size_t)nt * n);
     for (int t = 0; t < n_q; t++) c->mod[t] = q[t];
     for (int t = 0; t < n_p; t++) c->mod[n_q + t] = p[t];
 #pragma omp parallel for
@@ -127,12 +127,11 @@ or_ctx *or_ctx_create(int log_n, int n_q, int n_p, const u32 *q, const u32 *p) {
         u64 psi = or_find_psi((u32)m, log_n);
         u64 psi_inv = invmod(psi, m);
         c->psi[t] = (u32)psi;
-        /* powers psi^i for i < N, then scatter to bit-reversed index */
+        /* powers psi^i and psi^-i for i < N */
         u64 pw = 1, pwi = 1;
         for (int i = 0; i < n; i++) {
-            u32 r = brv((u32)i, log_n);
-            c->psi_rev[(size_t)t * n + r] = (u32)pw;
-            c->psi_inv_rev[(size_t)t * n + r] = (u32)pwi;
+            c->psi_pow[(size_t)t * n + i] = (u32)pw;
+            c->psi_inv_pow[(size_t)t * n + i] = (u32)pwi;
             pw = mulmod(pw, psi, m);
             pwi = mulmod(pwi, psi_inv, m);
         }
@@ -142,52 +141,62 @@ or_ctx *or_ctx_create(int log_n, int n_q, int n_p, const u32 *q, const u32 *p) {
 
 void or_ctx_destroy(or_ctx *c) {
     if (!c) return;
-    free(c->mod); free(c->psi); free(c->psi_rev); free(c->psi_inv_rev); free(c);
+    free(c->mod); free(c->psi); free(c->psi_pow); free(c->psi_inv_pow); free(c);
 }
 
 u32 or_ctx_psi(const or_ctx *c, int t) { return c->psi[t]; }
 
 /* ------------------------------------------------------------------ NTT
  * Negacyclic NTT, defined as  A[k] = sum_{n<N} a[n] * psi^((2*brv(k)+1)*n)  mod q.
- * Computed with the iterative Cooley-Tukey schedule that merges the psi powers into the
- * twiddles (stage with m butterfly groups uses psi^brv(m+i) for group i); its output is in
- * bit-reversed order, i.e. exactly the definition above.  The inverse undoes each stage in
- * reverse order, (X, Y) -> (X+Y, (X-Y)*psi^-brv(m+i)), then multiplies by N^-1.
+ * Factored as the definition reads: with b[n] = a[n] psi^n and omega = psi^2 (a primitive N-th
+ * root of unity), A[k] = B[brv(k)] where B[j] = sum_n b[n] omega^(n j) is the cyclic DFT of b.
+ * B is computed by the textbook iterative radix-2 decimation in time (inputs permuted to
+ * bit-reversed order, then stages of length 2, 4, ..., N with twiddle powers of
+ * omega^(N/len)), and read back at the bit-reversed index.  The inverse reads B[j] = A[brv(j)],
+ * runs the same transform with omega^-1, multiplies by N^-1 and untwists by psi^-n.
  */
-void or_ntt_fwd_limb(const or_ctx *c, int t, u32 *a) {
-    int n = c->n;
-    u64 q = c->mod[t];
-    const u32 *tw = c->psi_rev + (size_t)t * n;
-    for (int m = 1, half = n / 2; m < n; m *= 2, half /= 2) {
-        for (int i = 0; i < m; i++) {
-            u64 w = tw[m + i];
-            int j1 = 2 * i * half;
-            for (int j = j1; j < j1 + half; j++) {
-                u64 u = a[j], v = mulmod(a[j + half], w, q);
-                a[j] = (u32)((u + v) % q);
-                a[j + half] = (u32)((u + q - v) % q);
+static void cyclic_dft(u32 *x, int n, int log_n, u64 omega, u64 q) {
+    for (int i = 0; i < n; i++) {                     /* bit-reversal permutation */
+        int r = (int)brv((u32)i, log_n);
+        if (r > i) { u32 tmp = x[i]; x[i] = x[r]; x[r] = tmp; }
+    }
+    for (int len = 2; len <= n; len *= 2) {
+        u64 w_len = 1;                                /* omega^(N/len) */
+        for (int e = 0; e < n / len; e++) w_len = mulmod(w_len, omega, q);
+        for (int start = 0; start < n; start += len) {
+            u64 w = 1;
+            for (int j = 0; j < len / 2; j++) {
+                u64 u = x[start + j], v = mulmod(x[start + j + len / 2], w, q);
+                x[start + j] = (u32)((u + v) % q);
+                x[start + j + len / 2] = (u32)((u + q - v) % q);
+                w = mulmod(w, w_len, q);
             }
         }
     }
 }
 
-void or_ntt_inv_limb(const or_ctx *c, int t, u32 *a) {
-    int n = c->n;
+void or_ntt_fwd_limb(const or_ctx *c, int t, u32 *a) {
+    int n = c->n, log_n = c->log_n;
     u64 q = c->mod[t];
-    const u32 *tw = c->psi_inv_rev + (size_t)t * n;
-    for (int m = n / 2, half = 1; m >= 1; m /= 2, half *= 2) {
-        for (int i = 0; i < m; i++) {
-            u64 w = tw[m + i];
-            int j1 = 2 * i * half;
-            for (int j = j1; j < j1 + half; j++) {
-                u64 u = a[j], v = a[j + half];
-                a[j] = (u32)((u + v) % q);
-                a[j + half] = (u32)mulmod((u + q - v) % q, w, q);
-            }
-        }
-    }
+    const u32 *pw = c->psi_pow + (size_t)t * n;
+    u32 *b = (u32 *)malloc(sizeof(u32) * (size_t)n);
+    for (int i = 0; i < n; i++) b[i] = (u32)mulmod(a[i], pw[i], q);
+    cyclic_dft(b, n, log_n, mulmod(c->psi[t], c->psi[t], q), q);
+    for (int k = 0; k < n; k++) a[k] = b[brv((u32)k, log_n)];
+    free(b);
+}
+
+void or_ntt_inv_limb(const or_ctx *c, int t, u32 *a) {
+    int n = c->n, log_n = c->log_n;
+    u64 q = c->mod[t];
+    const u32 *pwi = c->psi_inv_pow + (size_t)t * n;
+    u32 *b = (u32 *)malloc(sizeof(u32) * (size_t)n);
+    for (int j = 0; j < n; j++) b[j] = a[brv((u32)j, log_n)];
+    u64 psi_inv = pwi[1 % n];
+    cyclic_dft(b, n, log_n, mulmod(psi_inv, psi_inv, q), q);
     u64 n_inv = invmod((u64)n % q, q);
-    for (int j = 0; j < n; j++) a[j] = (u32)mulmod(a[j], n_inv, q);
+    for (int i = 0; i < n; i++) a[i] = (u32)mulmod(mulmod(b[i], n_inv, q), pwi[i], q);
+    free(b);
 }
 
 /* batch over limbs first_limb .. first_limb+n_limbs-1 of a [limb][N] buffer whose row 0 is
