@@ -1018,7 +1018,7 @@ INFO_DESCRIPTIONS = {
     "coeff-to-slot": "N=2^16, 36+12 primes, dnum 4, from level 24; step = CoeffToSlot in 3 levels of 5 radix-2 "
                      "stages, each an 8 baby x 8 giant step transform of 63 slot diagonals plus a rescale",
     "n14-hoisted8": "N=2^14, 12+4 primes, dnum 3, level 11; step = 8 units, each 8 hoisted rotations "
-                    "(+-1, +-2, +-4, +-8) + tensor + relin",
+                    "(+-1, +-2, +-4, +-8) + tensor + relin; the units' rotations as one ckks_rotate_hoisted_batch call",
     "n16-bsgs32": "N=2^16, 36+12 primes, dnum 4, level 24; step = 32 hoisted rotations of one ciphertext",
     "n16-stream64": "N=2^16, 36+12 primes, dnum 4, level 20; step = 64 pairs, each tensor + relin + "
                     "rotate by 2^(i mod 15)",
