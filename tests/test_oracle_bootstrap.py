@@ -83,3 +83,30 @@ def test_bootstrap_plans_are_the_dft_maps():
         for babies, giants, pt in s2c:
             y = bt.apply_bsgs(y, babies, giants, pt)
         assert np.allclose(y, bt.slot_to_coeff(z, log_n, levels), atol=1e-9)
+
+
+def test_monomial_half_is_the_negacyclic_product(oracle_mod):
+    """mul_monomial_half at N=2^4 (2 primes) against the negacyclic product with X^(N/2) by brute
+    force: c_k = sum_{i+j = k} a_i m_j - sum_{i+j = k+N} a_i m_j, m the monomial."""
+    from oracle import bootstrap as bt
+    log_n = 4
+    n = 1 << log_n
+    octx = oracle_mod.Ctx(log_n, 2, 1)
+    rng = np.random.default_rng(12)
+    level = 1
+    comps = [np.stack([rng.integers(0, q, size=n) for q in octx.q[: level + 1]]).astype(np.uint32)
+             for _ in range(2)]
+    ct = np.stack([octx.ntt_fwd(c, 0) for c in comps])
+    got = bt.mul_monomial_half(octx, ct, level)
+    for comp in range(2):
+        a = octx.ntt_inv(ct[comp], 0).astype(np.int64)
+        out = octx.ntt_inv(got[comp], 0).astype(np.int64)
+        for t, q in enumerate(octx.q[: level + 1]):
+            want = np.zeros(n, dtype=object)
+            for i in range(n):
+                k = i + n // 2
+                if k < n:
+                    want[k] += int(a[t, i])
+                else:
+                    want[k - n] -= int(a[t, i])
+            assert [int(v) % q for v in want] == [int(v) for v in out[t]]
